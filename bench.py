@@ -1,0 +1,541 @@
+"""Benchmark of the BEAM-masked MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl beam|reference]
+
+Workload (decode, Qwen3-30B-A3B-shaped bf16 layer): d=2048, E=128 experts,
+top-8, SwiGLU I=768, softmax renormalised over the Top-K, Zipf(1.1) expert
+skew, synthetic seeded data (dynamic_expert_routing_router_b200/inputs.py).
+The headline is T=128 tokens per step with the mask router keeping ~15% of the
+candidates (the paper's 1.23-of-8 operating point).  A step is one full layer
+forward (7 kernels) through the C ABI on one batch already resident in HBM;
+8 distinct token batches are cycled and L2 is flushed (256 MiB write) before
+every timed step.  Each step is timed with CUDA events on the launch stream,
+recorded by the library between its kernels, so the per-kernel times come from
+the same timed region.  The same line reports every kept fraction and T of the
+decode configuration next to the same kernels with the mask disabled, the
+end-to-end rate through host buffers, and the fp64 CPU oracle as a baseline.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica on
+its own batches (tokens are independent, no collective on the data path);
+time = max over ranks; value = all ranks' tokens / that time ("weak").
+
+--impl reference times the oracle (the plain fp64 CPU definition) on the same
+workload, a bounded sample per step, on the host cores of rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BEAM MoE-layer tokens/s & % roofline vs unmasked top-K, per kept fraction"
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+N_BATCHES = 8
+FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------- distributed --
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def reduce_time_and_units(seconds, units, world, device=None):
+    """(max seconds over ranks, sum of units over ranks)."""
+    if world <= 1:
+        return seconds, units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- peaks --
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=HBM_FALLBACK_GBS, bf16=BF16_FALLBACK_TFLOPS,
+                    bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, period_ms=100):
+        self.idx = gpu_index
+        self.proc = None
+        self.period = period_ms
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period), "-i", str(self.idx)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [c.strip() for c in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- workload --
+
+class Layer:
+    """The decode layer on one GPU: weights, token batches, mask routers."""
+
+    def __init__(self, T, device, rank, seed=0, share=None):
+        import torch
+        from dynamic_expert_routing_router_b200 import abi, inputs
+        self.torch, self.abi, self.inputs = torch, abi, inputs
+        self.sh = sh = inputs.QWEN3
+        self.T = T
+        self.device = device
+        if share is not None:  # same layer weights, another batch size
+            self.W1, self.W3, self.W2, self.Wg = share.W1, share.W3, share.W2, share.Wg
+            self.masks = share.masks
+        else:
+            self.W1, self.W3, self.W2 = inputs.make_experts(sh, seed=seed, device=device)
+            self.Wg = inputs.make_gate(sh, seed=seed, device=device)
+            self.masks = {}
+        self.xs = [inputs.make_tokens(sh, T, seed=1000 * (rank + 1) + b, device=device)
+                   for b in range(N_BATCHES)]
+        self.dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+        self.ws = abi.alloc_workspace(self.dsc, device)
+        self.out = torch.empty((T, sh.d), dtype=torch.bfloat16, device=device)
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def mask(self, f):
+        if f is None:
+            return None
+        if f not in self.masks:
+            self.masks[f] = self.inputs.make_mask(self.sh, f, seed=0, device=self.device)
+        return self.masks[f]
+
+    def routing_stats(self, f):
+        """Per batch: kept pairs P, experts touched U (from the library's counters)."""
+        torch = self.torch
+        Wm = self.mask(f)
+        stats = []
+        for x in self.xs:
+            self.abi.forward(self.dsc, x, self.Wg, Wm, self.W1, self.W3, self.W2, self.out,
+                             self.ws)
+            self.abi.check(self.dsc, self.ws)
+            v = self.abi.workspace_views(self.dsc, self.ws)
+            c = v["counts"].cpu()
+            stats.append(dict(P=int(c.sum()), U=int((c > 0).sum()),
+                              hist=v["hist"].cpu().tolist()))
+        torch.cuda.synchronize()
+        return stats
+
+
+def algorithmic(layer, st, masked):
+    """Bytes and flops the method must move/do per stage for one batch."""
+    sh, T = layer.sh, layer.T
+    d, E, I, K = sh.d, sh.E, sh.I, sh.K
+    P, U = st["P"], st["U"]
+    rows = 2 * E if masked else E
+    return {
+        "router_gemm": dict(bytes=rows * d * 2 + T * d * 2, flops=2 * T * d * rows, unit="tensor"),
+        "topk_mask": dict(bytes=T * rows * 4 + T * K * 8, flops=0, unit="hbm"),
+        "permute": dict(bytes=T * K * 4 + 2 * P * 4, flops=0, unit="hbm"),
+        "gather": dict(bytes=2 * P * d * 2, flops=0, unit="hbm"),
+        "gemm1_gate_up_swiglu": dict(bytes=U * 2 * I * d * 2 + P * d * 2 + P * I * 2,
+                                     flops=4 * d * I * P, unit="tensor"),
+        "gemm2_down": dict(bytes=U * d * I * 2 + P * I * 2 + P * d * 2, flops=2 * d * I * P,
+                           unit="tensor"),
+        "combine": dict(bytes=P * d * 2 + T * d * 2 + T * K * 8, flops=0, unit="hbm"),
+    }
+
+
+def layer_roofline_seconds(layer, st, masked, pk):
+    """t_roof = router + experts + permute/combine floors (HBM or tensor, whichever binds)."""
+    sh, T = layer.sh, layer.T
+    d, E, I = sh.d, sh.E, sh.I
+    P, U = st["P"], st["U"]
+    bw = pk["hbm"] * 1e9
+    tc = pk["bf16"] * 1e12
+    rows = 2 * E if masked else E
+    t = max((rows * d * 2 + T * d * 2) / bw, 2 * T * d * rows / tc)
+    t += max(U * 3 * d * I * 2 / bw, 6 * d * I * P / tc)
+    t += (P * d * 2 + T * d * 2) / bw
+    return t
+
+
+def time_steps(layer, f, steps, warmup, profiled=True, graph=False):
+    """Per-step device times (s) and per-stage times (s) over `steps` steps."""
+    torch, abi = layer.torch, layer.abi
+    Wm = layer.mask(f)
+    S = abi.FORWARD_STAGES
+    stream = torch.cuda.current_stream()
+    args = (layer.dsc, None, layer.Wg, Wm, layer.W1, layer.W3, layer.W2, layer.out, layer.ws)
+
+    def call(x, events=None):
+        a = list(args)
+        a[1] = x
+        if events is not None:
+            abi.forward_profiled(*a, events)
+        else:
+            abi.forward(*a)
+
+    graphs = None
+    if graph:
+        graphs = []
+        s = torch.cuda.Stream()
+        s.wait_stream(stream)
+        with torch.cuda.stream(s):
+            for b in range(N_BATCHES):
+                call(layer.xs[b])
+            s.synchronize()
+            for b in range(N_BATCHES):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    a = list(args)
+                    a[1] = layer.xs[b]
+                    abi.forward(*a, stream=s)
+                graphs.append(g)
+        torch.cuda.synchronize()
+    for i in range(warmup):
+        layer.flush.fill_(i & 255)
+        if graph:
+            graphs[i % N_BATCHES].replay()
+        else:
+            call(layer.xs[i % N_BATCHES])
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)] for _ in range(steps)]
+    for i in range(steps):
+        layer.flush.fill_(i & 255)
+        b = i % N_BATCHES
+        if graph:
+            evs[i][0].record()
+            graphs[b].replay()
+            evs[i][S].record()
+        elif profiled:
+            call(layer.xs[b], evs[i])
+        else:
+            evs[i][0].record()
+            call(layer.xs[b])
+            evs[i][S].record()
+    torch.cuda.synchronize()
+    step_s = [evs[i][0].elapsed_time(evs[i][S]) * 1e-3 for i in range(steps)]
+    stage_s = None
+    if profiled and not graph:
+        stage_s = [[evs[i][j].elapsed_time(evs[i][j + 1]) * 1e-3 for j in range(S)]
+                   for i in range(steps)]
+    abi.check(layer.dsc, layer.ws)
+    return step_s, stage_s
+
+
+def e2e_rate(layer, f, steps, warmup):
+    """Tokens/s through the C ABI with the batch in pinned host memory: H2D copy,
+    forward, D2H copy of the output, every step inside the timed region."""
+    torch = layer.torch
+    hx = [x.cpu().pin_memory() for x in layer.xs]
+    hout = torch.empty((layer.T, layer.sh.d), dtype=torch.bfloat16).pin_memory()
+    xdev = torch.empty_like(layer.xs[0])
+    Wm = layer.mask(f)
+
+    def step(i):
+        xdev.copy_(hx[i % N_BATCHES], non_blocking=True)
+        layer.abi.forward(layer.dsc, xdev, layer.Wg, Wm, layer.W1, layer.W3, layer.W2,
+                          layer.out, layer.ws)
+        hout.copy_(layer.out, non_blocking=True)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) * 1e-3
+    nbytes = layer.T * layer.sh.d * 2
+    return dict(value=layer.T * steps / sec, unit="tokens/s", h2d_bytes_per_step=nbytes,
+                d2h_bytes_per_step=nbytes)
+
+
+def cpu_baseline(layer, f, seconds, max_batches=None):
+    """The fp64 oracle (whole layer: logits, routing, mask, experts) on host cores,
+    on successive batches of the same workload until `seconds` have passed."""
+    import oracle
+    from dynamic_expert_routing_router_b200 import inputs
+    W = [inputs.host_array(t) for t in (layer.W1, layer.W3, layer.W2)]
+    Wg = inputs.host_array(layer.Wg)
+    Wm = layer.mask(f)
+    Wm = None if Wm is None else inputs.host_array(Wm)
+    xs = [inputs.host_array(x) for x in layer.xs]
+    sh = layer.sh
+    toks, t0, n = 0, time.perf_counter(), 0
+    while True:
+        oracle.forward(xs[n % len(xs)], Wg, Wm, *W, sh.K, sh.renorm, "bf16")
+        toks += layer.T
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_batches and n >= max_batches):
+            break
+    return dict(value=toks / el, unit="tokens/s", cores=oracle.max_threads(), kind="oracle",
+                sample=f"{n} batch(es) of T={layer.T} tokens (whole layer, fp64, kept pairs "
+                       f"only), {el:.1f} s")
+
+
+def run_beam(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    init_dist(world, "nccl")
+    pk = peaks()
+    T, f_head = args.T, args.kept
+
+    layer = Layer(T, device, rank)
+    st = layer.routing_stats(f_head)
+    P_mean = sum(s["P"] for s in st) / len(st)
+    U_mean = sum(s["U"] for s in st) / len(st)
+
+    # ---- headline timed region ------------------------------------------
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        step_s, stage_s = time_steps(layer, f_head, args.steps, args.warmup, profiled=True)
+        torch.cuda.synchronize()
+        barrier(world)
+    total = sum(step_s)
+    tmax, units = reduce_time_and_units(total, T * args.steps, world, device)
+    value = units / tmax
+
+    S = layer.abi.FORWARD_STAGES
+    names = [layer.abi.stage_name(j) for j in range(S)]
+    stage_mean = [sum(s[j] for s in stage_s) / len(stage_s) for j in range(S)]
+    step_mean = total / len(step_s)
+    kernels = {names[j]: dict(us=stage_mean[j] * 1e6, share=stage_mean[j] / step_mean)
+               for j in range(S)}
+    # dominant kernel vs its roofline (algorithmic bytes/flops averaged over batches)
+    dom = max(range(S), key=lambda j: stage_mean[j])
+    alg = [algorithmic(layer, st[i % N_BATCHES], True) for i in range(args.steps)]
+    a_bytes = sum(a[names[dom]]["bytes"] for a in alg) / len(alg)
+    a_flops = sum(a[names[dom]]["flops"] for a in alg) / len(alg)
+    t_dom = stage_mean[dom]
+    hbm_t = a_bytes / (pk["hbm"] * 1e9)
+    tc_t = a_flops / (pk["bf16"] * 1e12)
+    if tc_t > hbm_t:
+        achieved, peak, unit, bound = a_flops / t_dom / 1e12, pk["bf16"], "TFLOP/s", "tensor"
+    else:
+        achieved, peak, unit, bound = a_bytes / t_dom / 1e9, pk["hbm"], "GB/s", "hbm"
+    roofline = dict(kernel=names[dom], bound=bound, achieved=achieved, peak=peak, unit=unit,
+                    frac=achieved / peak, traffic=None, peak_source=pk["source"],
+                    algorithmic_bytes_per_launch=a_bytes, algorithmic_flops_per_launch=a_flops)
+    t_roof = sum(layer_roofline_seconds(layer, st[i % N_BATCHES], True, pk)
+                 for i in range(args.steps)) / args.steps
+
+    # graph-replayed headline (launch overhead removed)
+    g_step, _ = time_steps(layer, f_head, max(50, min(args.steps, 500)), 3, profiled=False,
+                           graph=True)
+    g_mean = sum(g_step) / len(g_step)
+
+    # ---- per kept fraction, next to the mask-disabled kernels -------------
+    sweep = []
+    if not args.no_sweep:
+        Ts = sorted(set([1, 8, 32, 128, T]))
+        for Tn in Ts:
+            lay = layer if Tn == T else Layer(Tn, device, rank, share=layer)
+            base = None
+            rows = []
+            for f in (None, 0.15, 0.35, 0.6, 1.0):
+                sts = lay.routing_stats(f)
+                gs, _ = time_steps(lay, f, 100, 5, profiled=False, graph=True)
+                tm = sum(gs) / len(gs)
+                troof = sum(layer_roofline_seconds(lay, s, f is not None, pk) for s in sts) / len(sts)
+                kept = sum(s["P"] for s in sts) / len(sts) / (Tn * lay.sh.K)
+                row = dict(T=Tn, kept_target=f if f is not None else "unmasked",
+                           kept_measured=round(kept, 4),
+                           experts_touched=sum(s["U"] for s in sts) / len(sts),
+                           tokens_per_s=Tn / tm, us_per_layer=tm * 1e6,
+                           roofline_us=troof * 1e6, roofline_frac=troof / tm)
+                if f is None:
+                    base = tm
+                else:
+                    row["speedup_vs_unmasked"] = base / tm
+                rows.append(row)
+            sweep += rows
+            if lay is not layer:
+                del lay
+
+    e2e = e2e_rate(layer, f_head, max(20, min(args.steps, 500)), 5)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(layer, f_head, args.cpu_seconds)
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tmax / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": (f"decode MoE layer, Qwen3-30B-A3B shape (d=2048, E=128, K=8, I=768, "
+                         f"renorm), T={T} tokens/step/GPU, mask kept ~{f_head:.0%}"),
+            "T": T, "kept_fraction_target": f_head,
+            "kept_fraction_measured": P_mean / (T * layer.sh.K),
+            "experts_touched_mean": U_mean, "kept_pairs_mean": P_mean,
+            "l2": "flushed (256 MiB write) before every timed step; 8 token batches cycled",
+            "timing": "CUDA events recorded by the library between its kernels, eager calls",
+            "parallelism": f"replicas x{world} (tokens independent, no collective)",
+        },
+        "ms_per_step_graph": g_mean * 1e3,
+        "layer_roofline": dict(us=t_roof * 1e6, frac_of_measured_step=t_roof / step_mean,
+                               frac_graph=t_roof / g_mean, peak_source=pk["source"]),
+        "roofline": roofline,
+        "kernels": kernels,
+        "per_kept_fraction": sweep,
+        "e2e": e2e,
+        "gpu_launches": S * args.steps,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from dynamic_expert_routing_router_b200 import inputs
+    sh = inputs.QWEN3
+    T, f = args.T, args.kept
+    W1, W3, W2 = (inputs.host_array(t) for t in inputs.make_experts(sh, seed=0, device="cpu"))
+    Wg = inputs.host_array(inputs.make_gate(sh, seed=0, device="cpu"))
+    Wm = inputs.host_array(inputs.make_mask(sh, f, seed=0, device="cpu"))
+    xs = [inputs.host_array(inputs.make_tokens(sh, T, seed=1000 + b, device="cpu"))
+          for b in range(N_BATCHES)]
+    # each step: one bounded sample of the batch (its first n tokens, whole layer)
+    n = min(T, args.ref_tokens)
+
+    def step(i):
+        oracle.forward(np.ascontiguousarray(xs[i % N_BATCHES][:n]), Wg, Wm, W1, W3, W2, sh.K,
+                       sh.renorm, "bf16")
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": (f"decode MoE layer, Qwen3-30B-A3B shape (d=2048, E=128, K=8, "
+                                f"I=768, renorm), T={T} tokens/step, mask kept ~{f:.0%}"),
+                   "T": T, "kept_fraction_target": f},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"first {n} tokens of each T={T} batch per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["beam", "reference"], default="beam")
+    ap.add_argument("--T", type=int, default=128)
+    ap.add_argument("--kept", type=float, default=0.15)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-tokens", type=int, default=32)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_beam(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,430 @@
+// beam_api.cu -- the C entry points of libbeam_moe.so: argument checks,
+// workspace layout, tensor-map encoding and the launch sequence of the BEAM
+// MoE layer (router GEMM -> top-K + mask -> grouping -> gather -> gate/up GEMM
+// + SwiGLU -> down GEMM -> combine).  Everything is stream-ordered; nothing
+// here synchronises the host except beam_moe_check, and nothing allocates.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "beam_internal.h"
+#include "beam_moe.h"
+
+using namespace beam;
+
+namespace {
+
+constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s per bounded wait
+constexpr int kMaxDevices = 64;
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+beam_status validate_desc(const beam_moe_desc *d) {
+    if (!d) return BEAM_ERR_INVALID_ARG;
+    if (d->T < 0 || d->d <= 0 || d->E <= 0 || d->I <= 0 || d->K <= 0) return BEAM_ERR_INVALID_ARG;
+    if (d->K > d->E || d->K > kMaxK || d->E > kMaxE) return BEAM_ERR_INVALID_ARG;
+    if (d->dtype != BEAM_BF16 && d->dtype != BEAM_F32) return BEAM_ERR_INVALID_ARG;
+    if (d->renorm_topk != 0 && d->renorm_topk != 1) return BEAM_ERR_INVALID_ARG;
+    if (d->dtype == BEAM_BF16) {
+        if (d->d % kBlockM != 0 || d->I % kBlockM != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    } else {
+        if (d->d % 8 != 0 || d->I % 8 != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    }
+    if ((long long)d->T * d->K > INT_MAX / 2) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    return BEAM_OK;
+}
+
+// Token-tile height of the expert GEMMs from the mean kept-or-not pairs per
+// expert (T*K/E): decode batches use thin tiles, prefill batches 128 rows.
+int choose_bn(const beam_moe_desc *d) {
+    const long long avg = cdiv((long long)d->T * d->K, d->E);
+    if (avg <= 16) return 16;
+    if (avg <= 32) return 32;
+    if (avg <= 64) return 64;
+    return 128;
+}
+
+beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
+    beam_status st = validate_desc(d);
+    if (st != BEAM_OK) return st;
+    std::memset(P, 0, sizeof(*P));
+    const long long T = d->T, K = d->K, E = d->E;
+    P->BN = choose_bn(d);
+    if (d->dtype == BEAM_BF16) {
+        // Router: enough (token tile x row block x split) units to cover the
+        // SMs at decode sizes, while the split partials stay smaller than the
+        // router weights; prefill needs no split.
+        P->router_bn = T >= 1024 ? 128 : T >= 256 ? 64 : T > 16 ? 32 : 16;
+        const long long n_tt = T > 0 ? cdiv(T, P->router_bn) : 1;
+        const long long base = n_tt * 2 * cdiv(E, kBlockM);
+        const long long nkb = d->d / kBlockK;
+        const long long cap_bytes = T > 0 ? d->d / (2 * T) : nkb;
+        int S = 1;
+        while (2LL * S <= nkb && nkb % (2LL * S) == 0 && base * 2 * S <= kNominalSMs &&
+               2LL * S <= (cap_bytes > 1 ? cap_bytes : 1))
+            S *= 2;
+        P->router_splits = S;
+    } else {
+        P->router_bn = 16;
+        P->router_splits = 1;
+    }
+    const long long p_cap = T * K + E * (P->BN - 1);
+    const long long tiles_cap = cdiv(T * K, P->BN) + E;
+    if (p_cap > INT_MAX / 2 || tiles_cap > INT_MAX / 2) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    P->p_cap = int(p_cap);
+    P->tiles_cap = int(tiles_cap);
+    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
+    size_t o = 0;
+    P->off_err = 0;
+    P->off_meta = 16;
+    P->off_counts = 256;
+    P->off_hist = align256(P->off_counts + 4 * size_t(E));
+    P->off_partial = align256(P->off_hist + 4 * size_t(K + 1));
+    P->off_idx = align256(P->off_partial + 4 * size_t(P->router_splits) * size_t(T) * 2 * size_t(E));
+    P->off_w = align256(P->off_idx + 4 * size_t(T * K));
+    P->off_pair = align256(P->off_w + 4 * size_t(T * K));
+    P->off_pair_pos = align256(P->off_pair + 4 * size_t(p_cap));
+    P->off_tiles = align256(P->off_pair_pos + 4 * size_t(T * K));
+    P->off_xp = align256(P->off_tiles + 16 * size_t(tiles_cap));
+    P->off_h = align256(P->off_xp + es * size_t(p_cap) * size_t(d->d));
+    P->off_y = align256(P->off_h + es * size_t(p_cap) * size_t(d->I));
+    o = align256(P->off_y + es * size_t(p_cap) * size_t(d->d));
+    P->workspace_bytes = o;
+    return BEAM_OK;
+}
+
+int sm_count() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return kNominalSMs;
+    if (dev < 0 || dev >= kMaxDevices) return kNominalSMs;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = kNominalSMs;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows, inner] matrix, box = 64 x box_rows,
+// 128-byte swizzle (matches the UMMA descriptors in tc_gemm.cu), zero fill.
+bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
+               unsigned long long rows, unsigned box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn || rows == 0) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {unsigned(kBlockK), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct Recorder {
+    void *const *events;
+    cudaStream_t st;
+    cudaError_t rec(int i) const {
+        if (!events) return cudaSuccess;
+        return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+    }
+};
+
+#define BEAM_TRY_CUDA(expr)                          \
+    do {                                             \
+        cudaError_t e_ = (expr);                     \
+        if (e_ != cudaSuccess) return BEAM_ERR_CUDA; \
+    } while (0)
+
+struct RouteOut {
+    int *idx;
+    float *w;
+    int *counts;
+    int *hist;
+    float *logits;
+};
+
+// Stages 0-1: router GEMM into the split partials, then top-K + mask.
+beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, const void *x,
+                         const void *Wg, const void *Wm, const RouteOut &ro, char *ws,
+                         cudaStream_t st, const Recorder &rec, int n_sm) {
+    float *partial = reinterpret_cast<float *>(ws + P.off_partial);
+    int *hdr = reinterpret_cast<int *>(ws);  // err + meta (8 ints)
+    ZeroRegion zero[3] = {{hdr, 8}, {ro.counts, d->E}, {ro.hist, ro.hist ? d->K + 1 : 0}};
+    BEAM_TRY_CUDA(rec.rec(0));
+    if (d->dtype == BEAM_BF16) {
+        CUtensorMap mWg, mWm, mX;
+        if (!make_tmap(&mWg, Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mWm, Wm ? Wm : Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mX, x, d->d, d->T, P.router_bn)) return BEAM_ERR_CUDA;
+        TcGemmArgs a;
+        std::memset(&a, 0, sizeof(a));
+        const int mb_per = int(cdiv(d->E, kBlockM));
+        a.n_mb_gate = mb_per;
+        a.n_mb = Wm ? 2 * mb_per : mb_per;
+        a.n_tt = int(cdiv(d->T, P.router_bn));
+        a.nk = d->d / kBlockK / P.router_splits;
+        a.n_units = a.n_mb * a.n_tt * P.router_splits;
+        a.T = d->T;
+        a.E = d->E;
+        a.out = partial;
+        a.out_ld = 2LL * d->E;
+        a.out_split_stride = (long long)d->T * 2 * d->E;
+        a.err = hdr;
+        a.zero[0] = zero[0];
+        a.zero[1] = zero[1];
+        a.zero[2] = zero[2];
+        a.timeout_ns = kWaitTimeoutNs;
+        const int grid = a.n_units < n_sm ? a.n_units : n_sm;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_ROUTER, P.router_bn, mWg, mWm, mX, a, grid, st));
+    } else {
+        BEAM_TRY_CUDA(launch_router_f32(static_cast<const float *>(x), static_cast<const float *>(Wg),
+                                        static_cast<const float *>(Wm), d->T, d->d, d->E, partial,
+                                        zero, st));
+    }
+    BEAM_TRY_CUDA(rec.rec(1));
+    TopkArgs t;
+    t.partial = partial;
+    t.S = P.router_splits;
+    t.T = d->T;
+    t.E = d->E;
+    t.K = d->K;
+    t.renorm = d->renorm_topk;
+    t.has_mask = Wm != nullptr;
+    t.logits = ro.logits;
+    t.idx = ro.idx;
+    t.w = ro.w;
+    t.counts = ro.counts;
+    t.hist = ro.hist;
+    BEAM_TRY_CUDA(launch_topk_mask(t, n_sm, st));
+    return BEAM_OK;
+}
+
+beam_status check_ws(const beam_moe_plan_info &P, const void *ws, size_t bytes) {
+    if (!ws || !aligned16(ws) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return BEAM_ERR_WORKSPACE;
+    if (bytes < P.workspace_bytes) return BEAM_ERR_WORKSPACE;
+    return BEAM_OK;
+}
+
+beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, const void *Wm,
+                         const void *W1, const void *W3, const void *W2, void *out, void *workspace,
+                         size_t ws_bytes, void *stream, void *const *events) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(d, &P);
+    if (s != BEAM_OK) return s;
+    if (!x || !Wg || !W1 || !W3 || !W2 || !out) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x, Wg, W1, W3, W2, static_cast<const void *>(out)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    if (Wm && !aligned16(Wm)) return BEAM_ERR_INVALID_ARG;
+    s = check_ws(P, workspace, ws_bytes);
+    if (s != BEAM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Recorder rec{events, st};
+    if (d->T == 0) {
+        for (int i = 0; i <= BEAM_MOE_FORWARD_STAGES; ++i) BEAM_TRY_CUDA(rec.rec(i));
+        return BEAM_OK;
+    }
+    const int n_sm = sm_count();
+    char *ws = static_cast<char *>(workspace);
+    int *err = reinterpret_cast<int *>(ws + P.off_err);
+    int *meta = reinterpret_cast<int *>(ws + P.off_meta);
+    int *counts = reinterpret_cast<int *>(ws + P.off_counts);
+    int *hist = reinterpret_cast<int *>(ws + P.off_hist);
+    int *idx = reinterpret_cast<int *>(ws + P.off_idx);
+    float *w = reinterpret_cast<float *>(ws + P.off_w);
+    int *pair = reinterpret_cast<int *>(ws + P.off_pair);
+    int *pair_pos = reinterpret_cast<int *>(ws + P.off_pair_pos);
+    int4 *tiles = reinterpret_cast<int4 *>(ws + P.off_tiles);
+    void *xp = ws + P.off_xp;
+    void *h = ws + P.off_h;
+    void *y = ws + P.off_y;
+
+    const RouteOut ro{idx, w, counts, hist, nullptr};
+    s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
+    if (s != BEAM_OK) return s;
+
+    BEAM_TRY_CUDA(rec.rec(2));
+    PermuteArgs pa{idx, counts, d->T, d->K, d->E, P.BN, pair, pair_pos, tiles, meta, err};
+    BEAM_TRY_CUDA(launch_permute(pa, st));
+
+    BEAM_TRY_CUDA(rec.rec(3));
+    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
+    BEAM_TRY_CUDA(launch_gather(x, pair, meta, d->K, (long long)es * d->d, P.p_cap, xp, n_sm, st));
+
+    if (d->dtype == BEAM_BF16) {
+        CUtensorMap mW1, mW3, mW2, mXp, mH;
+        if (!make_tmap(&mW1, W1, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mW3, W3, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mW2, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mXp, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mH, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+
+        TcGemmArgs g;
+        std::memset(&g, 0, sizeof(g));
+        g.meta = meta;
+        g.tiles = tiles;
+        g.err = err;
+        g.timeout_ns = kWaitTimeoutNs;
+
+        BEAM_TRY_CUDA(rec.rec(4));
+        g.n_mb = d->I / kBlockM;
+        g.nk = d->d / kBlockK;
+        g.a_rows_per_expert = d->I;
+        g.out = h;
+        g.out_ld = d->I;
+        long long units = (long long)P.tiles_cap * g.n_mb;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, mW1, mW3, mXp, g,
+                                     int(units < n_sm ? units : n_sm), st));
+
+        BEAM_TRY_CUDA(rec.rec(5));
+        g.n_mb = d->d / kBlockM;
+        g.nk = d->I / kBlockK;
+        g.a_rows_per_expert = d->d;
+        g.out = y;
+        g.out_ld = d->d;
+        units = (long long)P.tiles_cap * g.n_mb;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, P.BN, mW2, mW2, mH, g,
+                                     int(units < n_sm ? units : n_sm), st));
+    } else {
+        BEAM_TRY_CUDA(rec.rec(4));
+        BEAM_TRY_CUDA(launch_gemm1_f32(static_cast<const float *>(xp), static_cast<const float *>(W1),
+                                       static_cast<const float *>(W3), tiles, meta, P.tiles_cap,
+                                       d->d, d->I, static_cast<float *>(h), st));
+        BEAM_TRY_CUDA(rec.rec(5));
+        BEAM_TRY_CUDA(launch_gemm2_f32(static_cast<const float *>(h), static_cast<const float *>(W2),
+                                       tiles, meta, P.tiles_cap, d->d, d->I,
+                                       static_cast<float *>(y), st));
+    }
+
+    BEAM_TRY_CUDA(rec.rec(6));
+    BEAM_TRY_CUDA(launch_combine(d->dtype, y, idx, w, pair_pos, d->T, d->K, d->d, out, n_sm, st));
+    BEAM_TRY_CUDA(rec.rec(7));
+    return BEAM_OK;
+}
+
+const char *const kStageNames[BEAM_MOE_FORWARD_STAGES] = {
+    "router_gemm", "topk_mask", "permute", "gather", "gemm1_gate_up_swiglu", "gemm2_down",
+    "combine"};
+
+}  // namespace
+
+extern "C" {
+
+size_t beam_moe_workspace_size(const beam_moe_desc *desc) {
+    beam_moe_plan_info P;
+    if (make_plan(desc, &P) != BEAM_OK) return 0;
+    return P.workspace_bytes;
+}
+
+beam_status beam_moe_plan(const beam_moe_desc *desc, beam_moe_plan_info *info) {
+    if (!info) return BEAM_ERR_INVALID_ARG;
+    return make_plan(desc, info);
+}
+
+beam_status beam_moe_route(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                           const void *W_mask, int32_t *topk_idx, float *topk_w,
+                           int32_t *expert_counts, int32_t *kept_hist, float *logits,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(desc, &P);
+    if (s != BEAM_OK) return s;
+    if (!x || !W_gate || !topk_idx || !topk_w || !expert_counts) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x, W_gate, static_cast<const void *>(topk_idx),
+                          static_cast<const void *>(topk_w), static_cast<const void *>(expert_counts)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    if ((W_mask && !aligned16(W_mask)) || (kept_hist && !aligned16(kept_hist)) ||
+        (logits && !aligned16(logits)))
+        return BEAM_ERR_INVALID_ARG;
+    s = check_ws(P, workspace, workspace_bytes);
+    if (s != BEAM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (desc->T == 0) {
+        BEAM_TRY_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * desc->E, st));
+        if (kept_hist)
+            BEAM_TRY_CUDA(cudaMemsetAsync(kept_hist, 0, sizeof(int32_t) * (desc->K + 1), st));
+        return BEAM_OK;
+    }
+    const RouteOut ro{topk_idx, topk_w, expert_counts, kept_hist, logits};
+    const Recorder rec{nullptr, st};
+    return launch_route(desc, P, x, W_gate, W_mask, ro, static_cast<char *>(workspace), st, rec,
+                        sm_count());
+}
+
+beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                             const void *W_mask, const void *W1, const void *W3, const void *W2,
+                             void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, out, workspace, workspace_bytes,
+                        stream, nullptr);
+}
+
+beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
+                                      const void *W_gate, const void *W_mask, const void *W1,
+                                      const void *W3, const void *W2, void *out, void *workspace,
+                                      size_t workspace_bytes, void *stream,
+                                      void *const *events) {
+    if (!events) return BEAM_ERR_INVALID_ARG;
+    for (int i = 0; i <= BEAM_MOE_FORWARD_STAGES; ++i)
+        if (!events[i]) return BEAM_ERR_INVALID_ARG;
+    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, out, workspace, workspace_bytes,
+                        stream, events);
+}
+
+beam_status beam_moe_check(const beam_moe_desc *desc, void *workspace, void *stream) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(desc, &P);
+    if (s != BEAM_OK) return s;
+    if (!workspace) return BEAM_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BEAM_ERR_CUDA;
+    int err = 0;
+    if (cudaMemcpy(&err, static_cast<char *>(workspace) + P.off_err, sizeof(int),
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return BEAM_ERR_CUDA;
+    if (err == DEV_ERR_TIMEOUT) return BEAM_ERR_TIMEOUT;
+    if (err != 0) return BEAM_ERR_INTERNAL;
+    return BEAM_OK;
+}
+
+const char *beam_status_str(beam_status status) {
+    switch (status) {
+        case BEAM_OK: return "BEAM_OK";
+        case BEAM_ERR_INVALID_ARG: return "BEAM_ERR_INVALID_ARG";
+        case BEAM_ERR_UNSUPPORTED_SHAPE: return "BEAM_ERR_UNSUPPORTED_SHAPE";
+        case BEAM_ERR_WORKSPACE: return "BEAM_ERR_WORKSPACE";
+        case BEAM_ERR_CUDA: return "BEAM_ERR_CUDA";
+        case BEAM_ERR_TIMEOUT: return "BEAM_ERR_TIMEOUT";
+        case BEAM_ERR_INTERNAL: return "BEAM_ERR_INTERNAL";
+    }
+    return "BEAM_ERR_UNKNOWN";
+}
+
+const char *beam_moe_stage_name(int stage) {
+    if (stage < 0 || stage >= BEAM_MOE_FORWARD_STAGES) return nullptr;
+    return kStageNames[stage];
+}
+
+}  // extern "C"

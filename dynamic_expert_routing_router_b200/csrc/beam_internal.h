@@ -1,0 +1,101 @@
+// beam_internal.h -- launch interface between the C-ABI host code
+// (beam_api.cu) and the kernels (tc_gemm.cu, simt_kernels.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "beam_moe.h"
+
+namespace beam {
+
+// Device error word values (workspace `err`).
+enum : int { DEV_OK = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_INTERNAL = 2 };
+
+// Roles of the tensor-core GEMM kernel.
+enum TcMode : int {
+    MODE_ROUTER = 0,  // logits: [W_gate | W_mask] rows x token rows, split over d
+    MODE_GEMM1 = 1,   // SiLU(W1 x) * (W3 x) per kept pair  -> H
+    MODE_GEMM2 = 2    // W2 h per kept pair                  -> Y
+};
+
+constexpr int kBlockM = 128;   // weight rows per tile (the MMA's M)
+constexpr int kBlockK = 64;    // reduction elements per stage: one 128-byte bf16 row
+constexpr int kNominalSMs = 148;
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 16;
+
+struct ZeroRegion {
+    int *ptr;
+    int count;
+};
+
+// Arguments of the tensor-core GEMM (all three modes).
+struct TcGemmArgs {
+    int n_mb;            // weight-row blocks per token tile
+    int nk;              // k-blocks per unit
+    int n_tt;            // router: token tiles
+    int n_mb_gate;       // router: m-blocks read from W_gate; the rest from W_mask
+    int n_units;         // router: number of units (GEMMs take it from meta[0])
+    int T, E;            // router: tokens and experts (logit columns 2E)
+    int a_rows_per_expert;  // GEMM1: I, GEMM2: d
+    const int *meta;     // GEMMs: meta[0] = tiles in the tile list
+    const int4 *tiles;   // GEMMs: (expert, first row, valid rows, 0)
+    void *out;           // router: f32 partial [S][T][2E]; GEMM1: H; GEMM2: Y (bf16)
+    long long out_ld;    // elements per output row
+    long long out_split_stride;  // router: elements per split slab
+    int *err;            // device error word
+    ZeroRegion zero[3];  // router: regions CTA 0 clears for the later kernels
+    unsigned long long timeout_ns;
+};
+
+cudaError_t launch_tc_gemm(int mode, int bn, const CUtensorMap &a0, const CUtensorMap &a1,
+                           const CUtensorMap &b, const TcGemmArgs &args, int grid,
+                           cudaStream_t stream);
+
+// Top-K + softmax + mask + aggregation (one warp per token).
+struct TopkArgs {
+    const float *partial;  // [S][T][2E]
+    int S, T, E, K, renorm, has_mask;
+    float *logits;         // [T][2E] or NULL
+    int *idx;              // [T][K]
+    float *w;              // [T][K]
+    int *counts;           // [E]
+    int *hist;             // [K+1] or NULL
+};
+cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream);
+
+// Expert grouping: one block per expert.
+struct PermuteArgs {
+    const int *idx;
+    const int *counts;
+    int T, K, E, BN;
+    int *pair, *pair_pos;
+    int4 *tiles;
+    int *meta;
+    int *err;
+};
+cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
+
+// Gather token rows into expert order (row_bytes multiple of 16).
+cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
+                          long long row_bytes, int p_cap, void *xp, int n_sm,
+                          cudaStream_t stream);
+
+// out[t] = sum_k w[t,k] * Y[pair_pos[t,k]] over kept k, fp32 accumulation.
+cudaError_t launch_combine(int dtype, const void *Y, const int *idx, const float *w,
+                           const int *pair_pos, int T, int K, int d, void *out, int n_sm,
+                           cudaStream_t stream);
+
+// fp32 SIMT path (BEAM_F32).
+cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,
+                              int E, float *partial, const ZeroRegion (&zero)[3],
+                              cudaStream_t stream);
+cudaError_t launch_gemm1_f32(const float *xp, const float *W1, const float *W3, const int4 *tiles,
+                             const int *meta, int tiles_cap, int d, int I, float *H,
+                             cudaStream_t stream);
+cudaError_t launch_gemm2_f32(const float *H, const float *W2, const int4 *tiles, const int *meta,
+                             int tiles_cap, int d, int I, float *Y, cudaStream_t stream);
+
+}  // namespace beam

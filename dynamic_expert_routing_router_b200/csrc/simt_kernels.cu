@@ -1,0 +1,481 @@
+// simt_kernels.cu -- the CUDA-core stages of the BEAM MoE layer:
+//   topk_mask   Top-K, softmax, binary mask and aggregation per token
+//               (BEAM §3.2 Eq. 4-7), per-expert counts and kept histogram
+//   permute     expert-token grouping of the kept pairs only (masked pairs
+//               are left out of the count, so they are never scheduled)
+//   gather      token rows copied into expert order for the grouped GEMMs
+//   combine     y = sum_k w_k * E_{c_k}(x) over kept candidates (Eq. 8)
+// and the fp32 path (router and expert GEMMs on CUDA cores) for BEAM_F32.
+#include <cuda_bf16.h>
+
+#include <climits>
+
+#include "beam_internal.h"
+#include "beam_ptx.cuh"
+
+namespace beam {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ------------------------------------------------------------ top-K + mask --
+//
+// One warp per token.  Lane l holds the logits of experts l, l+32, ...; the
+// router's split-K partial sums are added in split order.  K rounds of a
+// warp arg-max (ties -> lower expert id) give the candidates in descending
+// order.  renorm: softmax over the candidates (Eq. 4); else over all E.
+// The mask keeps candidate k iff its pre-sigmoid value z >= 0 (Eq. 6; NaN
+// is not kept); w = g * m (Eq. 7).  Counts and the histogram are gathered in
+// shared memory and added to global memory once per block.
+template <int EPL>
+__global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a) {
+    __shared__ int s_counts[kMaxE];
+    __shared__ int s_hist[kMaxK + 1];
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_counts[i] = 0;
+    if (threadIdx.x <= a.K) s_hist[threadIdx.x] = 0;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int warps = blockDim.x >> 5;
+    const long long E2 = 2LL * a.E;
+    const long long slab = (long long)a.T * E2;
+
+    for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < a.T; t += gridDim.x * warps) {
+        float r[EPL], z[EPL];
+        unsigned taken = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int j = lane + 32 * i;
+            r[i] = -INFINITY;
+            z[i] = 0.0f;
+            if (j < a.E) {
+                const float *pr = a.partial + (long long)t * E2 + j;
+                float rs = 0.0f, zs = 0.0f;
+                for (int s = 0; s < a.S; ++s) {
+                    rs += pr[s * slab];
+                    if (a.has_mask) zs += pr[s * slab + a.E];
+                }
+                if (a.logits) {
+                    a.logits[(long long)t * E2 + j] = rs;
+                    if (a.has_mask) a.logits[(long long)t * E2 + a.E + j] = zs;
+                }
+                r[i] = (rs != rs) ? -INFINITY : rs;  // NaN never wins a slot
+                z[i] = zs;
+            } else {
+                taken |= 1u << i;
+            }
+        }
+
+        int my_cand = -1;
+        float my_e = 0.0f, my_z = 0.0f, rmax = 0.0f, denom = 0.0f;
+        for (int k = 0; k < a.K; ++k) {
+            float bv = -INFINITY, bz = 0.0f;
+            int bi = INT_MAX;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int j = lane + 32 * i;
+                if (!((taken >> i) & 1u) && (r[i] > bv || (r[i] == bv && j < bi))) {
+                    bv = r[i];
+                    bi = j;
+                    bz = z[i];
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, bv, off);
+                const int oi = __shfl_xor_sync(kFull, bi, off);
+                const float oz = __shfl_xor_sync(kFull, bz, off);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                    bz = oz;
+                }
+            }
+            if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
+            if (k == 0) rmax = bv;
+            const float ek = expf(bv - rmax);
+            denom += ek;
+            if (lane == k) {
+                my_cand = bi;
+                my_e = ek;
+                my_z = bz;
+            }
+        }
+        if (!a.renorm) {
+            float part = 0.0f;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (lane + 32 * i < a.E) part += expf(r[i] - rmax);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
+            denom = part;  // identical on every lane (pairwise sums commute exactly)
+        }
+        const bool kept = (lane < a.K) && (!a.has_mask || my_z >= 0.0f);
+        if (lane < a.K) {
+            const float g = my_e / denom;
+            a.idx[(long long)t * a.K + lane] = kept ? my_cand : -1;
+            a.w[(long long)t * a.K + lane] = kept ? g : 0.0f;
+            if (kept) atomicAdd(&s_counts[my_cand], 1);
+        }
+        const int nkept = __popc(__ballot_sync(kFull, kept));
+        if (lane == 0) atomicAdd(&s_hist[nkept], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x)
+        if (s_counts[i]) atomicAdd(&a.counts[i], s_counts[i]);
+    if (a.hist && threadIdx.x <= a.K && s_hist[threadIdx.x]) atomicAdd(&a.hist[threadIdx.x], s_hist[threadIdx.x]);
+}
+
+// ----------------------------------------------------------------- permute --
+//
+// Block e lists the kept pairs of expert e in token order.  Every block
+// derives the padded offsets from counts[] (exclusive sums over lower
+// experts), so no separate scan kernel is needed.  Rows of expert e:
+// [off_e, off_e + roundup(count_e, BN)); padding rows get pair = -1.  The
+// tile list holds one entry per BN rows of a non-empty expert.
+constexpr int kPermThreads = 256;
+
+__device__ __forceinline__ int block_sum_256(int v, int *s_red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    __syncthreads();
+    if (lane == 0) s_red[warp] = v;
+    __syncthreads();
+    int total = 0;
+#pragma unroll
+    for (int i = 0; i < kPermThreads / 32; ++i) total += s_red[i];
+    return total;
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs a) {
+    __shared__ int s_red[kPermThreads / 32];
+    __shared__ int s_wcnt[kPermThreads / 32];
+    __shared__ int s_wpre[kPermThreads / 32];
+    __shared__ int s_total;
+    const int e = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    int c = 0;
+    if (tid < a.E) c = a.counts[tid];
+    const int padded = (c + a.BN - 1) / a.BN * a.BN;
+    const int ntile = (c + a.BN - 1) / a.BN;
+    const int off_e = block_sum_256(tid < e ? padded : 0, s_red);
+    const int toff_e = block_sum_256(tid < e ? ntile : 0, s_red);
+    if (e == 0) {
+        const int tot_rows = block_sum_256(padded, s_red);
+        const int tot_tiles = block_sum_256(ntile, s_red);
+        const int tot_pairs = block_sum_256(c, s_red);
+        if (tid == 0) {
+            a.meta[0] = tot_tiles;
+            a.meta[1] = tot_rows;
+            a.meta[2] = tot_pairs;
+        }
+    }
+    const int count_e = a.counts[e];
+
+    int running = 0;
+    for (int base = 0; base < a.T; base += kPermThreads) {
+        const int t = base + tid;
+        int km = -1;
+        if (t < a.T) {
+            const int *row = a.idx + (long long)t * a.K;
+            for (int k = 0; k < a.K; ++k)
+                if (row[k] == e) km = k;
+        }
+        const unsigned bal = __ballot_sync(kFull, km >= 0);
+        if (lane == 0) s_wcnt[warp] = __popc(bal);
+        __syncthreads();
+        if (tid == 0) {
+            int acc = 0;
+            for (int i = 0; i < kPermThreads / 32; ++i) {
+                s_wpre[i] = acc;
+                acc += s_wcnt[i];
+            }
+            s_total = acc;
+        }
+        __syncthreads();
+        if (km >= 0) {
+            const int pos = off_e + running + s_wpre[warp] + __popc(bal & ((1u << lane) - 1u));
+            a.pair[pos] = t * a.K + km;
+            a.pair_pos[(long long)t * a.K + km] = pos;
+        }
+        running += s_total;
+        __syncthreads();
+    }
+    if (tid == 0 && running != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
+
+    const int padded_e = (count_e + a.BN - 1) / a.BN * a.BN;
+    for (int r = count_e + tid; r < padded_e; r += kPermThreads) a.pair[off_e + r] = -1;
+    const int ntile_e = padded_e / a.BN;
+    for (int j = tid; j < ntile_e; j += kPermThreads) {
+        const int rows = min(a.BN, count_e - j * a.BN);
+        a.tiles[toff_e + j] = make_int4(e, off_e + j * a.BN, rows, 0);
+    }
+}
+
+// ------------------------------------------------------------------ gather --
+// One warp per permuted row, 16-byte vectors; padding rows are skipped (they
+// only feed padding columns of the GEMMs, which are never stored).
+__global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *pair,
+                                                     const int *meta, int K, int row_vec,
+                                                     uint4 *xp) {
+    const int rows = meta[1];
+    const int lane = threadIdx.x & 31;
+    for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
+        const int pr = pair[r];
+        if (pr < 0) continue;
+        const uint4 *src = x + (long long)(pr / K) * row_vec;
+        uint4 *dst = xp + (long long)r * row_vec;
+        for (int v = lane; v < row_vec; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+// ----------------------------------------------------------------- combine --
+// One block per token; each thread owns 8 consecutive features.  The kept
+// candidates are added in slot order k = 0..K-1 in fp32, then rounded once.
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8]) {
+    uint4 raw;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = raw;
+}
+__device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <typename Tv>
+__global__ void __launch_bounds__(256) combine_kernel(const Tv *Y, const int *idx, const float *w,
+                                                      const int *pair_pos, int T, int K, int d,
+                                                      Tv *out) {
+    __shared__ int s_row[kMaxK];
+    __shared__ float s_w[kMaxK];
+    const int nvec = d / 8;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < K) {
+            const long long o = (long long)t * K + threadIdx.x;
+            const int id = idx[o];
+            s_row[threadIdx.x] = id >= 0 ? pair_pos[o] : -1;
+            s_w[threadIdx.x] = w[o];
+        }
+        __syncthreads();
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int k = 0; k < K; ++k) {
+                const int row = s_row[k];
+                if (row < 0) continue;
+                float y[8];
+                load8(Y + (long long)row * d + v * 8, y);
+                const float wk = s_w[k];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
+            }
+            store8(out + (long long)t * d + v * 8, acc);
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------- fp32 path -----
+// Plain shared-memory tiled SIMT kernels for BEAM_F32 (small layers).  Each
+// output is one fp32 accumulator summed over the reduction index in order.
+constexpr int kT = 16;
+
+__global__ void __launch_bounds__(256) router_f32_kernel(const float *x, const float *Wg,
+                                                         const float *Wm, int T, int d, int E,
+                                                         int J, float *logits, ZeroRegion z0,
+                                                         ZeroRegion z1, ZeroRegion z2) {
+    if (blockIdx.x == 0 && blockIdx.y == 0) {
+        const int tid = threadIdx.y * kT + threadIdx.x;
+        const ZeroRegion zr[3] = {z0, z1, z2};
+        for (int r = 0; r < 3; ++r)
+            if (zr[r].ptr)
+                for (int i = tid; i < zr[r].count; i += kT * kT) zr[r].ptr[i] = 0;
+    }
+    __shared__ float xs[kT][kT + 1];
+    __shared__ float ws[kT][kT + 1];
+    const int t = blockIdx.x * kT + threadIdx.y;
+    const int j = blockIdx.y * kT + threadIdx.x;
+    const int jl = blockIdx.y * kT + threadIdx.y;  // weight row this thread loads
+    const float *wrow = nullptr;
+    if (jl < J) wrow = jl < E ? Wg + (long long)jl * d : Wm + (long long)(jl - E) * d;
+    float acc = 0.0f;
+    for (int k0 = 0; k0 < d; k0 += kT) {
+        const int tl = blockIdx.x * kT + threadIdx.y;
+        const int k = k0 + threadIdx.x;
+        xs[threadIdx.y][threadIdx.x] = (tl < T && k < d) ? x[(long long)tl * d + k] : 0.0f;
+        ws[threadIdx.y][threadIdx.x] = (wrow && k < d) ? wrow[k] : 0.0f;
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kT; ++kk) acc = fmaf(xs[threadIdx.y][kk], ws[threadIdx.x][kk], acc);
+        __syncthreads();
+    }
+    if (t < T && j < J) logits[(long long)t * 2 * E + j] = acc;
+}
+
+__device__ __forceinline__ float silu_mul_f32(float g, float u) {
+    return g / (1.0f + expf(-g)) * u;
+}
+
+// GEMM1 (fp32): H[row] = SiLU(xp[row] W1_e^T) * (xp[row] W3_e^T) for the rows
+// of one tile; block (column block, tile).
+__global__ void __launch_bounds__(256) gemm1_f32_kernel(const float *xp, const float *W1,
+                                                        const float *W3, const int4 *tiles,
+                                                        const int *meta, int d, int I, float *H) {
+    const int ti = blockIdx.x;
+    if (ti >= meta[0]) return;
+    const int4 tile = tiles[ti];
+    const int e = tile.x, row0 = tile.y, rows = tile.z;
+    __shared__ float xs[kT][kT + 1];
+    __shared__ float w1s[kT][kT + 1];
+    __shared__ float w3s[kT][kT + 1];
+    const int col = blockIdx.y * kT + threadIdx.x;
+    const int wl = blockIdx.y * kT + threadIdx.y;  // weight row this thread loads
+    for (int rr = 0; rr < rows; rr += kT) {
+        float ga = 0.0f, ub = 0.0f;
+        for (int k0 = 0; k0 < d; k0 += kT) {
+            const int k = k0 + threadIdx.x;
+            const int r = rr + threadIdx.y;
+            xs[threadIdx.y][threadIdx.x] =
+                (r < rows && k < d) ? xp[(long long)(row0 + r) * d + k] : 0.0f;
+            const bool okw = wl < I && k < d;
+            w1s[threadIdx.y][threadIdx.x] = okw ? W1[((long long)e * I + wl) * d + k] : 0.0f;
+            w3s[threadIdx.y][threadIdx.x] = okw ? W3[((long long)e * I + wl) * d + k] : 0.0f;
+            __syncthreads();
+#pragma unroll
+            for (int kk = 0; kk < kT; ++kk) {
+                ga = fmaf(xs[threadIdx.y][kk], w1s[threadIdx.x][kk], ga);
+                ub = fmaf(xs[threadIdx.y][kk], w3s[threadIdx.x][kk], ub);
+            }
+            __syncthreads();
+        }
+        const int r = rr + threadIdx.y;
+        if (r < rows && col < I) H[(long long)(row0 + r) * I + col] = silu_mul_f32(ga, ub);
+    }
+}
+
+// GEMM2 (fp32): Y[row] = H[row] W2_e^T.
+__global__ void __launch_bounds__(256) gemm2_f32_kernel(const float *H, const float *W2,
+                                                        const int4 *tiles, const int *meta, int d,
+                                                        int I, float *Y) {
+    const int ti = blockIdx.x;
+    if (ti >= meta[0]) return;
+    const int4 tile = tiles[ti];
+    const int e = tile.x, row0 = tile.y, rows = tile.z;
+    __shared__ float hs[kT][kT + 1];
+    __shared__ float w2s[kT][kT + 1];
+    const int col = blockIdx.y * kT + threadIdx.x;
+    const int wl = blockIdx.y * kT + threadIdx.y;
+    for (int rr = 0; rr < rows; rr += kT) {
+        float acc = 0.0f;
+        for (int k0 = 0; k0 < I; k0 += kT) {
+            const int k = k0 + threadIdx.x;
+            const int r = rr + threadIdx.y;
+            hs[threadIdx.y][threadIdx.x] =
+                (r < rows && k < I) ? H[(long long)(row0 + r) * I + k] : 0.0f;
+            w2s[threadIdx.y][threadIdx.x] =
+                (wl < d && k < I) ? W2[((long long)e * d + wl) * I + k] : 0.0f;
+            __syncthreads();
+#pragma unroll
+            for (int kk = 0; kk < kT; ++kk) acc = fmaf(hs[threadIdx.y][kk], w2s[threadIdx.x][kk], acc);
+            __syncthreads();
+        }
+        const int r = rr + threadIdx.y;
+        if (r < rows && col < d) Y[(long long)(row0 + r) * d + col] = acc;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
+    if (a.T <= 0) return cudaSuccess;
+    const int warps = 8;
+    int blocks = (a.T + warps - 1) / warps;
+    if (blocks > 2 * n_sm) blocks = 2 * n_sm;
+    const int epl = (a.E + 31) / 32;
+    if (epl <= 1) topk_mask_kernel<1><<<blocks, 256, 0, stream>>>(a);
+    else if (epl <= 2) topk_mask_kernel<2><<<blocks, 256, 0, stream>>>(a);
+    else if (epl <= 4) topk_mask_kernel<4><<<blocks, 256, 0, stream>>>(a);
+    else topk_mask_kernel<8><<<blocks, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {
+    permute_kernel<<<a.E, kPermThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
+                          long long row_bytes, int p_cap, void *xp, int n_sm,
+                          cudaStream_t stream) {
+    int blocks = (p_cap + 7) / 8;
+    if (blocks > 8 * n_sm) blocks = 8 * n_sm;
+    if (blocks <= 0) return cudaSuccess;
+    gather_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4 *>(x), pair, meta, K,
+                                              int(row_bytes / 16), static_cast<uint4 *>(xp));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(int dtype, const void *Y, const int *idx, const float *w,
+                           const int *pair_pos, int T, int K, int d, void *out, int n_sm,
+                           cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    int threads = d / 8;
+    threads = threads >= 256 ? 256 : ((threads + 31) / 32) * 32;
+    int blocks = T < 8 * n_sm ? T : 8 * n_sm;
+    if (dtype == BEAM_BF16)
+        combine_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(Y), idx, w, pair_pos, T, K, d,
+            static_cast<__nv_bfloat16 *>(out));
+    else
+        combine_kernel<float><<<blocks, threads, 0, stream>>>(static_cast<const float *>(Y), idx, w,
+                                                             pair_pos, T, K, d,
+                                                             static_cast<float *>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,
+                              int E, float *partial, const ZeroRegion (&zero)[3],
+                              cudaStream_t stream) {
+    const int J = Wm ? 2 * E : E;
+    dim3 grid(T > 0 ? (T + kT - 1) / kT : 1, (J + kT - 1) / kT);
+    router_f32_kernel<<<grid, dim3(kT, kT), 0, stream>>>(x, Wg, Wm, T, d, E, J, partial, zero[0],
+                                                         zero[1], zero[2]);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm1_f32(const float *xp, const float *W1, const float *W3, const int4 *tiles,
+                             const int *meta, int tiles_cap, int d, int I, float *H,
+                             cudaStream_t stream) {
+    dim3 grid(tiles_cap, (I + kT - 1) / kT);
+    gemm1_f32_kernel<<<grid, dim3(kT, kT), 0, stream>>>(xp, W1, W3, tiles, meta, d, I, H);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm2_f32(const float *H, const float *W2, const int4 *tiles, const int *meta,
+                             int tiles_cap, int d, int I, float *Y, cudaStream_t stream) {
+    dim3 grid(tiles_cap, (d + kT - 1) / kT);
+    gemm2_f32_kernel<<<grid, dim3(kT, kT), 0, stream>>>(H, W2, tiles, meta, d, I, Y);
+    return cudaGetLastError();
+}
+
+}  // namespace beam

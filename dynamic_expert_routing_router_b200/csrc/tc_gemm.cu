@@ -1,0 +1,331 @@
+// tc_gemm.cu -- grouped GEMMs of the BEAM MoE layer on the sm_100a tensor
+// cores (tcgen05.mma, fp32 accumulators in TMEM, operands staged by TMA).
+//
+// One persistent, warp-specialised kernel serves three roles:
+//   MODE_ROUTER  logits  r = x W_gate, z = x W_mask   (BEAM §3.2 steps 1-2)
+//   MODE_GEMM1   H = SiLU(x W1_e^T) * (x W3_e^T)      (Eq. 3, gate/up + SwiGLU)
+//   MODE_GEMM2   Y = H W2_e^T                          (Eq. 3, down projection)
+//
+// Orientation: the weight rows are the MMA's M operand (128 rows per tile)
+// and the tokens are its N operand (BN = 16..128 per tile), D = W * X^T.  A
+// decode step touches few tokens per expert, so the weights (the bytes that
+// matter) fill the 128-row side; a prefill tile uses BN = 128 tokens.
+// The GEMMs run only over the tile list built from KEPT pairs: an expert
+// without kept pairs has no tile, and TMA never reads its weights.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer (one thread): weight tile(s) + token tile per stage
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2..5  epilogue: TMEM -> registers -> activation -> global memory
+// Pipelines: a STAGES-deep shared-memory ring (full/empty mbarriers) and a
+// 2-deep TMEM accumulator ring (tfull/tempty), so the epilogue of one unit
+// overlaps the MMAs of the next.  Every wait is bounded (beam_ptx.cuh); on
+// expiry the CTA records DEV_ERR_TIMEOUT, drains its own copies and MMAs,
+// frees TMEM and returns.
+#include <cuda_bf16.h>
+
+#include "beam_internal.h"
+#include "beam_ptx.cuh"
+
+namespace beam {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kUmmaK = 16;  // K of one kind::f16 MMA
+
+template <int NUM_A, int BN>
+struct TcCfg {
+    static constexpr uint32_t A_BYTES = kBlockM * kBlockK * 2;  // 16 KB
+    static constexpr uint32_t B_BYTES = BN * kBlockK * 2;
+    static constexpr uint32_t STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    static constexpr int STAGES_FIT = int((220u * 1024u) / STAGE_BYTES);
+    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+    static constexpr uint32_t ACC_COLS = NUM_A * BN;  // fp32 columns per accumulator
+    static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+    static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
+    static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
+                  "TMEM allocation must be a power of two in [32, 512]");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+    static_assert(STAGES >= 2, "pipeline too shallow");
+    static_assert(SMEM_BYTES <= 227u * 1024u, "shared memory");
+};
+
+struct Unit {
+    int mb;     // weight-row block
+    int a_row;  // first row of the A (weight) tile in its 2D tensor map
+    int b_row;  // first row of the B (token) tile
+    int kb0;    // first k-block
+    int sel;    // router: 0 = W_gate rows, 1 = W_mask rows
+    int tt, s;  // router: token tile, split
+    int rows;   // GEMMs: valid token rows of the tile
+};
+
+template <int MODE, int BN>
+__device__ __forceinline__ Unit decode_unit(int u, const TcGemmArgs &p) {
+    Unit w;
+    w.mb = u % p.n_mb;
+    const int rest = u / p.n_mb;
+    if (MODE == MODE_ROUTER) {
+        w.tt = rest % p.n_tt;
+        w.s = rest / p.n_tt;
+        w.sel = w.mb >= p.n_mb_gate ? 1 : 0;
+        w.a_row = (w.sel ? w.mb - p.n_mb_gate : w.mb) * kBlockM;
+        w.b_row = w.tt * BN;
+        w.kb0 = w.s * p.nk;
+        w.rows = 0;
+    } else {
+        const int4 t = p.tiles[rest];
+        w.a_row = t.x * p.a_rows_per_expert + w.mb * kBlockM;
+        w.b_row = t.y;
+        w.rows = t.z;
+        w.kb0 = 0;
+        w.sel = 0;
+        w.tt = w.s = 0;
+    }
+    return w;
+}
+
+__device__ __forceinline__ void signal_abort(int *err, int *abort_flag) {
+    atomicExch(err, DEV_ERR_TIMEOUT);
+    *reinterpret_cast<volatile int *>(abort_flag) = 1;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return g / (1.0f + __expf(-g)) * u;
+}
+
+template <int MODE, int NUM_A, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                   const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const TcGemmArgs p) {
+    using C = TcCfg<NUM_A, BN>;
+    constexpr int STAGES = C::STAGES;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    // 1024-byte aligned start of the stage ring (SWIZZLE_128B atoms).
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_units = (MODE == MODE_ROUTER) ? p.n_units : p.meta[0] * p.n_mb;
+    const volatile int *abort_flag = &abort_sh;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 128);
+        }
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA0);
+        tma_prefetch_desc(&tmA1);
+        tma_prefetch_desc(&tmB);
+    }
+    if (MODE == MODE_ROUTER && blockIdx.x == 0) {
+        // Per-call counters of the later kernels start at zero.
+        for (int r = 0; r < 3; ++r)
+            if (p.zero[r].ptr)
+                for (int i = threadIdx.x; i < p.zero[r].count; i += blockDim.x) p.zero[r].ptr[i] = 0;
+    }
+    if (warp == 1) tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+                const Unit w = decode_unit<MODE, BN>(u, p);
+                const CUtensorMap *am = (MODE == MODE_ROUTER && w.sel) ? &tmA1 : &tmA0;
+                for (int kb = 0; kb < p.nk; ++kb, ++it) {
+                    const int s = int(it % STAGES);
+                    const uint32_t ph = ((it / STAGES) & 1u) ^ 1u;
+                    if (!mbar_wait_bounded(&empty_bar[s], ph, abort_flag, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
+                    const int kx = (w.kb0 + kb) * kBlockK;
+                    tma_load_2d(st, am, kx, w.a_row, &full_bar[s]);
+                    if (NUM_A == 2) tma_load_2d(st + C::A_BYTES, &tmA1, kx, w.a_row, &full_bar[s]);
+                    tma_load_2d(st + NUM_A * C::A_BYTES, &tmB, kx, w.b_row, &full_bar[s]);
+                }
+            }
+            if (!ok) {
+                signal_abort(p.err, &abort_sh);
+                // Let this CTA's own copies land before it can exit.
+                for (uint32_t j = (it > uint32_t(STAGES) ? it - STAGES : 0u); j < it; ++j)
+                    mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1u, nullptr,
+                                      p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            constexpr uint32_t IDESC = umma_idesc_bf16_f32(kBlockM, BN);
+            uint32_t it = 0, lu = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++lu) {
+                const uint32_t a = lu & 1u;
+                if (!mbar_wait_bounded(&tempty_bar[a], ((lu >> 1) & 1u) ^ 1u, abort_flag,
+                                       p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d0 = tmem_base + a * C::ACC_COLS;
+                for (int kb = 0; kb < p.nk; ++kb, ++it) {
+                    const int s = int(it % STAGES);
+                    if (!mbar_wait_bounded(&full_bar[s], (it / STAGES) & 1u, abort_flag,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t sa = smem_u32(smem + size_t(s) * C::STAGE_BYTES);
+                    const uint32_t sb = sa + NUM_A * C::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
+                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bdesc = umma_desc_sw128(sb + kk * 32);
+                        umma_bf16(d0, umma_desc_sw128(sa + kk * 32), bdesc, IDESC, acc);
+                        if (NUM_A == 2)
+                            umma_bf16(d0 + BN, umma_desc_sw128(sa + C::A_BYTES + kk * 32), bdesc,
+                                      IDESC, acc);
+                    }
+                    umma_commit(&empty_bar[s]);  // stage reusable once these MMAs finish
+                }
+                if (!ok) break;
+                umma_commit(&tfull_bar[a]);  // accumulator complete
+            }
+            if (!ok) {
+                signal_abort(p.err, &abort_sh);
+                umma_commit(&drain_bar);  // wait for the MMAs already issued
+                mbar_wait_bounded(&drain_bar, 0u, nullptr, p.timeout_ns);
+            }
+        }
+    } else {
+        // --------------------------------------------------- epilogue --
+        const int q = warp & 3;          // TMEM lane quadrant this warp may access
+        const int row = q * 32 + lane;   // row within the 128-row weight tile
+        uint32_t lu = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++lu) {
+            const Unit w = decode_unit<MODE, BN>(u, p);
+            const uint32_t a = lu & 1u;
+            bool ok = mbar_wait_bounded(&tfull_bar[a], (lu >> 1) & 1u, abort_flag, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                if (lane == 0) signal_abort(p.err, &abort_sh);
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + a * C::ACC_COLS;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t g[16], v[16];
+                tmem_ld_16(tb + c0, g);
+                if (NUM_A == 2) tmem_ld_16(tb + BN + c0, v);
+                tmem_ld_wait();
+                reg_fence_16(g);
+                if (NUM_A == 2) reg_fence_16(v);
+                if (MODE == MODE_ROUTER) {
+                    const int jr = (w.sel ? w.mb - p.n_mb_gate : w.mb) * kBlockM + row;
+                    if (jr < p.E) {
+                        const int j = w.sel ? p.E + jr : jr;
+                        float *out = static_cast<float *>(p.out) + w.s * p.out_split_stride + j;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int t = w.tt * BN + c0 + c;
+                            if (t < p.T) out[(long long)t * p.out_ld] = __uint_as_float(g[c]);
+                        }
+                    }
+                } else {
+                    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
+                                         (long long)w.b_row * p.out_ld + w.mb * kBlockM + row;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (c0 + c < w.rows) {
+                            float val = __uint_as_float(g[c]);
+                            if (MODE == MODE_GEMM1) val = silu_mul(val, __uint_as_float(v[c]));
+                            out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(val);
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&tempty_bar[a]);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <int MODE, int NUM_A, int BN>
+cudaError_t launch_cfg(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                       const TcGemmArgs &args, int grid, cudaStream_t stream) {
+    using C = TcCfg<NUM_A, BN>;
+    auto kern = tc_gemm_kernel<MODE, NUM_A, BN>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b, args);
+    return cudaGetLastError();
+}
+
+template <int MODE, int NUM_A>
+cudaError_t launch_bn(int bn, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                      const TcGemmArgs &args, int grid, cudaStream_t stream) {
+    switch (bn) {
+        case 16: return launch_cfg<MODE, NUM_A, 16>(a0, a1, b, args, grid, stream);
+        case 32: return launch_cfg<MODE, NUM_A, 32>(a0, a1, b, args, grid, stream);
+        case 64: return launch_cfg<MODE, NUM_A, 64>(a0, a1, b, args, grid, stream);
+        case 128: return launch_cfg<MODE, NUM_A, 128>(a0, a1, b, args, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gemm(int mode, int bn, const CUtensorMap &a0, const CUtensorMap &a1,
+                           const CUtensorMap &b, const TcGemmArgs &args, int grid,
+                           cudaStream_t stream) {
+    if (grid <= 0) return cudaSuccess;
+    switch (mode) {
+        case MODE_ROUTER: return launch_bn<MODE_ROUTER, 1>(bn, a0, a1, b, args, grid, stream);
+        case MODE_GEMM1: return launch_bn<MODE_GEMM1, 2>(bn, a0, a1, b, args, grid, stream);
+        case MODE_GEMM2: return launch_bn<MODE_GEMM2, 1>(bn, a0, a1, b, args, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace beam

@@ -1,0 +1,166 @@
+/*
+ * beam_moe.h -- C ABI of the BEAM-masked MoE layer forward pass (B200, sm_100a).
+ *
+ * The operation is the MoE layer of "BEAM: Binary Expert Activation Masking
+ * for Dynamic Routing in MoE" (arXiv 2605.14438), §3.2, for one batch of T
+ * tokens x [T, d]:
+ *
+ *   r = x W_gate                 main-router logits                (step 1)
+ *   g = Softmax(Top-K(r))        candidate weights                 (Eq. 1/4)
+ *   m = [sigmoid(x W_mask) >= 0.5] on the K candidates             (Eq. 5-6)
+ *   w = g * m                    no renormalisation after the mask (Eq. 7)
+ *   y = sum_k w_k E_{c_k}(x)     only kept (token, expert) pairs   (Eq. 8)
+ *   E_e(x) = (SiLU(x W1_e^T) * (x W3_e^T)) W2_e^T                  (Eq. 3)
+ *
+ * A token whose candidates are all masked gets y = 0 (it passes the layer
+ * through the residual, which stays the caller's).  A masked pair is never
+ * scheduled, so an expert without kept pairs has none of its weights read.
+ *
+ * Conventions (all entry points):
+ *  - Layouts are row-major and contiguous: x [T,d]; W_gate, W_mask [E,d]
+ *    (row e = column e of the paper's d x N matrices); W1 (gate), W3 (up)
+ *    [E,I,d]; W2 (down) [E,d,I]; out [T,d].
+ *  - dtype BEAM_BF16: x, weights and out are bfloat16; accumulation is fp32;
+ *    the SwiGLU activations H and the per-pair expert outputs are rounded to
+ *    bf16 once each.  dtype BEAM_F32: everything fp32.  Logits, softmax
+ *    weights and the combine are fp32 in both.
+ *  - Every pointer except the host descriptor is a DEVICE pointer, 16-byte
+ *    aligned.  The caller owns every buffer, including the workspace; the
+ *    library allocates nothing and keeps no state between calls.
+ *  - Every launch is ordered on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and the calls never synchronise the host, except
+ *    beam_moe_check.  Argument and shape errors are returned before anything
+ *    is launched; a failed launch returns BEAM_ERR_CUDA.
+ *  - Constraints: 1 <= K <= min(E, 16), E <= 256, T >= 0.  BEAM_BF16 needs
+ *    d % 128 == 0 and I % 128 == 0; BEAM_F32 needs d % 8 == 0 and I % 8 == 0
+ *    (else BEAM_ERR_UNSUPPORTED_SHAPE).  T*K and the workspace rows must fit
+ *    in int32.
+ *  - Top-K ties go to the lower expert index; candidates are listed by
+ *    descending logit (the paper does not fix either).  The mask test is taken
+ *    on the pre-sigmoid value, z >= 0 <=> sigmoid(z) >= 0.5 (Eq. 6); NaN is
+ *    not kept.  Non-finite inputs are the caller's responsibility.
+ */
+#ifndef BEAM_MOE_H
+#define BEAM_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BEAM_OK = 0,
+    BEAM_ERR_INVALID_ARG = 1,       /* NULL / misaligned pointer, bad K, E, dtype, ... */
+    BEAM_ERR_UNSUPPORTED_SHAPE = 2, /* d or I not a multiple of the tile width */
+    BEAM_ERR_WORKSPACE = 3,         /* workspace NULL, misaligned or too small */
+    BEAM_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+    BEAM_ERR_TIMEOUT = 5,           /* a bounded device-side wait gave up */
+    BEAM_ERR_INTERNAL = 6           /* a device-side consistency check failed */
+} beam_status;
+
+typedef enum { BEAM_BF16 = 0, BEAM_F32 = 1 } beam_dtype;
+
+/* One MoE layer call: T tokens of width d, E experts, top-K, SwiGLU width I.
+ * renorm_topk = 1: softmax over the K largest logits (Eq. 4, sums to 1).
+ * renorm_topk = 0: softmax over all E logits, restricted to the K largest. */
+typedef struct {
+    int T, d, E, I, K;
+    int dtype;       /* beam_dtype */
+    int renorm_topk; /* 0 or 1 */
+} beam_moe_desc;
+
+/* Workspace layout chosen for a descriptor (byte offsets from the workspace
+ * base).  Exposed so that tests and tools can read the intermediate arrays
+ * after beam_moe_forward; none of it is needed to call the layer.
+ *   err       int32      device error word (0 = ok), read by beam_moe_check
+ *   meta      int32[4]   [0] tiles in the tile list, [1] padded rows,
+ *                        [2] kept pairs P, [3] reserved
+ *   counts    int32[E]   kept pairs per expert
+ *   hist      int32[K+1] tokens by number of kept candidates
+ *   partial   f32[S][T][2E] router partial logits (S = router_splits)
+ *   idx       int32[T][K] candidate expert, -1 where masked
+ *   w         f32[T][K]   g * m
+ *   pair      int32[p_cap] permuted row -> t*K + k (-1 on padding rows);
+ *             expert e owns rows [off_e, off_e + roundup(counts[e], BN)),
+ *             experts in ascending order, tokens ascending inside
+ *   pair_pos  int32[T][K] permuted row of a kept pair (undefined if masked)
+ *   tiles     int32[tiles_cap][4] (expert, first row, valid rows, 0)
+ *   xp        [p_cap][d]  gathered token rows (dtype)
+ *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
+ *   y         [p_cap][d]  expert output per pair (dtype)                    */
+typedef struct {
+    int BN;            /* token rows per expert tile; the padding unit */
+    int router_bn;     /* token rows per router tile */
+    int router_splits; /* router split-K factor S */
+    int p_cap;         /* rows of xp / h / y / pair */
+    int tiles_cap;     /* entries of the tile list */
+    int reserved;
+    size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
+        off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y;
+    size_t workspace_bytes;
+} beam_moe_plan_info;
+
+/* Number of kernel launches of one beam_moe_forward call (the stages below). */
+#define BEAM_MOE_FORWARD_STAGES 7
+
+/* Bytes of device workspace beam_moe_forward needs for `desc` (0 on a bad
+ * descriptor).  Grows with T: O(T*K*(2d + I)) for the permuted activations. */
+size_t beam_moe_workspace_size(const beam_moe_desc *desc);
+
+/* Fill `info` with the workspace layout for `desc`.  Host only. */
+beam_status beam_moe_plan(const beam_moe_desc *desc, beam_moe_plan_info *info);
+
+/* Routing alone: §3.2 steps 1-3 and Eq. (7).
+ *   x, W_gate [E,d], W_mask [E,d] or NULL (mask disabled: all candidates kept)
+ *   topk_idx  int32 [T,K]  candidate expert id, -1 where masked      (written)
+ *   topk_w    f32   [T,K]  g * m                                     (written)
+ *   expert_counts int32 [E] kept pairs per expert                    (written)
+ *   kept_hist int32 [K+1] tokens by kept count, or NULL              (written)
+ *   logits    f32 [T,2E] or NULL: r in columns [0,E), the mask pre-activation
+ *             z in [E,2E) (not written when W_mask is NULL)          (written)
+ *   workspace of beam_moe_workspace_size(desc) bytes (partial logits).
+ * Uses the same kernels, tiling and summation order as beam_moe_forward, so
+ * both take bitwise identical routing decisions for the same inputs. */
+beam_status beam_moe_route(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                           const void *W_mask, int32_t *topk_idx, float *topk_w,
+                           int32_t *expert_counts, int32_t *kept_hist, float *logits,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* The whole layer, Eq. (4)-(8): out [T,d] = sum of kept experts' outputs
+ * weighted by g * m.  W_mask NULL runs the same kernels with the mask test
+ * off (vanilla Top-K MoE).  Launches BEAM_MOE_FORWARD_STAGES kernels:
+ * router GEMM, top-K + mask, grouping, row gather, gate/up GEMM + SwiGLU,
+ * down GEMM, weighted combine.  No host synchronisation; capturable into a
+ * CUDA graph. */
+beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                             const void *W_mask, const void *W1, const void *W3,
+                             const void *W2, void *out, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/* beam_moe_forward that also records `events[i]` (cudaEvent_t, created by the
+ * caller) on `stream` before stage i and events[BEAM_MOE_FORWARD_STAGES]
+ * after the last one, so the caller can time each kernel with
+ * cudaEventElapsedTime.  Same launches and results as beam_moe_forward. */
+beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
+                                      const void *W_gate, const void *W_mask,
+                                      const void *W1, const void *W3, const void *W2,
+                                      void *out, void *workspace, size_t workspace_bytes,
+                                      void *stream, void *const *events);
+
+/* Synchronise `stream`, then read the workspace error word written by the last
+ * call: BEAM_OK, BEAM_ERR_TIMEOUT (a bounded device wait expired, the kernel
+ * returned early) or BEAM_ERR_INTERNAL (a device consistency check failed). */
+beam_status beam_moe_check(const beam_moe_desc *desc, void *workspace, void *stream);
+
+/* Static, NUL-terminated name of a status code. */
+const char *beam_status_str(beam_status status);
+
+/* Name of forward stage i (0 <= i < BEAM_MOE_FORWARD_STAGES), else NULL. */
+const char *beam_moe_stage_name(int stage);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -13,6 +13,10 @@ def pytest_configure(config):
 
 
 @pytest.fixture(scope="session", autouse=True)
-def _build_oracle():
+def _build_libraries():
+    """Build the CPU oracle and the CUDA library in-tree when missing or stale
+    (nvcc cross-compiles for sm_100a without a GPU)."""
     import oracle
+    from dynamic_expert_routing_router_b200 import build
     oracle.build()
+    build.build()

@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments before touching a GPU (these tests run without one)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from dynamic_expert_routing_router_b200 import abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(beam_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_entry_point():
+    names = _declared_functions()
+    assert "beam_moe_forward" in names and "beam_moe_route" in names
+    L = abi.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_and_stage_names():
+    assert abi.status_str(0) == "BEAM_OK"
+    assert abi.status_str(5) == "BEAM_ERR_TIMEOUT"
+    assert [abi.stage_name(i) for i in range(abi.FORWARD_STAGES)] == [
+        "router_gemm", "topk_mask", "permute", "gather", "gemm1_gate_up_swiglu",
+        "gemm2_down", "combine"]
+    assert abi.stage_name(abi.FORWARD_STAGES) is None
+
+
+def test_plan_layout_is_consistent():
+    for T in (0, 1, 8, 32, 128, 8192):
+        dsc = abi.desc(T, 2048, 128, 768, 8, "bf16", 1)
+        P = abi.plan(dsc)
+        assert P["BN"] in (16, 32, 64, 128)
+        assert P["p_cap"] == T * 8 + 128 * (P["BN"] - 1)
+        offs = [P[k] for k in ("off_counts", "off_hist", "off_partial", "off_idx", "off_w",
+                               "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h",
+                               "off_y")]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert P["off_y"] + 2 * P["p_cap"] * 2048 <= P["workspace_bytes"]
+        assert abi.workspace_size(dsc) == P["workspace_bytes"]
+        assert (2048 // 64) % P["router_splits"] == 0
+    assert abi.plan(abi.desc(8192, 2048, 128, 768, 8))["BN"] == 128
+    assert abi.plan(abi.desc(128, 2048, 128, 768, 8))["BN"] == 16
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(K=0), 1), (dict(K=17, E=32), 1), (dict(E=300, K=8), 1), (dict(K=9, E=8), 1),
+    (dict(dtype=7), 1), (dict(renorm=2), 1), (dict(T=-1), 1),
+    (dict(d=2000), 2), (dict(I=700), 2),
+])
+def test_bad_descriptors_are_rejected(bad, code):
+    args = dict(T=4, d=2048, E=128, I=768, K=8, dtype="bf16", renorm=1)
+    args.update(bad)
+    dsc = abi.desc(**args)
+    assert abi.workspace_size(dsc) == 0
+    with pytest.raises(abi.BeamError) as ei:
+        abi.plan(dsc)
+    assert ei.value.status == code
+
+
+def test_f32_shape_rule():
+    assert abi.workspace_size(abi.desc(4, 128, 8, 256, 2, "f32", 0)) > 0
+    assert abi.workspace_size(abi.desc(4, 132, 8, 256, 2, "f32", 0)) == 0  # d % 8
+
+
+def _call_forward(dsc, ptrs, ws_bytes):
+    L = abi.lib()
+    vp = ctypes.c_void_p
+    return L.beam_moe_forward(ctypes.byref(dsc), *[vp(p) if p else None for p in ptrs],
+                              ctypes.c_size_t(ws_bytes), None)
+
+
+def test_argument_errors_return_before_any_launch():
+    dsc = abi.desc(4, 2048, 128, 768, 8, "bf16", 1)
+    need = abi.workspace_size(dsc)
+    good = [4096 * (i + 1) for i in range(8)]  # x Wg Wm W1 W3 W2 out ws (never dereferenced)
+    # NULL weight
+    p = list(good)
+    p[3] = 0
+    assert _call_forward(dsc, p, need) == 1
+    # misaligned x
+    p = list(good)
+    p[0] += 8
+    assert _call_forward(dsc, p, need) == 1
+    # workspace too small, NULL, misaligned
+    assert _call_forward(dsc, good, need - 1) == 3
+    p = list(good)
+    p[7] = 0
+    assert _call_forward(dsc, p, need) == 3
+    p = list(good)
+    p[7] += 16
+    assert _call_forward(dsc, p, need) == 3

@@ -1,0 +1,315 @@
+"""CUDA library vs. the fp64 oracle, through the C ABI, on B200.
+
+Workloads: the tiny fp32 layer (d=128, E=8, K=2, I=256, no renorm), the
+Qwen3-30B-A3B-shaped bf16 layer at decode (T = 1..128) and prefill (T = 8192)
+for several kept fractions, the large fine-grained layer (d=7168, E=256,
+I=2048), and edge shapes (E not a multiple of 128, K = 1, K = 16, ragged T,
+T = 0, renorm off).  See tests/_parity.py for the bars.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dynamic_expert_routing_router_b200 import abi, inputs
+
+from _parity import (assert_grouping_bitexact, assert_routing_bitexact, assert_values,
+                     compact_experts, gpu_forward, gpu_route, host, oracle_from_logits,
+                     oracle_values)
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def qwen3_experts():
+    torch.cuda.init()
+    return inputs.make_experts(inputs.QWEN3, seed=0, device=DEV)
+
+
+@pytest.fixture(scope="module")
+def qwen3_experts_host(qwen3_experts):
+    return tuple(host(W) for W in qwen3_experts)
+
+
+def _tiny(gamma):
+    L = inputs.make_tiny(T=64, seed=0, gamma=gamma, device="cpu")
+    return {k: v.to(DEV) for k, v in L.items()}
+
+
+# ------------------------------------------------------------------ tiny --
+
+def test_tiny_f32_layer_matches_oracle():
+    gamma = json.load(open(os.path.join(HERE, "golden", "tiny_gamma.json")))["gamma"]
+    L = _tiny(gamma)
+    sh = inputs.TINY
+    dsc = abi.desc(64, sh.d, sh.E, sh.I, sh.K, "f32", sh.renorm)
+    g = gpu_route(dsc, L["x"], L["W_gate"], L["W_mask"])
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
+    assert_routing_bitexact(g, o)
+    # GPU fp32 logits against the oracle's fp64 logits
+    r, z = oracle.logits(host(L["x"]), host(L["W_gate"]), host(L["W_mask"]), "f32")
+    np.testing.assert_allclose(g["logits"], np.concatenate([r, z], 1), rtol=0, atol=1e-5)
+    kept = (g["idx"] >= 0).mean()
+    assert 0.35 <= kept <= 0.65, kept
+    out, ws = gpu_forward(dsc, L["x"], L["W_gate"], L["W_mask"], L["W1"], L["W3"], L["W2"])
+    views = abi.workspace_views(dsc, ws)
+    assert np.array_equal(views["idx"].cpu().numpy(), g["idx"])
+    assert_grouping_bitexact(dsc, views, g["idx"])
+    ref = oracle_values(L["x"], L["W1"], L["W3"], L["W2"], g["idx"], o["w"], "f32")
+    assert_values(out, ref, g["idx"], "f32")
+
+
+def test_tiny_f32_zero_mask_is_vanilla_topk_bitwise():
+    L = _tiny(0.0)
+    sh = inputs.TINY
+    dsc = abi.desc(64, sh.d, sh.E, sh.I, sh.K, "f32", sh.renorm)
+    Wz = torch.zeros_like(L["W_mask"])
+    out0, _ = gpu_forward(dsc, L["x"], L["W_gate"], Wz, L["W1"], L["W3"], L["W2"])
+    outn, _ = gpu_forward(dsc, L["x"], L["W_gate"], None, L["W1"], L["W3"], L["W2"])
+    assert torch.equal(out0, outn)
+    g = gpu_route(dsc, L["x"], L["W_gate"], Wz)
+    assert (g["idx"] >= 0).all() and g["hist"][sh.K] == 64
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, False)
+    ref = oracle_values(L["x"], L["W1"], L["W3"], L["W2"], o["idx"], o["w"], "f32")
+    assert_values(outn, ref, o["idx"], "f32")
+
+
+# ---------------------------------------------------------------- decode --
+
+DECODE = [(T, f) for T in (1, 8, 32, 128) for f in (0.15, 0.35, 0.6, 1.0)]
+
+
+@pytest.mark.parametrize("T,f", DECODE)
+def test_qwen3_decode_matches_oracle(T, f, qwen3_experts, qwen3_experts_host):
+    sh = inputs.QWEN3
+    W1, W3, W2 = qwen3_experts
+    x = inputs.make_tokens(sh, T, seed=100 + T, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = inputs.make_mask(sh, f, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    g = gpu_route(dsc, x, Wg, Wm)
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
+    assert_routing_bitexact(g, o)
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    views = abi.workspace_views(dsc, ws)
+    assert np.array_equal(views["idx"].cpu().numpy(), g["idx"])
+    assert np.array_equal(views["w"].cpu().numpy(), g["w"])
+    assert_grouping_bitexact(dsc, views, g["idx"])
+    n = min(T, 32)
+    h1, h3, h2 = qwen3_experts_host
+    ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16", 0, n)
+    assert_values(out, ref, g["idx"], "bf16", rows=slice(0, n))
+    if f >= 1.0:
+        assert (g["idx"] >= 0).all()
+
+
+# --------------------------------------------------------------- prefill --
+
+@pytest.mark.parametrize("f", [0.15, 0.35, 1.0])
+def test_qwen3_prefill_matches_oracle(f, qwen3_experts, qwen3_experts_host):
+    sh = inputs.QWEN3
+    T = 8192
+    W1, W3, W2 = qwen3_experts
+    x = inputs.make_tokens(sh, T, seed=7, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = inputs.make_mask(sh, f, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    g = gpu_route(dsc, x, Wg, Wm)
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
+    assert_routing_bitexact(g, o)
+    # histogram over 0..K kept experts covers the whole batch
+    assert g["hist"].sum() == T and len(g["hist"]) == sh.K + 1
+    kept = (g["idx"] >= 0).mean()
+    if f < 1.0:
+        assert abs(kept - f) < 0.05, kept
+        assert g["hist"][0] >= 0.01 * T, g["hist"]  # >= 1% of tokens fully masked
+    else:
+        assert g["hist"][sh.K] == T
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    views = abi.workspace_views(dsc, ws)
+    assert np.array_equal(views["idx"].cpu().numpy(), g["idx"])
+    assert_grouping_bitexact(dsc, views, g["idx"])
+    h1, h3, h2 = qwen3_experts_host
+    for t0 in (0, T - 40):  # first rows and the ragged end
+        ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16", t0, t0 + 40)
+        assert_values(out, ref, g["idx"], "bf16", rows=slice(t0, t0 + 40))
+
+
+# ------------------------------------------------------------ invariants --
+
+def test_zero_mask_equals_no_mask_bitwise_bf16(qwen3_experts):
+    sh = inputs.QWEN3
+    W1, W3, W2 = qwen3_experts
+    for T in (32, 1024):
+        x = inputs.make_tokens(sh, T, seed=3, device=DEV)
+        Wg = inputs.make_gate(sh, seed=0, device=DEV)
+        dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+        out0, ws0 = gpu_forward(dsc, x, Wg, torch.zeros_like(Wg), W1, W3, W2)
+        outn, wsn = gpu_forward(dsc, x, Wg, None, W1, W3, W2)
+        assert torch.equal(out0, outn)
+        assert (abi.workspace_views(dsc, ws0)["idx"] >= 0).all()
+
+
+def test_unused_experts_are_never_read(qwen3_experts):
+    """NaN in every expert without a kept pair changes nothing (bitwise)."""
+    sh = inputs.QWEN3
+    T = 32
+    x = inputs.make_tokens(sh, T, seed=11, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = inputs.make_mask(sh, 0.15, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    W1, W3, W2 = (W.clone() for W in qwen3_experts)
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    counts = abi.workspace_views(dsc, ws)["counts"].cpu()
+    unused = torch.nonzero(counts == 0).flatten().to(DEV)
+    assert len(unused) > sh.E // 2
+    for W in (W1, W3, W2):
+        W.index_fill_(0, unused, float("nan"))
+    out2, _ = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    assert torch.isfinite(out2.float()).all()
+    assert torch.equal(out, out2)
+
+
+def test_all_masked_batch_outputs_zero(qwen3_experts):
+    sh = inputs.QWEN3
+    T = 64
+    W1, W3, W2 = qwen3_experts
+    x = inputs.make_tokens(sh, T, seed=5, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = torch.zeros_like(Wg)
+    Wm[:, sh.d - 1] = -1.0  # z = -1 for every expert (bias feature x[d-1] = 1)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    v = abi.workspace_views(dsc, ws)
+    assert (v["idx"] == -1).all() and v["hist"][0].item() == T and v["meta"][0].item() == 0
+    assert (out.float() == 0).all()
+
+
+def test_route_and_forward_agree_and_are_deterministic(qwen3_experts):
+    sh = inputs.QWEN3
+    W1, W3, W2 = qwen3_experts
+    T = 200  # ragged against every tile size
+    x = inputs.make_tokens(sh, T, seed=21, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = inputs.make_mask(sh, 0.35, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    g = gpu_route(dsc, x, Wg, Wm)
+    out1, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    out2, _ = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2, ws=ws)
+    assert torch.equal(out1, out2)
+    v = abi.workspace_views(dsc, ws)
+    assert np.array_equal(v["idx"].cpu().numpy(), g["idx"])
+    assert np.array_equal(v["counts"].cpu().numpy(), g["counts"])
+
+
+def test_cuda_graph_replay_matches_eager(qwen3_experts):
+    sh = inputs.QWEN3
+    W1, W3, W2 = qwen3_experts
+    T = 128
+    x = inputs.make_tokens(sh, T, seed=31, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = inputs.make_mask(sh, 0.35, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    ref, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    out = torch.empty_like(ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        abi.forward(dsc, x, Wg, Wm, W1, W3, W2, out, ws, stream=s)  # warm-up
+        s.synchronize()
+        with torch.cuda.graph(graph, stream=s):
+            abi.forward(dsc, x, Wg, Wm, W1, W3, W2, out, ws, stream=s)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    # new inputs written into the captured buffers are picked up
+    x2 = inputs.make_tokens(sh, T, seed=32, device=DEV)
+    x.copy_(x2)
+    graph.replay()
+    torch.cuda.synchronize()
+    ref2, _ = gpu_forward(dsc, x2, Wg, Wm, W1, W3, W2)
+    assert torch.equal(out, ref2)
+
+
+# ----------------------------------------------------------- edge shapes --
+
+EDGE = [
+    # (name, T, d, E, I, K, renorm, f)
+    ("qwen15_like_E60", 40, 2048, 60, 1408, 4, 0, 0.35),
+    ("dsv2lite_like_E64", 33, 2048, 64, 1408, 6, 1, 0.5),
+    ("top1", 17, 1024, 32, 256, 1, 1, 0.5),
+    ("top16_E256", 9, 512, 256, 384, 16, 1, 0.6),
+    ("ragged_T3_renorm0", 3, 2048, 128, 768, 8, 0, 0.35),
+    ("T1_all_kept", 1, 2048, 128, 768, 8, 1, 1.0),
+    ("bn64_T600", 600, 1024, 128, 256, 8, 1, 0.35),
+    ("bn32_T400", 400, 2048, 128, 768, 8, 1, 0.6),
+]
+
+
+@pytest.mark.parametrize("name,T,d,E,I,K,renorm,f", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_shapes_match_oracle(name, T, d, E, I, K, renorm, f):
+    sh = inputs.Shape(d=d, E=E, K=K, I=I, renorm=renorm, dtype="bf16")
+    x = inputs.make_tokens(sh, T, seed=T, device=DEV)
+    Wg = inputs.make_gate(sh, seed=1, device=DEV)
+    Wm = inputs.make_mask(sh, f, seed=1, device=DEV)
+    W1, W3, W2 = inputs.make_experts(sh, seed=1, device=DEV)
+    dsc = abi.desc(T, d, E, I, K, "bf16", renorm)
+    g = gpu_route(dsc, x, Wg, Wm)
+    o = oracle_from_logits(g["logits"], E, K, renorm, True)
+    assert_routing_bitexact(g, o)
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    views = abi.workspace_views(dsc, ws)
+    assert_grouping_bitexact(dsc, views, g["idx"])
+    ref = oracle_values(x, W1, W3, W2, g["idx"], o["w"], "bf16")
+    assert_values(out, ref, g["idx"], "bf16")
+
+
+def test_empty_batch_is_a_no_op():
+    sh = inputs.QWEN3
+    dsc = abi.desc(0, sh.d, sh.E, sh.I, sh.K, "bf16", 1)
+    ws = abi.alloc_workspace(dsc, DEV)
+    x = torch.empty((0, sh.d), dtype=torch.bfloat16, device=DEV)
+    W = torch.empty((16,), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((0, sh.d), dtype=torch.bfloat16, device=DEV)
+    abi.forward(dsc, x if x.numel() else W, W, None, W, W, W, out if out.numel() else W, ws)
+    abi.check(dsc, ws)
+
+
+# ----------------------------------------------------------------- large --
+
+@pytest.mark.parametrize("T,f", [(16, 0.15), (16, 0.5), (4096, 0.15), (4096, 0.5)])
+def test_large_layer_matches_oracle(T, f, large_layer):
+    sh = inputs.LARGE
+    W1, W3, W2, Wg = large_layer
+    x = inputs.make_tokens(sh, T, seed=40 + T, device=DEV)
+    Wm = inputs.make_mask(sh, f, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    g = gpu_route(dsc, x, Wg, Wm)
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
+    assert_routing_bitexact(g, o)
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    views = abi.workspace_views(dsc, ws)
+    assert_grouping_bitexact(dsc, views, g["idx"])
+    n = 6
+    c1, c3, c2, cidx = compact_experts(W1, W3, W2, g["idx"][:n])
+    xs = host(x[:n])
+    ref = oracle.experts(xs, c1, c3, c2, cidx, o["w"][:n], "bf16")
+    assert_values(out, ref, g["idx"], "bf16", rows=slice(0, n))
+
+
+@pytest.fixture(scope="module")
+def large_layer():
+    sh = inputs.LARGE
+    W1, W3, W2 = inputs.make_experts(sh, seed=0, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV, zipf=None)
+    yield W1, W3, W2, Wg
+    del W1, W3, W2
+    torch.cuda.empty_cache()
