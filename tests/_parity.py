@@ -6,7 +6,10 @@ bit-exact when the oracle is fed the library's own fp32 logits; values are
 compared with the oracle's fp64 expert math applied to those decisions:
   bf16: max|out - ref| <= 2e-2 * RMS(ref)
   fp32: max|out - ref| <= 1e-4 * max|ref|
-and tokens with no kept candidate must be exactly 0 in both.
+and tokens with no kept candidate must be exactly 0 in both.  RMS(ref) is
+taken over the tokens that keep at least one expert: the all-masked tokens are
+exactly 0 on both sides (checked separately) and at low kept fractions they
+are most of the batch, which would shrink the scale the bound is stated in.
 """
 import numpy as np
 import torch
@@ -95,7 +98,8 @@ def assert_values(out, ref, idx, dtype, rows=None):
     assert (o[empty] == 0).all() and (ref[empty] == 0).all(), "all-masked tokens must be 0"
     diff = np.abs(o - ref).max() if o.size else 0.0
     if dtype == "bf16":
-        rms = np.sqrt((ref ** 2).mean()) if ref.size else 0.0
+        act = ref[~empty]
+        rms = np.sqrt((act ** 2).mean()) if act.size else 0.0
         assert diff <= BF16_TOL_RMS * rms + 1e-30, (diff, rms)
     else:
         mx = np.abs(ref).max() if ref.size else 0.0
