@@ -184,6 +184,6 @@ def workspace_views(dsc, workspace) -> dict:
         tiles=view(P["off_tiles"], 4 * P["tiles_cap"], torch.int32, 4).view(-1, 4),
         xp=view(P["off_xp"], P["p_cap"] * dsc.d, dt, es).view(P["p_cap"], dsc.d),
         h=view(P["off_h"], P["p_cap"] * dsc.I, dt, es).view(P["p_cap"], dsc.I),
-        y=view(P["off_y"], P["p_cap"] * dsc.d, dt, es).view(P["p_cap"], dsc.d),
+        y=view(P["off_y"], P["p_cap"] * dsc.d, torch.float32, 4).view(P["p_cap"], dsc.d),
         plan=P,
     )

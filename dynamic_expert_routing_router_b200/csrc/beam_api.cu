@@ -95,7 +95,7 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
     P->off_xp = align256(P->off_tiles + 16 * size_t(tiles_cap));
     P->off_h = align256(P->off_xp + es * size_t(p_cap) * size_t(d->d));
     P->off_y = align256(P->off_h + es * size_t(p_cap) * size_t(d->I));
-    o = align256(P->off_y + es * size_t(p_cap) * size_t(d->d));
+    o = align256(P->off_y + 4 * size_t(p_cap) * size_t(d->d));  // Y is fp32
     P->workspace_bytes = o;
     return BEAM_OK;
 }
@@ -261,7 +261,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     int4 *tiles = reinterpret_cast<int4 *>(ws + P.off_tiles);
     void *xp = ws + P.off_xp;
     void *h = ws + P.off_h;
-    void *y = ws + P.off_y;
+    float *y = reinterpret_cast<float *>(ws + P.off_y);
 
     const RouteOut ro{idx, w, counts, hist, nullptr};
     s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
@@ -316,8 +316,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
                                        d->d, d->I, static_cast<float *>(h), st));
         BEAM_TRY_CUDA(rec.rec(5));
         BEAM_TRY_CUDA(launch_gemm2_f32(static_cast<const float *>(h), static_cast<const float *>(W2),
-                                       tiles, meta, P.tiles_cap, d->d, d->I,
-                                       static_cast<float *>(y), st));
+                                       tiles, meta, P.tiles_cap, d->d, d->I, y, st));
     }
 
     BEAM_TRY_CUDA(rec.rec(6));

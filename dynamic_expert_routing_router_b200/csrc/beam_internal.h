@@ -42,7 +42,7 @@ struct TcGemmArgs {
     int a_rows_per_expert;  // GEMM1: I, GEMM2: d
     const int *meta;     // GEMMs: meta[0] = tiles in the tile list
     const int4 *tiles;   // GEMMs: (expert, first row, valid rows, 0)
-    void *out;           // router: f32 partial [S][T][2E]; GEMM1: H; GEMM2: Y (bf16)
+    void *out;           // router: f32 partial [S][T][2E]; GEMM1: H (bf16); GEMM2: Y (f32)
     long long out_ld;    // elements per output row
     long long out_split_stride;  // router: elements per split slab
     int *err;            // device error word
@@ -83,8 +83,9 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
                           long long row_bytes, int p_cap, void *xp, int n_sm,
                           cudaStream_t stream);
 
-// out[t] = sum_k w[t,k] * Y[pair_pos[t,k]] over kept k, fp32 accumulation.
-cudaError_t launch_combine(int dtype, const void *Y, const int *idx, const float *w,
+// out[t] = sum_k w[t,k] * Y[pair_pos[t,k]] over kept k; Y fp32, fp32 sums,
+// one rounding to the output dtype.
+cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
                            const int *pair_pos, int T, int K, int d, void *out, int n_sm,
                            cudaStream_t stream);
 

@@ -234,17 +234,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *
 
 // ----------------------------------------------------------------- combine --
 // One block per token; each thread owns 8 consecutive features.  The kept
-// candidates are added in slot order k = 0..K-1 in fp32, then rounded once.
-__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
-    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
-    }
-}
+// candidates' fp32 expert outputs are added in slot order k = 0..K-1 in fp32,
+// then rounded once to the output type.
 __device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
     const float4 a = *reinterpret_cast<const float4 *>(p);
     const float4 b = *reinterpret_cast<const float4 *>(p + 4);
@@ -263,10 +254,10 @@ __device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
     *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <typename Tv>
-__global__ void __launch_bounds__(256) combine_kernel(const Tv *Y, const int *idx, const float *w,
-                                                      const int *pair_pos, int T, int K, int d,
-                                                      Tv *out) {
+template <typename Tout>
+__global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int *idx,
+                                                      const float *w, const int *pair_pos, int T,
+                                                      int K, int d, Tout *out) {
     __shared__ int s_row[kMaxK];
     __shared__ float s_w[kMaxK];
     const int nvec = d / 8;
@@ -435,7 +426,7 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine(int dtype, const void *Y, const int *idx, const float *w,
+cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
                            const int *pair_pos, int T, int K, int d, void *out, int n_sm,
                            cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
@@ -444,11 +435,9 @@ cudaError_t launch_combine(int dtype, const void *Y, const int *idx, const float
     int blocks = T < 8 * n_sm ? T : 8 * n_sm;
     if (dtype == BEAM_BF16)
         combine_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(Y), idx, w, pair_pos, T, K, d,
-            static_cast<__nv_bfloat16 *>(out));
+            Y, idx, w, pair_pos, T, K, d, static_cast<__nv_bfloat16 *>(out));
     else
-        combine_kernel<float><<<blocks, threads, 0, stream>>>(static_cast<const float *>(Y), idx, w,
-                                                             pair_pos, T, K, d,
+        combine_kernel<float><<<blocks, threads, 0, stream>>>(Y, idx, w, pair_pos, T, K, d,
                                                              static_cast<float *>(out));
     return cudaGetLastError();
 }

@@ -4,7 +4,7 @@
 // One persistent, warp-specialised kernel serves three roles:
 //   MODE_ROUTER  logits  r = x W_gate, z = x W_mask   (BEAM §3.2 steps 1-2)
 //   MODE_GEMM1   H = SiLU(x W1_e^T) * (x W3_e^T)      (Eq. 3, gate/up + SwiGLU)
-//   MODE_GEMM2   Y = H W2_e^T                          (Eq. 3, down projection)
+//   MODE_GEMM2   Y = H W2_e^T  (fp32 out)              (Eq. 3, down projection)
 //
 // Orientation: the weight rows are the MMA's M operand (128 rows per tile)
 // and the tokens are its N operand (BN = 16..128 per tile), D = W * X^T.  A
@@ -263,17 +263,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (t < p.T) out[(long long)t * p.out_ld] = __uint_as_float(g[c]);
                         }
                     }
-                } else {
+                } else if (MODE == MODE_GEMM1) {
+                    // H (bf16): the next GEMM's operand.
                     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
                                          (long long)w.b_row * p.out_ld + w.mb * kBlockM + row;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        if (c0 + c < w.rows) {
-                            float val = __uint_as_float(g[c]);
-                            if (MODE == MODE_GEMM1) val = silu_mul(val, __uint_as_float(v[c]));
-                            out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(val);
-                        }
-                    }
+                    for (int c = 0; c < 16; ++c)
+                        if (c0 + c < w.rows)
+                            out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(
+                                silu_mul(__uint_as_float(g[c]), __uint_as_float(v[c])));
+                } else {
+                    // Y (fp32): rounded once, after the weighted combine.
+                    float *out = static_cast<float *>(p.out) + (long long)w.b_row * p.out_ld +
+                                 w.mb * kBlockM + row;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (c0 + c < w.rows) out[(long long)(c0 + c) * p.out_ld] = __uint_as_float(g[c]);
                 }
             }
             tc_fence_before_sync();

@@ -21,8 +21,9 @@
  *    (row e = column e of the paper's d x N matrices); W1 (gate), W3 (up)
  *    [E,I,d]; W2 (down) [E,d,I]; out [T,d].
  *  - dtype BEAM_BF16: x, weights and out are bfloat16; accumulation is fp32;
- *    the SwiGLU activations H and the per-pair expert outputs are rounded to
- *    bf16 once each.  dtype BEAM_F32: everything fp32.  Logits, softmax
+ *    the SwiGLU activations H (the second GEMM's operand) are rounded to bf16
+ *    once; the per-pair expert outputs stay fp32 and the weighted sum is
+ *    rounded to bf16 once.  dtype BEAM_F32: everything fp32.  Logits, softmax
  *    weights and the combine are fp32 in both.
  *  - Every pointer except the host descriptor is a DEVICE pointer, 16-byte
  *    aligned.  The caller owns every buffer, including the workspace; the
@@ -89,7 +90,7 @@ typedef struct {
  *   tiles     int32[tiles_cap][4] (expert, first row, valid rows, 0)
  *   xp        [p_cap][d]  gathered token rows (dtype)
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
- *   y         [p_cap][d]  expert output per pair (dtype)                    */
+ *   y         f32[p_cap][d] expert output per pair                           */
 typedef struct {
     int BN;            /* token rows per expert tile; the padding unit */
     int router_bn;     /* token rows per router tile */
