@@ -244,7 +244,8 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     if (s != BEAM_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Recorder rec{events, st};
-    if (d->T == 0) {
+    if (d->T == 0) {  // nothing to compute; leave a clean error word and counters
+        BEAM_TRY_CUDA(cudaMemsetAsync(workspace, 0, P.off_partial, st));
         for (int i = 0; i <= BEAM_MOE_FORWARD_STAGES; ++i) BEAM_TRY_CUDA(rec.rec(i));
         return BEAM_OK;
     }
@@ -362,6 +363,7 @@ beam_status beam_moe_route(const beam_moe_desc *desc, const void *x, const void 
     if (s != BEAM_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (desc->T == 0) {
+        BEAM_TRY_CUDA(cudaMemsetAsync(workspace, 0, P.off_partial, st));
         BEAM_TRY_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * desc->E, st));
         if (kept_hist)
             BEAM_TRY_CUDA(cudaMemsetAsync(kept_hist, 0, sizeof(int32_t) * (desc->K + 1), st));
