@@ -272,6 +272,10 @@ def time_steps(layer, f, steps, warmup, profiled=True, graph=False):
             call(layer.xs[i % N_BATCHES])
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)] for _ in range(steps)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
     for i in range(steps):
         layer.flush.fill_(i & 255)
         b = i % N_BATCHES
