@@ -231,71 +231,52 @@ def layer_roofline_seconds(layer, st, masked, pk):
     return t
 
 
-def time_steps(layer, f, steps, warmup, profiled=True, graph=False):
-    """Per-step device times (s) and per-stage times (s) over `steps` steps."""
+def time_steps(layer, f, steps, warmup):
+    """GPU time of `steps` layer steps: per step (s) and per stage (s).
+
+    One CUDA graph per token batch holds the whole forward with the library's
+    stage events as event nodes.  Each step: flush L2, replay, synchronise,
+    read the events, so step and kernel times are pure device time on the
+    launch stream, free of host launch gaps."""
     torch, abi = layer.torch, layer.abi
     Wm = layer.mask(f)
     S = abi.FORWARD_STAGES
-    stream = torch.cuda.current_stream()
-    args = (layer.dsc, None, layer.Wg, Wm, layer.W1, layer.W3, layer.W2, layer.out, layer.ws)
-
-    def call(x, events=None):
-        a = list(args)
-        a[1] = x
-        if events is not None:
-            abi.forward_profiled(*a, events)
-        else:
-            abi.forward(*a)
-
-    graphs = None
-    if graph:
-        graphs = []
-        s = torch.cuda.Stream()
-        s.wait_stream(stream)
-        with torch.cuda.stream(s):
-            for b in range(N_BATCHES):
-                call(layer.xs[b])
-            s.synchronize()
-            for b in range(N_BATCHES):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=s):
-                    a = list(args)
-                    a[1] = layer.xs[b]
-                    abi.forward(*a, stream=s)
-                graphs.append(g)
-        torch.cuda.synchronize()
-    for i in range(warmup):
-        layer.flush.fill_(i & 255)
-        if graph:
-            graphs[i % N_BATCHES].replay()
-        else:
-            call(layer.xs[i % N_BATCHES])
-    torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)]
+           for _ in range(N_BATCHES)]
     for row in evs:  # torch creates the CUDA event on first record
         for e in row:
             e.record()
     torch.cuda.synchronize()
-    for i in range(steps):
-        layer.flush.fill_(i & 255)
-        b = i % N_BATCHES
-        if graph:
-            evs[i][0].record()
-            graphs[b].replay()
-            evs[i][S].record()
-        elif profiled:
-            call(layer.xs[b], evs[i])
-        else:
-            evs[i][0].record()
-            call(layer.xs[b])
-            evs[i][S].record()
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for b in range(N_BATCHES):
+            abi.forward(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1, layer.W3, layer.W2,
+                        layer.out, layer.ws, stream=s)
+        s.synchronize()
+        for b in range(N_BATCHES):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                abi.forward_profiled(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1, layer.W3,
+                                     layer.W2, layer.out, layer.ws, evs[b], stream=s)
+            graphs.append(g)
     torch.cuda.synchronize()
-    step_s = [evs[i][0].elapsed_time(evs[i][S]) * 1e-3 for i in range(steps)]
-    stage_s = None
-    if profiled and not graph:
-        stage_s = [[evs[i][j].elapsed_time(evs[i][j + 1]) * 1e-3 for j in range(S)]
-                   for i in range(steps)]
+    for i in range(warmup):
+        layer.flush.fill_(i & 255)
+        graphs[i % N_BATCHES].replay()
+    torch.cuda.synchronize()
+    step_s, stage_s = [], []
+    for i in range(steps):
+        b = i % N_BATCHES
+        layer.flush.fill_(i & 255)
+        graphs[b].replay()
+        torch.cuda.synchronize()
+        e = evs[b]
+        stage_s.append([e[j].elapsed_time(e[j + 1]) * 1e-3 for j in range(S)])
+        step_s.append(e[0].elapsed_time(e[S]) * 1e-3)
     abi.check(layer.dsc, layer.ws)
+    del graphs
     return step_s, stage_s
 
 
@@ -371,7 +352,7 @@ def run_beam(args):
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
-        step_s, stage_s = time_steps(layer, f_head, args.steps, args.warmup, profiled=True)
+        step_s, stage_s = time_steps(layer, f_head, args.steps, args.warmup)
         torch.cuda.synchronize()
         barrier(world)
     total = sum(step_s)
@@ -402,11 +383,6 @@ def run_beam(args):
     t_roof = sum(layer_roofline_seconds(layer, st[i % N_BATCHES], True, pk)
                  for i in range(args.steps)) / args.steps
 
-    # graph-replayed headline (launch overhead removed)
-    g_step, _ = time_steps(layer, f_head, max(50, min(args.steps, 500)), 3, profiled=False,
-                           graph=True)
-    g_mean = sum(g_step) / len(g_step)
-
     # ---- per kept fraction, next to the mask-disabled kernels -------------
     sweep = []
     if not args.no_sweep:
@@ -417,7 +393,7 @@ def run_beam(args):
             rows = []
             for f in (None, 0.15, 0.35, 0.6, 1.0):
                 sts = lay.routing_stats(f)
-                gs, _ = time_steps(lay, f, 100, 5, profiled=False, graph=True)
+                gs, _ = time_steps(lay, f, args.sweep_steps, 5)
                 tm = sum(gs) / len(gs)
                 troof = sum(layer_roofline_seconds(lay, s, f is not None, pk) for s in sts) / len(sts)
                 kept = sum(s["P"] for s in sts) / len(sts) / (Tn * lay.sh.K)
@@ -454,12 +430,12 @@ def run_beam(args):
             "kept_fraction_measured": P_mean / (T * layer.sh.K),
             "experts_touched_mean": U_mean, "kept_pairs_mean": P_mean,
             "l2": "flushed (256 MiB write) before every timed step; 8 token batches cycled",
-            "timing": "CUDA events recorded by the library between its kernels, eager calls",
+            "timing": ("CUDA graph replay per step; CUDA events recorded by the library "
+                       "between its kernels (graph event nodes) give step and kernel times"),
             "parallelism": f"replicas x{world} (tokens independent, no collective)",
         },
-        "ms_per_step_graph": g_mean * 1e3,
-        "layer_roofline": dict(us=t_roof * 1e6, frac_of_measured_step=t_roof / step_mean,
-                               frac_graph=t_roof / g_mean, peak_source=pk["source"]),
+        "layer_roofline": dict(us=t_roof * 1e6, frac=t_roof / step_mean,
+                               peak_source=pk["source"]),
         "roofline": roofline,
         "kernels": kernels,
         "per_kept_fraction": sweep,
@@ -523,12 +499,13 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["beam", "reference"], default="beam")
     ap.add_argument("--T", type=int, default=128)
     ap.add_argument("--kept", type=float, default=0.15)
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--sweep-steps", type=int, default=100)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=32)

@@ -144,12 +144,16 @@ bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
     return r == CUDA_SUCCESS;
 }
 
+// Records the caller's timing events between stages.  External records
+// become event nodes when the call is captured into a CUDA graph, so the
+// per-kernel times can also be read from graph replays.
 struct Recorder {
     void *const *events;
     cudaStream_t st;
     cudaError_t rec(int i) const {
         if (!events) return cudaSuccess;
-        return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+        return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,
+                                        cudaEventRecordExternal);
     }
 };
 

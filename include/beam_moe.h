@@ -143,7 +143,9 @@ beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const voi
 /* beam_moe_forward that also records `events[i]` (cudaEvent_t, created by the
  * caller) on `stream` before stage i and events[BEAM_MOE_FORWARD_STAGES]
  * after the last one, so the caller can time each kernel with
- * cudaEventElapsedTime.  Same launches and results as beam_moe_forward. */
+ * cudaEventElapsedTime.  The records are "external" (cudaEventRecordExternal):
+ * captured into a CUDA graph they become event nodes that every replay
+ * re-records.  Same launches and results as beam_moe_forward. */
 beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
                                       const void *W_gate, const void *W_mask,
                                       const void *W1, const void *W3, const void *W2,
