@@ -231,18 +231,22 @@ def layer_roofline_seconds(layer, st, masked, pk):
     return t
 
 
-def time_steps(layer, f, steps, warmup):
-    """GPU time of `steps` layer steps: per step (s) and per stage (s).
+def time_steps(layer, f, steps, warmup, profiled=False, only=None):
+    """GPU time of `steps` layer steps: per step (s) and, if `profiled`, per
+    stage (s).
 
-    One CUDA graph per token batch holds the whole forward with the library's
-    stage events as event nodes.  Each step: flush L2, replay, synchronise,
-    read the events, so step and kernel times are pure device time on the
-    launch stream, free of host launch gaps."""
+    One CUDA graph per token batch holds the whole forward.  Each step: flush
+    L2, replay, synchronise, read the events; the times are device time on the
+    launch stream, free of host launch gaps.  Without `profiled` the events
+    bracket the replay.  With it, the library records its stage events inside
+    the graph (event nodes) between the kernels; those records lengthen the
+    step by a few microseconds each, so they are used for the per-kernel
+    breakdown only.  `only` = j records just the events around stage j."""
     torch, abi = layer.torch, layer.abi
     Wm = layer.mask(f)
     S = abi.FORWARD_STAGES
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)]
-           for _ in range(N_BATCHES)]
+           for _ in range(N_BATCHES if profiled else 1)]
     for row in evs:  # torch creates the CUDA event on first record
         for e in row:
             e.record()
@@ -258,8 +262,15 @@ def time_steps(layer, f, steps, warmup):
         for b in range(N_BATCHES):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                abi.forward_profiled(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1, layer.W3,
-                                     layer.W2, layer.out, layer.ws, evs[b], stream=s)
+                if profiled:
+                    ev = evs[b] if only is None else [
+                        e if j in (only, only + 1) else None for j, e in enumerate(evs[b])]
+                    abi.forward_profiled(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1,
+                                         layer.W3, layer.W2, layer.out, layer.ws, ev,
+                                         stream=s)
+                else:
+                    abi.forward(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1, layer.W3,
+                                layer.W2, layer.out, layer.ws, stream=s)
             graphs.append(g)
     torch.cuda.synchronize()
     for i in range(warmup):
@@ -270,10 +281,19 @@ def time_steps(layer, f, steps, warmup):
     for i in range(steps):
         b = i % N_BATCHES
         layer.flush.fill_(i & 255)
-        graphs[b].replay()
+        if profiled:
+            graphs[b].replay()
+        else:
+            evs[0][0].record()
+            graphs[b].replay()
+            evs[0][S].record()
         torch.cuda.synchronize()
-        e = evs[b]
-        stage_s.append([e[j].elapsed_time(e[j + 1]) * 1e-3 for j in range(S)])
+        e = evs[b] if profiled else evs[0]
+        if profiled and only is not None:
+            stage_s.append(e[only].elapsed_time(e[only + 1]) * 1e-3)
+            continue
+        if profiled:
+            stage_s.append([e[j].elapsed_time(e[j + 1]) * 1e-3 for j in range(S)])
         step_s.append(e[0].elapsed_time(e[S]) * 1e-3)
     abi.check(layer.dsc, layer.ws)
     del graphs
@@ -352,9 +372,11 @@ def run_beam(args):
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
-        step_s, stage_s = time_steps(layer, f_head, args.steps, args.warmup)
+        step_s, _ = time_steps(layer, f_head, args.steps, args.warmup)
         torch.cuda.synchronize()
         barrier(world)
+        # per-kernel breakdown: the same steps with the library's stage events
+        prof_s, stage_s = time_steps(layer, f_head, args.steps, args.warmup, profiled=True)
     total = sum(step_s)
     tmax, units = reduce_time_and_units(total, T * args.steps, world, device)
     value = units / tmax
@@ -363,14 +385,17 @@ def run_beam(args):
     names = [layer.abi.stage_name(j) for j in range(S)]
     stage_mean = [sum(s[j] for s in stage_s) / len(stage_s) for j in range(S)]
     step_mean = total / len(step_s)
-    kernels = {names[j]: dict(us=stage_mean[j] * 1e6, share=stage_mean[j] / step_mean)
+    prof_mean = sum(prof_s) / len(prof_s)
+    kernels = {names[j]: dict(us=stage_mean[j] * 1e6, share=stage_mean[j] / prof_mean)
                for j in range(S)}
     # dominant kernel vs its roofline (algorithmic bytes/flops averaged over batches)
     dom = max(range(S), key=lambda j: stage_mean[j])
     alg = [algorithmic(layer, st[i % N_BATCHES], True) for i in range(args.steps)]
     a_bytes = sum(a[names[dom]]["bytes"] for a in alg) / len(alg)
     a_flops = sum(a[names[dom]]["flops"] for a in alg) / len(alg)
-    t_dom = stage_mean[dom]
+    # the dominant kernel alone between two events (least perturbed timing)
+    _, dom_s = time_steps(layer, f_head, args.steps, args.warmup, profiled=True, only=dom)
+    t_dom = sum(dom_s) / len(dom_s)
     hbm_t = a_bytes / (pk["hbm"] * 1e9)
     tc_t = a_flops / (pk["bf16"] * 1e12)
     if tc_t > hbm_t:
@@ -379,6 +404,7 @@ def run_beam(args):
         achieved, peak, unit, bound = a_bytes / t_dom / 1e9, pk["hbm"], "GB/s", "hbm"
     roofline = dict(kernel=names[dom], bound=bound, achieved=achieved, peak=peak, unit=unit,
                     frac=achieved / peak, traffic=None, peak_source=pk["source"],
+                    us_per_launch=t_dom * 1e6,
                     algorithmic_bytes_per_launch=a_bytes, algorithmic_flops_per_launch=a_flops)
     t_roof = sum(layer_roofline_seconds(layer, st[i % N_BATCHES], True, pk)
                  for i in range(args.steps)) / args.steps
@@ -430,14 +456,18 @@ def run_beam(args):
             "kept_fraction_measured": P_mean / (T * layer.sh.K),
             "experts_touched_mean": U_mean, "kept_pairs_mean": P_mean,
             "l2": "flushed (256 MiB write) before every timed step; 8 token batches cycled",
-            "timing": ("CUDA graph replay per step; CUDA events recorded by the library "
-                       "between its kernels (graph event nodes) give step and kernel times"),
+            "timing": ("one CUDA graph replay per step, CUDA events around it on the launch "
+                       "stream; kernel times from a second pass with event nodes"),
             "parallelism": f"replicas x{world} (tokens independent, no collective)",
         },
         "layer_roofline": dict(us=t_roof * 1e6, frac=t_roof / step_mean,
                                peak_source=pk["source"]),
         "roofline": roofline,
         "kernels": kernels,
+        "kernels_note": ("per-kernel device time between the library's stage events "
+                         f"(a second pass of {args.steps} steps with event nodes in the "
+                         f"graph: {prof_mean * 1e6:.1f} us/step vs {step_mean * 1e6:.1f} "
+                         "without them)"),
         "per_kept_fraction": sweep,
         "e2e": e2e,
         "gpu_launches": S * args.steps,

@@ -148,8 +148,10 @@ def forward(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, stream=None):
 
 
 def forward_profiled(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, events, stream=None):
-    """`events`: FORWARD_STAGES + 1 torch.cuda.Event(enable_timing=True)."""
-    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    """`events`: FORWARD_STAGES + 1 torch.cuda.Event(enable_timing=True) or None
+    (None records nothing at that point)."""
+    arr = (ctypes.c_void_p * len(events))(*[None if e is None else e.cuda_event
+                                             for e in events])
     _ok(lib().beam_moe_forward_profiled(ctypes.byref(dsc), _ptr(x), _ptr(W_gate), _ptr(W_mask),
                                         _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out),
                                         _ptr(workspace), workspace.numel(), _stream(stream),

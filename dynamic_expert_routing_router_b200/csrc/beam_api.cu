@@ -67,7 +67,8 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
         const long long nkb = d->d / kBlockK;
         const long long cap_bytes = T > 0 ? d->d / (2 * T) : nkb;
         int S = 1;
-        while (2LL * S <= nkb && nkb % (2LL * S) == 0 && base * 2 * S <= kNominalSMs &&
+        while (2LL * S <= kMaxRouterSplits && 2LL * S <= nkb && nkb % (2LL * S) == 0 &&
+               base * 2 * S <= kNominalSMs &&
                2LL * S <= (cap_bytes > 1 ? cap_bytes : 1))
             S *= 2;
         P->router_splits = S;
@@ -151,7 +152,7 @@ struct Recorder {
     void *const *events;
     cudaStream_t st;
     cudaError_t rec(int i) const {
-        if (!events) return cudaSuccess;
+        if (!events || !events[i]) return cudaSuccess;
         return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,
                                         cudaEventRecordExternal);
     }
@@ -392,8 +393,6 @@ beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
                                       size_t workspace_bytes, void *stream,
                                       void *const *events) {
     if (!events) return BEAM_ERR_INVALID_ARG;
-    for (int i = 0; i <= BEAM_MOE_FORWARD_STAGES; ++i)
-        if (!events[i]) return BEAM_ERR_INVALID_ARG;
     return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, out, workspace, workspace_bytes,
                         stream, events);
 }

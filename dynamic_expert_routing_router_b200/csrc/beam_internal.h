@@ -25,6 +25,7 @@ constexpr int kBlockK = 64;    // reduction elements per stage: one 128-byte bf1
 constexpr int kNominalSMs = 148;
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 16;
+constexpr int kMaxRouterSplits = 32;  // top-K sums the split partials unrolled
 
 struct ZeroRegion {
     int *ptr;

@@ -28,7 +28,7 @@ constexpr unsigned kFull = 0xffffffffu;
 // The mask keeps candidate k iff its pre-sigmoid value z >= 0 (Eq. 6; NaN
 // is not kept); w = g * m (Eq. 7).  Counts and the histogram are gathered in
 // shared memory and added to global memory once per block.
-template <int EPL>
+template <int EPL, int S>
 __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a) {
     __shared__ int s_counts[kMaxE];
     __shared__ int s_hist[kMaxK + 1];
@@ -50,11 +50,20 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a) {
             r[i] = -INFINITY;
             z[i] = 0.0f;
             if (j < a.E) {
+                // All S partials are loaded before they are added (S is a
+                // compile-time constant), then summed in split order.
                 const float *pr = a.partial + (long long)t * E2 + j;
+                float pr_r[S], pr_z[S];
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    pr_r[s] = __ldg(pr + s * slab);
+                    pr_z[s] = a.has_mask ? __ldg(pr + s * slab + a.E) : 0.0f;
+                }
                 float rs = 0.0f, zs = 0.0f;
-                for (int s = 0; s < a.S; ++s) {
-                    rs += pr[s * slab];
-                    if (a.has_mask) zs += pr[s * slab + a.E];
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    rs += pr_r[s];
+                    zs += pr_z[s];
                 }
                 if (a.logits) {
                     a.logits[(long long)t * E2 + j] = rs;
@@ -397,17 +406,30 @@ __global__ void __launch_bounds__(256) gemm2_f32_kernel(const float *H, const fl
 
 }  // namespace
 
+template <int EPL>
+cudaError_t launch_topk_s(const TopkArgs &a, int blocks, cudaStream_t stream) {
+    switch (a.S) {
+        case 1: topk_mask_kernel<EPL, 1><<<blocks, 256, 0, stream>>>(a); break;
+        case 2: topk_mask_kernel<EPL, 2><<<blocks, 256, 0, stream>>>(a); break;
+        case 4: topk_mask_kernel<EPL, 4><<<blocks, 256, 0, stream>>>(a); break;
+        case 8: topk_mask_kernel<EPL, 8><<<blocks, 256, 0, stream>>>(a); break;
+        case 16: topk_mask_kernel<EPL, 16><<<blocks, 256, 0, stream>>>(a); break;
+        case 32: topk_mask_kernel<EPL, 32><<<blocks, 256, 0, stream>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
     if (a.T <= 0) return cudaSuccess;
     const int warps = 8;
     int blocks = (a.T + warps - 1) / warps;
     if (blocks > 2 * n_sm) blocks = 2 * n_sm;
     const int epl = (a.E + 31) / 32;
-    if (epl <= 1) topk_mask_kernel<1><<<blocks, 256, 0, stream>>>(a);
-    else if (epl <= 2) topk_mask_kernel<2><<<blocks, 256, 0, stream>>>(a);
-    else if (epl <= 4) topk_mask_kernel<4><<<blocks, 256, 0, stream>>>(a);
-    else topk_mask_kernel<8><<<blocks, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    if (epl <= 1) return launch_topk_s<1>(a, blocks, stream);
+    if (epl <= 2) return launch_topk_s<2>(a, blocks, stream);
+    if (epl <= 4) return launch_topk_s<4>(a, blocks, stream);
+    return launch_topk_s<8>(a, blocks, stream);
 }
 
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {

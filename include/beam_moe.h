@@ -145,7 +145,9 @@ beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const voi
  * after the last one, so the caller can time each kernel with
  * cudaEventElapsedTime.  The records are "external" (cudaEventRecordExternal):
  * captured into a CUDA graph they become event nodes that every replay
- * re-records.  Same launches and results as beam_moe_forward. */
+ * re-records.  A NULL entry records nothing at that point (each record costs
+ * a few microseconds of device time, so time one kernel with just the two
+ * events around it).  Same launches and results as beam_moe_forward. */
 beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
                                       const void *W_gate, const void *W_mask,
                                       const void *W1, const void *W3, const void *W2,
