@@ -66,6 +66,8 @@ def lib():
         L.beam_moe_forward_profiled.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                 ctypes.POINTER(vp)]
         L.beam_moe_check.argtypes = [pd, vp, vp]
+        L.beam_moe_route_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.beam_moe_route_noalloc.restype = i32
         L.beam_status_str.argtypes = [i32]
         L.beam_status_str.restype = ctypes.c_char_p
         L.beam_moe_stage_name.argtypes = [i32]
@@ -139,6 +141,18 @@ def route(dsc, x, W_gate, W_mask, topk_idx, topk_w, counts, hist=None, logits=No
                              _ptr(logits), _ptr(workspace),
                              workspace.numel() if workspace is not None else 0,
                              _stream(stream)), "beam_moe_route")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def route_noalloc(dsc, x, W_gate, W_mask, topk_idx, topk_w, counts, hist=None, logits=None,
+                  stream=None):
+    """beam_moe_route without a caller workspace (scratch in the library's own
+    fixed device array); for callers that cannot allocate device memory."""
+    _ok(lib().beam_moe_route_noalloc(ctypes.byref(dsc), _ptr(x), _ptr(W_gate), _ptr(W_mask),
+                                     _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(hist),
+                                     _ptr(logits), _stream(stream)), "beam_moe_route_noalloc")
 
 
 def forward(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, stream=None):

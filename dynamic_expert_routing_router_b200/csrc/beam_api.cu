@@ -331,6 +331,50 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     return BEAM_OK;
 }
 
+}  // namespace
+
+namespace beam {
+
+size_t route_scratch_bytes(const beam_moe_desc *desc) {
+    beam_moe_plan_info P;
+    if (make_plan(desc, &P) != BEAM_OK) return 0;
+    return P.off_idx;  // header + router partials: all the routing call uses
+}
+
+beam_status route_into_scratch(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                               const void *W_mask, int32_t *topk_idx, float *topk_w,
+                               int32_t *expert_counts, int32_t *kept_hist, float *logits,
+                               void *scratch, size_t scratch_bytes, cudaStream_t st) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(desc, &P);
+    if (s != BEAM_OK) return s;
+    if (!x || !W_gate || !topk_idx || !topk_w || !expert_counts) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x, W_gate, static_cast<const void *>(topk_idx),
+                          static_cast<const void *>(topk_w), static_cast<const void *>(expert_counts)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    if ((W_mask && !aligned16(W_mask)) || (kept_hist && !aligned16(kept_hist)) ||
+        (logits && !aligned16(logits)))
+        return BEAM_ERR_INVALID_ARG;
+    if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u) != 0 ||
+        scratch_bytes < P.off_idx)
+        return BEAM_ERR_WORKSPACE;
+    if (desc->T == 0) {
+        BEAM_TRY_CUDA(cudaMemsetAsync(scratch, 0, P.off_partial, st));
+        BEAM_TRY_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * desc->E, st));
+        if (kept_hist)
+            BEAM_TRY_CUDA(cudaMemsetAsync(kept_hist, 0, sizeof(int32_t) * (desc->K + 1), st));
+        return BEAM_OK;
+    }
+    const RouteOut ro{topk_idx, topk_w, expert_counts, kept_hist, logits};
+    const Recorder rec{nullptr, st};
+    return launch_route(desc, P, x, W_gate, W_mask, ro, static_cast<char *>(scratch), st, rec,
+                        sm_count());
+}
+
+}  // namespace beam
+
+namespace {
+
 const char *const kStageNames[BEAM_MOE_FORWARD_STAGES] = {
     "router_gemm", "topk_mask", "permute", "gather", "gemm1_gate_up_swiglu", "gemm2_down",
     "combine"};

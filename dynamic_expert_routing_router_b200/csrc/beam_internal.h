@@ -100,4 +100,12 @@ cudaError_t launch_gemm1_f32(const float *xp, const float *W1, const float *W3, 
 cudaError_t launch_gemm2_f32(const float *H, const float *W2, const int4 *tiles, const int *meta,
                              int tiles_cap, int d, int I, float *Y, cudaStream_t stream);
 
+// Routing (the two kernels of beam_moe_route) into caller-provided scratch
+// of at least route_scratch_bytes(desc) bytes, 256-byte aligned.
+size_t route_scratch_bytes(const beam_moe_desc *desc);  // 0 on a bad descriptor
+beam_status route_into_scratch(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                               const void *W_mask, int32_t *topk_idx, float *topk_w,
+                               int32_t *expert_counts, int32_t *kept_hist, float *logits,
+                               void *scratch, size_t scratch_bytes, cudaStream_t stream);
+
 }  // namespace beam

@@ -154,6 +154,37 @@ beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
                                       void *out, void *workspace, size_t workspace_bytes,
                                       void *stream, void *const *events);
 
+/* Bytes of the fixed device array behind beam_moe_route_noalloc (16 MiB). */
+#define BEAM_MOE_ROUTE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* beam_moe_route for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a service of this library.
+ *
+ * Who needs it: code running while a stream is captured into a CUDA graph in
+ * the global or thread-local capture mode (cudaMalloc is illegal there and
+ * breaks the capture), and plugins inside a runtime whose memory pool owns
+ * the device memory and does not let extensions allocate.  The caller still
+ * passes every input and output exactly as for beam_moe_route; the scratch
+ * (router partial logits, error word, counters) lives in a file-scope device
+ * array of BEAM_MOE_ROUTE_NOALLOC_SCRATCH_BYTES that every GPU loading the
+ * library holds until the process exits.  Nothing here calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *  - Size limit: the call needs beam_moe_plan(desc)->off_idx bytes of
+ *    scratch; larger batches return BEAM_ERR_WORKSPACE before any launch (for
+ *    d=2048, E=128 every T up to 8192 fits).
+ *  - The first call on a device looks the array's address up on that device
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array: calls whose kernels may overlap on the GPU
+ *    (different streams, or concurrent host threads) race on it and must be
+ *    ordered by the caller.  Each call clears what must start at zero.
+ *  - Same kernels and results as beam_moe_route; beam_moe_check does not
+ *    apply (there is no caller workspace to read). */
+beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
+                                   const void *W_gate, const void *W_mask, int32_t *topk_idx,
+                                   float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
+                                   float *logits, void *stream);
+
 /* Synchronise `stream`, then read the workspace error word written by the last
  * call: BEAM_OK, BEAM_ERR_TIMEOUT (a bounded device wait expired, the kernel
  * returned early) or BEAM_ERR_INTERNAL (a device consistency check failed). */
