@@ -282,9 +282,13 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     BEAM_TRY_CUDA(launch_gather(x, pair, meta, d->K, (long long)es * d->d, P.p_cap, xp, n_sm, st));
 
     if (d->dtype == BEAM_BF16) {
+        // Thin token tiles: gate and up rows interleaved in one 128-row tile
+        // (twice the work units); 128-token tiles: two 128-row weight tiles.
+        const bool interleave = P.BN < 128;
+        const unsigned wbox = interleave ? kBlockM / 2 : kBlockM;
         CUtensorMap mW1, mW3, mW2, mXp, mH;
-        if (!make_tmap(&mW1, W1, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mW3, W3, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mW1, W1, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&mW3, W3, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
         if (!make_tmap(&mW2, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
         if (!make_tmap(&mXp, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
         if (!make_tmap(&mH, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
@@ -297,14 +301,14 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         g.timeout_ns = kWaitTimeoutNs;
 
         BEAM_TRY_CUDA(rec.rec(4));
-        g.n_mb = d->I / kBlockM;
+        g.n_mb = d->I / int(wbox);
         g.nk = d->d / kBlockK;
         g.a_rows_per_expert = d->I;
         g.out = h;
         g.out_ld = d->I;
         long long units = (long long)P.tiles_cap * g.n_mb;
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, mW1, mW3, mXp, g,
-                                     int(units < n_sm ? units : n_sm), st));
+        BEAM_TRY_CUDA(launch_tc_gemm(interleave ? MODE_GEMM1_IL : MODE_GEMM1, P.BN, mW1, mW3, mXp,
+                                     g, int(units < n_sm ? units : n_sm), st));
 
         BEAM_TRY_CUDA(rec.rec(5));
         g.n_mb = d->d / kBlockM;

@@ -17,7 +17,8 @@ enum : int { DEV_OK = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_INTERNAL = 2 };
 enum TcMode : int {
     MODE_ROUTER = 0,  // logits: [W_gate | W_mask] rows x token rows, split over d
     MODE_GEMM1 = 1,   // SiLU(W1 x) * (W3 x) per kept pair  -> H
-    MODE_GEMM2 = 2    // W2 h per kept pair                  -> Y
+    MODE_GEMM2 = 2,   // W2 h per kept pair                  -> Y
+    MODE_GEMM1_IL = 3 // GEMM1 with 64 rows of W1 and 64 of W3 interleaved in one tile
 };
 
 constexpr int kBlockM = 128;   // weight rows per tile (the MMA's M)

@@ -4,6 +4,11 @@
 // One persistent, warp-specialised kernel serves three roles:
 //   MODE_ROUTER  logits  r = x W_gate, z = x W_mask   (BEAM §3.2 steps 1-2)
 //   MODE_GEMM1   H = SiLU(x W1_e^T) * (x W3_e^T)      (Eq. 3, gate/up + SwiGLU)
+//                two 128-row weight tiles (W1, W3), two accumulators
+//   MODE_GEMM1_IL the same with 64 rows of W1 and the matching 64 rows of W3
+//                in one 128-row tile and one accumulator: twice the work units
+//                for thin token tiles; the epilogue warps pair gate and up
+//                rows through shared memory
 //   MODE_GEMM2   Y = H W2_e^T  (fp32 out)              (Eq. 3, down projection)
 //
 // Orientation: the weight rows are the MMA's M operand (128 rows per tile)
@@ -34,14 +39,18 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kUmmaK = 16;  // K of one kind::f16 MMA
 
-template <int NUM_A, int BN>
+constexpr int kXchLd = 17;  // padded row of the gate/up exchange buffer (floats)
+
+template <int NUM_A, int BN, bool XCH>
 struct TcCfg {
     static constexpr uint32_t A_BYTES = kBlockM * kBlockK * 2;  // 16 KB
     static constexpr uint32_t B_BYTES = BN * kBlockK * 2;
     static constexpr uint32_t STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
-    static constexpr int STAGES_FIT = int((220u * 1024u) / STAGE_BYTES);
+    static constexpr uint32_t XCH_BYTES = XCH ? kBlockM * kXchLd * 4 : 0;
+    static constexpr int STAGES_FIT = int((220u * 1024u - XCH_BYTES) / STAGE_BYTES);
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+    static constexpr uint32_t SMEM_BYTES =
+        STAGES * STAGE_BYTES + XCH_BYTES + 1024;  // + alignment slack
     static constexpr uint32_t ACC_COLS = NUM_A * BN;  // fp32 columns per accumulator
     static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
     static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
@@ -62,6 +71,11 @@ struct Unit {
     int rows;   // GEMMs: valid token rows of the tile
 };
 
+// Named barrier of the four epilogue warps (barrier 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_sync() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
 template <int MODE, int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const TcGemmArgs &p) {
     Unit w;
@@ -77,7 +91,8 @@ __device__ __forceinline__ Unit decode_unit(int u, const TcGemmArgs &p) {
         w.rows = 0;
     } else {
         const int4 t = p.tiles[rest];
-        w.a_row = t.x * p.a_rows_per_expert + w.mb * kBlockM;
+        const int rows_per_mb = (MODE == MODE_GEMM1_IL) ? kBlockM / 2 : kBlockM;
+        w.a_row = t.x * p.a_rows_per_expert + w.mb * rows_per_mb;
         w.b_row = t.y;
         w.rows = t.z;
         w.kb0 = 0;
@@ -101,10 +116,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                    const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const TcGemmArgs p) {
-    using C = TcCfg<NUM_A, BN>;
+    using C = TcCfg<NUM_A, BN, MODE == MODE_GEMM1_IL>;
     constexpr int STAGES = C::STAGES;
 
     extern __shared__ uint8_t smem_raw[];
+    __shared__ int xvote[4];
     __shared__ __align__(8) uint64_t full_bar[STAGES];
     __shared__ __align__(8) uint64_t empty_bar[STAGES];
     __shared__ __align__(8) uint64_t tfull_bar[2];
@@ -170,7 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
                     const int kx = (w.kb0 + kb) * kBlockK;
-                    tma_load_2d(st, am, kx, w.a_row, &full_bar[s]);
+                    if (MODE == MODE_GEMM1_IL) {
+                        // rows 0..63: W1 (gate), rows 64..127: W3 (up), same I rows
+                        tma_load_2d(st, &tmA0, kx, w.a_row, &full_bar[s]);
+                        tma_load_2d(st + C::A_BYTES / 2, &tmA1, kx, w.a_row, &full_bar[s]);
+                    } else {
+                        tma_load_2d(st, am, kx, w.a_row, &full_bar[s]);
+                    }
                     if (NUM_A == 2) tma_load_2d(st + C::A_BYTES, &tmA1, kx, w.a_row, &full_bar[s]);
                     tma_load_2d(st + NUM_A * C::A_BYTES, &tmB, kx, w.b_row, &full_bar[s]);
                 }
@@ -238,6 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t a = lu & 1u;
             bool ok = mbar_wait_bounded(&tfull_bar[a], (lu >> 1) & 1u, abort_flag, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
+            if (MODE == MODE_GEMM1_IL) {
+                // The four warps meet at named barriers below: agree first.
+                if (lane == 0) xvote[warp - 2] = ok ? 1 : 0;
+                epilogue_sync();
+                ok = xvote[0] && xvote[1] && xvote[2] && xvote[3];
+            }
             if (!ok) {
                 if (lane == 0) signal_abort(p.err, &abort_sh);
                 break;
@@ -263,6 +291,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (t < p.T) out[(long long)t * p.out_ld] = __uint_as_float(g[c]);
                         }
                     }
+                } else if (MODE == MODE_GEMM1_IL) {
+                    // TMEM rows 0..63 hold gate, 64..127 up, for I rows mb*64 + r.
+                    float *xch = reinterpret_cast<float *>(smem + size_t(STAGES) * C::STAGE_BYTES);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) xch[row * kXchLd + c] = __uint_as_float(g[c]);
+                    epilogue_sync();
+                    const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
+                    const int r = et & 63, half = et >> 6;
+                    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
+                                         (long long)w.b_row * p.out_ld + w.mb * (kBlockM / 2) + r;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const int c = half * 8 + cc;
+                        if (c0 + c < w.rows)
+                            out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(
+                                silu_mul(xch[r * kXchLd + c], xch[(64 + r) * kXchLd + c]));
+                    }
+                    epilogue_sync();
                 } else if (MODE == MODE_GEMM1) {
                     // H (bf16): the next GEMM's operand.
                     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
@@ -298,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int MODE, int NUM_A, int BN>
 cudaError_t launch_cfg(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                        const TcGemmArgs &args, int grid, cudaStream_t stream) {
-    using C = TcCfg<NUM_A, BN>;
+    using C = TcCfg<NUM_A, BN, MODE == MODE_GEMM1_IL>;
     auto kern = tc_gemm_kernel<MODE, NUM_A, BN>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM_BYTES));
@@ -328,6 +374,7 @@ cudaError_t launch_tc_gemm(int mode, int bn, const CUtensorMap &a0, const CUtens
     switch (mode) {
         case MODE_ROUTER: return launch_bn<MODE_ROUTER, 1>(bn, a0, a1, b, args, grid, stream);
         case MODE_GEMM1: return launch_bn<MODE_GEMM1, 2>(bn, a0, a1, b, args, grid, stream);
+        case MODE_GEMM1_IL: return launch_bn<MODE_GEMM1_IL, 1>(bn, a0, a1, b, args, grid, stream);
         case MODE_GEMM2: return launch_bn<MODE_GEMM2, 1>(bn, a0, a1, b, args, grid, stream);
         default: return cudaErrorInvalidValue;
     }
