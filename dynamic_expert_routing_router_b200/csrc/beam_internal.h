@@ -28,6 +28,25 @@ constexpr int kMaxE = 256;
 constexpr int kMaxK = 16;
 constexpr int kMaxRouterSplits = 32;  // top-K sums the split partials unrolled
 
+// Launch with programmatic stream serialization (PDL): the kernel may begin
+// its prologue while the previous kernel in the stream finishes; every kernel
+// of this library waits (griddep_wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 struct ZeroRegion {
     int *ptr;
     int count;

@@ -19,6 +19,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialization may start while its
+// predecessor in the stream is still running.  It must call griddep_wait()
+// before touching any global memory its predecessor writes or reads; after
+// that it lets its own successor start launching.  Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

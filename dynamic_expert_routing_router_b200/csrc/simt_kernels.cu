@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a) {
     for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_counts[i] = 0;
     if (threadIdx.x <= a.K) s_hist[threadIdx.x] = 0;
     __syncthreads();
+    griddep_wait();
+    griddep_launch_dependents();
 
     const int lane = threadIdx.x & 31;
     const int warps = blockDim.x >> 5;
@@ -165,6 +167,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     __shared__ int s_total;
     const int e = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    griddep_launch_dependents();
 
     int c = 0;
     if (tid < a.E) c = a.counts[tid];
@@ -230,6 +234,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
 __global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *pair,
                                                      const int *meta, int K, int row_vec,
                                                      uint4 *xp) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int rows = meta[1];
     const int lane = threadIdx.x & 31;
     for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
@@ -270,6 +276,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
     __shared__ int s_row[kMaxK];
     __shared__ float s_w[kMaxK];
     const int nvec = d / 8;
+    griddep_wait();
+    griddep_launch_dependents();
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < K) {
             const long long o = (long long)t * K + threadIdx.x;
@@ -409,15 +417,14 @@ __global__ void __launch_bounds__(256) gemm2_f32_kernel(const float *H, const fl
 template <int EPL>
 cudaError_t launch_topk_s(const TopkArgs &a, int blocks, cudaStream_t stream) {
     switch (a.S) {
-        case 1: topk_mask_kernel<EPL, 1><<<blocks, 256, 0, stream>>>(a); break;
-        case 2: topk_mask_kernel<EPL, 2><<<blocks, 256, 0, stream>>>(a); break;
-        case 4: topk_mask_kernel<EPL, 4><<<blocks, 256, 0, stream>>>(a); break;
-        case 8: topk_mask_kernel<EPL, 8><<<blocks, 256, 0, stream>>>(a); break;
-        case 16: topk_mask_kernel<EPL, 16><<<blocks, 256, 0, stream>>>(a); break;
-        case 32: topk_mask_kernel<EPL, 32><<<blocks, 256, 0, stream>>>(a); break;
+        case 1: return launch_pdl(topk_mask_kernel<EPL, 1>, dim3(blocks), dim3(256), 0, stream, a);
+        case 2: return launch_pdl(topk_mask_kernel<EPL, 2>, dim3(blocks), dim3(256), 0, stream, a);
+        case 4: return launch_pdl(topk_mask_kernel<EPL, 4>, dim3(blocks), dim3(256), 0, stream, a);
+        case 8: return launch_pdl(topk_mask_kernel<EPL, 8>, dim3(blocks), dim3(256), 0, stream, a);
+        case 16: return launch_pdl(topk_mask_kernel<EPL, 16>, dim3(blocks), dim3(256), 0, stream, a);
+        case 32: return launch_pdl(topk_mask_kernel<EPL, 32>, dim3(blocks), dim3(256), 0, stream, a);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
@@ -433,8 +440,7 @@ cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
 }
 
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {
-    permute_kernel<<<a.E, kPermThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, stream, a);
 }
 
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
@@ -443,9 +449,9 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
     int blocks = (p_cap + 7) / 8;
     if (blocks > 8 * n_sm) blocks = 8 * n_sm;
     if (blocks <= 0) return cudaSuccess;
-    gather_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4 *>(x), pair, meta, K,
-                                              int(row_bytes / 16), static_cast<uint4 *>(xp));
-    return cudaGetLastError();
+    return launch_pdl(gather_kernel, dim3(blocks), dim3(256), 0, stream,
+                      static_cast<const uint4 *>(x), pair, meta, K, int(row_bytes / 16),
+                      static_cast<uint4 *>(xp));
 }
 
 cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
@@ -456,12 +462,10 @@ cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const floa
     threads = threads >= 256 ? 256 : ((threads + 31) / 32) * 32;
     int blocks = T < 8 * n_sm ? T : 8 * n_sm;
     if (dtype == BEAM_BF16)
-        combine_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
-            Y, idx, w, pair_pos, T, K, d, static_cast<__nv_bfloat16 *>(out));
-    else
-        combine_kernel<float><<<blocks, threads, 0, stream>>>(Y, idx, w, pair_pos, T, K, d,
-                                                             static_cast<float *>(out));
-    return cudaGetLastError();
+        return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), 0, stream,
+                          Y, idx, w, pair_pos, T, K, d, static_cast<__nv_bfloat16 *>(out));
+    return launch_pdl(combine_kernel<float>, dim3(blocks), dim3(threads), 0, stream, Y, idx, w,
+                      pair_pos, T, K, d, static_cast<float *>(out));
 }
 
 cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,

@@ -135,7 +135,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_units = (MODE == MODE_ROUTER) ? p.n_units : p.meta[0] * p.n_mb;
     const volatile int *abort_flag = &abort_sh;
 
     if (threadIdx.x == 0) {
@@ -156,17 +155,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmA1);
         tma_prefetch_desc(&tmB);
     }
+    if (warp == 1) tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    // Everything above is private to the CTA; global memory only from here.
+    griddep_wait();
+    griddep_launch_dependents();
     if (MODE == MODE_ROUTER && blockIdx.x == 0) {
         // Per-call counters of the later kernels start at zero.
         for (int r = 0; r < 3; ++r)
             if (p.zero[r].ptr)
                 for (int i = threadIdx.x; i < p.zero[r].count; i += blockDim.x) p.zero[r].ptr[i] = 0;
     }
-    if (warp == 1) tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = tmem_base_sh;
+    const int n_units = (MODE == MODE_ROUTER) ? p.n_units : p.meta[0] * p.n_mb;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -349,8 +353,7 @@ cudaError_t launch_cfg(const CUtensorMap &a0, const CUtensorMap &a1, const CUten
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM_BYTES));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b, args);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM_BYTES, stream, a0, a1, b, args);
 }
 
 template <int MODE, int NUM_A>
