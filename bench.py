@@ -383,6 +383,10 @@ def run_beam(args):
 
     S = layer.abi.FORWARD_STAGES
     names = [layer.abi.stage_name(j) for j in range(S)]
+    n_kernels = layer.abi.kernel_count(layer.dsc)
+    fused = n_kernels == S - 1  # decode tiles: both expert GEMMs in one launch (stage 4)
+    if fused:
+        names[4] = "experts_fused_gate_up_down"
     stage_mean = [sum(s[j] for s in stage_s) / len(stage_s) for j in range(S)]
     step_mean = total / len(step_s)
     prof_mean = sum(prof_s) / len(prof_s)
@@ -391,6 +395,12 @@ def run_beam(args):
     # dominant kernel vs its roofline (algorithmic bytes/flops averaged over batches)
     dom = max(range(S), key=lambda j: stage_mean[j])
     alg = [algorithmic(layer, st[i % N_BATCHES], True) for i in range(args.steps)]
+    if fused:
+        for a in alg:
+            g1, g2 = a.pop("gemm1_gate_up_swiglu"), a.pop("gemm2_down")
+            a[names[4]] = dict(bytes=g1["bytes"] + g2["bytes"], flops=g1["flops"] + g2["flops"],
+                               unit="tensor")
+            a["gemm2_down"] = dict(bytes=0, flops=0, unit="hbm")
     a_bytes = sum(a[names[dom]]["bytes"] for a in alg) / len(alg)
     a_flops = sum(a[names[dom]]["flops"] for a in alg) / len(alg)
     # the dominant kernel alone between two events (least perturbed timing)
@@ -470,7 +480,7 @@ def run_beam(args):
                          "without them)"),
         "per_kept_fraction": sweep,
         "e2e": e2e,
-        "gpu_launches": S * args.steps,
+        "gpu_launches": n_kernels * args.steps,
         "clocks": clocks,
     }
     if cpu is not None:

@@ -41,7 +41,7 @@ class PlanInfo(ctypes.Structure):
                [(n, ctypes.c_size_t) for n in (
                    "off_err", "off_meta", "off_counts", "off_hist", "off_partial", "off_idx",
                    "off_w", "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h", "off_y",
-                   "workspace_bytes")]
+                   "off_tile_done", "workspace_bytes")]
 
 
 _lib = None
@@ -68,6 +68,8 @@ def lib():
         L.beam_moe_check.argtypes = [pd, vp, vp]
         L.beam_moe_route_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.beam_moe_route_noalloc.restype = i32
+        L.beam_moe_forward_kernel_count.argtypes = [pd]
+        L.beam_moe_forward_kernel_count.restype = i32
         L.beam_status_str.argtypes = [i32]
         L.beam_status_str.restype = ctypes.c_char_p
         L.beam_moe_stage_name.argtypes = [i32]
@@ -117,6 +119,11 @@ def stage_name(i: int):
 
 def workspace_size(dsc: Desc) -> int:
     return int(lib().beam_moe_workspace_size(ctypes.byref(dsc)))
+
+
+def kernel_count(dsc: Desc) -> int:
+    """Kernel launches of one forward call for this descriptor."""
+    return int(lib().beam_moe_forward_kernel_count(ctypes.byref(dsc)))
 
 
 def plan(dsc: Desc) -> dict:

@@ -96,10 +96,14 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
     P->off_xp = align256(P->off_tiles + 16 * size_t(tiles_cap));
     P->off_h = align256(P->off_xp + es * size_t(p_cap) * size_t(d->d));
     P->off_y = align256(P->off_h + es * size_t(p_cap) * size_t(d->I));
-    o = align256(P->off_y + 4 * size_t(p_cap) * size_t(d->d));  // Y is fp32
+    P->off_tile_done = align256(P->off_y + 4 * size_t(p_cap) * size_t(d->d));  // Y is fp32
+    o = align256(P->off_tile_done + 4 * size_t(tiles_cap));
     P->workspace_bytes = o;
     return BEAM_OK;
 }
+
+// Decode-sized token tiles run both expert GEMMs as one fused launch.
+bool fused_experts(const beam_moe_plan_info &P) { return P.BN < 128; }
 
 int sm_count() {
     static int cache[kMaxDevices] = {0};
@@ -181,10 +185,12 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
     ZeroRegion zero[3] = {{hdr, 8}, {ro.counts, d->E}, {ro.hist, ro.hist ? d->K + 1 : 0}};
     BEAM_TRY_CUDA(rec.rec(0));
     if (d->dtype == BEAM_BF16) {
-        CUtensorMap mWg, mWm, mX;
-        if (!make_tmap(&mWg, Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mWm, Wm ? Wm : Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mX, x, d->d, d->T, P.router_bn)) return BEAM_ERR_CUDA;
+        TcMaps maps;
+        if (!make_tmap(&maps.a0, Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.a1, Wm ? Wm : Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b, x, d->d, d->T, P.router_bn)) return BEAM_ERR_CUDA;
+        maps.a2 = maps.a0;
+        maps.b2 = maps.b;
         TcGemmArgs a;
         std::memset(&a, 0, sizeof(a));
         const int mb_per = int(cdiv(d->E, kBlockM));
@@ -204,7 +210,7 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
         a.zero[2] = zero[2];
         a.timeout_ns = kWaitTimeoutNs;
         const int grid = a.n_units < n_sm ? a.n_units : n_sm;
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_ROUTER, P.router_bn, mWg, mWm, mX, a, grid, st));
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_ROUTER, P.router_bn, maps, a, grid, st));
     } else {
         BEAM_TRY_CUDA(launch_router_f32(static_cast<const float *>(x), static_cast<const float *>(Wg),
                                         static_cast<const float *>(Wm), d->T, d->d, d->E, partial,
@@ -265,6 +271,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     int *pair = reinterpret_cast<int *>(ws + P.off_pair);
     int *pair_pos = reinterpret_cast<int *>(ws + P.off_pair_pos);
     int4 *tiles = reinterpret_cast<int4 *>(ws + P.off_tiles);
+    int *tile_done = reinterpret_cast<int *>(ws + P.off_tile_done);
     void *xp = ws + P.off_xp;
     void *h = ws + P.off_h;
     float *y = reinterpret_cast<float *>(ws + P.off_y);
@@ -274,7 +281,8 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     if (s != BEAM_OK) return s;
 
     BEAM_TRY_CUDA(rec.rec(2));
-    PermuteArgs pa{idx, counts, d->T, d->K, d->E, P.BN, pair, pair_pos, tiles, meta, err};
+    PermuteArgs pa{idx, counts, d->T, d->K, d->E, P.BN, pair, pair_pos, tiles, tile_done, meta,
+                   err};
     BEAM_TRY_CUDA(launch_permute(pa, st));
 
     BEAM_TRY_CUDA(rec.rec(3));
@@ -282,16 +290,17 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     BEAM_TRY_CUDA(launch_gather(x, pair, meta, d->K, (long long)es * d->d, P.p_cap, xp, n_sm, st));
 
     if (d->dtype == BEAM_BF16) {
-        // Thin token tiles: gate and up rows interleaved in one 128-row tile
-        // (twice the work units); 128-token tiles: two 128-row weight tiles.
-        const bool interleave = P.BN < 128;
-        const unsigned wbox = interleave ? kBlockM / 2 : kBlockM;
-        CUtensorMap mW1, mW3, mW2, mXp, mH;
-        if (!make_tmap(&mW1, W1, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mW3, W3, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mW2, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mXp, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&mH, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        // Thin token tiles (decode): gate and up rows interleaved in one
+        // 128-row tile, and both expert GEMMs in one fused launch.  128-token
+        // tiles (prefill): two 128-row weight tiles per unit, two launches.
+        const bool fused = fused_experts(P);
+        const unsigned wbox = fused ? kBlockM / 2 : kBlockM;
+        TcMaps maps;
+        if (!make_tmap(&maps.a0, W1, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.a1, W3, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.a2, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b2, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
 
         TcGemmArgs g;
         std::memset(&g, 0, sizeof(g));
@@ -299,26 +308,42 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         g.tiles = tiles;
         g.err = err;
         g.timeout_ns = kWaitTimeoutNs;
-
-        BEAM_TRY_CUDA(rec.rec(4));
         g.n_mb = d->I / int(wbox);
         g.nk = d->d / kBlockK;
         g.a_rows_per_expert = d->I;
         g.out = h;
         g.out_ld = d->I;
-        long long units = (long long)P.tiles_cap * g.n_mb;
-        BEAM_TRY_CUDA(launch_tc_gemm(interleave ? MODE_GEMM1_IL : MODE_GEMM1, P.BN, mW1, mW3, mXp,
-                                     g, int(units < n_sm ? units : n_sm), st));
 
-        BEAM_TRY_CUDA(rec.rec(5));
-        g.n_mb = d->d / kBlockM;
-        g.nk = d->I / kBlockK;
-        g.a_rows_per_expert = d->d;
-        g.out = y;
-        g.out_ld = d->d;
-        units = (long long)P.tiles_cap * g.n_mb;
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, P.BN, mW2, mW2, mH, g,
-                                     int(units < n_sm ? units : n_sm), st));
+        BEAM_TRY_CUDA(rec.rec(4));
+        if (fused) {
+            g.n_mb2 = d->d / kBlockM;
+            g.nk2 = d->I / kBlockK;
+            g.a_rows2 = d->d;
+            g.out2 = y;
+            g.out2_ld = d->d;
+            g.tile_done = tile_done;
+            const long long units = (long long)P.tiles_cap * (g.n_mb + g.n_mb2);
+            BEAM_TRY_CUDA(launch_tc_gemm(MODE_EXPERTS, P.BN, maps, g,
+                                         int(units < n_sm ? units : n_sm), st));
+            BEAM_TRY_CUDA(rec.rec(5));  // the down GEMM ran inside the fused launch
+        } else {
+            long long units = (long long)P.tiles_cap * g.n_mb;
+            BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, maps, g,
+                                         int(units < n_sm ? units : n_sm), st));
+            BEAM_TRY_CUDA(rec.rec(5));
+            TcMaps m2 = maps;
+            m2.a0 = maps.a2;
+            m2.a1 = maps.a2;
+            m2.b = maps.b2;
+            g.n_mb = d->d / kBlockM;
+            g.nk = d->I / kBlockK;
+            g.a_rows_per_expert = d->d;
+            g.out = y;
+            g.out_ld = d->d;
+            units = (long long)P.tiles_cap * g.n_mb;
+            BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, P.BN, m2, g,
+                                         int(units < n_sm ? units : n_sm), st));
+        }
     } else {
         BEAM_TRY_CUDA(rec.rec(4));
         BEAM_TRY_CUDA(launch_gemm1_f32(static_cast<const float *>(xp), static_cast<const float *>(W1),
@@ -472,6 +497,14 @@ const char *beam_status_str(beam_status status) {
         case BEAM_ERR_INTERNAL: return "BEAM_ERR_INTERNAL";
     }
     return "BEAM_ERR_UNKNOWN";
+}
+
+int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
+    beam_moe_plan_info P;
+    if (make_plan(desc, &P) != BEAM_OK) return 0;
+    if (desc->T == 0) return 0;
+    return (desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 1
+                                                          : BEAM_MOE_FORWARD_STAGES;
 }
 
 const char *beam_moe_stage_name(int stage) {

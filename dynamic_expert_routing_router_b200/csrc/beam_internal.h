@@ -18,7 +18,14 @@ enum TcMode : int {
     MODE_ROUTER = 0,  // logits: [W_gate | W_mask] rows x token rows, split over d
     MODE_GEMM1 = 1,   // SiLU(W1 x) * (W3 x) per kept pair  -> H
     MODE_GEMM2 = 2,   // W2 h per kept pair                  -> Y
-    MODE_GEMM1_IL = 3 // GEMM1 with 64 rows of W1 and 64 of W3 interleaved in one tile
+    MODE_GEMM1_IL = 3, // GEMM1 with 64 rows of W1 and 64 of W3 interleaved in one tile
+    MODE_EXPERTS = 4   // MODE_GEMM1_IL units then MODE_GEMM2 units in one launch
+};
+
+// Tensor maps of one tensor-core launch.  a0/a1/b: the (first) GEMM's weight
+// tile(s) and token tile; a2/b2: the down projection's in MODE_EXPERTS.
+struct TcMaps {
+    CUtensorMap a0, a1, b, a2, b2;
 };
 
 constexpr int kBlockM = 128;   // weight rows per tile (the MMA's M)
@@ -69,10 +76,14 @@ struct TcGemmArgs {
     int *err;            // device error word
     ZeroRegion zero[3];  // router: regions CTA 0 clears for the later kernels
     unsigned long long timeout_ns;
+    // MODE_EXPERTS: the down projection that follows the gate/up units
+    int n_mb2, nk2, a_rows2;  // d/128 row blocks, I/64 k-blocks, d rows per expert
+    void *out2;               // Y (f32)
+    long long out2_ld;
+    int *tile_done;           // per tile: gate/up units whose H rows are published
 };
 
-cudaError_t launch_tc_gemm(int mode, int bn, const CUtensorMap &a0, const CUtensorMap &a1,
-                           const CUtensorMap &b, const TcGemmArgs &args, int grid,
+cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,
                            cudaStream_t stream);
 
 // Top-K + softmax + mask + aggregation (one warp per token).
@@ -94,6 +105,7 @@ struct PermuteArgs {
     int T, K, E, BN;
     int *pair, *pair_pos;
     int4 *tiles;
+    int *tile_done;  // cleared for every tile written (MODE_EXPERTS counters)
     int *meta;
     int *err;
 };

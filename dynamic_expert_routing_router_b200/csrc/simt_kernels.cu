@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     for (int j = tid; j < ntile_e; j += kPermThreads) {
         const int rows = min(a.BN, count_e - j * a.BN);
         a.tiles[toff_e + j] = make_int4(e, off_e + j * a.BN, rows, 0);
+        a.tile_done[toff_e + j] = 0;
     }
 }
 

@@ -1,15 +1,19 @@
 // tc_gemm.cu -- grouped GEMMs of the BEAM MoE layer on the sm_100a tensor
 // cores (tcgen05.mma, fp32 accumulators in TMEM, operands staged by TMA).
 //
-// One persistent, warp-specialised kernel serves three roles:
-//   MODE_ROUTER  logits  r = x W_gate, z = x W_mask   (BEAM §3.2 steps 1-2)
-//   MODE_GEMM1   H = SiLU(x W1_e^T) * (x W3_e^T)      (Eq. 3, gate/up + SwiGLU)
-//                two 128-row weight tiles (W1, W3), two accumulators
+// One persistent, warp-specialised kernel serves every role:
+//   MODE_ROUTER   logits  r = x W_gate, z = x W_mask   (BEAM §3.2 steps 1-2)
+//   MODE_GEMM1    H = SiLU(x W1_e^T) * (x W3_e^T)      (Eq. 3, gate/up + SwiGLU)
+//                 two 128-row weight tiles (W1, W3), two accumulators
 //   MODE_GEMM1_IL the same with 64 rows of W1 and the matching 64 rows of W3
-//                in one 128-row tile and one accumulator: twice the work units
-//                for thin token tiles; the epilogue warps pair gate and up
-//                rows through shared memory
-//   MODE_GEMM2   Y = H W2_e^T  (fp32 out)              (Eq. 3, down projection)
+//                 in one 128-row tile and one accumulator (twice the units);
+//                 the epilogue warps pair gate and up rows through shared memory
+//   MODE_GEMM2    Y = H W2_e^T  (fp32 out)              (Eq. 3, down projection)
+//   MODE_EXPERTS  MODE_GEMM1_IL units followed by MODE_GEMM2 units in one
+//                 launch: a down-projection unit of a token tile starts once
+//                 every gate/up unit of that tile has published its rows of H
+//                 (per-tile counter), so the second GEMM fills the first one's
+//                 tail instead of waiting for a kernel boundary.
 //
 // Orientation: the weight rows are the MMA's M operand (128 rows per tile)
 // and the tokens are its N operand (BN = 16..128 per tile), D = W * X^T.  A
@@ -27,6 +31,10 @@
 // overlaps the MMAs of the next.  Every wait is bounded (beam_ptx.cuh); on
 // expiry the CTA records DEV_ERR_TIMEOUT, drains its own copies and MMAs,
 // frees TMEM and returns.
+//
+// MODE_EXPERTS cannot deadlock: a CTA issues all of its gate/up units before
+// any of its down units, gate/up units wait on nothing outside their CTA, and
+// the grid never exceeds the CTAs that fit on the GPU at once (one per SM).
 #include <cuda_bf16.h>
 
 #include "beam_internal.h"
@@ -38,7 +46,6 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kUmmaK = 16;  // K of one kind::f16 MMA
-
 constexpr int kXchLd = 17;  // padded row of the gate/up exchange buffer (floats)
 
 template <int NUM_A, int BN, bool XCH>
@@ -61,11 +68,20 @@ struct TcCfg {
     static_assert(SMEM_BYTES <= 227u * 1024u, "shared memory");
 };
 
+template <int MODE>
+struct ModeTraits {
+    static constexpr int NUM_A = MODE == MODE_GEMM1 ? 2 : 1;
+    static constexpr bool XCH = MODE == MODE_GEMM1_IL || MODE == MODE_EXPERTS;
+};
+
 struct Unit {
+    int phase;  // MODE_EXPERTS: 0 = gate/up unit, 1 = down unit; else 0
+    int ti;     // tile index (GEMMs)
     int mb;     // weight-row block
     int a_row;  // first row of the A (weight) tile in its 2D tensor map
     int b_row;  // first row of the B (token) tile
     int kb0;    // first k-block
+    int nk;     // k-blocks of this unit
     int sel;    // router: 0 = W_gate rows, 1 = W_mask rows
     int tt, s;  // router: token tile, split
     int rows;   // GEMMs: valid token rows of the tile
@@ -77,11 +93,17 @@ __device__ __forceinline__ void epilogue_sync() {
 }
 
 template <int MODE, int BN>
-__device__ __forceinline__ Unit decode_unit(int u, const TcGemmArgs &p) {
+__device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs &p) {
     Unit w;
-    w.mb = u % p.n_mb;
-    const int rest = u / p.n_mb;
+    w.phase = 0;
+    w.sel = 0;
+    w.tt = w.s = 0;
+    w.kb0 = 0;
+    w.nk = p.nk;
     if (MODE == MODE_ROUTER) {
+        w.mb = u % p.n_mb;
+        const int rest = u / p.n_mb;
+        w.ti = 0;
         w.tt = rest % p.n_tt;
         w.s = rest / p.n_tt;
         w.sel = w.mb >= p.n_mb_gate ? 1 : 0;
@@ -89,16 +111,27 @@ __device__ __forceinline__ Unit decode_unit(int u, const TcGemmArgs &p) {
         w.b_row = w.tt * BN;
         w.kb0 = w.s * p.nk;
         w.rows = 0;
-    } else {
-        const int4 t = p.tiles[rest];
-        const int rows_per_mb = (MODE == MODE_GEMM1_IL) ? kBlockM / 2 : kBlockM;
-        w.a_row = t.x * p.a_rows_per_expert + w.mb * rows_per_mb;
-        w.b_row = t.y;
-        w.rows = t.z;
-        w.kb0 = 0;
-        w.sel = 0;
-        w.tt = w.s = 0;
+        return w;
     }
+    int v = u, n_mb = p.n_mb, rows_per_mb = kBlockM, a_rows = p.a_rows_per_expert;
+    if (MODE == MODE_GEMM1_IL) rows_per_mb = kBlockM / 2;
+    if (MODE == MODE_EXPERTS) {
+        if (u < n_first) {
+            rows_per_mb = kBlockM / 2;
+        } else {
+            w.phase = 1;
+            v = u - n_first;
+            n_mb = p.n_mb2;
+            a_rows = p.a_rows2;
+            w.nk = p.nk2;
+        }
+    }
+    w.mb = v % n_mb;
+    w.ti = v / n_mb;
+    const int4 t = p.tiles[w.ti];
+    w.a_row = t.x * a_rows + w.mb * rows_per_mb;
+    w.b_row = t.y;
+    w.rows = t.z;
     return w;
 }
 
@@ -111,12 +144,31 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return g / (1.0f + __expf(-g)) * u;
 }
 
-template <int MODE, int NUM_A, int BN>
+// Bounded wait until *ctr >= need (acquire at GPU scope).
+__device__ __forceinline__ bool wait_counter_bounded(const int *ctr, int need,
+                                                     const volatile int *abort_flag,
+                                                     uint64_t timeout_ns) {
+    uint64_t t0 = 0;
+    for (uint32_t spin = 0; spin < (1u << 24); ++spin) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= need) return true;
+        if ((spin & 31u) == 0) {
+            if (*abort_flag) return false;
+            const uint64_t t = globaltimer_ns();
+            if (spin == 0) t0 = t;
+            else if (t - t0 > timeout_ns) return false;
+        }
+        __nanosleep(100);
+    }
+    return false;
+}
+
+template <int MODE, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
-                   const __grid_constant__ CUtensorMap tmA1,
-                   const __grid_constant__ CUtensorMap tmB, const TcGemmArgs p) {
-    using C = TcCfg<NUM_A, BN, MODE == MODE_GEMM1_IL>;
+    tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcGemmArgs p) {
+    constexpr int NUM_A = ModeTraits<MODE>::NUM_A;
+    using C = TcCfg<NUM_A, BN, ModeTraits<MODE>::XCH>;
     constexpr int STAGES = C::STAGES;
 
     extern __shared__ uint8_t smem_raw[];
@@ -151,9 +203,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA0);
-        tma_prefetch_desc(&tmA1);
-        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&maps.a0);
+        tma_prefetch_desc(&maps.a1);
+        tma_prefetch_desc(&maps.b);
+        if (MODE == MODE_EXPERTS) {
+            tma_prefetch_desc(&maps.a2);
+            tma_prefetch_desc(&maps.b2);
+        }
     }
     if (warp == 1) tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
     tc_fence_before_sync();
@@ -170,7 +226,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.zero[r].ptr)
                 for (int i = threadIdx.x; i < p.zero[r].count; i += blockDim.x) p.zero[r].ptr[i] = 0;
     }
-    const int n_units = (MODE == MODE_ROUTER) ? p.n_units : p.meta[0] * p.n_mb;
+    const int ntiles = (MODE == MODE_ROUTER) ? 0 : p.meta[0];
+    const int n_first = ntiles * p.n_mb;  // units of the first GEMM
+    const int n_units = (MODE == MODE_ROUTER)    ? p.n_units
+                        : (MODE == MODE_EXPERTS) ? n_first + ntiles * p.n_mb2
+                                                 : n_first;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -178,9 +238,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-                const Unit w = decode_unit<MODE, BN>(u, p);
-                const CUtensorMap *am = (MODE == MODE_ROUTER && w.sel) ? &tmA1 : &tmA0;
-                for (int kb = 0; kb < p.nk; ++kb, ++it) {
+                const Unit w = decode_unit<MODE, BN>(u, n_first, p);
+                const CUtensorMap *am = &maps.a0;
+                const CUtensorMap *bm = &maps.b;
+                if (MODE == MODE_ROUTER && w.sel) am = &maps.a1;
+                if (MODE == MODE_EXPERTS && w.phase == 1) {
+                    // H rows of this tile come from other CTAs' gate/up units.
+                    if (!wait_counter_bounded(p.tile_done + w.ti, p.n_mb, abort_flag,
+                                              p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    am = &maps.a2;
+                    bm = &maps.b2;
+                }
+                const bool interleaved =
+                    MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
+                for (int kb = 0; kb < w.nk; ++kb, ++it) {
                     const int s = int(it % STAGES);
                     const uint32_t ph = ((it / STAGES) & 1u) ^ 1u;
                     if (!mbar_wait_bounded(&empty_bar[s], ph, abort_flag, p.timeout_ns)) {
@@ -190,15 +265,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
                     const int kx = (w.kb0 + kb) * kBlockK;
-                    if (MODE == MODE_GEMM1_IL) {
+                    if (interleaved) {
                         // rows 0..63: W1 (gate), rows 64..127: W3 (up), same I rows
-                        tma_load_2d(st, &tmA0, kx, w.a_row, &full_bar[s]);
-                        tma_load_2d(st + C::A_BYTES / 2, &tmA1, kx, w.a_row, &full_bar[s]);
+                        tma_load_2d(st, &maps.a0, kx, w.a_row, &full_bar[s]);
+                        tma_load_2d(st + C::A_BYTES / 2, &maps.a1, kx, w.a_row, &full_bar[s]);
                     } else {
                         tma_load_2d(st, am, kx, w.a_row, &full_bar[s]);
                     }
-                    if (NUM_A == 2) tma_load_2d(st + C::A_BYTES, &tmA1, kx, w.a_row, &full_bar[s]);
-                    tma_load_2d(st + NUM_A * C::A_BYTES, &tmB, kx, w.b_row, &full_bar[s]);
+                    if (NUM_A == 2)
+                        tma_load_2d(st + C::A_BYTES, &maps.a1, kx, w.a_row, &full_bar[s]);
+                    tma_load_2d(st + NUM_A * C::A_BYTES, bm, kx, w.b_row, &full_bar[s]);
                 }
             }
             if (!ok) {
@@ -216,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0, lu = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++lu) {
+                const int nk = (MODE == MODE_EXPERTS && u >= n_first) ? p.nk2 : p.nk;
                 const uint32_t a = lu & 1u;
                 if (!mbar_wait_bounded(&tempty_bar[a], ((lu >> 1) & 1u) ^ 1u, abort_flag,
                                        p.timeout_ns)) {
@@ -224,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d0 = tmem_base + a * C::ACC_COLS;
-                for (int kb = 0; kb < p.nk; ++kb, ++it) {
+                for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = int(it % STAGES);
                     if (!mbar_wait_bounded(&full_bar[s], (it / STAGES) & 1u, abort_flag,
                                            p.timeout_ns)) {
@@ -260,11 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = q * 32 + lane;   // row within the 128-row weight tile
         uint32_t lu = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++lu) {
-            const Unit w = decode_unit<MODE, BN>(u, p);
+            const Unit w = decode_unit<MODE, BN>(u, n_first, p);
             const uint32_t a = lu & 1u;
             bool ok = mbar_wait_bounded(&tfull_bar[a], (lu >> 1) & 1u, abort_flag, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
-            if (MODE == MODE_GEMM1_IL) {
+            if (ModeTraits<MODE>::XCH) {
                 // The four warps meet at named barriers below: agree first.
                 if (lane == 0) xvote[warp - 2] = ok ? 1 : 0;
                 epilogue_sync();
@@ -276,6 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + a * C::ACC_COLS;
+            const bool gate_up_il =
+                MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
+            const bool down = MODE == MODE_GEMM2 || (MODE == MODE_EXPERTS && w.phase == 1);
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 16) {
                 uint32_t g[16], v[16];
@@ -295,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (t < p.T) out[(long long)t * p.out_ld] = __uint_as_float(g[c]);
                         }
                     }
-                } else if (MODE == MODE_GEMM1_IL) {
+                } else if (gate_up_il) {
                     // TMEM rows 0..63 hold gate, 64..127 up, for I rows mb*64 + r.
                     float *xch = reinterpret_cast<float *>(smem + size_t(STAGES) * C::STAGE_BYTES);
 #pragma unroll
@@ -322,17 +402,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (c0 + c < w.rows)
                             out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(
                                 silu_mul(__uint_as_float(g[c]), __uint_as_float(v[c])));
-                } else {
+                } else if (down) {
                     // Y (fp32): rounded once, after the weighted combine.
-                    float *out = static_cast<float *>(p.out) + (long long)w.b_row * p.out_ld +
+                    void *base = (MODE == MODE_EXPERTS) ? p.out2 : p.out;
+                    const long long ld = (MODE == MODE_EXPERTS) ? p.out2_ld : p.out_ld;
+                    float *out = static_cast<float *>(base) + (long long)w.b_row * ld +
                                  w.mb * kBlockM + row;
 #pragma unroll
                     for (int c = 0; c < 16; ++c)
-                        if (c0 + c < w.rows) out[(long long)(c0 + c) * p.out_ld] = __uint_as_float(g[c]);
+                        if (c0 + c < w.rows) out[(long long)(c0 + c) * ld] = __uint_as_float(g[c]);
                 }
             }
             tc_fence_before_sync();
             mbar_arrive(&tempty_bar[a]);
+            if (MODE == MODE_EXPERTS && w.phase == 0) {
+                // Publish this unit's rows of H to the down units of the tile.
+                __threadfence();
+                epilogue_sync();
+                if (threadIdx.x == 64)
+                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.tile_done + w.ti)
+                                 : "memory");
+            }
         }
     }
 
@@ -345,40 +435,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int MODE, int NUM_A, int BN>
-cudaError_t launch_cfg(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
-                       const TcGemmArgs &args, int grid, cudaStream_t stream) {
-    using C = TcCfg<NUM_A, BN, MODE == MODE_GEMM1_IL>;
-    auto kern = tc_gemm_kernel<MODE, NUM_A, BN>;
+template <int MODE, int BN>
+cudaError_t launch_cfg(const TcMaps &maps, const TcGemmArgs &args, int grid,
+                       cudaStream_t stream) {
+    using C = TcCfg<ModeTraits<MODE>::NUM_A, BN, ModeTraits<MODE>::XCH>;
+    auto kern = tc_gemm_kernel<MODE, BN>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM_BYTES));
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM_BYTES, stream, a0, a1, b, args);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM_BYTES, stream, maps, args);
 }
 
-template <int MODE, int NUM_A>
-cudaError_t launch_bn(int bn, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
-                      const TcGemmArgs &args, int grid, cudaStream_t stream) {
+template <int MODE>
+cudaError_t launch_bn(int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,
+                      cudaStream_t stream) {
     switch (bn) {
-        case 16: return launch_cfg<MODE, NUM_A, 16>(a0, a1, b, args, grid, stream);
-        case 32: return launch_cfg<MODE, NUM_A, 32>(a0, a1, b, args, grid, stream);
-        case 64: return launch_cfg<MODE, NUM_A, 64>(a0, a1, b, args, grid, stream);
-        case 128: return launch_cfg<MODE, NUM_A, 128>(a0, a1, b, args, grid, stream);
+        case 16: return launch_cfg<MODE, 16>(maps, args, grid, stream);
+        case 32: return launch_cfg<MODE, 32>(maps, args, grid, stream);
+        case 64: return launch_cfg<MODE, 64>(maps, args, grid, stream);
+        case 128: return launch_cfg<MODE, 128>(maps, args, grid, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_tc_gemm(int mode, int bn, const CUtensorMap &a0, const CUtensorMap &a1,
-                           const CUtensorMap &b, const TcGemmArgs &args, int grid,
+cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,
                            cudaStream_t stream) {
     if (grid <= 0) return cudaSuccess;
     switch (mode) {
-        case MODE_ROUTER: return launch_bn<MODE_ROUTER, 1>(bn, a0, a1, b, args, grid, stream);
-        case MODE_GEMM1: return launch_bn<MODE_GEMM1, 2>(bn, a0, a1, b, args, grid, stream);
-        case MODE_GEMM1_IL: return launch_bn<MODE_GEMM1_IL, 1>(bn, a0, a1, b, args, grid, stream);
-        case MODE_GEMM2: return launch_bn<MODE_GEMM2, 1>(bn, a0, a1, b, args, grid, stream);
+        case MODE_ROUTER: return launch_bn<MODE_ROUTER>(bn, maps, args, grid, stream);
+        case MODE_GEMM1: return launch_bn<MODE_GEMM1>(bn, maps, args, grid, stream);
+        case MODE_GEMM2: return launch_bn<MODE_GEMM2>(bn, maps, args, grid, stream);
+        case MODE_GEMM1_IL: return launch_bn<MODE_GEMM1_IL>(bn, maps, args, grid, stream);
+        case MODE_EXPERTS: return launch_bn<MODE_EXPERTS>(bn, maps, args, grid, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -88,6 +88,7 @@ typedef struct {
  *             experts in ascending order, tokens ascending inside
  *   pair_pos  int32[T][K] permuted row of a kept pair (undefined if masked)
  *   tiles     int32[tiles_cap][4] (expert, first row, valid rows, 0)
+ *   tile_done int32[tiles_cap] gate/up units finished per tile (fused path)
  *   xp        [p_cap][d]  gathered token rows (dtype)
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
  *   y         f32[p_cap][d] expert output per pair                           */
@@ -99,11 +100,15 @@ typedef struct {
     int tiles_cap;     /* entries of the tile list */
     int reserved;
     size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
-        off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y;
+        off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done;
     size_t workspace_bytes;
 } beam_moe_plan_info;
 
-/* Number of kernel launches of one beam_moe_forward call (the stages below). */
+/* Stage slots of one beam_moe_forward call (router GEMM, top-K + mask,
+ * grouping, gather, gate/up GEMM, down GEMM, combine).  With token tiles
+ * thinner than 128 rows (decode batches) the two expert GEMMs run as one
+ * fused launch in the gate/up slot and the down slot is empty; see
+ * beam_moe_forward_kernel_count. */
 #define BEAM_MOE_FORWARD_STAGES 7
 
 /* Bytes of device workspace beam_moe_forward needs for `desc` (0 on a bad
@@ -184,6 +189,10 @@ beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
                                    const void *W_gate, const void *W_mask, int32_t *topk_idx,
                                    float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
                                    float *logits, void *stream);
+
+/* Kernel launches one beam_moe_forward call makes for `desc` (6 or 7), or 0
+ * on a bad descriptor. */
+int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last
  * call: BEAM_OK, BEAM_ERR_TIMEOUT (a bounded device wait expired, the kernel
