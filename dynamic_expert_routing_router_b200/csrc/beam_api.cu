@@ -322,6 +322,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
             g.out2 = y;
             g.out2_ld = d->d;
             g.tile_done = tile_done;
+            g.work_ctr = meta + 3;
             const long long units = (long long)P.tiles_cap * (g.n_mb + g.n_mb2);
             BEAM_TRY_CUDA(launch_tc_gemm(MODE_EXPERTS, P.BN, maps, g,
                                          int(units < n_sm ? units : n_sm), st));

@@ -81,6 +81,7 @@ struct TcGemmArgs {
     void *out2;               // Y (f32)
     long long out2_ld;
     int *tile_done;           // per tile: gate/up units whose H rows are published
+    int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
 };
 
 cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,

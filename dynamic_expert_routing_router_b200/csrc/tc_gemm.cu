@@ -32,9 +32,14 @@
 // expiry the CTA records DEV_ERR_TIMEOUT, drains its own copies and MMAs,
 // frees TMEM and returns.
 //
-// MODE_EXPERTS cannot deadlock: a CTA issues all of its gate/up units before
-// any of its down units, gate/up units wait on nothing outside their CTA, and
-// the grid never exceeds the CTAs that fit on the GPU at once (one per SM).
+// MODE_EXPERTS hands units out dynamically: the producer takes the next index
+// from a global counter (all gate/up units first, then the smaller down
+// units, so the tail is made of small units) and passes it to the MMA and
+// epilogue warps through a 4-slot ring in shared memory.  It cannot deadlock:
+// indices are handed out in increasing order, so every gate/up unit a down
+// unit waits for was already taken by a running CTA whose producer issued
+// all of that unit's loads before taking another index, and gate/up units
+// wait on nothing outside their CTA.  The other modes deal units round-robin.
 #include <cuda_bf16.h>
 
 #include "beam_internal.h"
@@ -172,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int STAGES = C::STAGES;
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ int xvote[4];
+    __shared__ int xvote[4];   // epilogue warps: "accumulator arrived" votes
+    __shared__ int uvote[4];   // epilogue warps: "unit received / hand-out over" votes
     __shared__ __align__(8) uint64_t full_bar[STAGES];
     __shared__ __align__(8) uint64_t empty_bar[STAGES];
     __shared__ __align__(8) uint64_t tfull_bar[2];
@@ -180,6 +186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    constexpr bool DYN = MODE == MODE_EXPERTS;  // dynamic unit hand-out
+    constexpr int kRing = 4;
+    __shared__ int unit_ring[kRing];
+    __shared__ __align__(8) uint64_t unit_full[kRing];
+    __shared__ __align__(8) uint64_t unit_empty[kRing];
 
     // 1024-byte aligned start of the stage ring (SWIZZLE_128B atoms).
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -199,6 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tempty_bar[a], 128);
         }
         mbar_init(&drain_bar, 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&unit_full[i], 1);
+            mbar_init(&unit_empty[i], 1 + 4);  // MMA thread + one lane per epilogue warp
+        }
         abort_sh = 0;
         fence_barrier_init();
     }
@@ -237,7 +252,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+            for (uint32_t lu = 0;; ++lu) {
+                int u = blockIdx.x + int(lu) * gridDim.x;
+                if (DYN) {
+                    const int slot = int(lu % kRing);
+                    if (!mbar_wait_bounded(&unit_empty[slot], ((lu / kRing) & 1u) ^ 1u, abort_flag,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    u = atomicAdd(p.work_ctr, 1);
+                    if (u >= n_units) u = -1;
+                    unit_ring[slot] = u;
+                    mbar_arrive(&unit_full[slot]);
+                    if (u < 0) break;
+                } else if (u >= n_units) {
+                    break;
+                }
                 const Unit w = decode_unit<MODE, BN>(u, n_first, p);
                 const CUtensorMap *am = &maps.a0;
                 const CUtensorMap *bm = &maps.b;
@@ -276,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(st + C::A_BYTES, &maps.a1, kx, w.a_row, &full_bar[s]);
                     tma_load_2d(st + NUM_A * C::A_BYTES, bm, kx, w.b_row, &full_bar[s]);
                 }
+                if (!ok) break;
             }
             if (!ok) {
                 signal_abort(p.err, &abort_sh);
@@ -289,9 +321,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------- MMA issuer --
         if (lane == 0) {
             constexpr uint32_t IDESC = umma_idesc_bf16_f32(kBlockM, BN);
-            uint32_t it = 0, lu = 0;
+            uint32_t it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++lu) {
+            for (uint32_t lu = 0;; ++lu) {
+                int u = blockIdx.x + int(lu) * gridDim.x;
+                if (DYN) {
+                    const int slot = int(lu % kRing);
+                    if (!mbar_wait_bounded(&unit_full[slot], (lu / kRing) & 1u, abort_flag,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    u = unit_ring[slot];
+                    mbar_arrive(&unit_empty[slot]);
+                    if (u < 0) break;
+                } else if (u >= n_units) {
+                    break;
+                }
                 const int nk = (MODE == MODE_EXPERTS && u >= n_first) ? p.nk2 : p.nk;
                 const uint32_t a = lu & 1u;
                 if (!mbar_wait_bounded(&tempty_bar[a], ((lu >> 1) & 1u) ^ 1u, abort_flag,
@@ -335,11 +381,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         // --------------------------------------------------- epilogue --
         const int q = warp & 3;          // TMEM lane quadrant this warp may access
         const int row = q * 32 + lane;   // row within the 128-row weight tile
-        uint32_t lu = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++lu) {
+        for (uint32_t lu = 0;; ++lu) {
+            int u = blockIdx.x + int(lu) * gridDim.x;
+            bool ok = true;
+            if (DYN) {
+                const int slot = int(lu % kRing);
+                ok = mbar_wait_bounded(&unit_full[slot], (lu / kRing) & 1u, abort_flag,
+                                       p.timeout_ns);
+                ok = __all_sync(0xffffffffu, ok);
+                if (ok) {
+                    u = unit_ring[slot];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&unit_empty[slot]);
+                }
+            } else if (u >= n_units) {
+                break;  // round-robin: the same u in every epilogue warp
+            }
+            if (DYN) {
+                // The four warps must leave together (they meet at named
+                // barriers): agree on "all got a unit", "hand-out finished".
+                // Each vote array is written only after barriers that every
+                // warp passes after its last read of it.
+                if (lane == 0) uvote[warp - 2] = ok ? (u < 0 ? 2 : 1) : 0;
+                epilogue_sync();
+                const int v0 = uvote[0], v1 = uvote[1], v2 = uvote[2], v3 = uvote[3];
+                if (!(v0 && v1 && v2 && v3)) {
+                    if (lane == 0) signal_abort(p.err, &abort_sh);
+                    break;
+                }
+                if (v0 == 2 || v1 == 2 || v2 == 2 || v3 == 2) break;
+            }
             const Unit w = decode_unit<MODE, BN>(u, n_first, p);
             const uint32_t a = lu & 1u;
-            bool ok = mbar_wait_bounded(&tfull_bar[a], (lu >> 1) & 1u, abort_flag, p.timeout_ns);
+            ok = mbar_wait_bounded(&tfull_bar[a], (lu >> 1) & 1u, abort_flag, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (ModeTraits<MODE>::XCH) {
                 // The four warps meet at named barriers below: agree first.

@@ -77,7 +77,8 @@ typedef struct {
  * after beam_moe_forward; none of it is needed to call the layer.
  *   err       int32      device error word (0 = ok), read by beam_moe_check
  *   meta      int32[4]   [0] tiles in the tile list, [1] padded rows,
- *                        [2] kept pairs P, [3] reserved
+ *                        [2] kept pairs P, [3] work counter of the fused
+ *                        expert kernel (units handed out so far)
  *   counts    int32[E]   kept pairs per expert
  *   hist      int32[K+1] tokens by number of kept candidates
  *   partial   f32[S][T][2E] router partial logits (S = router_splits)
