@@ -21,17 +21,22 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------ top-K + mask --
 //
-// One warp per token.  Lane l holds the logits of experts l, l+32, ...; the
-// router's split-K partial sums are added in split order.  K rounds of a
-// warp arg-max (ties -> lower expert id) give the candidates in descending
-// order.  renorm: softmax over the candidates (Eq. 4); else over all E.
-// The mask keeps candidate k iff its pre-sigmoid value z >= 0 (Eq. 6; NaN
-// is not kept); w = g * m (Eq. 7).  Counts and the histogram are gathered in
-// shared memory and added to global memory once per block.
-template <int EPL, int S>
-__global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a) {
+// A block takes `tpb` tokens at a time.  Phase 1: all threads add the router's
+// split-K partial logits for those tokens (independent float4 loads, summed in
+// split order) into shared memory, and export them when asked.  Phase 2: one
+// warp per token; lane l holds the logits of experts l, l+32, ...  K rounds of
+// a warp arg-max (ties -> lower expert id) give the candidates in descending
+// order.  renorm: softmax over the candidates (Eq. 4); else over all E.  The
+// mask keeps candidate k iff its pre-sigmoid value z >= 0 (Eq. 6; NaN is not
+// kept); w = g * m (Eq. 7).  Counts and the histogram are gathered in shared
+// memory and added to global memory once per block.
+constexpr int kTopkMaxTok = 8;
+
+template <int EPL>
+__global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tpb) {
     __shared__ int s_counts[kMaxE];
     __shared__ int s_hist[kMaxK + 1];
+    __shared__ __align__(16) float s_logit[kTopkMaxTok][2 * kMaxE];
     for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_counts[i] = 0;
     if (threadIdx.x <= a.K) s_hist[threadIdx.x] = 0;
     __syncthreads();
@@ -39,100 +44,120 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a) {
     griddep_launch_dependents();
 
     const int lane = threadIdx.x & 31;
-    const int warps = blockDim.x >> 5;
-    const long long E2 = 2LL * a.E;
+    const int warp = threadIdx.x >> 5;
+    const int E2 = 2 * a.E;
+    const int cols = a.has_mask ? E2 : a.E;  // columns that hold logits
     const long long slab = (long long)a.T * E2;
+    const bool vec = (E2 % 4 == 0) && (cols % 4 == 0);
 
-    for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < a.T; t += gridDim.x * warps) {
-        float r[EPL], z[EPL];
-        unsigned taken = 0;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int j = lane + 32 * i;
-            r[i] = -INFINITY;
-            z[i] = 0.0f;
-            if (j < a.E) {
-                // All S partials are loaded before they are added (S is a
-                // compile-time constant), then summed in split order.
-                const float *pr = a.partial + (long long)t * E2 + j;
-                float pr_r[S], pr_z[S];
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    pr_r[s] = __ldg(pr + s * slab);
-                    pr_z[s] = a.has_mask ? __ldg(pr + s * slab + a.E) : 0.0f;
+    for (int t0 = blockIdx.x * tpb; t0 < a.T; t0 += gridDim.x * tpb) {
+        const int nt = min(tpb, a.T - t0);
+        // ---- phase 1: split sums -> shared memory
+        if (vec) {
+            const int c4n = cols / 4;
+            for (int v = threadIdx.x; v < nt * c4n; v += blockDim.x) {
+                const int tt = v / c4n, c4 = v - tt * c4n;
+                const float4 *pr =
+                    reinterpret_cast<const float4 *>(a.partial + (long long)(t0 + tt) * E2) + c4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+                for (int sp = 0; sp < a.S; ++sp) {
+                    const float4 q = __ldg(pr + sp * (slab / 4));
+                    acc.x += q.x;
+                    acc.y += q.y;
+                    acc.z += q.z;
+                    acc.w += q.w;
                 }
-                float rs = 0.0f, zs = 0.0f;
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    rs += pr_r[s];
-                    zs += pr_z[s];
-                }
-                if (a.logits) {
-                    a.logits[(long long)t * E2 + j] = rs;
-                    if (a.has_mask) a.logits[(long long)t * E2 + a.E + j] = zs;
-                }
-                r[i] = (rs != rs) ? -INFINITY : rs;  // NaN never wins a slot
-                z[i] = zs;
-            } else {
-                taken |= 1u << i;
+                reinterpret_cast<float4 *>(&s_logit[tt][0])[c4] = acc;
+                if (a.logits)
+                    reinterpret_cast<float4 *>(a.logits + (long long)(t0 + tt) * E2)[c4] = acc;
+            }
+        } else {
+            for (int v = threadIdx.x; v < nt * cols; v += blockDim.x) {
+                const int tt = v / cols, c = v - tt * cols;
+                const float *pr = a.partial + (long long)(t0 + tt) * E2 + c;
+                float acc = 0.0f;
+                for (int sp = 0; sp < a.S; ++sp) acc += __ldg(pr + sp * slab);
+                s_logit[tt][c] = acc;
+                if (a.logits) a.logits[(long long)(t0 + tt) * E2 + c] = acc;
             }
         }
-
-        int my_cand = -1;
-        float my_e = 0.0f, my_z = 0.0f, rmax = 0.0f, denom = 0.0f;
-        for (int k = 0; k < a.K; ++k) {
-            float bv = -INFINITY, bz = 0.0f;
-            int bi = INT_MAX;
+        __syncthreads();
+        // ---- phase 2: one warp per token
+        if (warp < nt) {
+            const int t = t0 + warp;
+            float r[EPL], z[EPL];
+            unsigned taken = 0;
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int j = lane + 32 * i;
-                if (!((taken >> i) & 1u) && (r[i] > bv || (r[i] == bv && j < bi))) {
-                    bv = r[i];
-                    bi = j;
-                    bz = z[i];
+                r[i] = -INFINITY;
+                z[i] = 0.0f;
+                if (j < a.E) {
+                    const float rs = s_logit[warp][j];
+                    r[i] = (rs != rs) ? -INFINITY : rs;  // NaN never wins a slot
+                    if (a.has_mask) z[i] = s_logit[warp][a.E + j];
+                } else {
+                    taken |= 1u << i;
                 }
             }
+
+            int my_cand = -1;
+            float my_e = 0.0f, my_z = 0.0f, rmax = 0.0f, denom = 0.0f;
+            for (int k = 0; k < a.K; ++k) {
+                float bv = -INFINITY, bz = 0.0f;
+                int bi = INT_MAX;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(kFull, bv, off);
-                const int oi = __shfl_xor_sync(kFull, bi, off);
-                const float oz = __shfl_xor_sync(kFull, bz, off);
-                if (ov > bv || (ov == bv && oi < bi)) {
-                    bv = ov;
-                    bi = oi;
-                    bz = oz;
+                for (int i = 0; i < EPL; ++i) {
+                    const int j = lane + 32 * i;
+                    if (!((taken >> i) & 1u) && (r[i] > bv || (r[i] == bv && j < bi))) {
+                        bv = r[i];
+                        bi = j;
+                        bz = z[i];
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(kFull, bv, off);
+                    const int oi = __shfl_xor_sync(kFull, bi, off);
+                    const float oz = __shfl_xor_sync(kFull, bz, off);
+                    if (ov > bv || (ov == bv && oi < bi)) {
+                        bv = ov;
+                        bi = oi;
+                        bz = oz;
+                    }
+                }
+                if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
+                if (k == 0) rmax = bv;
+                const float ek = expf(bv - rmax);
+                denom += ek;
+                if (lane == k) {
+                    my_cand = bi;
+                    my_e = ek;
+                    my_z = bz;
                 }
             }
-            if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
-            if (k == 0) rmax = bv;
-            const float ek = expf(bv - rmax);
-            denom += ek;
-            if (lane == k) {
-                my_cand = bi;
-                my_e = ek;
-                my_z = bz;
+            if (!a.renorm) {
+                float part = 0.0f;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (lane + 32 * i < a.E) part += expf(r[i] - rmax);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
+                denom = part;  // identical on every lane (pairwise sums commute exactly)
             }
+            const bool kept = (lane < a.K) && (!a.has_mask || my_z >= 0.0f);
+            if (lane < a.K) {
+                const float g = my_e / denom;
+                a.idx[(long long)t * a.K + lane] = kept ? my_cand : -1;
+                a.w[(long long)t * a.K + lane] = kept ? g : 0.0f;
+                if (kept) atomicAdd(&s_counts[my_cand], 1);
+            }
+            const int nkept = __popc(__ballot_sync(kFull, kept));
+            if (lane == 0) atomicAdd(&s_hist[nkept], 1);
         }
-        if (!a.renorm) {
-            float part = 0.0f;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (lane + 32 * i < a.E) part += expf(r[i] - rmax);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
-            denom = part;  // identical on every lane (pairwise sums commute exactly)
-        }
-        const bool kept = (lane < a.K) && (!a.has_mask || my_z >= 0.0f);
-        if (lane < a.K) {
-            const float g = my_e / denom;
-            a.idx[(long long)t * a.K + lane] = kept ? my_cand : -1;
-            a.w[(long long)t * a.K + lane] = kept ? g : 0.0f;
-            if (kept) atomicAdd(&s_counts[my_cand], 1);
-        }
-        const int nkept = __popc(__ballot_sync(kFull, kept));
-        if (lane == 0) atomicAdd(&s_hist[nkept], 1);
+        __syncthreads();  // s_logit is rewritten by the next tokens
     }
-    __syncthreads();
     for (int i = threadIdx.x; i < a.E; i += blockDim.x)
         if (s_counts[i]) atomicAdd(&a.counts[i], s_counts[i]);
     if (a.hist && threadIdx.x <= a.K && s_hist[threadIdx.x]) atomicAdd(&a.hist[threadIdx.x], s_hist[threadIdx.x]);
@@ -415,29 +440,22 @@ __global__ void __launch_bounds__(256) gemm2_f32_kernel(const float *H, const fl
 
 }  // namespace
 
-template <int EPL>
-cudaError_t launch_topk_s(const TopkArgs &a, int blocks, cudaStream_t stream) {
-    switch (a.S) {
-        case 1: return launch_pdl(topk_mask_kernel<EPL, 1>, dim3(blocks), dim3(256), 0, stream, a);
-        case 2: return launch_pdl(topk_mask_kernel<EPL, 2>, dim3(blocks), dim3(256), 0, stream, a);
-        case 4: return launch_pdl(topk_mask_kernel<EPL, 4>, dim3(blocks), dim3(256), 0, stream, a);
-        case 8: return launch_pdl(topk_mask_kernel<EPL, 8>, dim3(blocks), dim3(256), 0, stream, a);
-        case 16: return launch_pdl(topk_mask_kernel<EPL, 16>, dim3(blocks), dim3(256), 0, stream, a);
-        case 32: return launch_pdl(topk_mask_kernel<EPL, 32>, dim3(blocks), dim3(256), 0, stream, a);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
     if (a.T <= 0) return cudaSuccess;
-    const int warps = 8;
-    int blocks = (a.T + warps - 1) / warps;
-    if (blocks > 2 * n_sm) blocks = 2 * n_sm;
+    // Tokens per block: one at decode sizes (more blocks, more loads in
+    // flight), up to kTopkMaxTok for large batches.
+    int tpb = (a.T + 127) / 128;
+    if (tpb > kTopkMaxTok) tpb = kTopkMaxTok;
+    int blocks = (a.T + tpb - 1) / tpb;
+    if (blocks > 8 * n_sm) blocks = 8 * n_sm;
     const int epl = (a.E + 31) / 32;
-    if (epl <= 1) return launch_topk_s<1>(a, blocks, stream);
-    if (epl <= 2) return launch_topk_s<2>(a, blocks, stream);
-    if (epl <= 4) return launch_topk_s<4>(a, blocks, stream);
-    return launch_topk_s<8>(a, blocks, stream);
+    if (epl <= 1)
+        return launch_pdl(topk_mask_kernel<1>, dim3(blocks), dim3(256), 0, stream, a, tpb);
+    if (epl <= 2)
+        return launch_pdl(topk_mask_kernel<2>, dim3(blocks), dim3(256), 0, stream, a, tpb);
+    if (epl <= 4)
+        return launch_pdl(topk_mask_kernel<4>, dim3(blocks), dim3(256), 0, stream, a, tpb);
+    return launch_pdl(topk_mask_kernel<8>, dim3(blocks), dim3(256), 0, stream, a, tpb);
 }
 
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {
