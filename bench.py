@@ -384,7 +384,7 @@ def run_beam(args):
     S = layer.abi.FORWARD_STAGES
     names = [layer.abi.stage_name(j) for j in range(S)]
     n_kernels = layer.abi.kernel_count(layer.dsc)
-    fused = layer.abi.plan(layer.dsc)["BN"] < 128  # decode tiles: one expert launch (stage 4)
+    fused = n_kernels == S - 1  # decode tiles: both expert GEMMs in one launch (stage 4)
     if fused:
         names[4] = "experts_fused_gate_up_down"
     stage_mean = [sum(s[j] for s in stage_s) / len(stage_s) for j in range(S)]

@@ -286,9 +286,8 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     BEAM_TRY_CUDA(launch_permute(pa, st));
 
     BEAM_TRY_CUDA(rec.rec(3));
-    if (d->dtype != BEAM_BF16) {  // bf16: the expert kernels read the rows from x themselves
-        BEAM_TRY_CUDA(launch_gather(x, pair, meta, d->K, 4LL * d->d, P.p_cap, xp, n_sm, st));
-    }
+    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
+    BEAM_TRY_CUDA(launch_gather(x, pair, meta, d->K, (long long)es * d->d, P.p_cap, xp, n_sm, st));
 
     if (d->dtype == BEAM_BF16) {
         // Thin token tiles (decode): gate and up rows interleaved in one
@@ -314,10 +313,6 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         g.a_rows_per_expert = d->I;
         g.out = h;
         g.out_ld = d->I;
-        g.gx = x;
-        g.pair = pair;
-        g.K = d->K;
-        g.d = d->d;
 
         BEAM_TRY_CUDA(rec.rec(4));
         if (fused) {
@@ -509,9 +504,8 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     beam_moe_plan_info P;
     if (make_plan(desc, &P) != BEAM_OK) return 0;
     if (desc->T == 0) return 0;
-    if (desc->dtype != BEAM_BF16) return BEAM_MOE_FORWARD_STAGES;
-    // bf16: no gather launch; decode tiles also fuse the two expert GEMMs
-    return fused_experts(P) ? BEAM_MOE_FORWARD_STAGES - 2 : BEAM_MOE_FORWARD_STAGES - 1;
+    return (desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 1
+                                                          : BEAM_MOE_FORWARD_STAGES;
 }
 
 const char *beam_moe_stage_name(int stage) {

@@ -82,11 +82,6 @@ struct TcGemmArgs {
     long long out2_ld;
     int *tile_done;           // per tile: gate/up units whose H rows are published
     int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
-    // MODE_GEMM1 / MODE_EXPERTS gate/up units: token rows loaded straight from
-    // x (row pair[r] / K) instead of a gathered copy
-    const void *gx;
-    const int *pair;
-    int K, d;
 };
 
 cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,

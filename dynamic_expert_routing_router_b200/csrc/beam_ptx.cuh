@@ -103,31 +103,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *t
         : "memory");
 }
 
-// 16-byte asynchronous copy global -> shared (L2 only), the thread's own
-// completion tracked by cp_async_mbar_arrive_noinc.
-__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
-                 "l"(gmem_src)
-                 : "memory");
-}
-
-// Arrive on `bar` once every cp.async this thread issued so far has landed.
-// The arrival counts against the barrier's expected count (.noinc).
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-// Orders shared-memory writes of the generic proxy (cp.async, st.shared) that
-// this thread has observed before later async-proxy reads (tcgen05.mma).
-__device__ __forceinline__ void fence_proxy_async_shared() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // -------------------------------------------------------------- tcgen05 --
 
 __device__ __forceinline__ void tc_fence_before_sync() {

@@ -23,10 +23,7 @@
 // without kept pairs has no tile, and TMA never reads its weights.
 //
 // Warp roles (192 threads, one CTA per SM):
-//   warp 0      producer: lane 0 issues the TMA loads of the weight tile(s)
-//               (and of the token tile where it is a plain matrix: router
-//               tokens, H); for gate/up units all 32 lanes copy the tile's
-//               token rows straight from x with cp.async, by their pair index
+//   warp 0      TMA producer (one thread): weight tile(s) + token tile per stage
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..5  epilogue: TMEM -> registers -> activation -> global memory
 // Pipelines: a STAGES-deep shared-memory ring (full/empty mbarriers) and a
@@ -80,11 +77,7 @@ template <int MODE>
 struct ModeTraits {
     static constexpr int NUM_A = MODE == MODE_GEMM1 ? 2 : 1;
     static constexpr bool XCH = MODE == MODE_GEMM1_IL || MODE == MODE_EXPERTS;
-    // Gate/up units load their token rows from x with cp.async (no gathered copy).
-    static constexpr bool GATHER = MODE == MODE_GEMM1 || MODE == MODE_EXPERTS;
 };
-
-constexpr unsigned kFullMask = 0xffffffffu;
 
 struct Unit {
     int phase;  // MODE_EXPERTS: 0 = gate/up unit, 1 = down unit; else 0
@@ -198,8 +191,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int unit_ring[kRing];
     __shared__ __align__(8) uint64_t unit_full[kRing];
     __shared__ __align__(8) uint64_t unit_empty[kRing];
-    constexpr bool GATHER = ModeTraits<MODE>::GATHER;
-    __shared__ int tok_s[GATHER ? BN : 1];  // token of each row of the current tile
 
     // 1024-byte aligned start of the stage ring (SWIZZLE_128B atoms).
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -211,9 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            // GATHER: the TMA issuer's expect_tx arrival + one cp.async arrival
-            // per producer lane.
-            mbar_init(&full_bar[s], GATHER ? 1 + 32 : 1);
+            mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -259,81 +248,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  : n_first;
 
     if (warp == 0) {
-        // ---------------------------------------------------- producer --
-        // Lane 0 takes the units, does the waits and issues the TMA loads; with
-        // GATHER all 32 lanes also copy the tile's token rows from x.
-        uint32_t it = 0;
-        bool ok = true;
-        const __nv_bfloat16 *xg = static_cast<const __nv_bfloat16 *>(p.gx);
-        for (uint32_t lu = 0;; ++lu) {
-            int u = blockIdx.x + int(lu) * gridDim.x;
-            if (DYN) {
-                int uu = -1, good = 1;
-                if (lane == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (uint32_t lu = 0;; ++lu) {
+                int u = blockIdx.x + int(lu) * gridDim.x;
+                if (DYN) {
                     const int slot = int(lu % kRing);
                     if (!mbar_wait_bounded(&unit_empty[slot], ((lu / kRing) & 1u) ^ 1u, abort_flag,
                                            p.timeout_ns)) {
-                        good = 0;
-                    } else {
-                        uu = atomicAdd(p.work_ctr, 1);
-                        if (uu >= n_units) uu = -1;
-                        unit_ring[slot] = uu;
-                        mbar_arrive(&unit_full[slot]);
+                        ok = false;
+                        break;
                     }
-                }
-                good = __shfl_sync(kFullMask, good, 0);
-                u = __shfl_sync(kFullMask, uu, 0);
-                if (!good) {
-                    ok = false;
+                    u = atomicAdd(p.work_ctr, 1);
+                    if (u >= n_units) u = -1;
+                    unit_ring[slot] = u;
+                    mbar_arrive(&unit_full[slot]);
+                    if (u < 0) break;
+                } else if (u >= n_units) {
                     break;
                 }
-                if (u < 0) break;
-            } else if (u >= n_units) {
-                break;
-            }
-            const Unit w = decode_unit<MODE, BN>(u, n_first, p);
-            const CUtensorMap *am = &maps.a0;
-            const CUtensorMap *bm = &maps.b;
-            if (MODE == MODE_ROUTER && w.sel) am = &maps.a1;
-            if (MODE == MODE_EXPERTS && w.phase == 1) {
-                // H rows of this tile come from other CTAs' gate/up units.
-                int good = 1;
-                if (lane == 0) {
-                    good = wait_counter_bounded(p.tile_done + w.ti, p.n_mb, abort_flag,
-                                                p.timeout_ns);
+                const Unit w = decode_unit<MODE, BN>(u, n_first, p);
+                const CUtensorMap *am = &maps.a0;
+                const CUtensorMap *bm = &maps.b;
+                if (MODE == MODE_ROUTER && w.sel) am = &maps.a1;
+                if (MODE == MODE_EXPERTS && w.phase == 1) {
+                    // H rows of this tile come from other CTAs' gate/up units.
+                    if (!wait_counter_bounded(p.tile_done + w.ti, p.n_mb, abort_flag,
+                                              p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
                     asm volatile("fence.proxy.async.global;" ::: "memory");
+                    am = &maps.a2;
+                    bm = &maps.b2;
                 }
-                if (!__shfl_sync(kFullMask, good, 0)) {
-                    ok = false;
-                    break;
-                }
-                am = &maps.a2;
-                bm = &maps.b2;
-            }
-            const bool interleaved =
-                MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
-            const bool gather = GATHER && w.phase == 0;
-            if (gather) {
-                for (int r = lane; r < BN; r += 32) {
-                    const int pr = r < w.rows ? p.pair[w.b_row + r] : -1;
-                    tok_s[r] = pr < 0 ? -1 : pr / p.K;
-                }
-                __syncwarp();
-            }
-            for (int kb = 0; kb < w.nk; ++kb, ++it) {
-                const int s = int(it % STAGES);
-                const uint32_t ph = ((it / STAGES) & 1u) ^ 1u;
-                int good = 1;
-                if (lane == 0) good = mbar_wait_bounded(&empty_bar[s], ph, abort_flag, p.timeout_ns);
-                if (!__shfl_sync(kFullMask, good, 0)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
-                const int kx = (w.kb0 + kb) * kBlockK;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full_bar[s], gather ? NUM_A * C::A_BYTES
-                                                               : C::STAGE_BYTES);
+                const bool interleaved =
+                    MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
+                for (int kb = 0; kb < w.nk; ++kb, ++it) {
+                    const int s = int(it % STAGES);
+                    const uint32_t ph = ((it / STAGES) & 1u) ^ 1u;
+                    if (!mbar_wait_bounded(&empty_bar[s], ph, abort_flag, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
+                    const int kx = (w.kb0 + kb) * kBlockK;
                     if (interleaved) {
                         // rows 0..63: W1 (gate), rows 64..127: W3 (up), same I rows
                         tma_load_2d(st, &maps.a0, kx, w.a_row, &full_bar[s]);
@@ -343,31 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (NUM_A == 2)
                         tma_load_2d(st + C::A_BYTES, &maps.a1, kx, w.a_row, &full_bar[s]);
-                    if (!gather) tma_load_2d(st + NUM_A * C::A_BYTES, bm, kx, w.b_row, &full_bar[s]);
+                    tma_load_2d(st + NUM_A * C::A_BYTES, bm, kx, w.b_row, &full_bar[s]);
                 }
-                if (gather) {
-                    // Row r, 16-byte chunk c lands where a 128-byte-swizzled TMA
-                    // box would put it: r * 128 + ((c ^ (r % 8)) * 16).
-                    uint8_t *sb = st + NUM_A * C::A_BYTES;
-#pragma unroll
-                    for (int j = 0; j < BN / 4; ++j) {
-                        const int q = lane + 32 * j;
-                        const int r = q >> 3, c = q & 7;
-                        const int tok = tok_s[r];
-                        if (tok >= 0)
-                            cp_async_16(sb + r * 128 + ((c ^ (r & 7)) << 4),
-                                        xg + (long long)tok * p.d + kx + c * 8);
-                    }
-                }
-                if (GATHER) cp_async_mbar_arrive_noinc(&full_bar[s]);
+                if (!ok) break;
             }
-            if (!ok) break;
-        }
-        if (!ok) {
-            if (GATHER) cp_async_wait_all();  // this lane's own copies land first
-            if (lane == 0) {
+            if (!ok) {
                 signal_abort(p.err, &abort_sh);
-                // Let this CTA's own TMA copies land before it can exit.
+                // Let this CTA's own copies land before it can exit.
                 for (uint32_t j = (it > uint32_t(STAGES) ? it - STAGES : 0u); j < it; ++j)
                     mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1u, nullptr,
                                       p.timeout_ns);
@@ -410,7 +354,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (GATHER) fence_proxy_async_shared();  // cp.async rows -> MMA reads
                     tc_fence_after_sync();
                     const uint32_t sa = smem_u32(smem + size_t(s) * C::STAGE_BYTES);
                     const uint32_t sb = sa + NUM_A * C::A_BYTES;

@@ -90,8 +90,7 @@ typedef struct {
  *   pair_pos  int32[T][K] permuted row of a kept pair (undefined if masked)
  *   tiles     int32[tiles_cap][4] (expert, first row, valid rows, 0)
  *   tile_done int32[tiles_cap] gate/up units finished per tile (fused path)
- *   xp        [p_cap][d]  gathered token rows (fp32 layer only; the bf16
- *                         expert kernels read x directly)
+ *   xp        [p_cap][d]  gathered token rows (dtype)
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
  *   y         f32[p_cap][d] expert output per pair                           */
 typedef struct {
@@ -107,11 +106,10 @@ typedef struct {
 } beam_moe_plan_info;
 
 /* Stage slots of one beam_moe_forward call (router GEMM, top-K + mask,
- * grouping, gather, gate/up GEMM, down GEMM, combine).  In the bf16 layer
- * the expert kernels read the token rows from x themselves, so the gather
- * slot is empty, and with token tiles thinner than 128 rows (decode batches)
- * the two expert GEMMs run as one fused launch in the gate/up slot, leaving
- * the down slot empty too; see beam_moe_forward_kernel_count. */
+ * grouping, gather, gate/up GEMM, down GEMM, combine).  With token tiles
+ * thinner than 128 rows (decode batches) the two expert GEMMs run as one
+ * fused launch in the gate/up slot and the down slot is empty; see
+ * beam_moe_forward_kernel_count. */
 #define BEAM_MOE_FORWARD_STAGES 7
 
 /* Bytes of device workspace beam_moe_forward needs for `desc` (0 on a bad
@@ -193,9 +191,8 @@ beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
                                    float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
                                    float *logits, void *stream);
 
-/* Kernel launches one beam_moe_forward call makes for `desc`: 5 (bf16,
- * decode-sized tiles), 6 (bf16, 128-row tiles) or 7 (fp32); 0 for T = 0 or a
- * bad descriptor. */
+/* Kernel launches one beam_moe_forward call makes for `desc` (6 or 7), or 0
+ * on a bad descriptor. */
 int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last
