@@ -103,3 +103,11 @@ def test_argument_errors_return_before_any_launch():
     p = list(good)
     p[7] += 16
     assert _call_forward(dsc, p, need) == 3
+
+
+def test_kernel_count_per_path():
+    assert abi.kernel_count(abi.desc(128, 2048, 128, 768, 8, "bf16", 1)) == 6  # fused experts
+    assert abi.kernel_count(abi.desc(8192, 2048, 128, 768, 8, "bf16", 1)) == 7
+    assert abi.kernel_count(abi.desc(64, 128, 8, 256, 2, "f32", 0)) == 7
+    assert abi.kernel_count(abi.desc(0, 2048, 128, 768, 8, "bf16", 1)) == 0
+    assert abi.kernel_count(abi.desc(4, 2000, 128, 768, 8, "bf16", 1)) == 0
