@@ -213,17 +213,31 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     }
     const int count_e = a.counts[e];
 
+    // Each pass: thread i owns tokens base + 4i .. base + 4i + 3 (token order =
+    // thread order); a token matches expert e in at most one slot.
+    constexpr int kTokPerThread = 4;
     int running = 0;
-    for (int base = 0; base < a.T; base += kPermThreads) {
-        const int t = base + tid;
-        int km = -1;
-        if (t < a.T) {
-            const int *row = a.idx + (long long)t * a.K;
-            for (int k = 0; k < a.K; ++k)
-                if (row[k] == e) km = k;
+    for (int base = 0; base < a.T; base += kPermThreads * kTokPerThread) {
+        int km[kTokPerThread];
+        int cnt = 0;
+#pragma unroll
+        for (int q = 0; q < kTokPerThread; ++q) {
+            const int t = base + tid * kTokPerThread + q;
+            km[q] = -1;
+            if (t < a.T) {
+                const int *row = a.idx + (long long)t * a.K;
+                for (int k = 0; k < a.K; ++k)
+                    if (row[k] == e) km[q] = k;
+            }
+            cnt += km[q] >= 0;
         }
-        const unsigned bal = __ballot_sync(kFull, km >= 0);
-        if (lane == 0) s_wcnt[warp] = __popc(bal);
+        int incl = cnt;  // warp inclusive scan of the per-thread counts
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int nb = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += nb;
+        }
+        if (lane == 31) s_wcnt[warp] = incl;
         __syncthreads();
         if (tid == 0) {
             int acc = 0;
@@ -234,10 +248,15 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
             s_total = acc;
         }
         __syncthreads();
-        if (km >= 0) {
-            const int pos = off_e + running + s_wpre[warp] + __popc(bal & ((1u << lane) - 1u));
-            a.pair[pos] = t * a.K + km;
-            a.pair_pos[(long long)t * a.K + km] = pos;
+        int pos = off_e + running + s_wpre[warp] + incl - cnt;
+#pragma unroll
+        for (int q = 0; q < kTokPerThread; ++q) {
+            if (km[q] >= 0) {
+                const int t = base + tid * kTokPerThread + q;
+                a.pair[pos] = t * a.K + km[q];
+                a.pair_pos[(long long)t * a.K + km[q]] = pos;
+                ++pos;
+            }
         }
         running += s_total;
         __syncthreads();
@@ -269,7 +288,16 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *
         if (pr < 0) continue;
         const uint4 *src = x + (long long)(pr / K) * row_vec;
         uint4 *dst = xp + (long long)r * row_vec;
-        for (int v = lane; v < row_vec; v += 32) dst[v] = __ldg(src + v);
+        int v = lane;
+        for (; v + 96 < row_vec; v += 128) {  // four 16-byte loads in flight per lane
+            const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 32);
+            const uint4 a2 = __ldg(src + v + 64), a3 = __ldg(src + v + 96);
+            dst[v] = a0;
+            dst[v + 32] = a1;
+            dst[v + 64] = a2;
+            dst[v + 96] = a3;
+        }
+        for (; v < row_vec; v += 32) dst[v] = __ldg(src + v);
     }
 }
 
@@ -301,25 +329,43 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
                                                       int K, int d, Tout *out) {
     __shared__ int s_row[kMaxK];
     __shared__ float s_w[kMaxK];
+    __shared__ int s_n;
     const int nvec = d / 8;
     griddep_wait();
     griddep_launch_dependents();
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < K) {
-            const long long o = (long long)t * K + threadIdx.x;
-            const int id = idx[o];
-            s_row[threadIdx.x] = id >= 0 ? pair_pos[o] : -1;
-            s_w[threadIdx.x] = w[o];
+        if (threadIdx.x == 0) {  // kept candidates of token t, in slot order
+            int n = 0;
+            for (int k = 0; k < K; ++k) {
+                const long long o = (long long)t * K + k;
+                if (idx[o] >= 0) {
+                    s_row[n] = pair_pos[o];
+                    s_w[n] = w[o];
+                    ++n;
+                }
+            }
+            s_n = n;
         }
         __syncthreads();
+        const int n = s_n;
         for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int k = 0; k < K; ++k) {
-                const int row = s_row[k];
-                if (row < 0) continue;
+            int j = 0;
+            for (; j + 4 <= n; j += 4) {  // four rows in flight, added in slot order
+                float y[4][8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) load8(Y + (long long)s_row[j + q] * d + v * 8, y[q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float wk = s_w[j + q];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[q][i], acc[i]);
+                }
+            }
+            for (; j < n; ++j) {
                 float y[8];
-                load8(Y + (long long)row * d + v * 8, y);
-                const float wk = s_w[k];
+                load8(Y + (long long)s_row[j] * d + v * 8, y);
+                const float wk = s_w[j];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
             }
