@@ -187,8 +187,8 @@ __device__ __forceinline__ int block_sum_256(int v, int *s_red) {
 
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs a) {
     __shared__ int s_red[kPermThreads / 32];
-    __shared__ int s_wcnt[kPermThreads / 32];
-    __shared__ int s_wpre[kPermThreads / 32];
+    __shared__ int s_wcnt[4 * (kPermThreads / 32)];
+    __shared__ int s_wpre[4 * (kPermThreads / 32)];
     __shared__ int s_total;
     const int e = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -213,49 +213,45 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     }
     const int count_e = a.counts[e];
 
-    // Each pass: thread i owns tokens base + 4i .. base + 4i + 3 (token order =
-    // thread order); a token matches expert e in at most one slot.
-    constexpr int kTokPerThread = 4;
+    // Each pass covers kSub * 256 tokens as kSub coalesced sub-chunks (token
+    // base + q * 256 + tid); ranks follow (sub-chunk, warp, lane), i.e. token
+    // order.  A token matches expert e in at most one slot.
+    constexpr int kSub = 4;
+    constexpr int kWarps = kPermThreads / 32;
     int running = 0;
-    for (int base = 0; base < a.T; base += kPermThreads * kTokPerThread) {
-        int km[kTokPerThread];
-        int cnt = 0;
+    for (int base = 0; base < a.T; base += kPermThreads * kSub) {
+        int km[kSub];
+        unsigned bal[kSub];
 #pragma unroll
-        for (int q = 0; q < kTokPerThread; ++q) {
-            const int t = base + tid * kTokPerThread + q;
+        for (int q = 0; q < kSub; ++q) {
+            const int t = base + q * kPermThreads + tid;
             km[q] = -1;
             if (t < a.T) {
                 const int *row = a.idx + (long long)t * a.K;
                 for (int k = 0; k < a.K; ++k)
                     if (row[k] == e) km[q] = k;
             }
-            cnt += km[q] >= 0;
+            bal[q] = __ballot_sync(kFull, km[q] >= 0);
+            if (lane == 0) s_wcnt[q * kWarps + warp] = __popc(bal[q]);
         }
-        int incl = cnt;  // warp inclusive scan of the per-thread counts
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int nb = __shfl_up_sync(kFull, incl, off);
-            if (lane >= off) incl += nb;
-        }
-        if (lane == 31) s_wcnt[warp] = incl;
         __syncthreads();
         if (tid == 0) {
             int acc = 0;
-            for (int i = 0; i < kPermThreads / 32; ++i) {
+            for (int i = 0; i < kSub * kWarps; ++i) {
                 s_wpre[i] = acc;
                 acc += s_wcnt[i];
             }
             s_total = acc;
         }
         __syncthreads();
-        int pos = off_e + running + s_wpre[warp] + incl - cnt;
 #pragma unroll
-        for (int q = 0; q < kTokPerThread; ++q) {
+        for (int q = 0; q < kSub; ++q) {
             if (km[q] >= 0) {
-                const int t = base + tid * kTokPerThread + q;
+                const int t = base + q * kPermThreads + tid;
+                const int pos = off_e + running + s_wpre[q * kWarps + warp] +
+                                __popc(bal[q] & ((1u << lane) - 1u));
                 a.pair[pos] = t * a.K + km[q];
                 a.pair_pos[(long long)t * a.K + km[q]] = pos;
-                ++pos;
             }
         }
         running += s_total;
