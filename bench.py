@@ -384,8 +384,7 @@ def run_beam(args):
     S = layer.abi.FORWARD_STAGES
     names = [layer.abi.stage_name(j) for j in range(S)]
     n_kernels = layer.abi.kernel_count(layer.dsc)
-    fused = layer.abi.plan(layer.dsc)["BN"] < 128  # decode tiles: one expert launch (stage 4)
-    names[1] = "route_group_topk_permute_gather"  # one cooperative launch (stages 1-3)
+    fused = n_kernels == S - 1  # decode tiles: both expert GEMMs in one launch (stage 4)
     if fused:
         names[4] = "experts_fused_gate_up_down"
     stage_mean = [sum(s[j] for s in stage_s) / len(stage_s) for j in range(S)]
@@ -396,11 +395,6 @@ def run_beam(args):
     # dominant kernel vs its roofline (algorithmic bytes/flops averaged over batches)
     dom = max(range(S), key=lambda j: stage_mean[j])
     alg = [algorithmic(layer, st[i % N_BATCHES], True) for i in range(args.steps)]
-    for a in alg:
-        parts = [a.pop(k) for k in ("topk_mask", "permute", "gather")]
-        a[names[1]] = dict(bytes=sum(x["bytes"] for x in parts), flops=0, unit="hbm")
-        a["permute"] = dict(bytes=0, flops=0, unit="hbm")
-        a["gather"] = dict(bytes=0, flops=0, unit="hbm")
     if fused:
         for a in alg:
             g1, g2 = a.pop("gemm1_gate_up_swiglu"), a.pop("gemm2_down")

@@ -176,13 +176,10 @@ struct RouteOut {
     float *logits;
 };
 
-// Stages 0-1: router GEMM into the split partials, then top-K + mask.  With
-// `defer_topk` the top-K launch is left to the caller (its arguments are
-// written there) so that it can run fused with the grouping.
+// Stages 0-1: router GEMM into the split partials, then top-K + mask.
 beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, const void *x,
                          const void *Wg, const void *Wm, const RouteOut &ro, char *ws,
-                         cudaStream_t st, const Recorder &rec, int n_sm,
-                         TopkArgs *defer_topk = nullptr) {
+                         cudaStream_t st, const Recorder &rec, int n_sm) {
     float *partial = reinterpret_cast<float *>(ws + P.off_partial);
     int *hdr = reinterpret_cast<int *>(ws);  // err + meta (8 ints)
     ZeroRegion zero[3] = {{hdr, 8}, {ro.counts, d->E}, {ro.hist, ro.hist ? d->K + 1 : 0}};
@@ -233,10 +230,6 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
     t.w = ro.w;
     t.counts = ro.counts;
     t.hist = ro.hist;
-    if (defer_topk) {
-        *defer_topk = t;
-        return BEAM_OK;
-    }
     BEAM_TRY_CUDA(launch_topk_mask(t, n_sm, st));
     return BEAM_OK;
 }
@@ -283,25 +276,18 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     void *h = ws + P.off_h;
     float *y = reinterpret_cast<float *>(ws + P.off_y);
 
-    // Router GEMM, then one cooperative launch for top-K + mask, grouping and
-    // the row gather (stage slots 1-3).
     const RouteOut ro{idx, w, counts, hist, nullptr};
-    GroupArgs ga;
-    std::memset(&ga, 0, sizeof(ga));
-    s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm, &ga.t);
+    s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
     if (s != BEAM_OK) return s;
-    ga.p = PermuteArgs{idx, counts, d->T, d->K, d->E, P.BN, pair, pair_pos, tiles, tile_done,
-                       meta, err};
-    ga.tpb = topk_tokens_per_block(d->T);
-    ga.x = x;
-    ga.xp = xp;
+
+    BEAM_TRY_CUDA(rec.rec(2));
+    PermuteArgs pa{idx, counts, d->T, d->K, d->E, P.BN, pair, pair_pos, tiles, tile_done, meta,
+                   err};
+    BEAM_TRY_CUDA(launch_permute(pa, st));
+
+    BEAM_TRY_CUDA(rec.rec(3));
     const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
-    ga.row_vec = int(es * d->d / 16);
-    ga.bar = reinterpret_cast<int *>(ws) + 1;  // header word 1, cleared by the router kernel
-    ga.timeout_ns = kWaitTimeoutNs;
-    BEAM_TRY_CUDA(launch_route_group(ga, n_sm, st));
-    BEAM_TRY_CUDA(rec.rec(2));  // grouping ran inside the fused launch
-    BEAM_TRY_CUDA(rec.rec(3));  // so did the gather
+    BEAM_TRY_CUDA(launch_gather(x, pair, meta, d->K, (long long)es * d->d, P.p_cap, xp, n_sm, st));
 
     if (d->dtype == BEAM_BF16) {
         // Thin token tiles (decode): gate and up rows interleaved in one
@@ -518,8 +504,8 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     beam_moe_plan_info P;
     if (make_plan(desc, &P) != BEAM_OK) return 0;
     if (desc->T == 0) return 0;
-    // router, fused top-K/grouping/gather, expert GEMM(s), combine
-    return (desc->dtype == BEAM_BF16 && fused_experts(P)) ? 4 : 5;
+    return (desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 1
+                                                          : BEAM_MOE_FORWARD_STAGES;
 }
 
 const char *beam_moe_stage_name(int stage) {

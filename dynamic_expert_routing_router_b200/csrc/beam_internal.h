@@ -112,21 +112,6 @@ struct PermuteArgs {
 };
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 
-// Top-K + mask, grouping and (when xp != NULL) the row gather in one
-// cooperative launch with grid-wide barriers between the phases.
-struct GroupArgs {
-    TopkArgs t;
-    PermuteArgs p;
-    int tpb;           // tokens per block in the top-K phase
-    const void *x;     // gather source rows
-    void *xp;          // gather destination (NULL: no gather phase)
-    int row_vec;       // 16-byte vectors per row
-    int *bar;          // barrier counter, 0 at launch
-    unsigned long long timeout_ns;
-};
-cudaError_t launch_route_group(const GroupArgs &g, int n_sm, cudaStream_t stream);
-int topk_tokens_per_block(int T);
-
 // Gather token rows into expert order (row_bytes multiple of 16).
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
                           long long row_bytes, int p_cap, void *xp, int n_sm,

@@ -32,32 +32,17 @@ constexpr unsigned kFull = 0xffffffffu;
 // memory and added to global memory once per block.
 constexpr int kTopkMaxTok = 8;
 
-struct __align__(16) TopkSmem {
-    float logit[kTopkMaxTok][2 * kMaxE];
-    int counts[kMaxE];
-    int hist[kMaxK + 1];
-};
-
-__device__ __forceinline__ void topk_init(const TopkArgs &a, TopkSmem &sm) {
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x) sm.counts[i] = 0;
-    if (threadIdx.x <= a.K) sm.hist[threadIdx.x] = 0;
-}
-
-// Counts and histogram of this block's tokens into global memory.
-__device__ __forceinline__ void topk_flush(const TopkArgs &a, TopkSmem &sm) {
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x)
-        if (sm.counts[i]) atomicAdd(&a.counts[i], sm.counts[i]);
-    if (a.hist && threadIdx.x <= a.K && sm.hist[threadIdx.x])
-        atomicAdd(&a.hist[threadIdx.x], sm.hist[threadIdx.x]);
-}
-
-// Token groups blk, blk + nblk, ... of `tpb` tokens each (whole block).
 template <int EPL>
-__device__ __forceinline__ void topk_tokens(const TopkArgs &a, int tpb, int blk, int nblk,
-                                            TopkSmem &sm) {
-    float(*s_logit)[2 * kMaxE] = sm.logit;
-    int *s_counts = sm.counts;
-    int *s_hist = sm.hist;
+__global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tpb) {
+    __shared__ int s_counts[kMaxE];
+    __shared__ int s_hist[kMaxK + 1];
+    __shared__ __align__(16) float s_logit[kTopkMaxTok][2 * kMaxE];
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_counts[i] = 0;
+    if (threadIdx.x <= a.K) s_hist[threadIdx.x] = 0;
+    __syncthreads();
+    griddep_wait();
+    griddep_launch_dependents();
+
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int E2 = 2 * a.E;
@@ -65,7 +50,7 @@ __device__ __forceinline__ void topk_tokens(const TopkArgs &a, int tpb, int blk,
     const long long slab = (long long)a.T * E2;
     const bool vec = (E2 % 4 == 0) && (cols % 4 == 0);
 
-    for (int t0 = blk * tpb; t0 < a.T; t0 += nblk * tpb) {
+    for (int t0 = blockIdx.x * tpb; t0 < a.T; t0 += gridDim.x * tpb) {
         const int nt = min(tpb, a.T - t0);
         // ---- phase 1: split sums -> shared memory
         if (vec) {
@@ -173,18 +158,9 @@ __device__ __forceinline__ void topk_tokens(const TopkArgs &a, int tpb, int blk,
         }
         __syncthreads();  // s_logit is rewritten by the next tokens
     }
-}
-
-template <int EPL>
-__global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tpb) {
-    __shared__ TopkSmem sm;
-    topk_init(a, sm);
-    __syncthreads();
-    griddep_wait();
-    griddep_launch_dependents();
-    topk_tokens<EPL>(a, tpb, blockIdx.x, gridDim.x, sm);
-    __syncthreads();
-    topk_flush(a, sm);
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x)
+        if (s_counts[i]) atomicAdd(&a.counts[i], s_counts[i]);
+    if (a.hist && threadIdx.x <= a.K && s_hist[threadIdx.x]) atomicAdd(&a.hist[threadIdx.x], s_hist[threadIdx.x]);
 }
 
 // ----------------------------------------------------------------- permute --
@@ -209,23 +185,18 @@ __device__ __forceinline__ int block_sum_256(int v, int *s_red) {
     return total;
 }
 
-struct PermSmem {
-    int red[kPermThreads / 32];
-    int wcnt[4 * (kPermThreads / 32)];
-    int wpre[4 * (kPermThreads / 32)];
-    int total;
-};
-
-// Expert e's kept pairs in token order (whole block).  Counts and top-K
-// indices may come from other blocks of the same kernel: read through L2.
-__device__ __forceinline__ void permute_expert(const PermuteArgs &a, int e, PermSmem &sm) {
-    int *s_red = sm.red;
-    int *s_wcnt = sm.wcnt;
-    int *s_wpre = sm.wpre;
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs a) {
+    __shared__ int s_red[kPermThreads / 32];
+    __shared__ int s_wcnt[4 * (kPermThreads / 32)];
+    __shared__ int s_wpre[4 * (kPermThreads / 32)];
+    __shared__ int s_total;
+    const int e = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    griddep_launch_dependents();
 
     int c = 0;
-    if (tid < a.E) c = __ldcg(a.counts + tid);
+    if (tid < a.E) c = a.counts[tid];
     const int padded = (c + a.BN - 1) / a.BN * a.BN;
     const int ntile = (c + a.BN - 1) / a.BN;
     const int off_e = block_sum_256(tid < e ? padded : 0, s_red);
@@ -240,7 +211,7 @@ __device__ __forceinline__ void permute_expert(const PermuteArgs &a, int e, Perm
             a.meta[2] = tot_pairs;
         }
     }
-    const int count_e = __ldcg(a.counts + e);
+    const int count_e = a.counts[e];
 
     // Each pass covers kSub * 256 tokens as kSub coalesced sub-chunks (token
     // base + q * 256 + tid); ranks follow (sub-chunk, warp, lane), i.e. token
@@ -258,7 +229,7 @@ __device__ __forceinline__ void permute_expert(const PermuteArgs &a, int e, Perm
             if (t < a.T) {
                 const int *row = a.idx + (long long)t * a.K;
                 for (int k = 0; k < a.K; ++k)
-                    if (__ldcg(row + k) == e) km[q] = k;
+                    if (row[k] == e) km[q] = k;
             }
             bal[q] = __ballot_sync(kFull, km[q] >= 0);
             if (lane == 0) s_wcnt[q * kWarps + warp] = __popc(bal[q]);
@@ -270,7 +241,7 @@ __device__ __forceinline__ void permute_expert(const PermuteArgs &a, int e, Perm
                 s_wpre[i] = acc;
                 acc += s_wcnt[i];
             }
-            sm.total = acc;
+            s_total = acc;
         }
         __syncthreads();
 #pragma unroll
@@ -283,7 +254,7 @@ __device__ __forceinline__ void permute_expert(const PermuteArgs &a, int e, Perm
                 a.pair_pos[(long long)t * a.K + km[q]] = pos;
             }
         }
-        running += sm.total;
+        running += s_total;
         __syncthreads();
     }
     if (tid == 0 && running != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
@@ -296,25 +267,20 @@ __device__ __forceinline__ void permute_expert(const PermuteArgs &a, int e, Perm
         a.tiles[toff_e + j] = make_int4(e, off_e + j * a.BN, rows, 0);
         a.tile_done[toff_e + j] = 0;
     }
-    __syncthreads();  // the shared scratch is reused by the next expert
-}
-
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs a) {
-    __shared__ PermSmem sm;
-    griddep_wait();
-    griddep_launch_dependents();
-    permute_expert(a, blockIdx.x, sm);
 }
 
 // ------------------------------------------------------------------ gather --
 // One warp per permuted row, 16-byte vectors; padding rows are skipped (they
 // only feed padding columns of the GEMMs, which are never stored).
-// Rows warp_id, warp_id + nwarps, ... of the grouped layout (one warp each).
-__device__ __forceinline__ void gather_rows(const uint4 *x, const int *pair, int rows, int K,
-                                            int row_vec, uint4 *xp, int warp_id, int nwarps) {
+__global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *pair,
+                                                     const int *meta, int K, int row_vec,
+                                                     uint4 *xp) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int rows = meta[1];
     const int lane = threadIdx.x & 31;
-    for (int r = warp_id; r < rows; r += nwarps) {
-        const int pr = __ldcg(pair + r);
+    for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
+        const int pr = pair[r];
         if (pr < 0) continue;
         const uint4 *src = x + (long long)(pr / K) * row_vec;
         uint4 *dst = xp + (long long)r * row_vec;
@@ -329,77 +295,6 @@ __device__ __forceinline__ void gather_rows(const uint4 *x, const int *pair, int
         }
         for (; v < row_vec; v += 32) dst[v] = __ldg(src + v);
     }
-}
-
-__global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *pair,
-                                                     const int *meta, int K, int row_vec,
-                                                     uint4 *xp) {
-    griddep_wait();
-    griddep_launch_dependents();
-    gather_rows(x, pair, meta[1], K, row_vec, xp, blockIdx.x * 8 + (threadIdx.x >> 5),
-                gridDim.x * 8);
-}
-
-// ------------------------------------------------ route + group (fused) --
-// One cooperative launch of the forward pass: top-K + mask for every token,
-// then the grouping of every expert, then the row gather -- separated by
-// grid-wide barriers.  Every block of a cooperative launch is resident at
-// once, so the barriers cannot wait for a block that never runs; each wait
-// is still bounded (DEV_ERR_TIMEOUT, the block returns).  Same arithmetic as
-// the three separate kernels (shared device functions).
-
-// Bounded wait until *ctr >= need (acquire at GPU scope).
-__device__ __forceinline__ bool wait_ge_bounded(const int *ctr, int need,
-                                                unsigned long long timeout_ns) {
-    uint64_t t0 = 0;
-    for (uint32_t spin = 0; spin < (1u << 24); ++spin) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-        if (v >= need) return true;
-        if ((spin & 31u) == 0) {
-            const uint64_t t = globaltimer_ns();
-            if (spin == 0) t0 = t;
-            else if (t - t0 > timeout_ns) return false;
-        }
-        __nanosleep(64);
-    }
-    return false;
-}
-
-// Grid-wide barrier number `round` (1, 2, ...) on a counter that starts at 0.
-__device__ __forceinline__ bool grid_barrier(int *ctr, int round, int *err,
-                                             unsigned long long timeout_ns, int *s_ok) {
-    __threadfence();  // this thread's writes before the arrival
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        atomicAdd(ctr, 1);
-        const bool ok = wait_ge_bounded(ctr, round * int(gridDim.x), timeout_ns);
-        if (!ok) atomicExch(err, DEV_ERR_TIMEOUT);
-        *s_ok = ok ? 1 : 0;
-    }
-    __syncthreads();
-    return *s_ok != 0;
-}
-
-template <int EPL>
-__global__ void __launch_bounds__(256) route_group_kernel(const GroupArgs g) {
-    __shared__ TopkSmem tsm;
-    __shared__ PermSmem psm;
-    __shared__ int s_ok;
-    topk_init(g.t, tsm);
-    __syncthreads();
-    griddep_wait();
-    griddep_launch_dependents();
-    topk_tokens<EPL>(g.t, g.tpb, blockIdx.x, gridDim.x, tsm);
-    __syncthreads();
-    topk_flush(g.t, tsm);
-    if (!grid_barrier(g.bar, 1, g.p.err, g.timeout_ns, &s_ok)) return;
-    for (int e = blockIdx.x; e < g.p.E; e += gridDim.x) permute_expert(g.p, e, psm);
-    if (g.xp == nullptr) return;  // the expert kernels read the token rows themselves
-    if (!grid_barrier(g.bar, 2, g.p.err, g.timeout_ns, &s_ok)) return;
-    gather_rows(static_cast<const uint4 *>(g.x), g.p.pair, __ldcg(g.p.meta + 1), g.p.K,
-                g.row_vec, static_cast<uint4 *>(g.xp), blockIdx.x * 8 + (threadIdx.x >> 5),
-                gridDim.x * 8);
 }
 
 // ----------------------------------------------------------------- combine --
@@ -591,7 +486,8 @@ cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
     if (a.T <= 0) return cudaSuccess;
     // Tokens per block: one at decode sizes (more blocks, more loads in
     // flight), up to kTopkMaxTok for large batches.
-    const int tpb = topk_tokens_per_block(a.T);
+    int tpb = (a.T + 127) / 128;
+    if (tpb > kTopkMaxTok) tpb = kTopkMaxTok;
     int blocks = (a.T + tpb - 1) / tpb;
     if (blocks > 8 * n_sm) blocks = 8 * n_sm;
     const int epl = (a.E + 31) / 32;
@@ -602,44 +498,6 @@ cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
     if (epl <= 4)
         return launch_pdl(topk_mask_kernel<4>, dim3(blocks), dim3(256), 0, stream, a, tpb);
     return launch_pdl(topk_mask_kernel<8>, dim3(blocks), dim3(256), 0, stream, a, tpb);
-}
-
-template <int EPL>
-cudaError_t launch_group_epl(const GroupArgs &g, int need_blocks, int n_sm, cudaStream_t stream) {
-    auto kern = route_group_kernel<EPL>;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
-    if (e != cudaSuccess) return e;
-    if (per_sm <= 0) return cudaErrorInvalidConfiguration;
-    int blocks = need_blocks;
-    if (blocks > per_sm * n_sm) blocks = per_sm * n_sm;  // all resident at once
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, g);
-}
-
-cudaError_t launch_route_group(const GroupArgs &g, int n_sm, cudaStream_t stream) {
-    if (g.t.T <= 0) return cudaSuccess;
-    int need = (g.t.T + g.tpb - 1) / g.tpb;
-    if (need < g.p.E) need = g.p.E;
-    const int epl = (g.t.E + 31) / 32;
-    if (epl <= 1) return launch_group_epl<1>(g, need, n_sm, stream);
-    if (epl <= 2) return launch_group_epl<2>(g, need, n_sm, stream);
-    if (epl <= 4) return launch_group_epl<4>(g, need, n_sm, stream);
-    return launch_group_epl<8>(g, need, n_sm, stream);
-}
-
-int topk_tokens_per_block(int T) {
-    int tpb = (T + 127) / 128;
-    return tpb > kTopkMaxTok ? kTopkMaxTok : tpb;
 }
 
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {

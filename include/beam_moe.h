@@ -106,11 +106,9 @@ typedef struct {
 } beam_moe_plan_info;
 
 /* Stage slots of one beam_moe_forward call (router GEMM, top-K + mask,
- * grouping, gather, gate/up GEMM, down GEMM, combine).  beam_moe_forward runs
- * top-K + mask, grouping and gather as one cooperative launch in the top-K
- * slot (the grouping and gather slots are empty), and with token tiles
+ * grouping, gather, gate/up GEMM, down GEMM, combine).  With token tiles
  * thinner than 128 rows (decode batches) the two expert GEMMs run as one
- * fused launch in the gate/up slot (the down slot is empty); see
+ * fused launch in the gate/up slot and the down slot is empty; see
  * beam_moe_forward_kernel_count. */
 #define BEAM_MOE_FORWARD_STAGES 7
 
@@ -193,8 +191,8 @@ beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
                                    float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
                                    float *logits, void *stream);
 
-/* Kernel launches one beam_moe_forward call makes for `desc`: 4 (bf16 with
- * decode-sized token tiles) or 5; 0 for T = 0 or a bad descriptor. */
+/* Kernel launches one beam_moe_forward call makes for `desc` (6 or 7), or 0
+ * on a bad descriptor. */
 int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last

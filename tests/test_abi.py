@@ -106,9 +106,8 @@ def test_argument_errors_return_before_any_launch():
 
 
 def test_kernel_count_per_path():
-    # router, fused top-K/grouping/gather, fused experts, combine
-    assert abi.kernel_count(abi.desc(128, 2048, 128, 768, 8, "bf16", 1)) == 4
-    assert abi.kernel_count(abi.desc(8192, 2048, 128, 768, 8, "bf16", 1)) == 5
-    assert abi.kernel_count(abi.desc(64, 128, 8, 256, 2, "f32", 0)) == 5
+    assert abi.kernel_count(abi.desc(128, 2048, 128, 768, 8, "bf16", 1)) == 6  # fused experts
+    assert abi.kernel_count(abi.desc(8192, 2048, 128, 768, 8, "bf16", 1)) == 7
+    assert abi.kernel_count(abi.desc(64, 128, 8, 256, 2, "f32", 0)) == 7
     assert abi.kernel_count(abi.desc(0, 2048, 128, 768, 8, "bf16", 1)) == 0
     assert abi.kernel_count(abi.desc(4, 2000, 128, 768, 8, "bf16", 1)) == 0
