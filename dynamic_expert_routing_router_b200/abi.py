@@ -31,7 +31,7 @@ class BeamError(RuntimeError):
 class Desc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d", ctypes.c_int), ("E", ctypes.c_int),
                 ("I", ctypes.c_int), ("K", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("renorm_topk", ctypes.c_int)]
+                ("renorm_topk", ctypes.c_int), ("mask_logit_threshold", ctypes.c_float)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -81,9 +81,18 @@ def lib():
     return _lib
 
 
-def desc(T, d, E, I, K, dtype="bf16", renorm=1) -> Desc:
+def tau_logit(tau: float) -> float:
+    """The descriptor's mask threshold for sigmoid(z) >= tau, as stored (fp32)."""
+    import math
+    import numpy as np
+    return float(np.float32(math.log(tau / (1.0 - tau))))
+
+
+def desc(T, d, E, I, K, dtype="bf16", renorm=1, tau=0.5) -> Desc:
+    """Layer descriptor; `tau` is the mask threshold of sigmoid(x W_mask)."""
     code = dtype if isinstance(dtype, int) else (BEAM_BF16 if dtype == "bf16" else BEAM_F32)
-    return Desc(int(T), int(d), int(E), int(I), int(K), int(code), int(renorm))
+    return Desc(int(T), int(d), int(E), int(I), int(K), int(code), int(renorm),
+                tau_logit(tau) if tau != 0.5 else 0.0)
 
 
 def _ptr(t):

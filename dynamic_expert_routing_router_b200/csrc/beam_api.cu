@@ -32,6 +32,7 @@ beam_status validate_desc(const beam_moe_desc *d) {
     if (d->K > d->E || d->K > kMaxK || d->E > kMaxE) return BEAM_ERR_INVALID_ARG;
     if (d->dtype != BEAM_BF16 && d->dtype != BEAM_F32) return BEAM_ERR_INVALID_ARG;
     if (d->renorm_topk != 0 && d->renorm_topk != 1) return BEAM_ERR_INVALID_ARG;
+    if (d->mask_logit_threshold != d->mask_logit_threshold) return BEAM_ERR_INVALID_ARG;  // NaN
     if (d->dtype == BEAM_BF16) {
         if (d->d % kBlockM != 0 || d->I % kBlockM != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;
     } else {
@@ -225,6 +226,7 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
     t.K = d->K;
     t.renorm = d->renorm_topk;
     t.has_mask = Wm != nullptr;
+    t.thr = d->mask_logit_threshold;
     t.logits = ro.logits;
     t.idx = ro.idx;
     t.w = ro.w;

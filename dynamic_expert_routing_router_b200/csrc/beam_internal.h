@@ -91,6 +91,7 @@ cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArg
 struct TopkArgs {
     const float *partial;  // [S][T][2E]
     int S, T, E, K, renorm, has_mask;
+    float thr;             // keep iff z >= thr (logit of the threshold tau)
     float *logits;         // [T][2E] or NULL
     int *idx;              // [T][K]
     float *w;              // [T][K]

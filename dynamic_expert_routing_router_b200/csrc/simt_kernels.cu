@@ -27,8 +27,8 @@ constexpr unsigned kFull = 0xffffffffu;
 // warp per token; lane l holds the logits of experts l, l+32, ...  K rounds of
 // a warp arg-max (ties -> lower expert id) give the candidates in descending
 // order.  renorm: softmax over the candidates (Eq. 4); else over all E.  The
-// mask keeps candidate k iff its pre-sigmoid value z >= 0 (Eq. 6; NaN is not
-// kept); w = g * m (Eq. 7).  Counts and the histogram are gathered in shared
+// mask keeps candidate k iff its pre-sigmoid value z >= thr = logit(tau)
+// (Eq. 6, tau = 0.5 <=> thr = 0; NaN is not kept); w = g * m (Eq. 7).  Counts and the histogram are gathered in shared
 // memory and added to global memory once per block.
 constexpr int kTopkMaxTok = 8;
 
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
                 for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
                 denom = part;  // identical on every lane (pairwise sums commute exactly)
             }
-            const bool kept = (lane < a.K) && (!a.has_mask || my_z >= 0.0f);
+            const bool kept = (lane < a.K) && (!a.has_mask || my_z >= a.thr);
             if (lane < a.K) {
                 const float g = my_e / denom;
                 a.idx[(long long)t * a.K + lane] = kept ? my_cand : -1;

@@ -65,11 +65,18 @@ typedef enum { BEAM_BF16 = 0, BEAM_F32 = 1 } beam_dtype;
 
 /* One MoE layer call: T tokens of width d, E experts, top-K, SwiGLU width I.
  * renorm_topk = 1: softmax over the K largest logits (Eq. 4, sums to 1).
- * renorm_topk = 0: softmax over all E logits, restricted to the K largest. */
+ * renorm_topk = 0: softmax over all E logits, restricted to the K largest.
+ * mask_logit_threshold: the binarisation threshold tau of Eq. (6) given as
+ *   its logit, ln(tau / (1 - tau)); a candidate is kept iff its mask
+ *   pre-activation z >= mask_logit_threshold (i.e. sigmoid(z) >= tau).
+ *   0 is the paper's tau = 0.5, so a zero-initialised descriptor keeps the
+ *   method's default; other values reproduce the threshold ablation (news
+ *   article on BEAM, §8).  Must not be NaN. */
 typedef struct {
     int T, d, E, I, K;
     int dtype;       /* beam_dtype */
     int renorm_topk; /* 0 or 1 */
+    float mask_logit_threshold;
 } beam_moe_desc;
 
 /* Workspace layout chosen for a descriptor (byte offsets from the workspace

@@ -50,8 +50,9 @@ def _load():
         p = ctypes.c_void_p
         i = ctypes.c_int
         lib.oracle_logits.argtypes = [i, i, i, i, p, p, p, p, p]
-        lib.oracle_route.argtypes = [i, i, i, i, p, p, p, p, p, p, p, p]
-        lib.oracle_route_f32.argtypes = [i, i, i, i, p, p, p, p, p, p, p, p]
+        d = ctypes.c_double
+        lib.oracle_route.argtypes = [i, i, i, i, d, p, p, p, p, p, p, p, p]
+        lib.oracle_route_f32.argtypes = [i, i, i, i, d, p, p, p, p, p, p, p, p]
         lib.oracle_permutation.argtypes = [i, i, i, p, p, p]
         lib.oracle_experts.argtypes = [i, i, i, i, i, i, p, p, p, p, p, p, i, i, p, i]
         lib.oracle_max_threads.argtypes = []
@@ -108,11 +109,13 @@ def logits(x, W_gate, W_mask, dtype):
     return r, z
 
 
-def route(r, z, K, renorm):
+def route(r, z, K, renorm, tau_logit=0.0):
     """Top-K, softmax, binary mask and aggregation from given logits.
 
     ``r``/``z`` may be float64 (oracle logits) or float32 (another
-    implementation's exported logits, widened exactly).  Returns a dict with
+    implementation's exported logits, widened exactly).  ``tau_logit`` is the
+    mask threshold tau of Eq. (6) as its logit (0 = tau 0.5): a candidate is
+    kept iff sigmoid(z) >= tau, i.e. z >= tau_logit.  Returns a dict with
     cand, g, idx, w, counts, hist.
     """
     lib = _load()
@@ -130,7 +133,8 @@ def route(r, z, K, renorm):
         r = np.ascontiguousarray(r, dtype=np.float64)
         z = None if z is None else np.ascontiguousarray(z, dtype=np.float64)
         fn = lib.oracle_route
-    _check(fn(T, E, K, int(renorm), _ptr(r), _ptr(z), _ptr(out["cand"]), _ptr(out["g"]),
+    _check(fn(T, E, K, int(renorm), float(tau_logit), _ptr(r), _ptr(z), _ptr(out["cand"]),
+              _ptr(out["g"]),
               _ptr(out["idx"]), _ptr(out["w"]), _ptr(out["counts"]), _ptr(out["hist"])),
            "route")
     return out
@@ -169,9 +173,9 @@ def experts(x, W1, W3, W2, idx, w, dtype, t_begin=0, t_end=None, nthreads=0):
     return y
 
 
-def forward(x, W_gate, W_mask, W1, W3, W2, K, renorm, dtype, nthreads=0):
+def forward(x, W_gate, W_mask, W1, W3, W2, K, renorm, dtype, nthreads=0, tau_logit=0.0):
     """The whole layer: logits, routing, mask, experts.  Returns (y, route dict, r, z)."""
     r, z = logits(x, W_gate, W_mask, dtype)
-    rt = route(r, z, K, renorm)
+    rt = route(r, z, K, renorm, tau_logit)
     y = experts(x, W1, W3, W2, rt["idx"], rt["w"], dtype, nthreads=nthreads)
     return y, rt, r, z

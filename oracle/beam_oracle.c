@@ -71,17 +71,20 @@ int oracle_logits(int T, int d, int E, int dtype, const void *x, const void *W_g
  * break ties; candidates are listed by descending logit and an exact tie goes
  * to the lower expert index, which makes the selection unique.
  *
- * Eq. (5)-(6): m = 1 iff sigmoid(z) >= 0.5.  sigmoid is monotone with
- * sigmoid(0) = 0.5 exactly, so the test is taken on the pre-activation as
- * z >= 0 (READING: the news article's "index becomes -1 when the raw value is
- * <= 0" contradicts both Eq. (6) and the zero-initialisation claim that every
- * candidate is kept, so Eq. (6) wins; -0.0 counts as >= 0).
+ * Eq. (5)-(6): m = 1 iff sigmoid(z) >= tau, with tau = 0.5 in the method and
+ * other values in the threshold ablation (news article, §8).  sigmoid is
+ * increasing, so the test is taken on the pre-activation as z >= logit(tau),
+ * which the caller passes as tau_logit (0 for tau = 0.5, where sigmoid(0) =
+ * 0.5 exactly).  READING: the news article's "index becomes -1 when the raw
+ * value is <= 0" contradicts both Eq. (6) and the zero-initialisation claim
+ * that every candidate is kept, so Eq. (6) wins; -0.0 counts as >= 0.
  *
  * Eq. (7): w = g * m with no renormalisation after the mask. */
-int oracle_route(int T, int E, int K, int renorm, const double *r, const double *z,
-                 int32_t *cand, double *g, int32_t *idx, double *w, int32_t *counts,
-                 int32_t *hist) {
+int oracle_route(int T, int E, int K, int renorm, double tau_logit, const double *r,
+                 const double *z, int32_t *cand, double *g, int32_t *idx, double *w,
+                 int32_t *counts, int32_t *hist) {
     if (T < 0 || E <= 0 || K <= 0 || K > E || !r || !idx) return -1;
+    if (isnan(tau_logit)) return -1;
     if (counts) memset(counts, 0, sizeof(int32_t) * (size_t)E);
     if (hist) memset(hist, 0, sizeof(int32_t) * (size_t)(K + 1));
     char *taken = (char *)malloc((size_t)E);
@@ -124,7 +127,7 @@ int oracle_route(int T, int E, int K, int renorm, const double *r, const double 
             int mk = 1;
             if (z) {
                 double zz = z[(size_t)t * E + c[k]];
-                mk = (zz >= 0.0) ? 1 : 0; /* NaN compares false: not kept */
+                mk = (zz >= tau_logit) ? 1 : 0; /* NaN compares false: not kept */
             }
             size_t o = (size_t)t * K + k;
             if (cand) cand[o] = c[k];
@@ -144,9 +147,9 @@ int oracle_route(int T, int E, int K, int renorm, const double *r, const double 
     return rc;
 }
 
-int oracle_route_f32(int T, int E, int K, int renorm, const float *r, const float *z,
-                     int32_t *cand, double *g, int32_t *idx, double *w, int32_t *counts,
-                     int32_t *hist) {
+int oracle_route_f32(int T, int E, int K, int renorm, double tau_logit, const float *r,
+                     const float *z, int32_t *cand, double *g, int32_t *idx, double *w,
+                     int32_t *counts, int32_t *hist) {
     if (T < 0 || E <= 0 || !r) return -1;
     size_t n = (size_t)T * E;
     double *rd = (double *)malloc(sizeof(double) * (n ? n : 1));
@@ -156,7 +159,7 @@ int oracle_route_f32(int T, int E, int K, int renorm, const float *r, const floa
         rd[i] = (double)r[i];
         if (z) zd[i] = (double)z[i];
     }
-    int rc = oracle_route(T, E, K, renorm, rd, zd, cand, g, idx, w, counts, hist);
+    int rc = oracle_route(T, E, K, renorm, tau_logit, rd, zd, cand, g, idx, w, counts, hist);
     free(rd);
     free(zd);
     return rc;

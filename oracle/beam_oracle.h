@@ -35,6 +35,10 @@ int oracle_logits(int T, int d, int E, int dtype, const void *x, const void *W_g
 
 /* Routing decisions and weights from given logits, Eq. (4)-(7).
  * r [T,E]; z [T,E] or NULL (mask disabled: every candidate kept).
+ * tau_logit: the binarisation threshold tau of Eq. (6) given as its logit,
+ * ln(tau / (1 - tau)); 0 is the paper's tau = 0.5.  sigmoid(z) >= tau holds
+ * exactly when z >= tau_logit (sigmoid is increasing), so the test is taken on
+ * z and both implementations compare against the same number.
  * renorm = 1: softmax over the Top-K entries (Eq. 4).  renorm = 0: softmax
  * over all E logits, restricted to the Top-K.
  * Outputs (any may be NULL except idx):
@@ -44,15 +48,15 @@ int oracle_logits(int T, int d, int E, int dtype, const void *x, const void *W_g
  *   w    [T,K]   g * m (Eq. 7, no renormalisation after the mask)
  *   counts [E]   kept (token, expert) pairs per expert
  *   hist [K+1]   tokens by number of kept candidates */
-int oracle_route(int T, int E, int K, int renorm, const double *r, const double *z,
-                 int32_t *cand, double *g, int32_t *idx, double *w, int32_t *counts,
-                 int32_t *hist);
+int oracle_route(int T, int E, int K, int renorm, double tau_logit, const double *r,
+                 const double *z, int32_t *cand, double *g, int32_t *idx, double *w,
+                 int32_t *counts, int32_t *hist);
 
 /* Same decisions fed with fp32 logits (as exported by another implementation):
  * r, z are float [T,E]; they are widened exactly to double first. */
-int oracle_route_f32(int T, int E, int K, int renorm, const float *r, const float *z,
-                     int32_t *cand, double *g, int32_t *idx, double *w, int32_t *counts,
-                     int32_t *hist);
+int oracle_route_f32(int T, int E, int K, int renorm, double tau_logit, const float *r,
+                     const float *z, int32_t *cand, double *g, int32_t *idx, double *w,
+                     int32_t *counts, int32_t *hist);
 
 /* Expert-token grouping: kept pairs listed expert by expert (ascending), and
  * within an expert by token (ascending).  Each entry is t*K + k.

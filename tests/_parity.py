@@ -56,10 +56,10 @@ def gpu_forward(dsc, x, Wg, Wm, W1, W3, W2, ws=None):
     return out, ws
 
 
-def oracle_from_logits(logits, E, K, renorm, has_mask):
+def oracle_from_logits(logits, E, K, renorm, has_mask, tau_logit=0.0):
     r = np.ascontiguousarray(logits[:, :E])
     z = np.ascontiguousarray(logits[:, E:]) if has_mask else None
-    return oracle.route(r, z, K, renorm)
+    return oracle.route(r, z, K, renorm, tau_logit)
 
 
 def assert_routing_bitexact(g, o):

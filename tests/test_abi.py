@@ -111,3 +111,10 @@ def test_kernel_count_per_path():
     assert abi.kernel_count(abi.desc(64, 128, 8, 256, 2, "f32", 0)) == 7
     assert abi.kernel_count(abi.desc(0, 2048, 128, 768, 8, "bf16", 1)) == 0
     assert abi.kernel_count(abi.desc(4, 2000, 128, 768, 8, "bf16", 1)) == 0
+
+
+def test_nan_mask_threshold_is_rejected():
+    dsc = abi.desc(4, 2048, 128, 768, 8, "bf16", 1)
+    dsc.mask_logit_threshold = float("nan")
+    assert abi.workspace_size(dsc) == 0
+    assert abi.tau_logit(0.5) == 0.0 and abi.tau_logit(0.9) > 2.19

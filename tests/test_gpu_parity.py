@@ -239,6 +239,35 @@ def test_cuda_graph_replay_matches_eager(qwen3_experts):
     assert torch.equal(out, ref2)
 
 
+# ---------------------------------------------------- threshold ablation --
+
+@pytest.mark.parametrize("tau", [0.3, 0.7])
+def test_mask_threshold_tau_matches_oracle(tau, qwen3_experts, qwen3_experts_host):
+    """Eq. (6) with tau != 0.5 (the paper's threshold ablation): decisions
+    bit-exact with the oracle fed the same logits and the same fp32 threshold,
+    values within the bar, kept fraction ordered by tau."""
+    sh = inputs.QWEN3
+    W1, W3, W2 = qwen3_experts
+    T = 64
+    x = inputs.make_tokens(sh, T, seed=77, device=DEV)
+    Wg = inputs.make_gate(sh, seed=0, device=DEV)
+    Wm = inputs.make_mask(sh, 0.5, seed=0, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm, tau=tau)
+    thr = dsc.mask_logit_threshold
+    assert thr != 0.0
+    g = gpu_route(dsc, x, Wg, Wm)
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True, tau_logit=thr)
+    assert_routing_bitexact(g, o)
+    base = gpu_route(abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm), x, Wg, Wm)
+    kept, kept05 = (g["idx"] >= 0).sum(), (base["idx"] >= 0).sum()
+    assert (kept < kept05) if tau > 0.5 else (kept > kept05)
+    out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
+    assert_grouping_bitexact(dsc, abi.workspace_views(dsc, ws), g["idx"])
+    h1, h3, h2 = qwen3_experts_host
+    ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16", 0, 24)
+    assert_values(out, ref, g["idx"], "bf16", rows=slice(0, 24))
+
+
 # ----------------------------------------------------------- edge shapes --
 
 EDGE = [

@@ -329,3 +329,25 @@ def test_figure3_shaped_example_closed_form():
     feat = [silu(0.5) * 0.5, silu(-1.5) * (-1.5), 0.0]
     expect = [(g[0] * s[0] + g[2] * s[3]) * f for f in feat]
     np.testing.assert_allclose(y[0], expect, rtol=1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.3, 0.5, 0.7, 0.9])
+def test_threshold_ablation_matches_sigmoid(tau):
+    """The threshold ablation (news article §8: tau in 0.1 .. 0.9): a candidate
+    is kept iff sigmoid(z) >= tau.  The oracle takes tau as its logit; checked
+    against scipy's expit away from the boundary, and kept fractions fall as tau
+    rises.  Catches a threshold applied to g instead of z, or the wrong side."""
+    T, E, K = 400, 16, 4
+    r = RNG.standard_normal((T, E))
+    z = RNG.standard_normal((T, E)) * 3.0
+    tl = math.log(tau / (1.0 - tau))
+    out = oracle.route(r, z, K, renorm=1, tau_logit=tl)
+    zc = np.take_along_axis(z, out["cand"], axis=1)
+    sig = expit(zc)
+    clear = np.abs(sig - tau) > 1e-9
+    assert ((out["idx"] >= 0) == (sig >= tau))[clear].all()
+    lo = oracle.route(r, z, K, renorm=1, tau_logit=math.log(0.05 / 0.95))
+    hi = oracle.route(r, z, K, renorm=1, tau_logit=math.log(0.95 / 0.05))
+    assert (lo["idx"] >= 0).sum() >= (out["idx"] >= 0).sum() >= (hi["idx"] >= 0).sum()
+    if tau == 0.5:
+        assert np.array_equal(out["idx"], oracle.route(r, z, K, renorm=1)["idx"])
