@@ -354,6 +354,74 @@ def cpu_baseline(layer, f, seconds, max_batches=None):
                        f"only), {el:.1f} s")
 
 
+def stack_bench(device, rank, Ts=(1, 64, 256), replays=5):
+    """Decode through the 48-layer stack (one set of seeded weights per layer,
+    ~58 GB of experts): per T, the stack time with each layer's mask router
+    and with the mask disabled.  Each layer's input is recorded from one eager
+    pass of the real chain (previous output + N(0, 0.1^2) noise, RMS 1), so
+    the timed CUDA graph of 48 forward calls routes exactly as the chain does
+    while the harness's own noise kernels stay out of the timing."""
+    import torch
+    from dynamic_expert_routing_router_b200 import abi, inputs
+    sh = inputs.QWEN3
+    L = inputs.STACK_LAYERS
+    layers = []
+    for l in range(L):
+        W1, W3, W2 = inputs.make_experts(sh, seed=0, device=device, layer=l)
+        Wg = inputs.make_gate(sh, seed=0, device=device, layer=l)
+        Wm = inputs.make_mask(sh, inputs.stack_kept_fraction(l), seed=0, device=device, layer=l)
+        layers.append((Wg, Wm, W1, W3, W2))
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    rows = []
+    for T in Ts:
+        dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+        ws = abi.alloc_workspace(dsc, device)
+        out = torch.empty((T, sh.d), dtype=torch.bfloat16, device=device)
+        res = {}
+        for masked in (True, False):
+            xs, kept = [], []
+            x = inputs.make_tokens(sh, T, seed=2000 * (rank + 1) + T, device=device)
+            for l, (Wg, Wm, W1, W3, W2) in enumerate(layers):
+                xs.append(x)
+                abi.forward(dsc, x, Wg, Wm if masked else None, W1, W3, W2, out, ws)
+                kept.append(abi.workspace_views(dsc, ws)["counts"].sum())
+                x = inputs.stack_next_input(out, l)
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for l, (Wg, Wm, W1, W3, W2) in enumerate(layers):
+                        abi.forward(dsc, xs[l], Wg, Wm if masked else None, W1, W3, W2, out, ws,
+                                    stream=s)
+            torch.cuda.synchronize()
+            times = []
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for i in range(replays + 1):
+                flush.fill_(i & 255)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                if i:
+                    times.append(e0.elapsed_time(e1) * 1e-3)
+            abi.check(dsc, ws)
+            del g
+            res[masked] = (sum(times) / len(times),
+                           float(torch.stack(kept).sum().item()) / (L * T * sh.K))
+        tm, fm = res[True]
+        tu, _ = res[False]
+        rows.append(dict(T=T, layers=L, us_per_stack=tm * 1e6, us_per_layer=tm / L * 1e6,
+                         tokens_per_s=T / tm, unmasked_us_per_stack=tu * 1e6,
+                         unmasked_tokens_per_s=T / tu, speedup_vs_unmasked=tu / tm,
+                         kept_fraction_mean=fm))
+    del layers
+    torch.cuda.empty_cache()
+    return dict(rows=rows, weights_gb=round(L * 3 * sh.E * sh.I * sh.d * 2 / 1e9, 1),
+                note="per-layer kept fractions drawn in [0.10, 0.60]; graph of 48 forwards")
+
+
 def run_beam(args):
     import torch
     rank, world, local = dist_env()
@@ -449,6 +517,10 @@ def run_beam(args):
 
     e2e = e2e_rate(layer, f_head, max(20, min(args.steps, 500)), 5)
 
+    stack = None
+    if not args.no_stack:
+        stack = stack_bench(device, rank)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(layer, f_head, args.cpu_seconds)
@@ -479,6 +551,7 @@ def run_beam(args):
                          f"graph: {prof_mean * 1e6:.1f} us/step vs {step_mean * 1e6:.1f} "
                          "without them)"),
         "per_kept_fraction": sweep,
+        "stack_48_layers": stack,
         "e2e": e2e,
         "gpu_launches": n_kernels * args.steps,
         "clocks": clocks,
@@ -545,6 +618,7 @@ def main(argv=None):
     ap.add_argument("--T", type=int, default=128)
     ap.add_argument("--kept", type=float, default=0.15)
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--sweep-steps", type=int, default=100)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

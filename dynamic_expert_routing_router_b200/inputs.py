@@ -158,3 +158,29 @@ def host_array(t: torch.Tensor):
     if t.dtype == torch.bfloat16:
         return bf16_bits(t)
     return t.detach().contiguous().cpu().to(torch.float32).numpy()
+
+
+# ------------------------------------------------------- 48-layer stack --
+# Decode through a stack of independent Qwen3-shaped layers: each layer has its
+# own seeded weights (seed + 1000 * layer) and its own mask router, drawn for a
+# kept fraction in [0.10, 0.60].  The next layer's input is the previous
+# layer's output plus N(0, 0.1^2) noise, rescaled to RMS 1 (the RMSNorm in
+# front of every MoE layer of these models) with the bias feature restored.
+STACK_LAYERS = 48
+_OFF_STACK_F, _OFF_STACK_NOISE = 9, 10
+
+
+def stack_kept_fraction(layer: int, seed: int = 0) -> float:
+    g = _gen("cpu", seed + layer * _LAYER_STRIDE + _OFF_STACK_F)
+    return float(0.10 + 0.50 * torch.rand((), generator=g).item())
+
+
+def stack_next_input(out: torch.Tensor, layer: int, seed: int = 0):
+    """Input of layer `layer` + 1 from the output of layer `layer`."""
+    noise = _normal(tuple(out.shape), 0.1, seed + layer * _LAYER_STRIDE + _OFF_STACK_NOISE,
+                    out.device, torch.float32)
+    x = out.float() + noise
+    if x.shape[0]:
+        x = x / x.pow(2).mean(dim=1, keepdim=True).sqrt().clamp_min(1e-6)
+    x[:, x.shape[1] - 1] = 1.0
+    return x.to(out.dtype)

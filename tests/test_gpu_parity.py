@@ -342,3 +342,36 @@ def large_layer():
     yield W1, W3, W2, Wg
     del W1, W3, W2
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------ 48-layer stack --
+
+def test_48_layer_decode_stack_matches_oracle():
+    """The 48-layer stack (48 x 1.2 GB of expert weights on the GPU): every
+    layer's routing is bit-exact with the oracle fed that layer's logits, and
+    every eighth layer's outputs match the oracle on sampled tokens, each layer
+    fed the GPU's own input (teacher forcing)."""
+    sh = inputs.QWEN3
+    T = 64
+    x = inputs.make_tokens(sh, T, seed=501, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    ws = abi.alloc_workspace(dsc, DEV)
+    kept = []
+    for layer in range(inputs.STACK_LAYERS):
+        W1, W3, W2 = inputs.make_experts(sh, seed=0, device=DEV, layer=layer)
+        Wg = inputs.make_gate(sh, seed=0, device=DEV, layer=layer)
+        Wm = inputs.make_mask(sh, inputs.stack_kept_fraction(layer), seed=0, device=DEV,
+                              layer=layer)
+        g = gpu_route(dsc, x, Wg, Wm)
+        o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
+        assert_routing_bitexact(g, o)
+        out, _ = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2, ws=ws)
+        if layer % 8 == 7:
+            n = 4
+            c1, c3, c2, cidx = compact_experts(W1, W3, W2, g["idx"][:n])
+            ref = oracle.experts(host(x[:n]), c1, c3, c2, cidx, o["w"][:n], "bf16")
+            assert_values(out, ref, g["idx"], "bf16", rows=slice(0, n))
+        kept.append((g["idx"] >= 0).mean())
+        x = inputs.stack_next_input(out, layer)
+        del W1, W3, W2
+    assert 0.05 < min(kept) and max(kept) < 0.7, kept
