@@ -56,8 +56,10 @@ def _load():
         lib.oracle_permutation.argtypes = [i, i, i, p, p, p]
         lib.oracle_experts.argtypes = [i, i, i, i, i, i, p, p, p, p, p, p, i, i, p, i]
         lib.oracle_max_threads.argtypes = []
+        lib.oracle_shared_experts.argtypes = [i, i, i, i, i, p, p, p, p, i, i, p, i]
         for f in (lib.oracle_logits, lib.oracle_route, lib.oracle_route_f32,
-                  lib.oracle_permutation, lib.oracle_experts, lib.oracle_max_threads):
+                  lib.oracle_permutation, lib.oracle_experts, lib.oracle_max_threads,
+                  lib.oracle_shared_experts):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -173,9 +175,32 @@ def experts(x, W1, W3, W2, idx, w, dtype, t_begin=0, t_end=None, nthreads=0):
     return y
 
 
-def forward(x, W_gate, W_mask, W1, W3, W2, K, renorm, dtype, nthreads=0, tau_logit=0.0):
-    """The whole layer: logits, routing, mask, experts.  Returns (y, route dict, r, z)."""
+def add_shared(y, x, W1s, W3s, W2s, dtype, t_begin=0, t_end=None, nthreads=0):
+    """y[t - t_begin] += sum_s SwiGLU shared expert s applied to x[t] (weight 1)."""
+    lib = _load()
+    x = _storage(x, dtype)
+    W1s, W3s, W2s = _storage(W1s, dtype), _storage(W3s, dtype), _storage(W2s, dtype)
+    T, d = x.shape
+    S, Is, d1 = W1s.shape
+    if d1 != d or W3s.shape != W1s.shape or W2s.shape != (S, d, Is):
+        raise ValueError("shared weights must be W1s,W3s [S,Is,d] and W2s [S,d,Is]")
+    if t_end is None:
+        t_end = T
+    if y.shape != (t_end - t_begin, d) or y.dtype != np.float64 or not y.flags.c_contiguous:
+        raise ValueError("y must be a contiguous float64 [t_end - t_begin, d] array")
+    _check(lib.oracle_shared_experts(T, d, S, Is, _code(dtype), _ptr(x), _ptr(W1s), _ptr(W3s),
+                                     _ptr(W2s), t_begin, t_end, _ptr(y), int(nthreads)),
+           "shared experts")
+    return y
+
+
+def forward(x, W_gate, W_mask, W1, W3, W2, K, renorm, dtype, nthreads=0, tau_logit=0.0,
+            shared=None):
+    """The whole layer: logits, routing, mask, experts (+ shared experts given as
+    (W1s, W3s, W2s)).  Returns (y, route dict, r, z)."""
     r, z = logits(x, W_gate, W_mask, dtype)
     rt = route(r, z, K, renorm, tau_logit)
     y = experts(x, W1, W3, W2, rt["idx"], rt["w"], dtype, nthreads=nthreads)
+    if shared is not None:
+        add_shared(y, x, *shared, dtype, nthreads=nthreads)
     return y, rt, r, z

@@ -245,3 +245,55 @@ int oracle_experts(int T, int d, int E, int I, int K, int dtype, const void *x,
     if (bad == 2 || bad == 3) return -2;
     return bad ? -1 : 0;
 }
+
+/* Shared experts: every token, weight 1, after the routed sum (see header). */
+int oracle_shared_experts(int T, int d, int n_shared, int Is, int dtype, const void *x,
+                          const void *W1s, const void *W3s, const void *W2s, int t_begin,
+                          int t_end, double *y, int nthreads) {
+    if (T < 0 || d <= 0 || n_shared < 0 || (n_shared > 0 && Is <= 0)) return -1;
+    if (n_shared == 0) return 0;
+    if (!x || !W1s || !W3s || !W2s || !y) return -1;
+    if (t_begin < 0 || t_end > T || t_begin > t_end) return -1;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_F32) return -1;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#else
+    nthreads = 1;
+#endif
+    int bad = 0;
+#pragma omp parallel num_threads(nthreads) reduction(| : bad)
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *h = (double *)malloc(sizeof(double) * (size_t)Is);
+        if (!xt || !h) bad = 1;
+#pragma omp for schedule(dynamic, 1)
+        for (int t = t_begin; t < t_end; ++t) {
+            if (!xt || !h) continue;
+            double *yt = y + (size_t)(t - t_begin) * d;
+            for (int j = 0; j < d; ++j) xt[j] = load_elem(x, dtype, (size_t)t * d + j);
+            for (int s = 0; s < n_shared; ++s) {
+                for (int i = 0; i < Is; ++i) {
+                    size_t row = ((size_t)s * Is + i) * d;
+                    double a = 0.0, b = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        a += xt[j] * load_elem(W1s, dtype, row + j);
+                        b += xt[j] * load_elem(W3s, dtype, row + j);
+                    }
+                    h[i] = a / (1.0 + exp(-a)) * b;
+                }
+                for (int j = 0; j < d; ++j) {
+                    size_t row = ((size_t)s * d + j) * Is;
+                    double acc = 0.0;
+                    for (int i = 0; i < Is; ++i) acc += h[i] * load_elem(W2s, dtype, row + i);
+                    yt[j] += acc;
+                }
+            }
+            for (int j = 0; j < d; ++j)
+                if (!isfinite(yt[j])) bad = 2;
+        }
+        free(xt);
+        free(h);
+    }
+    if (bad == 2 || bad == 3) return -2;
+    return bad ? -1 : 0;
+}

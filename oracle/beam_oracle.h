@@ -73,6 +73,15 @@ int oracle_experts(int T, int d, int E, int I, int K, int dtype, const void *x,
                    const void *W1, const void *W3, const void *W2, const int32_t *idx,
                    const double *w, int t_begin, int t_end, double *y, int nthreads);
 
+/* Shared experts (news article on BEAM, §5: models with always-on shared
+ * experts keep running them for every token, all-masked ones included).
+ * READING: each of the n_shared SwiGLU experts is added with weight 1 after
+ * the routed sum.  W1s, W3s [n_shared, Is, d]; W2s [n_shared, d, Is].
+ * Adds sum_s E_s(x_t) to y[t - t_begin] for t in [t_begin, t_end). */
+int oracle_shared_experts(int T, int d, int n_shared, int Is, int dtype, const void *x,
+                          const void *W1s, const void *W3s, const void *W2s, int t_begin,
+                          int t_end, double *y, int nthreads);
+
 /* Threads the OpenMP runtime would use by default (for reporting). */
 int oracle_max_threads(void);
 

@@ -351,3 +351,29 @@ def test_threshold_ablation_matches_sigmoid(tau):
     assert (lo["idx"] >= 0).sum() >= (out["idx"] >= 0).sum() >= (hi["idx"] >= 0).sum()
     if tau == 0.5:
         assert np.array_equal(out["idx"], oracle.route(r, z, K, renorm=1)["idx"])
+
+
+def test_shared_experts_run_for_every_token_with_weight_one():
+    """Shared experts (news article §5): always on, all-masked tokens
+    included.  With every candidate masked the layer output is exactly the sum
+    of the shared experts (numpy fp64); with a mask the shared part is the same
+    whatever the routed part is.  Catches shared experts skipped for
+    all-masked tokens, or scaled by a router weight."""
+    T, d, E, I, K, S, Is = 9, 16, 6, 12, 2, 3, 20
+    x, Wg, _, W1, W3, W2 = _rand_layer(T, d, E, I, RNG)
+    W1s = (RNG.standard_normal((S, Is, d)) / math.sqrt(d)).astype(np.float32)
+    W3s = (RNG.standard_normal((S, Is, d)) / math.sqrt(d)).astype(np.float32)
+    W2s = (RNG.standard_normal((S, d, Is)) / math.sqrt(Is)).astype(np.float32)
+    x = np.abs(x) + 0.1
+    Wm_all = -np.ones((E, d), np.float32)  # z = -sum(x) < 0: every candidate masked
+    y, rt, _, _ = oracle.forward(x, Wg, Wm_all, W1, W3, W2, K, 1, "f32",
+                                 shared=(W1s, W3s, W2s))
+    assert (rt["idx"] == -1).all()
+    ref = sum(_dense_expert(x, W1s, W3s, W2s, s) for s in range(S))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-13)
+    # routed + shared = routed alone + shared alone, for a partly kept mask
+    Wm = (RNG.standard_normal((E, d)) / math.sqrt(d)).astype(np.float32)
+    yr, rt2, _, _ = oracle.forward(x, Wg, Wm, W1, W3, W2, K, 1, "f32")
+    ys, _, _, _ = oracle.forward(x, Wg, Wm, W1, W3, W2, K, 1, "f32", shared=(W1s, W3s, W2s))
+    assert 0 < (rt2["idx"] >= 0).sum() < T * K
+    np.testing.assert_allclose(ys - yr, ref, rtol=1e-11, atol=1e-12)
