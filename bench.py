@@ -422,6 +422,75 @@ def stack_bench(device, rank, Ts=(1, 64, 256), replays=5):
                 note="per-layer kept fractions drawn in [0.10, 0.60]; graph of 48 forwards")
 
 
+def shared_bench(device, rank, Ts=(1, 128), steps=100, warmup=5):
+    """Decode layers with always-on shared experts (DeepSeekV2-Lite shape: E=64,
+    top-6, 2 shared; Qwen1.5-MoE shape: E=60, top-4, 4 shared; d=2048,
+    I=1408): per T, the layer time with the mask off, at ~15% kept, and with
+    every candidate masked (the floor: router + shared experts only)."""
+    import torch
+    from dynamic_expert_routing_router_b200 import abi, inputs
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    rows = []
+    for name, sh, S in (("deepseek_v2_lite_shape", inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED),
+                        ("qwen1.5_moe_shape", inputs.QWEN15_MOE, inputs.QWEN15_MOE_SHARED)):
+        W1, W3, W2 = inputs.make_experts(sh, seed=0, device=device)
+        W1s, W3s, W2s = inputs.make_shared_experts(sh, S, seed=0, device=device)
+        Wg = inputs.make_gate(sh, seed=0, device=device)
+        masks = {f: inputs.make_mask(sh, f, seed=0, device=device) for f in (0.15, 0.0)}
+        masks[None] = None
+        for T in Ts:
+            dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm, n_shared=S, I_shared=sh.I)
+            ws = abi.alloc_workspace(dsc, device)
+            out = torch.empty((T, sh.d), dtype=torch.bfloat16, device=device)
+            xs = [inputs.make_tokens(sh, T, seed=3000 * (rank + 1) + b, device=device)
+                  for b in range(N_BATCHES)]
+            res = {}
+            for f in (None, 0.15, 0.0):
+                kept = []
+                for x in xs:
+                    abi.forward_shared(dsc, x, Wg, masks[f], W1, W3, W2, W1s, W3s, W2s, out, ws)
+                    kept.append(abi.workspace_views(dsc, ws)["counts"].sum())
+                torch.cuda.synchronize()
+                s = torch.cuda.Stream()
+                s.wait_stream(torch.cuda.current_stream())
+                graphs = []
+                with torch.cuda.stream(s):
+                    for x in xs:
+                        g = torch.cuda.CUDAGraph()
+                        with torch.cuda.graph(g, stream=s):
+                            abi.forward_shared(dsc, x, Wg, masks[f], W1, W3, W2, W1s, W3s, W2s,
+                                               out, ws, stream=s)
+                        graphs.append(g)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                times = []
+                for i in range(warmup + steps):
+                    flush.fill_(i & 255)
+                    e0.record()
+                    graphs[i % N_BATCHES].replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    if i >= warmup:
+                        times.append(e0.elapsed_time(e1) * 1e-3)
+                abi.check(dsc, ws)
+                del graphs
+                res[f] = (sum(times) / len(times),
+                          float(torch.stack(kept).sum().item()) / (N_BATCHES * T * sh.K))
+            tu = res[None][0]
+            for f in (None, 0.15, 0.0):
+                t, kf = res[f]
+                row = dict(layer=name, n_shared=S, T=T,
+                           kept_target="unmasked" if f is None else f,
+                           kept_measured=round(kf, 4), us_per_layer=t * 1e6, tokens_per_s=T / t)
+                if f is not None:
+                    row["speedup_vs_unmasked"] = tu / t
+                rows.append(row)
+        del W1, W3, W2, W1s, W3s, W2s
+    torch.cuda.empty_cache()
+    return dict(rows=rows, note=("shared experts run for every token with weight 1 after the "
+                                 "routed sum; kept_target 0 = every candidate masked"))
+
+
 def run_beam(args):
     import torch
     rank, world, local = dist_env()
@@ -521,6 +590,10 @@ def run_beam(args):
     if not args.no_stack:
         stack = stack_bench(device, rank)
 
+    shared = None
+    if not args.no_shared:
+        shared = shared_bench(device, rank, steps=args.sweep_steps)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(layer, f_head, args.cpu_seconds)
@@ -552,6 +625,7 @@ def run_beam(args):
                          "without them)"),
         "per_kept_fraction": sweep,
         "stack_48_layers": stack,
+        "shared_experts": shared,
         "e2e": e2e,
         "gpu_launches": n_kernels * args.steps,
         "clocks": clocks,
@@ -619,6 +693,7 @@ def main(argv=None):
     ap.add_argument("--kept", type=float, default=0.15)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--no-shared", action="store_true")
     ap.add_argument("--sweep-steps", type=int, default=100)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -31,7 +31,8 @@ class BeamError(RuntimeError):
 class Desc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d", ctypes.c_int), ("E", ctypes.c_int),
                 ("I", ctypes.c_int), ("K", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("renorm_topk", ctypes.c_int), ("mask_logit_threshold", ctypes.c_float)]
+                ("renorm_topk", ctypes.c_int), ("mask_logit_threshold", ctypes.c_float),
+                ("n_shared", ctypes.c_int), ("I_shared", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -41,7 +42,7 @@ class PlanInfo(ctypes.Structure):
                [(n, ctypes.c_size_t) for n in (
                    "off_err", "off_meta", "off_counts", "off_hist", "off_partial", "off_idx",
                    "off_w", "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h", "off_y",
-                   "off_tile_done", "workspace_bytes")]
+                   "off_tile_done", "off_hs", "off_ys", "workspace_bytes")]
 
 
 _lib = None
@@ -63,6 +64,9 @@ def lib():
         L.beam_moe_plan.argtypes = [pd, ctypes.POINTER(PlanInfo)]
         L.beam_moe_route.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.beam_moe_forward.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.beam_moe_forward_shared.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                              vp]
+        L.beam_moe_forward_shared.restype = i32
         L.beam_moe_forward_profiled.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                 ctypes.POINTER(vp)]
         L.beam_moe_check.argtypes = [pd, vp, vp]
@@ -88,11 +92,12 @@ def tau_logit(tau: float) -> float:
     return float(np.float32(math.log(tau / (1.0 - tau))))
 
 
-def desc(T, d, E, I, K, dtype="bf16", renorm=1, tau=0.5) -> Desc:
-    """Layer descriptor; `tau` is the mask threshold of sigmoid(x W_mask)."""
+def desc(T, d, E, I, K, dtype="bf16", renorm=1, tau=0.5, n_shared=0, I_shared=0) -> Desc:
+    """Layer descriptor; `tau` is the mask threshold of sigmoid(x W_mask);
+    n_shared always-on shared experts of width I_shared."""
     code = dtype if isinstance(dtype, int) else (BEAM_BF16 if dtype == "bf16" else BEAM_F32)
     return Desc(int(T), int(d), int(E), int(I), int(K), int(code), int(renorm),
-                tau_logit(tau) if tau != 0.5 else 0.0)
+                tau_logit(tau) if tau != 0.5 else 0.0, int(n_shared), int(I_shared))
 
 
 def _ptr(t):
@@ -175,6 +180,16 @@ def forward(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, stream=None):
     _ok(lib().beam_moe_forward(ctypes.byref(dsc), _ptr(x), _ptr(W_gate), _ptr(W_mask),
                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), _ptr(workspace),
                                workspace.numel(), _stream(stream)), "beam_moe_forward")
+
+
+def forward_shared(dsc, x, W_gate, W_mask, W1, W3, W2, W1s, W3s, W2s, out, workspace,
+                   stream=None):
+    """The layer with dsc.n_shared always-on shared experts (weights W1s, W3s
+    [S, I_shared, d], W2s [S, d, I_shared])."""
+    _ok(lib().beam_moe_forward_shared(ctypes.byref(dsc), _ptr(x), _ptr(W_gate), _ptr(W_mask),
+                                      _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s), _ptr(W3s),
+                                      _ptr(W2s), _ptr(out), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)), "beam_moe_forward_shared")
 
 
 def forward_profiled(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, events, stream=None):

@@ -39,8 +39,18 @@ beam_status validate_desc(const beam_moe_desc *d) {
         if (d->d % 8 != 0 || d->I % 8 != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;
     }
     if ((long long)d->T * d->K > INT_MAX / 2) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    if (d->n_shared < 0 || d->n_shared > kMaxShared) return BEAM_ERR_INVALID_ARG;
+    if (d->n_shared > 0) {
+        if (d->I_shared <= 0) return BEAM_ERR_INVALID_ARG;
+        if (d->dtype != BEAM_BF16 || d->I_shared % kBlockM != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;
+        if ((long long)d->n_shared * d->T > INT_MAX / 2) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    }
     return BEAM_OK;
 }
+
+// Token-tile height of the shared experts' GEMMs (every token, every shared
+// expert): thin tiles spread a decode batch's weight stream over more SMs.
+int shared_bn(int T) { return T <= 16 ? 16 : T <= 256 ? 32 : 128; }
 
 // Token-tile height of the expert GEMMs from the mean kept-or-not pairs per
 // expert (T*K/E): decode batches use thin tiles, prefill batches 128 rows.
@@ -98,7 +108,10 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
     P->off_h = align256(P->off_xp + es * size_t(p_cap) * size_t(d->d));
     P->off_y = align256(P->off_h + es * size_t(p_cap) * size_t(d->I));
     P->off_tile_done = align256(P->off_y + 4 * size_t(p_cap) * size_t(d->d));  // Y is fp32
-    o = align256(P->off_tile_done + 4 * size_t(tiles_cap));
+    const size_t srows = size_t(d->n_shared) * size_t(T);  // shared rows: every token
+    P->off_hs = align256(P->off_tile_done + 4 * size_t(tiles_cap));
+    P->off_ys = align256(P->off_hs + es * srows * size_t(d->n_shared > 0 ? d->I_shared : 0));
+    o = align256(P->off_ys + 4 * srows * size_t(d->d));
     P->workspace_bytes = o;
     return BEAM_OK;
 }
@@ -244,7 +257,8 @@ beam_status check_ws(const beam_moe_plan_info &P, const void *ws, size_t bytes) 
 }
 
 beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, const void *Wm,
-                         const void *W1, const void *W3, const void *W2, void *out, void *workspace,
+                         const void *W1, const void *W3, const void *W2, const void *W1s,
+                         const void *W3s, const void *W2s, void *out, void *workspace,
                          size_t ws_bytes, void *stream, void *const *events) {
     beam_moe_plan_info P;
     beam_status s = make_plan(d, &P);
@@ -252,6 +266,11 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     if (!x || !Wg || !W1 || !W3 || !W2 || !out) return BEAM_ERR_INVALID_ARG;
     for (const void *p : {x, Wg, W1, W3, W2, static_cast<const void *>(out)})
         if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    if (d->n_shared > 0) {
+        if (!W1s || !W3s || !W2s) return BEAM_ERR_INVALID_ARG;
+        for (const void *p : {W1s, W3s, W2s})
+            if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    }
     if (Wm && !aligned16(Wm)) return BEAM_ERR_INVALID_ARG;
     s = check_ws(P, workspace, ws_bytes);
     if (s != BEAM_OK) return s;
@@ -357,8 +376,54 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
                                        tiles, meta, P.tiles_cap, d->d, d->I, y, st));
     }
 
+    float *ys = reinterpret_cast<float *>(ws + P.off_ys);
+    if (d->n_shared > 0) {
+        // Shared experts over every token (two dense launches; no grouping).
+        const int bn = shared_bn(d->T);
+        const int ntt = int(cdiv(d->T, bn));
+        void *hs = ws + P.off_hs;
+        const unsigned long long srows = (unsigned long long)d->n_shared * d->T;
+        TcMaps m1, m2;
+        if (!make_tmap(&m1.a0, W1s, d->d, (unsigned long long)d->n_shared * d->I_shared, kBlockM))
+            return BEAM_ERR_CUDA;
+        if (!make_tmap(&m1.a1, W3s, d->d, (unsigned long long)d->n_shared * d->I_shared, kBlockM))
+            return BEAM_ERR_CUDA;
+        if (!make_tmap(&m1.b, x, d->d, d->T, bn)) return BEAM_ERR_CUDA;
+        m1.a2 = m1.a0;
+        m1.b2 = m1.b;
+        if (!make_tmap(&m2.a0, W2s, d->I_shared, (unsigned long long)d->n_shared * d->d, kBlockM))
+            return BEAM_ERR_CUDA;
+        if (!make_tmap(&m2.b, hs, d->I_shared, srows, bn)) return BEAM_ERR_CUDA;
+        m2.a1 = m2.a0;
+        m2.a2 = m2.a0;
+        m2.b2 = m2.b;
+        TcGemmArgs g;
+        std::memset(&g, 0, sizeof(g));
+        g.err = err;
+        g.timeout_ns = kWaitTimeoutNs;
+        g.dense = 1;
+        g.dense_ntt = ntt;
+        g.dense_T = d->T;
+        g.n_mb = d->I_shared / kBlockM;
+        g.nk = d->d / kBlockK;
+        g.a_rows_per_expert = d->I_shared;
+        g.n_units = d->n_shared * ntt * g.n_mb;
+        g.out = hs;
+        g.out_ld = d->I_shared;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, bn, m1, g, g.n_units < n_sm ? g.n_units : n_sm, st));
+        g.dense_gemm2 = 1;
+        g.n_mb = d->d / kBlockM;
+        g.nk = d->I_shared / kBlockK;
+        g.a_rows_per_expert = d->d;
+        g.n_units = d->n_shared * ntt * g.n_mb;
+        g.out = ys;
+        g.out_ld = d->d;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, bn, m2, g, g.n_units < n_sm ? g.n_units : n_sm, st));
+    }
+
     BEAM_TRY_CUDA(rec.rec(6));
-    BEAM_TRY_CUDA(launch_combine(d->dtype, y, idx, w, pair_pos, d->T, d->K, d->d, out, n_sm, st));
+    BEAM_TRY_CUDA(launch_combine(d->dtype, y, idx, w, pair_pos, d->T, d->K, d->d, ys,
+                                 d->n_shared, out, n_sm, st));
     BEAM_TRY_CUDA(rec.rec(7));
     return BEAM_OK;
 }
@@ -459,8 +524,18 @@ beam_status beam_moe_route(const beam_moe_desc *desc, const void *x, const void 
 beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const void *W_gate,
                              const void *W_mask, const void *W1, const void *W3, const void *W2,
                              void *out, void *workspace, size_t workspace_bytes, void *stream) {
-    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, out, workspace, workspace_bytes,
-                        stream, nullptr);
+    if (desc && desc->n_shared != 0) return BEAM_ERR_INVALID_ARG;  // needs the shared weights
+    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, nullptr, nullptr, nullptr, out,
+                        workspace, workspace_bytes, stream, nullptr);
+}
+
+beam_status beam_moe_forward_shared(const beam_moe_desc *desc, const void *x,
+                                    const void *W_gate, const void *W_mask, const void *W1,
+                                    const void *W3, const void *W2, const void *W1s,
+                                    const void *W3s, const void *W2s, void *out,
+                                    void *workspace, size_t workspace_bytes, void *stream) {
+    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, W1s, W3s, W2s, out, workspace,
+                        workspace_bytes, stream, nullptr);
 }
 
 beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
@@ -469,8 +544,9 @@ beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
                                       size_t workspace_bytes, void *stream,
                                       void *const *events) {
     if (!events) return BEAM_ERR_INVALID_ARG;
-    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, out, workspace, workspace_bytes,
-                        stream, events);
+    if (desc && desc->n_shared != 0) return BEAM_ERR_INVALID_ARG;
+    return forward_impl(desc, x, W_gate, W_mask, W1, W3, W2, nullptr, nullptr, nullptr, out,
+                        workspace, workspace_bytes, stream, events);
 }
 
 beam_status beam_moe_check(const beam_moe_desc *desc, void *workspace, void *stream) {
@@ -506,8 +582,9 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     beam_moe_plan_info P;
     if (make_plan(desc, &P) != BEAM_OK) return 0;
     if (desc->T == 0) return 0;
-    return (desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 1
-                                                          : BEAM_MOE_FORWARD_STAGES;
+    const int shared = desc->n_shared > 0 ? 2 : 0;
+    return shared + ((desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 1
+                                                                     : BEAM_MOE_FORWARD_STAGES);
 }
 
 const char *beam_moe_stage_name(int stage) {

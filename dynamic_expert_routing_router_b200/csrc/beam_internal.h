@@ -33,7 +33,8 @@ constexpr int kBlockK = 64;    // reduction elements per stage: one 128-byte bf1
 constexpr int kNominalSMs = 148;
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 16;
-constexpr int kMaxRouterSplits = 32;  // top-K sums the split partials unrolled
+constexpr int kMaxRouterSplits = 32;
+constexpr int kMaxShared = 16;  // top-K sums the split partials unrolled
 
 // Launch with programmatic stream serialization (PDL): the kernel may begin
 // its prologue while the previous kernel in the stream finishes; every kernel
@@ -82,6 +83,10 @@ struct TcGemmArgs {
     long long out2_ld;
     int *tile_done;           // per tile: gate/up units whose H rows are published
     int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
+    // MODE_GEMM1 / MODE_GEMM2 over every token (shared experts): tile ti of
+    // n_units / n_mb is (shared expert ti / dense_ntt, token tile ti % dense_ntt);
+    // GEMM1 reads x rows, GEMM2 reads and both write rows s * T + token.
+    int dense, dense_ntt, dense_T, dense_gemm2;
 };
 
 cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,
@@ -121,8 +126,8 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
 // out[t] = sum_k w[t,k] * Y[pair_pos[t,k]] over kept k; Y fp32, fp32 sums,
 // one rounding to the output dtype.
 cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
-                           const int *pair_pos, int T, int K, int d, void *out, int n_sm,
-                           cudaStream_t stream);
+                           const int *pair_pos, int T, int K, int d, const float *Ys,
+                           int n_shared, void *out, int n_sm, cudaStream_t stream);
 
 // fp32 SIMT path (BEAM_F32).
 cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,

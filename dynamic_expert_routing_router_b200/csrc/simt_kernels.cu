@@ -322,7 +322,8 @@ __device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int *idx,
                                                       const float *w, const int *pair_pos, int T,
-                                                      int K, int d, Tout *out) {
+                                                      int K, int d, const float *Ys, int n_shared,
+                                                      Tout *out) {
     __shared__ int s_row[kMaxK];
     __shared__ float s_w[kMaxK];
     __shared__ int s_n;
@@ -364,6 +365,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
                 const float wk = s_w[j];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
+            }
+            for (int sx = 0; sx < n_shared; ++sx) {  // shared experts, weight 1, in order
+                float y[8];
+                load8(Ys + ((long long)sx * T + t) * d + v * 8, y);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] += y[i];
             }
             store8(out + (long long)t * d + v * 8, acc);
         }
@@ -516,17 +523,18 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
 }
 
 cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
-                           const int *pair_pos, int T, int K, int d, void *out, int n_sm,
-                           cudaStream_t stream) {
+                           const int *pair_pos, int T, int K, int d, const float *Ys,
+                           int n_shared, void *out, int n_sm, cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     int threads = d / 8;
     threads = threads >= 256 ? 256 : ((threads + 31) / 32) * 32;
     int blocks = T < 8 * n_sm ? T : 8 * n_sm;
     if (dtype == BEAM_BF16)
         return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), 0, stream,
-                          Y, idx, w, pair_pos, T, K, d, static_cast<__nv_bfloat16 *>(out));
+                          Y, idx, w, pair_pos, T, K, d, Ys, n_shared,
+                          static_cast<__nv_bfloat16 *>(out));
     return launch_pdl(combine_kernel<float>, dim3(blocks), dim3(threads), 0, stream, Y, idx, w,
-                      pair_pos, T, K, d, static_cast<float *>(out));
+                      pair_pos, T, K, d, Ys, n_shared, static_cast<float *>(out));
 }
 
 cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,

@@ -90,6 +90,7 @@ struct Unit {
     int sel;    // router: 0 = W_gate rows, 1 = W_mask rows
     int tt, s;  // router: token tile, split
     int rows;   // GEMMs: valid token rows of the tile
+    int out_row;  // GEMMs: first output row (= b_row except for dense units)
 };
 
 // Named barrier of the four epilogue warps (barrier 0 is __syncthreads).
@@ -116,6 +117,7 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs
         w.b_row = w.tt * BN;
         w.kb0 = w.s * p.nk;
         w.rows = 0;
+        w.out_row = 0;
         return w;
     }
     int v = u, n_mb = p.n_mb, rows_per_mb = kBlockM, a_rows = p.a_rows_per_expert;
@@ -133,9 +135,18 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs
     }
     w.mb = v % n_mb;
     w.ti = v / n_mb;
+    if ((MODE == MODE_GEMM1 || MODE == MODE_GEMM2) && p.dense) {
+        const int sx = w.ti / p.dense_ntt, t0 = (w.ti % p.dense_ntt) * BN;
+        w.a_row = sx * a_rows + w.mb * rows_per_mb;
+        w.out_row = sx * p.dense_T + t0;
+        w.b_row = p.dense_gemm2 ? w.out_row : t0;
+        w.rows = min(BN, p.dense_T - t0);
+        return w;
+    }
     const int4 t = p.tiles[w.ti];
     w.a_row = t.x * a_rows + w.mb * rows_per_mb;
     w.b_row = t.y;
+    w.out_row = t.y;
     w.rows = t.z;
     return w;
 }
@@ -241,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.zero[r].ptr)
                 for (int i = threadIdx.x; i < p.zero[r].count; i += blockDim.x) p.zero[r].ptr[i] = 0;
     }
-    const int ntiles = (MODE == MODE_ROUTER) ? 0 : p.meta[0];
+    const bool dense = (MODE == MODE_GEMM1 || MODE == MODE_GEMM2) && p.dense;
+    const int ntiles = (MODE == MODE_ROUTER) ? 0 : dense ? p.n_units / p.n_mb : p.meta[0];
     const int n_first = ntiles * p.n_mb;  // units of the first GEMM
     const int n_units = (MODE == MODE_ROUTER)    ? p.n_units
                         : (MODE == MODE_EXPERTS) ? n_first + ntiles * p.n_mb2
@@ -458,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
                     const int r = et & 63, half = et >> 6;
                     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
-                                         (long long)w.b_row * p.out_ld + w.mb * (kBlockM / 2) + r;
+                                         (long long)w.out_row * p.out_ld + w.mb * (kBlockM / 2) + r;
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc) {
                         const int c = half * 8 + cc;
@@ -470,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else if (MODE == MODE_GEMM1) {
                     // H (bf16): the next GEMM's operand.
                     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
-                                         (long long)w.b_row * p.out_ld + w.mb * kBlockM + row;
+                                         (long long)w.out_row * p.out_ld + w.mb * kBlockM + row;
 #pragma unroll
                     for (int c = 0; c < 16; ++c)
                         if (c0 + c < w.rows)
@@ -480,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // Y (fp32): rounded once, after the weighted combine.
                     void *base = (MODE == MODE_EXPERTS) ? p.out2 : p.out;
                     const long long ld = (MODE == MODE_EXPERTS) ? p.out2_ld : p.out_ld;
-                    float *out = static_cast<float *>(base) + (long long)w.b_row * ld +
+                    float *out = static_cast<float *>(base) + (long long)w.out_row * ld +
                                  w.mb * kBlockM + row;
 #pragma unroll
                     for (int c = 0; c < 16; ++c)

@@ -25,7 +25,9 @@ Workload recipe (all synthetic; the trained models of the paper are not used):
   W_mask[e] = N(0, 1/d) - gamma*mu, gamma calibrated offline by the oracle
   (tests/golden/tiny_gamma.json) to keep about half of the candidates.
 * Experts: W1 (gate), W3 (up) ~ N(0, 1/d) as [E, I, d]; W2 (down) ~ N(0, 1/I)
-  as [E, d, I].
+  as [E, d, I].  Shared experts (DeepSeekV2-Lite shape: 2 of them, Qwen1.5-MoE
+  shape: 4) are drawn the same way from their own seeds.
+* f = 0 (every candidate masked): W_mask = 0 except -1 in the bias column.
 
 Each tensor has its own seed (base seed + a fixed offset, plus 1000 per layer
 of a stack), drawn with a torch.Generator on the target device.
@@ -40,6 +42,7 @@ import torch
 
 # Per-tensor seed offsets.
 _OFF_X, _OFF_WG, _OFF_WM, _OFF_W1, _OFF_W3, _OFF_W2, _OFF_RANK, _OFF_MU = range(1, 9)
+_OFF_SHARED = 20
 _LAYER_STRIDE = 1000
 
 
@@ -56,6 +59,13 @@ class Shape:
 TINY = Shape(d=128, E=8, K=2, I=256, renorm=0, dtype="f32")
 QWEN3 = Shape(d=2048, E=128, K=8, I=768, renorm=1, dtype="bf16")
 LARGE = Shape(d=7168, E=256, K=8, I=2048, renorm=1, dtype="bf16")
+# Layers with always-on shared experts (the two such models of the BEAM
+# evaluation): routed experts and shared experts both of width I = 1408,
+# softmax over all experts restricted to the top-K (no renormalisation).
+DSV2_LITE = Shape(d=2048, E=64, K=6, I=1408, renorm=0, dtype="bf16")
+DSV2_LITE_SHARED = 2
+QWEN15_MOE = Shape(d=2048, E=60, K=4, I=1408, renorm=0, dtype="bf16")
+QWEN15_MOE_SHARED = 4
 
 
 def torch_dtype(shape: Shape):
@@ -106,6 +116,14 @@ def make_experts(shape: Shape, seed: int = 0, device="cpu", layer: int = 0):
     return W1, W3, W2
 
 
+def make_shared_experts(shape: Shape, n_shared: int, seed: int = 0, device="cpu",
+                        layer: int = 0):
+    """(W1s, W3s, W2s) of n_shared always-on experts of width shape.I, drawn
+    like the routed experts: [S, I, d], [S, I, d], [S, d, I]."""
+    sh = Shape(d=shape.d, E=n_shared, K=1, I=shape.I, renorm=shape.renorm, dtype=shape.dtype)
+    return make_experts(sh, seed=seed + _OFF_SHARED, device=device, layer=layer)
+
+
 def make_gate(shape: Shape, seed: int = 0, device="cpu", zipf: float | None = 1.1,
               layer: int = 0):
     """W_gate [E, d] ~ N(0, 1/d); with zipf, column d-1 = -zipf*ln(rank)."""
@@ -121,9 +139,14 @@ def make_gate(shape: Shape, seed: int = 0, device="cpu", zipf: float | None = 1.
 
 
 def make_mask(shape: Shape, f: float, seed: int = 0, device="cpu", layer: int = 0):
-    """W_mask [E, d] for a target kept fraction f (bias-feature recipe); f=1 -> zeros."""
+    """W_mask [E, d] for a target kept fraction f (bias-feature recipe); f=1 -> zeros;
+    f=0 -> zeros with -1 in the bias column (every mask pre-activation is -1)."""
     if f >= 1.0:
         return torch.zeros((shape.E, shape.d), dtype=torch_dtype(shape), device=device)
+    if f <= 0.0:
+        Wm = torch.zeros((shape.E, shape.d), dtype=torch.float32, device=device)
+        Wm[:, shape.d - 1] = -1.0
+        return Wm.to(torch_dtype(shape))
     base = seed + layer * _LAYER_STRIDE
     Wm = _normal((shape.E, shape.d), 1.0 / math.sqrt(shape.d), base + _OFF_WM, device,
                  torch.float32)

@@ -71,12 +71,19 @@ typedef enum { BEAM_BF16 = 0, BEAM_F32 = 1 } beam_dtype;
  *   pre-activation z >= mask_logit_threshold (i.e. sigmoid(z) >= tau).
  *   0 is the paper's tau = 0.5, so a zero-initialised descriptor keeps the
  *   method's default; other values reproduce the threshold ablation (news
- *   article on BEAM, §8).  Must not be NaN. */
+ *   article on BEAM, §8).  Must not be NaN.
+ * n_shared, I_shared: always-on shared experts (news article on BEAM, §5:
+ *   models such as Qwen1.5-MoE and DeepSeek-V2-Lite keep running them for
+ *   every token, all-masked tokens included), n_shared SwiGLU experts of
+ *   width I_shared, each added with weight 1 after the routed sum.  0 = none
+ *   (beam_moe_forward); > 0 needs beam_moe_forward_shared, BEAM_BF16,
+ *   n_shared <= 16 and I_shared % 128 == 0. */
 typedef struct {
     int T, d, E, I, K;
     int dtype;       /* beam_dtype */
     int renorm_topk; /* 0 or 1 */
     float mask_logit_threshold;
+    int n_shared, I_shared;
 } beam_moe_desc;
 
 /* Workspace layout chosen for a descriptor (byte offsets from the workspace
@@ -99,7 +106,9 @@ typedef struct {
  *   tile_done int32[tiles_cap] gate/up units finished per tile (fused path)
  *   xp        [p_cap][d]  gathered token rows (dtype)
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
- *   y         f32[p_cap][d] expert output per pair                           */
+ *   y         f32[p_cap][d] expert output per pair
+ *   hs        [n_shared*T][I_shared] shared experts' SwiGLU activations (dtype)
+ *   ys        f32[n_shared*T][d] shared experts' outputs                    */
 typedef struct {
     int BN;            /* token rows per expert tile; the padding unit */
     int router_bn;     /* token rows per router tile */
@@ -108,7 +117,8 @@ typedef struct {
     int tiles_cap;     /* entries of the tile list */
     int reserved;
     size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
-        off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done;
+        off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done, off_hs,
+        off_ys;
     size_t workspace_bytes;
 } beam_moe_plan_info;
 
@@ -152,6 +162,18 @@ beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const voi
                              const void *W_mask, const void *W1, const void *W3,
                              const void *W2, void *out, void *workspace,
                              size_t workspace_bytes, void *stream);
+
+/* beam_moe_forward with shared experts (desc->n_shared > 0): out = routed sum
+ * (Eq. 8) + sum over the shared experts of E_s(x), the shared experts run for
+ * every token.  W1s (gate), W3s (up) [n_shared, I_shared, d], W2s (down)
+ * [n_shared, d, I_shared], bf16.  Two more launches than beam_moe_forward
+ * (a gate/up and a down GEMM over all tokens), inside the down-GEMM stage slot.
+ * With n_shared == 0 it is beam_moe_forward (the shared pointers may be NULL). */
+beam_status beam_moe_forward_shared(const beam_moe_desc *desc, const void *x,
+                                    const void *W_gate, const void *W_mask, const void *W1,
+                                    const void *W3, const void *W2, const void *W1s,
+                                    const void *W3s, const void *W2s, void *out,
+                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* beam_moe_forward that also records `events[i]` (cudaEvent_t, created by the
  * caller) on `stream` before stage i and events[BEAM_MOE_FORWARD_STAGES]
@@ -198,8 +220,9 @@ beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
                                    float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
                                    float *logits, void *stream);
 
-/* Kernel launches one beam_moe_forward call makes for `desc` (6 or 7), or 0
- * on a bad descriptor. */
+/* Kernel launches one forward call makes for `desc`: 6 (bf16 with
+ * decode-sized token tiles) or 7, plus 2 with shared experts; 0 for T = 0 or
+ * a bad descriptor. */
 int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last

@@ -118,3 +118,22 @@ def test_nan_mask_threshold_is_rejected():
     dsc.mask_logit_threshold = float("nan")
     assert abi.workspace_size(dsc) == 0
     assert abi.tau_logit(0.5) == 0.0 and abi.tau_logit(0.9) > 2.19
+
+
+def test_shared_expert_descriptor_rules():
+    ok = abi.desc(64, 2048, 64, 1408, 6, "bf16", 1, n_shared=2, I_shared=1408)
+    P = abi.plan(ok)
+    assert P["off_ys"] > P["off_hs"] > P["off_tile_done"]
+    assert abi.kernel_count(ok) == abi.kernel_count(abi.desc(64, 2048, 64, 1408, 6)) + 2
+    for bad, code in ((dict(n_shared=17, I_shared=128), 1), (dict(n_shared=2, I_shared=0), 1),
+                      (dict(n_shared=2, I_shared=100), 2), (dict(n_shared=-1), 1)):
+        with pytest.raises(abi.BeamError) as ei:
+            abi.plan(abi.desc(8, 2048, 64, 1408, 6, "bf16", 1, **bad))
+        assert ei.value.status == code
+    with pytest.raises(abi.BeamError):
+        abi.plan(abi.desc(8, 128, 8, 256, 2, "f32", 0, n_shared=1, I_shared=256))
+    # beam_moe_forward refuses a descriptor with shared experts before any launch
+    L = abi.lib()
+    vp = ctypes.c_void_p
+    ptrs = [vp(4096 * (i + 1)) for i in range(8)]
+    assert L.beam_moe_forward(ctypes.byref(ok), *ptrs, ctypes.c_size_t(1 << 40), None) == 1

@@ -16,9 +16,9 @@ import torch
 import oracle
 from dynamic_expert_routing_router_b200 import abi, inputs
 
-from _parity import (assert_grouping_bitexact, assert_routing_bitexact, assert_values,
-                     compact_experts, gpu_forward, gpu_route, host, oracle_from_logits,
-                     oracle_values)
+from _parity import (BF16_TOL_RMS, assert_grouping_bitexact, assert_routing_bitexact,
+                     assert_values, bf16_excess, compact_experts, gpu_forward, gpu_route, host,
+                     oracle_from_logits, oracle_values)
 
 pytestmark = pytest.mark.gpu
 
@@ -375,3 +375,62 @@ def test_48_layer_decode_stack_matches_oracle():
         x = inputs.stack_next_input(out, layer)
         del W1, W3, W2
     assert 0.05 < min(kept) and max(kept) < 0.7, kept
+
+
+# -------------------------------------------------------- shared experts --
+
+SHARED = [
+    # (name, shape, n_shared, T, kept fraction)
+    ("dsv2lite_decode_T33", inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED, 33, 0.35),
+    ("dsv2lite_prefill_T2048", inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED, 2048, 0.35),
+    ("dsv2lite_decode_T300_renorm", inputs.Shape(2048, 64, 6, 1408, 1, "bf16"), 2, 300, 0.6),
+    ("qwen15_decode_T40", inputs.QWEN15_MOE, inputs.QWEN15_MOE_SHARED, 40, 0.15),
+    ("qwen15_decode_T1_unmasked", inputs.QWEN15_MOE, inputs.QWEN15_MOE_SHARED, 1, 1.0),
+]
+
+
+@pytest.mark.parametrize("name,sh,S,T,f", SHARED, ids=[c[0] for c in SHARED])
+def test_shared_experts_match_oracle(name, sh, S, T, f):
+    """Always-on shared experts (news article §5) on top of the masked routed
+    experts: routing bit-exact, outputs = routed sum + shared experts."""
+    d, E, K, I, renorm = sh.d, sh.E, sh.K, sh.I, sh.renorm
+    x = inputs.make_tokens(sh, T, seed=T + 5, device=DEV)
+    Wg = inputs.make_gate(sh, seed=3, device=DEV)
+    Wm = inputs.make_mask(sh, f, seed=3, device=DEV)
+    W1, W3, W2 = inputs.make_experts(sh, seed=3, device=DEV)
+    W1s, W3s, W2s = inputs.make_shared_experts(sh, S, seed=3, device=DEV)
+    dsc = abi.desc(T, d, E, I, K, "bf16", renorm, n_shared=S, I_shared=I)
+    g = gpu_route(dsc, x, Wg, Wm)
+    o = oracle_from_logits(g["logits"], E, K, renorm, True)
+    assert_routing_bitexact(g, o)
+    ws = abi.alloc_workspace(dsc, DEV)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, out, ws)
+    abi.check(dsc, ws)
+    n = min(T, 24)
+    for t0 in sorted({0, T - n}):
+        ref = oracle.experts(host(x), host(W1), host(W3), host(W2), g["idx"], o["w"], "bf16",
+                             t0, t0 + n)
+        oracle.add_shared(ref, host(x), host(W1s), host(W3s), host(W2s), "bf16", t0, t0 + n)
+        o_rows = out.float().cpu().numpy().astype(np.float64)[t0:t0 + n]
+        assert (bf16_excess(o_rows, ref) <= BF16_TOL_RMS).all()
+
+
+def test_shared_experts_serve_all_masked_tokens():
+    """Every candidate masked: the output is the shared experts alone."""
+    sh, S, T = inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED, 48
+    d, E, K, I = sh.d, sh.E, sh.K, sh.I
+    x = inputs.make_tokens(sh, T, seed=9, device=DEV)
+    Wg = inputs.make_gate(sh, seed=3, device=DEV)
+    Wm = inputs.make_mask(sh, 0.0, device=DEV)
+    W1, W3, W2 = inputs.make_experts(sh, seed=3, device=DEV)
+    W1s, W3s, W2s = inputs.make_shared_experts(sh, S, seed=3, device=DEV)
+    dsc = abi.desc(T, d, E, I, K, "bf16", sh.renorm, n_shared=S, I_shared=I)
+    ws = abi.alloc_workspace(dsc, DEV)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, out, ws)
+    abi.check(dsc, ws)
+    assert (abi.workspace_views(dsc, ws)["idx"] == -1).all()
+    ref = np.zeros((T, d))
+    oracle.add_shared(ref, host(x), host(W1s), host(W3s), host(W2s), "bf16")
+    assert (bf16_excess(out.float().cpu().numpy().astype(np.float64), ref) <= BF16_TOL_RMS).all()
