@@ -30,6 +30,7 @@ struct TcMaps {
 
 constexpr int kBlockM = 128;   // weight rows per tile (the MMA's M)
 constexpr int kBlockK = 64;    // reduction elements per stage: one 128-byte bf16 row
+constexpr int kRowBytes = kBlockK * 2;  // one swizzled row of a bf16 stage tile
 constexpr int kNominalSMs = 148;
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 16;
@@ -83,6 +84,7 @@ struct TcGemmArgs {
     long long out2_ld;
     int *tile_done;           // per tile: gate/up units whose H rows are published
     int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
+    const int *tile_tok;      // MODE_EXPERTS: per tile, BN token rows of x (gather4)
     // MODE_GEMM1 / MODE_GEMM2 over every token (shared experts): tile ti of
     // n_units / n_mb is (shared expert ti / dense_ntt, token tile ti % dense_ntt);
     // GEMM1 reads x rows, GEMM2 reads and both write rows s * T + token.
@@ -113,6 +115,7 @@ struct PermuteArgs {
     int *pair, *pair_pos;
     int4 *tiles;
     int *tile_done;  // cleared for every tile written (MODE_EXPERTS counters)
+    int *tile_tok;   // or null: per tile, the token of each of its BN rows (0 on padding)
     int *meta;
     int *err;
 };

@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
                                 __popc(bal[q] & ((1u << lane) - 1u));
                 a.pair[pos] = t * a.K + km[q];
                 a.pair_pos[(long long)t * a.K + km[q]] = pos;
+                if (a.tile_tok) a.tile_tok[(long long)toff_e * a.BN + (pos - off_e)] = t;
             }
         }
         running += s_total;
@@ -260,7 +261,10 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     if (tid == 0 && running != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
 
     const int padded_e = (count_e + a.BN - 1) / a.BN * a.BN;
-    for (int r = count_e + tid; r < padded_e; r += kPermThreads) a.pair[off_e + r] = -1;
+    for (int r = count_e + tid; r < padded_e; r += kPermThreads) {
+        a.pair[off_e + r] = -1;
+        if (a.tile_tok) a.tile_tok[(long long)toff_e * a.BN + r] = 0;  // any valid row of x
+    }
     const int ntile_e = padded_e / a.BN;
     for (int j = tid; j < ntile_e; j += kPermThreads) {
         const int rows = min(a.BN, count_e - j * a.BN);
