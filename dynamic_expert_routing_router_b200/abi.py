@@ -42,7 +42,7 @@ class PlanInfo(ctypes.Structure):
                [(n, ctypes.c_size_t) for n in (
                    "off_err", "off_meta", "off_counts", "off_hist", "off_partial", "off_idx",
                    "off_w", "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h", "off_y",
-                   "off_tile_done", "off_hs", "off_ys", "off_tile_tok", "workspace_bytes")]
+                   "off_tile_done", "off_hs", "off_ys", "workspace_bytes")]
 
 
 _lib = None

@@ -105,16 +105,13 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
     P->off_pair_pos = align256(P->off_pair + 4 * size_t(p_cap));
     P->off_tiles = align256(P->off_pair_pos + 4 * size_t(T * K));
     P->off_xp = align256(P->off_tiles + 16 * size_t(tiles_cap));
-    // bf16 decode tiles: the fused expert kernel reads token rows from x.
-    const bool direct_rows = d->dtype == BEAM_BF16 && P->BN < 128;
-    P->off_h = align256(P->off_xp + (direct_rows ? 0 : es * size_t(p_cap) * size_t(d->d)));
+    P->off_h = align256(P->off_xp + es * size_t(p_cap) * size_t(d->d));
     P->off_y = align256(P->off_h + es * size_t(p_cap) * size_t(d->I));
     P->off_tile_done = align256(P->off_y + 4 * size_t(p_cap) * size_t(d->d));  // Y is fp32
     const size_t srows = size_t(d->n_shared) * size_t(T);  // shared rows: every token
     P->off_hs = align256(P->off_tile_done + 4 * size_t(tiles_cap));
     P->off_ys = align256(P->off_hs + es * srows * size_t(d->n_shared > 0 ? d->I_shared : 0));
-    P->off_tile_tok = align256(P->off_ys + 4 * srows * size_t(d->d));
-    o = align256(P->off_tile_tok + (direct_rows ? 4 * size_t(tiles_cap) * size_t(P->BN) : 0));
+    o = align256(P->off_ys + 4 * srows * size_t(d->d));
     P->workspace_bytes = o;
     return BEAM_OK;
 }
@@ -304,19 +301,26 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
     if (s != BEAM_OK) return s;
 
-    // Thin token tiles (decode, bf16): gate and up rows interleaved in one
-    // 128-row tile, both expert GEMMs in one fused launch, and token rows read
-    // from x by that launch (no gather).  128-token tiles (prefill): two
-    // 128-row weight tiles per unit, two launches, rows gathered first.
+    // Thin token tiles (decode, bf16): the grouping kernel also copies the
+    // token rows (no gather launch), gate and up rows are interleaved in one
+    // 128-row tile, and both expert GEMMs run in one fused launch.  128-token
+    // tiles (prefill): rows gathered by their own kernel, two 128-row weight
+    // tiles per unit, two GEMM launches.
     const bool fused = d->dtype == BEAM_BF16 && fused_experts(P);
-    int *tile_tok = fused ? reinterpret_cast<int *>(ws + P.off_tile_tok) : nullptr;
+    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
+    const int row_vec = int(es * size_t(d->d) / 16);
     BEAM_TRY_CUDA(rec.rec(2));
-    PermuteArgs pa{idx,       counts,   d->T, d->K, d->E, P.BN, pair, pair_pos, tiles,
-                   tile_done, tile_tok, meta, err};
+    PermuteArgs pa{idx,      counts,    d->T,
+                   d->K,     d->E,      P.BN,
+                   pair,     pair_pos,  tiles,
+                   tile_done,
+                   fused ? static_cast<const uint4 *>(x) : nullptr,
+                   fused ? static_cast<uint4 *>(xp) : nullptr,
+                   row_vec,  fused ? kPermCopyBlocks : 1,
+                   meta,     err};
     BEAM_TRY_CUDA(launch_permute(pa, st));
 
     BEAM_TRY_CUDA(rec.rec(3));
-    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
     if (!fused)
         BEAM_TRY_CUDA(
             launch_gather(x, pair, meta, d->K, (long long)es * d->d, P.p_cap, xp, n_sm, st));
@@ -326,10 +330,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         TcMaps maps;
         if (!make_tmap(&maps.a0, W1, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.a1, W3, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
-        // Fused: rows of x one at a time (a gather4 box is one row high).
-        if (fused ? !make_tmap(&maps.b, x, d->d, d->T, 1)
-                  : !make_tmap(&maps.b, xp, d->d, P.p_cap, P.BN))
-            return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.a2, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.b2, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
 
@@ -354,7 +355,6 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
             g.out2_ld = d->d;
             g.tile_done = tile_done;
             g.work_ctr = meta + 3;
-            g.tile_tok = tile_tok;
             const long long units = (long long)P.tiles_cap * (g.n_mb + g.n_mb2);
             BEAM_TRY_CUDA(launch_tc_gemm(MODE_EXPERTS, P.BN, maps, g,
                                          int(units < n_sm ? units : n_sm), st));
@@ -594,7 +594,8 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     if (make_plan(desc, &P) != BEAM_OK) return 0;
     if (desc->T == 0) return 0;
     const int shared = desc->n_shared > 0 ? 2 : 0;
-    // Fused decode path: no gather launch and one launch for both GEMMs.
+    // Fused decode path: rows copied by the grouping kernel (no gather
+    // launch) and one launch for both expert GEMMs.
     return shared + ((desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 2
                                                                      : BEAM_MOE_FORWARD_STAGES);
 }

@@ -30,12 +30,12 @@ struct TcMaps {
 
 constexpr int kBlockM = 128;   // weight rows per tile (the MMA's M)
 constexpr int kBlockK = 64;    // reduction elements per stage: one 128-byte bf16 row
-constexpr int kRowBytes = kBlockK * 2;  // one swizzled row of a bf16 stage tile
 constexpr int kNominalSMs = 148;
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 16;
-constexpr int kMaxRouterSplits = 32;
-constexpr int kMaxShared = 16;  // top-K sums the split partials unrolled
+constexpr int kMaxRouterSplits = 32;  // top-K sums the split partials unrolled
+constexpr int kMaxShared = 16;        // shared experts per layer
+constexpr int kPermCopyBlocks = 4;    // grouping blocks per expert when they copy rows
 
 // Launch with programmatic stream serialization (PDL): the kernel may begin
 // its prologue while the previous kernel in the stream finishes; every kernel
@@ -84,7 +84,6 @@ struct TcGemmArgs {
     long long out2_ld;
     int *tile_done;           // per tile: gate/up units whose H rows are published
     int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
-    const int *tile_tok;      // MODE_EXPERTS: per tile, BN token rows of x (gather4)
     // MODE_GEMM1 / MODE_GEMM2 over every token (shared experts): tile ti of
     // n_units / n_mb is (shared expert ti / dense_ntt, token tile ti % dense_ntt);
     // GEMM1 reads x rows, GEMM2 reads and both write rows s * T + token.
@@ -115,7 +114,12 @@ struct PermuteArgs {
     int *pair, *pair_pos;
     int4 *tiles;
     int *tile_done;  // cleared for every tile written (MODE_EXPERTS counters)
-    int *tile_tok;   // or null: per tile, the token of each of its BN rows (0 on padding)
+    // Optional row copy (fused decode path): x rows into grouped order, done by
+    // R blocks per expert instead of a separate gather launch.  x, xp null: none.
+    const uint4 *x;
+    uint4 *xp;
+    int row_vec;  // 16-byte vectors per row
+    int R;        // blocks per expert (>= 1)
     int *meta;
     int *err;
 };

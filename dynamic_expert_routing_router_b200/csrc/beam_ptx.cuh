@@ -103,20 +103,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *t
         : "memory");
 }
 
-// Four rows (r0..r3) of a 2D tensor, columns [x, x + box width), in one
-// copy: the tensor map's box is one row high, and the rows land one after
-// another at smem_dst in the map's swizzled layout.  x obeys the same 16-byte
-// rule as a tiled load; the row indices must lie inside the tensor.
-__device__ __forceinline__ void tma_gather4_2d(void *smem_dst, const CUtensorMap *tm, int x,
-                                               int r0, int r1, int r2, int r3, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(smem_u32(bar))
-        : "memory");
-}
-
 // -------------------------------------------------------------- tcgen05 --
 
 __device__ __forceinline__ void tc_fence_before_sync() {

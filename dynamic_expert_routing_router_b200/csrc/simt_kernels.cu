@@ -170,6 +170,10 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
 // experts), so no separate scan kernel is needed.  Rows of expert e:
 // [off_e, off_e + roundup(count_e, BN)); padding rows get pair = -1.  The
 // tile list holds one entry per BN rows of a non-empty expert.
+//
+// With a row copy (x, xp set), R blocks share an expert: each one repeats the
+// listing (identical values, so the duplicate writes agree) and then copies
+// every R-th group of its rows of x into xp, one warp per row.
 constexpr int kPermThreads = 256;
 
 __device__ __forceinline__ int block_sum_256(int v, int *s_red) {
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     __shared__ int s_wcnt[4 * (kPermThreads / 32)];
     __shared__ int s_wpre[4 * (kPermThreads / 32)];
     __shared__ int s_total;
-    const int e = blockIdx.x;
+    const int e = blockIdx.x / a.R, replica = blockIdx.x % a.R;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_wait();
     griddep_launch_dependents();
@@ -252,7 +256,6 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
                                 __popc(bal[q] & ((1u << lane) - 1u));
                 a.pair[pos] = t * a.K + km[q];
                 a.pair_pos[(long long)t * a.K + km[q]] = pos;
-                if (a.tile_tok) a.tile_tok[(long long)toff_e * a.BN + (pos - off_e)] = t;
             }
         }
         running += s_total;
@@ -261,15 +264,31 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     if (tid == 0 && running != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
 
     const int padded_e = (count_e + a.BN - 1) / a.BN * a.BN;
-    for (int r = count_e + tid; r < padded_e; r += kPermThreads) {
-        a.pair[off_e + r] = -1;
-        if (a.tile_tok) a.tile_tok[(long long)toff_e * a.BN + r] = 0;  // any valid row of x
-    }
+    for (int r = count_e + tid; r < padded_e; r += kPermThreads) a.pair[off_e + r] = -1;
     const int ntile_e = padded_e / a.BN;
     for (int j = tid; j < ntile_e; j += kPermThreads) {
         const int rows = min(a.BN, count_e - j * a.BN);
         a.tiles[toff_e + j] = make_int4(e, off_e + j * a.BN, rows, 0);
         a.tile_done[toff_e + j] = 0;
+    }
+    if (a.xp == nullptr) return;
+    // Row copy.  The pair entries read back were written by this block (the
+    // listing loop ends with a barrier); padding rows are not copied, they
+    // only feed padding columns of the GEMMs, which are never stored.
+    for (int r = replica * kWarps + warp; r < count_e; r += a.R * kWarps) {
+        const int pr = a.pair[off_e + r];
+        const uint4 *src = a.x + (long long)(pr / a.K) * a.row_vec;
+        uint4 *dst = a.xp + (long long)(off_e + r) * a.row_vec;
+        int v = lane;
+        for (; v + 96 < a.row_vec; v += 128) {  // four 16-byte loads in flight per lane
+            const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 32);
+            const uint4 a2 = __ldg(src + v + 64), a3 = __ldg(src + v + 96);
+            dst[v] = a0;
+            dst[v + 32] = a1;
+            dst[v + 64] = a2;
+            dst[v + 96] = a3;
+        }
+        for (; v < a.row_vec; v += 32) dst[v] = __ldg(src + v);
     }
 }
 
@@ -512,7 +531,7 @@ cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream) {
 }
 
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {
-    return launch_pdl(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, stream, a);
+    return launch_pdl(permute_kernel, dim3(a.E * a.R), dim3(kPermThreads), 0, stream, a);
 }
 
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,

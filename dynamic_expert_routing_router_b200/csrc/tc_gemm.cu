@@ -298,14 +298,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const bool interleaved =
                     MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
-                // Gate/up units of the fused kernel read their BN token rows
-                // of x directly (the rows of tile ti, in grouped order).
-                int4 tok[MODE == MODE_EXPERTS ? BN / 4 : 1];
-                if (MODE == MODE_EXPERTS && w.phase == 0) {
-                    const int4 *tt = reinterpret_cast<const int4 *>(p.tile_tok + (long long)w.ti * BN);
-#pragma unroll
-                    for (int g = 0; g < BN / 4; ++g) tok[g] = tt[g];
-                }
                 for (int kb = 0; kb < w.nk; ++kb, ++it) {
                     const int s = int(it % STAGES);
                     const uint32_t ph = ((it / STAGES) & 1u) ^ 1u;
@@ -325,15 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (NUM_A == 2)
                         tma_load_2d(st + C::A_BYTES, &maps.a1, kx, w.a_row, &full_bar[s]);
-                    if (MODE == MODE_EXPERTS && w.phase == 0) {
-                        // Token rows straight from x, four per copy.
-#pragma unroll
-                        for (int g = 0; g < BN / 4; ++g)
-                            tma_gather4_2d(st + NUM_A * C::A_BYTES + g * 4 * kRowBytes, bm, kx,
-                                           tok[g].x, tok[g].y, tok[g].z, tok[g].w, &full_bar[s]);
-                    } else {
-                        tma_load_2d(st + NUM_A * C::A_BYTES, bm, kx, w.b_row, &full_bar[s]);
-                    }
+                    tma_load_2d(st + NUM_A * C::A_BYTES, bm, kx, w.b_row, &full_bar[s]);
                 }
                 if (!ok) break;
             }

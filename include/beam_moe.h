@@ -104,15 +104,11 @@ typedef struct {
  *   pair_pos  int32[T][K] permuted row of a kept pair (undefined if masked)
  *   tiles     int32[tiles_cap][4] (expert, first row, valid rows, 0)
  *   tile_done int32[tiles_cap] gate/up units finished per tile (fused path)
- *   xp        [p_cap][d]  gathered token rows (dtype); empty (0 bytes) when
- *             BN < 128 and dtype is bf16: the fused expert kernel reads the
- *             token rows of x itself, through tile_tok
+ *   xp        [p_cap][d]  gathered token rows (dtype)
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
  *   y         f32[p_cap][d] expert output per pair
  *   hs        [n_shared*T][I_shared] shared experts' SwiGLU activations (dtype)
- *   ys        f32[n_shared*T][d] shared experts' outputs
- *   tile_tok  int32[tiles_cap][BN] token of each tile row (0 on padding);
- *             bf16 with BN < 128 only, else empty                           */
+ *   ys        f32[n_shared*T][d] shared experts' outputs                    */
 typedef struct {
     int BN;            /* token rows per expert tile; the padding unit */
     int router_bn;     /* token rows per router tile */
@@ -122,7 +118,7 @@ typedef struct {
     int reserved;
     size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
         off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done, off_hs,
-        off_ys, off_tile_tok;
+        off_ys;
     size_t workspace_bytes;
 } beam_moe_plan_info;
 
