@@ -297,3 +297,240 @@ int oracle_shared_experts(int T, int d, int n_shared, int Is, int dtype, const v
     if (bad == 2 || bad == 3) return -2;
     return bad ? -1 : 0;
 }
+
+/* Training-mode backward (see header).  Phase 1, per token: the forward of
+ * every candidate (a = x W1^T, b = x W3^T, h = SiLU(a) (.) b, e = h W2^T), then
+ *   u_k    = <dy, e_k>
+ *   dm_k   = g_k u_k                         (through w = g m, Eq. 7; STE term)
+ *   dz_k   = (dm_k + beta) s_k (1 - s_k)     (s = sigmoid(z), Eq. 5; dm/ds = 1)
+ *   dg_k   = m_k u_k
+ *   dr     = softmax backward of dg (over the candidates when renorm, Eq. 4;
+ *            over all E logits otherwise)
+ * and, for kept candidates, the expert backward with upstream w_k dy:
+ *   dh = W2^T (w_k dy), da = dh (.) b (.) SiLU'(a), db = dh (.) SiLU(a),
+ *   dx += W1^T da + W3^T db.
+ * dx also gets W_gate^T dr and W_mask^T dz.  Phase 2 sums the weight
+ * gradients over tokens (ascending) and slots (ascending). */
+static double sigmoid_d(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+int oracle_backward(int T, int d, int E, int I, int K, int renorm, int dtype, double tau_logit,
+                    double beta, int ste, const void *x, const void *W_gate, const void *W_mask,
+                    const void *W1, const void *W3, const void *W2, const void *dy, int n_sel,
+                    const int32_t *sel, double *dx, double *dWg, double *dWm, double *dW1,
+                    double *dW3, double *dW2, double *u, double *dz, int nthreads) {
+    if (T < 0 || d <= 0 || E <= 0 || I <= 0 || K <= 0 || K > E) return -1;
+    if (!x || !W_gate || !W1 || !W3 || !W2 || !dy || !dx || !dWg) return -1;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_F32) return -1;
+    if (sel == NULL) n_sel = E;
+    if (n_sel < 0) return -1;
+    for (int s = 0; sel && s < n_sel; ++s)
+        if (sel[s] < 0 || sel[s] >= E) return -1;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#else
+    nthreads = 1;
+#endif
+    const size_t TK = (size_t)T * K, TE = (size_t)T * E;
+    double *r = (double *)malloc(sizeof(double) * (TE ? TE : 1));
+    double *zl = (double *)malloc(sizeof(double) * (TE ? TE : 1));
+    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (TK ? TK : 1));
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (TK ? TK : 1));
+    double *g = (double *)malloc(sizeof(double) * (TK ? TK : 1));
+    double *w = (double *)malloc(sizeof(double) * (TK ? TK : 1));
+    double *uk = (double *)malloc(sizeof(double) * (TK ? TK : 1));
+    double *dzk = (double *)malloc(sizeof(double) * (TK ? TK : 1));
+    double *dr = (double *)malloc(sizeof(double) * (TE ? TE : 1));
+    double *hs = (double *)malloc(sizeof(double) * (TK ? TK : 1) * I);
+    double *das = (double *)malloc(sizeof(double) * (TK ? TK : 1) * I);
+    double *dbs = (double *)malloc(sizeof(double) * (TK ? TK : 1) * I);
+    int rc = 0;
+    if (!r || !zl || !cand || !idx || !g || !w || !uk || !dzk || !dr || !hs || !das || !dbs) {
+        rc = -1;
+        goto done;
+    }
+    rc = oracle_logits(T, d, E, dtype, x, W_gate, W_mask, r, W_mask ? zl : NULL);
+    if (rc) goto done;
+    rc = oracle_route(T, E, K, renorm, tau_logit, r, W_mask ? zl : NULL, cand, g, idx, w, NULL,
+                      NULL);
+    if (rc) goto done;
+
+    int bad = 0;
+#pragma omp parallel num_threads(nthreads) reduction(| : bad)
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dyt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *a = (double *)malloc(sizeof(double) * (size_t)I);
+        double *b = (double *)malloc(sizeof(double) * (size_t)I);
+        double *dh = (double *)malloc(sizeof(double) * (size_t)I);
+        double *dg = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!xt || !dyt || !a || !b || !dh || !dg) bad = 1;
+#pragma omp for schedule(dynamic, 1)
+        for (int t = 0; t < T; ++t) {
+            if (bad & 1) continue;
+            for (int j = 0; j < d; ++j) {
+                xt[j] = load_elem(x, dtype, (size_t)t * d + j);
+                dyt[j] = load_elem(dy, dtype, (size_t)t * d + j);
+            }
+            double *dxt = dx + (size_t)t * d;
+            for (int j = 0; j < d; ++j) dxt[j] = 0.0;
+            for (int k = 0; k < K; ++k) {
+                const size_t o = (size_t)t * K + k;
+                const int e = cand[o];
+                double *h = hs + o * I, *da = das + o * I, *db = dbs + o * I;
+                for (int i = 0; i < I; ++i) {
+                    size_t row = ((size_t)e * I + i) * d;
+                    double ai = 0.0, bi = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        ai += xt[j] * load_elem(W1, dtype, row + j);
+                        bi += xt[j] * load_elem(W3, dtype, row + j);
+                    }
+                    a[i] = ai;
+                    b[i] = bi;
+                    h[i] = ai * sigmoid_d(ai) * bi;
+                }
+                double uu = 0.0;
+                for (int j = 0; j < d; ++j) {
+                    size_t row = ((size_t)e * d + j) * I;
+                    double ej = 0.0;
+                    for (int i = 0; i < I; ++i) ej += h[i] * load_elem(W2, dtype, row + i);
+                    uu += dyt[j] * ej;
+                }
+                uk[o] = uu;
+                const int kept = idx[o] >= 0;
+                dg[k] = kept ? uu : 0.0;
+                if (W_mask) {
+                    const double sg = sigmoid_d(zl[(size_t)t * E + e]);
+                    const double dm = ste ? g[o] * uu : 0.0;
+                    dzk[o] = (dm + beta) * sg * (1.0 - sg);
+                } else {
+                    dzk[o] = 0.0;
+                }
+                if (!kept) {
+                    for (int i = 0; i < I; ++i) da[i] = db[i] = 0.0;
+                    continue;
+                }
+                /* Expert backward with upstream w_k dy. */
+                for (int i = 0; i < I; ++i) dh[i] = 0.0;
+                for (int j = 0; j < d; ++j) {
+                    size_t row = ((size_t)e * d + j) * I;
+                    const double c = w[o] * dyt[j];
+                    for (int i = 0; i < I; ++i) dh[i] += c * load_elem(W2, dtype, row + i);
+                }
+                for (int i = 0; i < I; ++i) {
+                    const double sa = sigmoid_d(a[i]);
+                    da[i] = dh[i] * b[i] * sa * (1.0 + a[i] * (1.0 - sa));
+                    db[i] = dh[i] * a[i] * sa;
+                }
+                for (int i = 0; i < I; ++i) {
+                    size_t row = ((size_t)e * I + i) * d;
+                    for (int j = 0; j < d; ++j)
+                        dxt[j] += da[i] * load_elem(W1, dtype, row + j) +
+                                  db[i] * load_elem(W3, dtype, row + j);
+                }
+            }
+            /* Softmax backward: g_k = p_{c_k}; dL/dr_e = p_e (dg_e - sum_k g_k dg_k). */
+            double sdot = 0.0;
+            for (int k = 0; k < K; ++k) sdot += g[(size_t)t * K + k] * dg[k];
+            double *drt = dr + (size_t)t * E;
+            for (int e = 0; e < E; ++e) drt[e] = 0.0;
+            if (renorm) {
+                for (int k = 0; k < K; ++k) {
+                    const size_t o = (size_t)t * K + k;
+                    drt[cand[o]] = g[o] * (dg[k] - sdot);
+                }
+            } else {
+                const double *rt = r + (size_t)t * E;
+                const double mx = rt[cand[(size_t)t * K]];
+                double den = 0.0;
+                for (int e = 0; e < E; ++e) den += exp(rt[e] - mx);
+                for (int e = 0; e < E; ++e) drt[e] = -exp(rt[e] - mx) / den * sdot;
+                for (int k = 0; k < K; ++k) {
+                    const size_t o = (size_t)t * K + k;
+                    drt[cand[o]] += g[o] * dg[k];
+                }
+            }
+            for (int e = 0; e < E; ++e) {
+                if (drt[e] == 0.0) continue;
+                for (int j = 0; j < d; ++j)
+                    dxt[j] += drt[e] * load_elem(W_gate, dtype, (size_t)e * d + j);
+            }
+            if (W_mask) {
+                for (int k = 0; k < K; ++k) {
+                    const size_t o = (size_t)t * K + k;
+                    for (int j = 0; j < d; ++j)
+                        dxt[j] += dzk[o] * load_elem(W_mask, dtype, (size_t)cand[o] * d + j);
+                }
+            }
+            for (int j = 0; j < d; ++j)
+                if (!isfinite(dxt[j])) bad |= 2;
+        }
+        free(xt);
+        free(dyt);
+        free(a);
+        free(b);
+        free(dh);
+        free(dg);
+    }
+    if (bad & 1) { rc = -1; goto done; }
+    if (bad) { rc = -2; goto done; }
+
+    /* Router gradients: dWg[e] = sum_t dr[t][e] x_t; dWm[e] = sum over the
+     * (t, k) with c = e of dz x_t. */
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int e = 0; e < E; ++e) {
+        double *gw = dWg + (size_t)e * d;
+        double *mw = W_mask && dWm ? dWm + (size_t)e * d : NULL;
+        for (int j = 0; j < d; ++j) {
+            gw[j] = 0.0;
+            if (mw) mw[j] = 0.0;
+        }
+        for (int t = 0; t < T; ++t) {
+            const double c = dr[(size_t)t * E + e];
+            if (c != 0.0)
+                for (int j = 0; j < d; ++j) gw[j] += c * load_elem(x, dtype, (size_t)t * d + j);
+            if (!mw) continue;
+            for (int k = 0; k < K; ++k) {
+                const size_t o = (size_t)t * K + k;
+                if (cand[o] != e) continue;
+                for (int j = 0; j < d; ++j)
+                    mw[j] += dzk[o] * load_elem(x, dtype, (size_t)t * d + j);
+            }
+        }
+    }
+
+    /* Expert weight gradients of the selected experts, kept pairs only. */
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+    for (int s = 0; s < n_sel; ++s) {
+        const int e = sel ? sel[s] : s;
+        double *g1 = dW1 ? dW1 + (size_t)s * I * d : NULL;
+        double *g3 = dW3 ? dW3 + (size_t)s * I * d : NULL;
+        double *g2 = dW2 ? dW2 + (size_t)s * d * I : NULL;
+        if (g1) memset(g1, 0, sizeof(double) * (size_t)I * d);
+        if (g3) memset(g3, 0, sizeof(double) * (size_t)I * d);
+        if (g2) memset(g2, 0, sizeof(double) * (size_t)d * I);
+        for (int t = 0; t < T; ++t) {
+            for (int k = 0; k < K; ++k) {
+                const size_t o = (size_t)t * K + k;
+                if (idx[o] != e) continue; /* masked or another expert */
+                const double *da = das + o * I, *db = dbs + o * I, *h = hs + o * I;
+                for (int i = 0; i < I; ++i)
+                    for (int j = 0; j < d; ++j) {
+                        const double xj = load_elem(x, dtype, (size_t)t * d + j);
+                        if (g1) g1[(size_t)i * d + j] += da[i] * xj;
+                        if (g3) g3[(size_t)i * d + j] += db[i] * xj;
+                    }
+                if (g2)
+                    for (int j = 0; j < d; ++j) {
+                        const double c = w[o] * load_elem(dy, dtype, (size_t)t * d + j);
+                        for (int i = 0; i < I; ++i) g2[(size_t)j * I + i] += c * h[i];
+                    }
+            }
+        }
+    }
+    if (u) memcpy(u, uk, sizeof(double) * TK);
+    if (dz) memcpy(dz, dzk, sizeof(double) * TK);
+done:
+    free(r); free(zl); free(cand); free(idx); free(g); free(w); free(uk); free(dzk); free(dr);
+    free(hs); free(das); free(dbs);
+    return rc;
+}

@@ -82,6 +82,28 @@ int oracle_shared_experts(int T, int d, int n_shared, int Is, int dtype, const v
                           const void *W1s, const void *W3s, const void *W2s, int t_begin,
                           int t_end, double *y, int nthreads);
 
+/* Training-mode backward of the layer (news article on BEAM, §4: the
+ * straight-through estimator and the sparsity penalty).  Objective:
+ *   L = sum_t <dy_t, y_t> + beta * sum_t sum_{k<K} sigmoid(z_{t,c_k})
+ * with y the forward of Eq. (8).  READINGS (the pages describe both terms in
+ * words only): the estimator passes the gradient straight through the
+ * threshold of Eq. (6), dm/dm_hat = 1, and keeps the sigmoid's derivative; the
+ * penalty adds up the K candidates' m_hat of every token.  Every candidate's
+ * expert is evaluated, kept or not, because u_{t,k} = <dy_t, E_{c_k}(x_t)>
+ * enters the mask gradient of a masked candidate too.  ste = 0 leaves the
+ * straight-through term out: the exact gradient of L with the candidates and
+ * the mask held fixed, which finite differences can check.
+ * Inputs in the storage dtype (dy too); W_mask may be NULL (no mask: m = 1,
+ * no penalty).  Outputs fp64, overwritten: dx [T,d]; dWg, dWm [E,d] (dWm
+ * untouched without a mask); u, dz [T,K] or NULL; the expert gradients of the
+ * n_sel experts listed in sel (sel NULL: all E in order), each NULL-able:
+ * dW1, dW3 [n_sel,I,d], dW2 [n_sel,d,I].  Returns -2 on a non-finite value. */
+int oracle_backward(int T, int d, int E, int I, int K, int renorm, int dtype, double tau_logit,
+                    double beta, int ste, const void *x, const void *W_gate, const void *W_mask,
+                    const void *W1, const void *W3, const void *W2, const void *dy, int n_sel,
+                    const int32_t *sel, double *dx, double *dWg, double *dWm, double *dW1,
+                    double *dW3, double *dW2, double *u, double *dz, int nthreads);
+
 /* Threads the OpenMP runtime would use by default (for reporting). */
 int oracle_max_threads(void);
 
