@@ -501,6 +501,81 @@ def shared_bench(device, rank, Ts=(1, 128), steps=100, warmup=5):
                                  "routed sum; kept_target 0 = every candidate masked"))
 
 
+def backward_bench(layer, f, steps, warmup, pk):
+    """Training-mode backward of the decode layer (straight-through estimator,
+    penalty beta = 0.01): one CUDA graph per token batch, L2 flushed before each
+    replay.  Algorithmic bytes: the router weights, every candidate expert's
+    W1/W3/W2 (read once), x and dy, dx, and a read-modify-write of the fp32
+    gradients of the router and of the experts with a kept pair."""
+    torch, abi, inputs = layer.torch, layer.abi, layer.inputs
+    sh, T = layer.sh, layer.T
+    d, E, I, K = sh.d, sh.E, sh.I, sh.K
+    Wm = layer.mask(f)
+    dev = layer.device
+    dys = [inputs.make_upstream_grad(sh, T, seed=500 + b, device=dev) for b in range(N_BATCHES)]
+    z = lambda *s_: torch.zeros(s_, dtype=torch.float32, device=dev)  # noqa: E731
+    dx, dWg, dWm = z(T, d), z(E, d), z(E, d)
+    dW1, dW3, dW2 = z(E, I, d), z(E, I, d), z(E, d, I)
+    ws = abi.alloc_backward_workspace(layer.dsc, dev)
+    beta = 0.01
+    P = abi.plan(layer.dsc)
+    # Experts with a kept pair (the library's counters after each call) and
+    # candidate experts (routing with the mask disabled: every top-K entry).
+    u_cand, u_kept = [], []
+    r_idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    r_w = torch.empty((T, K), dtype=torch.float32, device=dev)
+    r_cnt = torch.empty((E,), dtype=torch.int32, device=dev)
+    r_ws = abi.alloc_workspace(layer.dsc, dev)
+    for b in range(N_BATCHES):
+        abi.backward(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1, layer.W3, layer.W2, dys[b],
+                     beta, dx, dWg, dWm, dW1, dW3, dW2, ws)
+        abi.check(layer.dsc, ws)
+        kept = ws[P["off_counts"]:P["off_counts"] + 4 * E].view(torch.int32)
+        u_kept.append(int((kept > 0).sum()))
+        abi.route(layer.dsc, layer.xs[b], layer.Wg, None, r_idx, r_w, r_cnt, None, None, r_ws)
+        u_cand.append(int((r_cnt > 0).sum()))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graphs = []
+    with torch.cuda.stream(s):
+        for b in range(N_BATCHES):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                abi.backward(layer.dsc, layer.xs[b], layer.Wg, Wm, layer.W1, layer.W3, layer.W2,
+                             dys[b], beta, dx, dWg, dWm, dW1, dW3, dW2, ws, stream=s)
+            graphs.append(g)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for i in range(warmup + steps):
+        flush_l2(layer.flush, i)
+        e0.record()
+        graphs[i % N_BATCHES].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) * 1e-3)
+    abi.check(layer.dsc, ws)
+    del graphs
+    t = sum(times) / len(times)
+    uc = sum(u_cand) / len(u_cand)
+    uk = sum(u_kept) / len(u_kept)
+    wbytes = 3 * I * d * 2
+    alg = (2 * E * d * 2 + uc * wbytes + 2 * T * d * 2 + T * d * 4 +
+           2 * (2 * E * d * 4) + 2 * uk * 3 * I * d * 4)
+    roof = alg / (pk["hbm"] * 1e9)
+    out = dict(T=T, kept_target=f, us_per_call=t * 1e6, tokens_per_s=T / t,
+               candidate_experts_mean=uc, kept_experts_mean=uk,
+               algorithmic_bytes=alg, roofline_us=roof * 1e6, roofline_frac=roof / t,
+               bound="hbm", peak_source=pk["source"], launches=abi.backward_kernel_count(layer.dsc),
+               note=("weight gradients fp32, accumulated; every candidate's expert is "
+                     "evaluated (its u enters the mask gradient)"))
+    del dW1, dW3, dW2, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_beam(args):
     import torch
     rank, world, local = dist_env()
@@ -607,6 +682,10 @@ def run_beam(args):
     if not args.no_shared:
         shared = shared_bench(device, rank, steps=args.sweep_steps)
 
+    backward = None
+    if not args.no_backward:
+        backward = backward_bench(layer, f_head, args.sweep_steps, 5, pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(layer, f_head, args.cpu_seconds)
@@ -640,6 +719,7 @@ def run_beam(args):
         "per_kept_fraction": sweep,
         "stack_48_layers": stack,
         "shared_experts": shared,
+        "backward": backward,
         "e2e": e2e,
         "gpu_launches": n_kernels * args.steps,
         "clocks": clocks,
@@ -708,6 +788,7 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-shared", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--sweep-steps", type=int, default=100)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

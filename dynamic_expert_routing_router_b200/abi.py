@@ -74,6 +74,13 @@ def lib():
         L.beam_moe_route_noalloc.restype = i32
         L.beam_moe_forward_kernel_count.argtypes = [pd]
         L.beam_moe_forward_kernel_count.restype = i32
+        L.beam_moe_backward_workspace_size.argtypes = [pd]
+        L.beam_moe_backward_workspace_size.restype = sz
+        L.beam_moe_backward.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                        vp, vp, vp, vp, sz, vp]
+        L.beam_moe_backward.restype = i32
+        L.beam_moe_backward_kernel_count.argtypes = [pd]
+        L.beam_moe_backward_kernel_count.restype = i32
         L.beam_status_str.argtypes = [i32]
         L.beam_status_str.restype = ctypes.c_char_p
         L.beam_moe_stage_name.argtypes = [i32]
@@ -138,6 +145,36 @@ def workspace_size(dsc: Desc) -> int:
 def kernel_count(dsc: Desc) -> int:
     """Kernel launches of one forward call for this descriptor."""
     return int(lib().beam_moe_forward_kernel_count(ctypes.byref(dsc)))
+
+
+def backward_workspace_size(dsc: Desc) -> int:
+    return int(lib().beam_moe_backward_workspace_size(ctypes.byref(dsc)))
+
+
+def backward_kernel_count(dsc: Desc) -> int:
+    """Kernel launches of one backward call for this descriptor."""
+    return int(lib().beam_moe_backward_kernel_count(ctypes.byref(dsc)))
+
+
+def alloc_backward_workspace(dsc: Desc, device=None):
+    """A uint8 torch tensor of backward_workspace_size(dsc) bytes on `device`."""
+    import torch
+    n = backward_workspace_size(dsc)
+    if n == 0:
+        raise BeamError(1, "beam_moe_backward_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def backward(dsc, x, W_gate, W_mask, W1, W3, W2, dy, beta, dx, dW_gate, dW_mask, dW1, dW3, dW2,
+             workspace, stream=None):
+    """Training-mode gradients (straight-through estimator, beta-weighted
+    penalty on the candidates' mask scores).  dx is overwritten; the weight
+    gradients (fp32, shaped like their weights) are accumulated into."""
+    _ok(lib().beam_moe_backward(ctypes.byref(dsc), _ptr(x), _ptr(W_gate), _ptr(W_mask),
+                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), ctypes.c_float(beta),
+                                _ptr(dx), _ptr(dW_gate), _ptr(dW_mask), _ptr(dW1), _ptr(dW3),
+                                _ptr(dW2), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "beam_moe_backward")
 
 
 def plan(dsc: Desc) -> dict:

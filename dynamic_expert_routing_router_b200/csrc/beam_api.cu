@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -188,6 +189,9 @@ struct RouteOut {
     int *counts;
     int *hist;
     float *logits;
+    int *cand = nullptr;        // training: every candidate
+    float *gk = nullptr;        // training: softmax weight before the mask
+    int *counts_all = nullptr;  // training: candidates per expert (caller zeroes)
 };
 
 // Stages 0-1: router GEMM into the split partials, then top-K + mask.
@@ -245,6 +249,9 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
     t.w = ro.w;
     t.counts = ro.counts;
     t.hist = ro.hist;
+    t.cand = ro.cand;
+    t.gk = ro.gk;
+    t.counts_all = ro.counts_all;
     BEAM_TRY_CUDA(launch_topk_mask(t, n_sm, st));
     return BEAM_OK;
 }
@@ -439,6 +446,193 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     return BEAM_OK;
 }
 
+// ------------------------------------------------------------ backward --
+// The backward workspace is the forward plan (its grouping now holds every
+// candidate: T*K pairs fit p_cap) followed by the training-only arrays.
+struct BwdPlan {
+    size_t off_cand, off_gk, off_counts_all, off_logits, off_dyp, off_A, off_B, off_da, off_db,
+        off_dxp, off_u, off_dz, off_dr, bytes;
+};
+
+beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan *B) {
+    beam_status s = make_plan(d, P);
+    if (s != BEAM_OK) return s;
+    if (d->n_shared != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;  // shared experts: forward only
+    const size_t T = size_t(d->T), K = size_t(d->K), E = size_t(d->E), I = size_t(d->I);
+    const size_t dd = size_t(d->d), pc = size_t(P->p_cap);
+    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
+    size_t o = P->workspace_bytes;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align256(o + bytes);
+        return at;
+    };
+    B->off_cand = take(4 * T * K);
+    B->off_gk = take(4 * T * K);
+    B->off_counts_all = take(4 * E);
+    B->off_logits = take(4 * T * 2 * E);
+    B->off_dyp = take(es * pc * dd);
+    B->off_A = take(4 * pc * I);
+    B->off_B = take(4 * pc * I);
+    B->off_da = take(4 * pc * I);
+    B->off_db = take(4 * pc * I);
+    B->off_dxp = take(4 * pc * dd);
+    B->off_u = take(4 * T * K);
+    B->off_dz = take(4 * T * K);
+    B->off_dr = take(4 * T * E);
+    B->bytes = o;
+    return BEAM_OK;
+}
+
+beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg, const void *Wm,
+                          const void *W1, const void *W3, const void *W2, const void *dy,
+                          float beta, float *dx, float *dWg, float *dWm, float *dW1, float *dW3,
+                          float *dW2, void *workspace, size_t ws_bytes, void *stream) {
+    beam_moe_plan_info P;
+    BwdPlan B;
+    beam_status s = make_bwd_plan(d, &P, &B);
+    if (s != BEAM_OK) return s;
+    if (!x || !Wg || !W1 || !W3 || !W2 || !dy || !dx || !dWg || !dW1 || !dW3 || !dW2)
+        return BEAM_ERR_INVALID_ARG;
+    if ((Wm == nullptr) != (dWm == nullptr) || !std::isfinite(beta)) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x, Wg, W1, W3, W2, dy, static_cast<const void *>(dx),
+                          static_cast<const void *>(dWg), static_cast<const void *>(dW1),
+                          static_cast<const void *>(dW3), static_cast<const void *>(dW2)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    if ((Wm && !aligned16(Wm)) || (dWm && !aligned16(dWm))) return BEAM_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < B.bytes)
+        return BEAM_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d->T == 0) {  // no token: no gradient; leave a clean error word
+        BEAM_TRY_CUDA(cudaMemsetAsync(workspace, 0, P.off_partial, st));
+        return BEAM_OK;
+    }
+    const int n_sm = sm_count();
+    char *ws = static_cast<char *>(workspace);
+    int *err = reinterpret_cast<int *>(ws + P.off_err);
+    int *meta = reinterpret_cast<int *>(ws + P.off_meta);
+    int *counts = reinterpret_cast<int *>(ws + P.off_counts);
+    int *hist = reinterpret_cast<int *>(ws + P.off_hist);
+    int *idx = reinterpret_cast<int *>(ws + P.off_idx);
+    float *w = reinterpret_cast<float *>(ws + P.off_w);
+    int *pair = reinterpret_cast<int *>(ws + P.off_pair);
+    int *pair_pos = reinterpret_cast<int *>(ws + P.off_pair_pos);
+    int4 *tiles = reinterpret_cast<int4 *>(ws + P.off_tiles);
+    int *tile_done = reinterpret_cast<int *>(ws + P.off_tile_done);
+    void *xp = ws + P.off_xp;
+    void *h = ws + P.off_h;
+    float *y = reinterpret_cast<float *>(ws + P.off_y);
+    int *cand = reinterpret_cast<int *>(ws + B.off_cand);
+    float *gk = reinterpret_cast<float *>(ws + B.off_gk);
+    int *counts_all = reinterpret_cast<int *>(ws + B.off_counts_all);
+    float *logits = reinterpret_cast<float *>(ws + B.off_logits);
+    void *dyp = ws + B.off_dyp;
+    float *A = reinterpret_cast<float *>(ws + B.off_A);
+    float *Bv = reinterpret_cast<float *>(ws + B.off_B);
+
+    // Routing, with every candidate and its pre-mask weight exported.
+    BEAM_TRY_CUDA(cudaMemsetAsync(counts_all, 0, sizeof(int) * size_t(d->E), st));
+    RouteOut ro{idx, w, counts, hist, logits};
+    ro.cand = cand;
+    ro.gk = gk;
+    ro.counts_all = counts_all;
+    s = launch_route(d, P, x, Wg, Wm, ro, ws, st, Recorder{nullptr, st}, n_sm);
+    if (s != BEAM_OK) return s;
+
+    // Every candidate grouped by expert (masked ones too: their expert
+    // outputs enter the mask gradient), with x and dy rows in that order.
+    const size_t es = d->dtype == BEAM_BF16 ? 2 : 4;
+    PermuteArgs pa{cand,      counts_all, d->T,
+                   d->K,      d->E,       P.BN,
+                   pair,      pair_pos,   tiles,
+                   tile_done, static_cast<const uint4 *>(x),
+                   static_cast<uint4 *>(xp),
+                   int(es * size_t(d->d) / 16), kPermCopyBlocks,
+                   meta,      err};
+    BEAM_TRY_CUDA(launch_permute(pa, st));
+    BEAM_TRY_CUDA(launch_gather(dy, pair, meta, d->K, (long long)es * d->d, P.p_cap, dyp, n_sm, st));
+
+    // Forward of every candidate: a, b (fp32), H, and Y = H W2^T.
+    if (d->dtype == BEAM_BF16) {
+        TcMaps maps;
+        if (!make_tmap(&maps.a0, W1, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.a1, W3, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        maps.a2 = maps.a0;
+        maps.b2 = maps.b;
+        TcGemmArgs g;
+        std::memset(&g, 0, sizeof(g));
+        g.meta = meta;
+        g.tiles = tiles;
+        g.err = err;
+        g.timeout_ns = kWaitTimeoutNs;
+        g.n_mb = d->I / kBlockM;
+        g.nk = d->d / kBlockK;
+        g.a_rows_per_expert = d->I;
+        g.out = h;
+        g.out_ld = d->I;
+        g.a_out = A;
+        g.b_out = Bv;
+        long long units = (long long)P.tiles_cap * g.n_mb;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, maps, g, int(units < n_sm ? units : n_sm), st));
+        TcMaps m2;
+        if (!make_tmap(&m2.a0, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&m2.b, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        m2.a1 = m2.a0;
+        m2.a2 = m2.a0;
+        m2.b2 = m2.b;
+        g.a_out = g.b_out = nullptr;
+        g.n_mb = d->d / kBlockM;
+        g.nk = d->I / kBlockK;
+        g.a_rows_per_expert = d->d;
+        g.out = y;
+        g.out_ld = d->d;
+        units = (long long)P.tiles_cap * g.n_mb;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, P.BN, m2, g, int(units < n_sm ? units : n_sm), st));
+    } else {
+        BEAM_TRY_CUDA(launch_gemm1_f32(static_cast<const float *>(xp), static_cast<const float *>(W1),
+                                       static_cast<const float *>(W3), tiles, meta, P.tiles_cap,
+                                       d->d, d->I, static_cast<float *>(h), st, A, Bv));
+        BEAM_TRY_CUDA(launch_gemm2_f32(static_cast<const float *>(h), static_cast<const float *>(W2),
+                                       tiles, meta, P.tiles_cap, d->d, d->I, y, st));
+    }
+
+    BwArgs a;
+    a.T = d->T;
+    a.d = d->d;
+    a.E = d->E;
+    a.I = d->I;
+    a.K = d->K;
+    a.renorm = d->renorm_topk;
+    a.has_mask = Wm != nullptr;
+    a.tiles_cap = P.tiles_cap;
+    a.beta = beta;
+    a.Y = y;
+    a.logits = logits;
+    a.cand = cand;
+    a.gk = gk;
+    a.idx = idx;
+    a.w = w;
+    a.pair = pair;
+    a.pair_pos = pair_pos;
+    a.tiles = tiles;
+    a.meta = meta;
+    a.counts_kept = counts;
+    a.counts_all = counts_all;
+    a.A = A;
+    a.B = Bv;
+    a.da = reinterpret_cast<float *>(ws + B.off_da);
+    a.db = reinterpret_cast<float *>(ws + B.off_db);
+    a.dxp = reinterpret_cast<float *>(ws + B.off_dxp);
+    a.u = reinterpret_cast<float *>(ws + B.off_u);
+    a.dz = reinterpret_cast<float *>(ws + B.off_dz);
+    a.dr = reinterpret_cast<float *>(ws + B.off_dr);
+    a.dx = dx;
+    BEAM_TRY_CUDA(launch_backward_stages(a, d->dtype, x, xp, dy, dyp, Wg, Wm, W1, W3, W2, dWg,
+                                         dWm, dW1, dW3, dW2, n_sm, st));
+    return BEAM_OK;
+}
+
 }  // namespace
 
 namespace beam {
@@ -490,6 +684,31 @@ const char *const kStageNames[BEAM_MOE_FORWARD_STAGES] = {
 }  // namespace
 
 extern "C" {
+
+size_t beam_moe_backward_workspace_size(const beam_moe_desc *desc) {
+    beam_moe_plan_info P;
+    BwdPlan B;
+    if (make_bwd_plan(desc, &P, &B) != BEAM_OK) return 0;
+    return B.bytes;
+}
+
+beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                              const void *W_mask, const void *W1, const void *W3, const void *W2,
+                              const void *dy, float beta, float *dx, float *dW_gate,
+                              float *dW_mask, float *dW1, float *dW3, float *dW2,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    return backward_impl(desc, x, W_gate, W_mask, W1, W3, W2, dy, beta, dx, dW_gate, dW_mask,
+                         dW1, dW3, dW2, workspace, workspace_bytes, stream);
+}
+
+int beam_moe_backward_kernel_count(const beam_moe_desc *desc) {
+    beam_moe_plan_info P;
+    BwdPlan B;
+    if (make_bwd_plan(desc, &P, &B) != BEAM_OK || desc->T == 0) return 0;
+    // router, top-K, grouping, dy gather, gate/up, down, then the seven
+    // CUDA-core stages (token, dh, dxp, dx, dW1/dW3, dW2, router weights)
+    return 13;
+}
 
 size_t beam_moe_workspace_size(const beam_moe_desc *desc) {
     beam_moe_plan_info P;

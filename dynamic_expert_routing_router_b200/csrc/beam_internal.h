@@ -36,6 +36,7 @@ constexpr int kMaxK = 16;
 constexpr int kMaxRouterSplits = 32;  // top-K sums the split partials unrolled
 constexpr int kMaxShared = 16;        // shared experts per layer
 constexpr int kPermCopyBlocks = 4;    // grouping blocks per expert when they copy rows
+constexpr int kMaxTileRows = 128;     // largest token tile (BN)
 
 // Launch with programmatic stream serialization (PDL): the kernel may begin
 // its prologue while the previous kernel in the stream finishes; every kernel
@@ -82,6 +83,7 @@ struct TcGemmArgs {
     int n_mb2, nk2, a_rows2;  // d/128 row blocks, I/64 k-blocks, d rows per expert
     void *out2;               // Y (f32)
     long long out2_ld;
+    float *a_out, *b_out;     // MODE_GEMM1 (or null): fp32 pre-activations, like H
     int *tile_done;           // per tile: gate/up units whose H rows are published
     int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
     // MODE_GEMM1 / MODE_GEMM2 over every token (shared experts): tile ti of
@@ -103,6 +105,12 @@ struct TopkArgs {
     float *w;              // [T][K]
     int *counts;           // [E]
     int *hist;             // [K+1] or NULL
+    // Training (backward) extras, each NULL-able: every candidate (masked or
+    // not) in slot order, its softmax weight before the mask, and candidate
+    // counts per expert (zeroed by the caller).
+    int *cand;             // [T][K]
+    float *gk;             // [T][K]
+    int *counts_all;       // [E]
 };
 cudaError_t launch_topk_mask(const TopkArgs &a, int n_sm, cudaStream_t stream);
 
@@ -136,13 +144,43 @@ cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const floa
                            const int *pair_pos, int T, int K, int d, const float *Ys,
                            int n_shared, void *out, int n_sm, cudaStream_t stream);
 
+// Training-mode backward (backward.cu).  Rows are those of the grouping of all
+// candidates (masked ones included); every array lives in the workspace.
+struct BwArgs {
+    int T, d, E, I, K, renorm, has_mask, tiles_cap;
+    float beta;
+    const float *Y;          // [p_cap][d] every candidate's expert output
+    const float *logits;     // [T][2E] router logits (r, then z)
+    const int *cand;         // [T][K] candidates
+    const float *gk;         // [T][K] softmax weights before the mask
+    const int *idx;          // [T][K] candidate or -1 (masked)
+    const float *w;          // [T][K] g * m
+    const int *pair;         // [p_cap] row -> t*K + k (-1 on padding)
+    const int *pair_pos;     // [T][K] row of a candidate
+    const int4 *tiles;       // tile list of the grouping
+    const int *meta;         // [0] tiles
+    const int *counts_kept;  // [E] kept pairs per expert
+    const int *counts_all;   // [E] candidates per expert
+    const float *A, *B;      // [p_cap][I] gate / up pre-activations
+    float *da, *db;          // [p_cap][I]
+    float *dxp;              // [p_cap][d] expert part of dx per kept row
+    float *u, *dz;           // [T][K]
+    float *dr;               // [T][E]
+    float *dx;               // [T][d]
+};
+cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
+                                   const void *dy, const void *dyp, const void *Wg,
+                                   const void *Wm, const void *W1, const void *W3,
+                                   const void *W2, float *dWg, float *dWm, float *dW1,
+                                   float *dW3, float *dW2, int n_sm, cudaStream_t st);
+
 // fp32 SIMT path (BEAM_F32).
 cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,
                               int E, float *partial, const ZeroRegion (&zero)[3],
                               cudaStream_t stream);
 cudaError_t launch_gemm1_f32(const float *xp, const float *W1, const float *W3, const int4 *tiles,
                              const int *meta, int tiles_cap, int d, int I, float *H,
-                             cudaStream_t stream);
+                             cudaStream_t stream, float *A = nullptr, float *B = nullptr);
 cudaError_t launch_gemm2_f32(const float *H, const float *W2, const int4 *tiles, const int *meta,
                              int tiles_cap, int d, int I, float *Y, cudaStream_t stream);
 

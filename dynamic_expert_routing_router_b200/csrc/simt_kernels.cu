@@ -35,9 +35,10 @@ constexpr int kTopkMaxTok = 8;
 template <int EPL>
 __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tpb) {
     __shared__ int s_counts[kMaxE];
+    __shared__ int s_counts_all[kMaxE];
     __shared__ int s_hist[kMaxK + 1];
     __shared__ __align__(16) float s_logit[kTopkMaxTok][2 * kMaxE];
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_counts[i] = 0;
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_counts[i] = s_counts_all[i] = 0;
     if (threadIdx.x <= a.K) s_hist[threadIdx.x] = 0;
     __syncthreads();
     griddep_wait();
@@ -152,14 +153,19 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
                 a.idx[(long long)t * a.K + lane] = kept ? my_cand : -1;
                 a.w[(long long)t * a.K + lane] = kept ? g : 0.0f;
                 if (kept) atomicAdd(&s_counts[my_cand], 1);
+                if (a.cand) a.cand[(long long)t * a.K + lane] = my_cand;
+                if (a.gk) a.gk[(long long)t * a.K + lane] = g;
+                if (a.counts_all) atomicAdd(&s_counts_all[my_cand], 1);
             }
             const int nkept = __popc(__ballot_sync(kFull, kept));
             if (lane == 0) atomicAdd(&s_hist[nkept], 1);
         }
         __syncthreads();  // s_logit is rewritten by the next tokens
     }
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x)
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) {
         if (s_counts[i]) atomicAdd(&a.counts[i], s_counts[i]);
+        if (a.counts_all && s_counts_all[i]) atomicAdd(&a.counts_all[i], s_counts_all[i]);
+    }
     if (a.hist && threadIdx.x <= a.K && s_hist[threadIdx.x]) atomicAdd(&a.hist[threadIdx.x], s_hist[threadIdx.x]);
 }
 
@@ -443,10 +449,12 @@ __device__ __forceinline__ float silu_mul_f32(float g, float u) {
 }
 
 // GEMM1 (fp32): H[row] = SiLU(xp[row] W1_e^T) * (xp[row] W3_e^T) for the rows
-// of one tile; block (column block, tile).
+// of one tile; block (column block, tile).  A, B (or null): the two
+// pre-activations as well, for the backward pass.
 __global__ void __launch_bounds__(256) gemm1_f32_kernel(const float *xp, const float *W1,
                                                         const float *W3, const int4 *tiles,
-                                                        const int *meta, int d, int I, float *H) {
+                                                        const int *meta, int d, int I, float *H,
+                                                        float *A, float *B) {
     const int ti = blockIdx.x;
     if (ti >= meta[0]) return;
     const int4 tile = tiles[ti];
@@ -475,7 +483,13 @@ __global__ void __launch_bounds__(256) gemm1_f32_kernel(const float *xp, const f
             __syncthreads();
         }
         const int r = rr + threadIdx.y;
-        if (r < rows && col < I) H[(long long)(row0 + r) * I + col] = silu_mul_f32(ga, ub);
+        if (r < rows && col < I) {
+            H[(long long)(row0 + r) * I + col] = silu_mul_f32(ga, ub);
+            if (A) {
+                A[(long long)(row0 + r) * I + col] = ga;
+                B[(long long)(row0 + r) * I + col] = ub;
+            }
+        }
     }
 }
 
@@ -572,9 +586,9 @@ cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, 
 
 cudaError_t launch_gemm1_f32(const float *xp, const float *W1, const float *W3, const int4 *tiles,
                              const int *meta, int tiles_cap, int d, int I, float *H,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, float *A, float *B) {
     dim3 grid(tiles_cap, (I + kT - 1) / kT);
-    gemm1_f32_kernel<<<grid, dim3(kT, kT), 0, stream>>>(xp, W1, W3, tiles, meta, d, I, H);
+    gemm1_f32_kernel<<<grid, dim3(kT, kT), 0, stream>>>(xp, W1, W3, tiles, meta, d, I, H, A, B);
     return cudaGetLastError();
 }
 

@@ -488,6 +488,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (c0 + c < w.rows)
                             out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(
                                 silu_mul(__uint_as_float(g[c]), __uint_as_float(v[c])));
+                    if (p.a_out) {  // training: both pre-activations in fp32
+                        const long long o = (long long)w.out_row * p.out_ld + w.mb * kBlockM + row;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            if (c0 + c < w.rows) {
+                                p.a_out[o + (long long)(c0 + c) * p.out_ld] = __uint_as_float(g[c]);
+                                p.b_out[o + (long long)(c0 + c) * p.out_ld] = __uint_as_float(v[c]);
+                            }
+                    }
                 } else if (down) {
                     // Y (fp32): rounded once, after the weighted combine.
                     void *base = (MODE == MODE_EXPERTS) ? p.out2 : p.out;

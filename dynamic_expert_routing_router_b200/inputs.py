@@ -43,6 +43,7 @@ import torch
 # Per-tensor seed offsets.
 _OFF_X, _OFF_WG, _OFF_WM, _OFF_W1, _OFF_W3, _OFF_W2, _OFF_RANK, _OFF_MU = range(1, 9)
 _OFF_SHARED = 20
+_OFF_DY = 30
 _LAYER_STRIDE = 1000
 
 
@@ -169,6 +170,11 @@ def make_tiny(T: int = 64, seed: int = 0, gamma: float | None = None, device="cp
     Wm = Wm - (0.0 if gamma is None else float(gamma)) * mu[None, :]
     W1, W3, W2 = make_experts(sh, seed, device)
     return dict(x=x, W_gate=Wg, W_mask=Wm, W1=W1, W3=W3, W2=W2, mu=mu)
+
+
+def make_upstream_grad(shape: Shape, T: int, seed: int = 0, device="cpu"):
+    """dy [T, d] for the backward pass: i.i.d. N(0, 1), in the layer's dtype."""
+    return _normal((T, shape.d), 1.0, seed + _OFF_DY, device, torch_dtype(shape))
 
 
 def bf16_bits(t: torch.Tensor):

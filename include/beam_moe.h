@@ -124,8 +124,9 @@ typedef struct {
 
 /* Stage slots of one beam_moe_forward call (router GEMM, top-K + mask,
  * grouping, gather, gate/up GEMM, down GEMM, combine).  With token tiles
- * thinner than 128 rows (decode batches) the two expert GEMMs run as one
- * fused launch in the gate/up slot and the down slot is empty; see
+ * thinner than 128 rows (decode batches, bf16) the grouping kernel copies the
+ * token rows itself, so the gather slot is empty, and the two expert GEMMs run
+ * as one fused launch in the gate/up slot, so the down slot is empty too; see
  * beam_moe_forward_kernel_count. */
 #define BEAM_MOE_FORWARD_STAGES 7
 
@@ -220,10 +221,48 @@ beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
                                    float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
                                    float *logits, void *stream);
 
-/* Kernel launches one forward call makes for `desc`: 6 (bf16 with
+/* Kernel launches one forward call makes for `desc`: 5 (bf16 with
  * decode-sized token tiles) or 7, plus 2 with shared experts; 0 for T = 0 or
  * a bad descriptor. */
 int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
+
+/* ------------------------------------------------------------ training --
+ * Backward pass of the layer for training the mask router (techwalker news
+ * article on BEAM, §4: the binary decision is trained through a
+ * straight-through estimator, and a penalty weighted by beta on the
+ * candidates' mask scores pushes towards fewer active experts).  The pages
+ * give both in words; the readings taken here:
+ *   objective  L = sum_t <dy_t, y_t> + beta * sum_t sum_{k<K} sigmoid(z_{t,c_k})
+ *              (the penalty adds up the K candidates' scores of every token;
+ *              divide beta by the token count for a mean)
+ *   estimator  the forward keeps the hard mask of Eq. (6); the backward
+ *              passes the gradient straight through the threshold
+ *              (dm/dsigmoid = 1) and keeps the sigmoid's slope
+ *   candidates every candidate's expert is evaluated, masked or not: candidate
+ *              k's mask gets g_k <dy, E_k(x)> through the estimator either way
+ *   weights    only kept candidates get expert-weight gradients (their
+ *              weight in Eq. 7 is g_k; a masked candidate's is 0)
+ * Arguments: the forward's inputs (same layouts, dtype of desc) and dy [T,d]
+ * in that dtype; beta finite.  desc->n_shared must be 0.
+ * Outputs, fp32, row-major like their weights:
+ *   dx [T,d]                       overwritten
+ *   dW_gate, dW_mask [E,d]         accumulated (+=); dW_mask NULL iff W_mask NULL
+ *   dW1, dW3 [E,I,d], dW2 [E,d,I]  accumulated (+=) for experts with at least
+ *                                  one kept pair; other experts' rows are not
+ *                                  touched (zero them once per step)
+ * Every sum runs in a fixed order: the gradients are bitwise repeatable.
+ * Workspace: beam_moe_backward_workspace_size bytes, 256-byte aligned; the
+ * caller owns it and every output.  Errors as for beam_moe_forward (shared
+ * experts: BEAM_ERR_UNSUPPORTED_SHAPE). */
+size_t beam_moe_backward_workspace_size(const beam_moe_desc *desc);
+beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const void *W_gate,
+                              const void *W_mask, const void *W1, const void *W3, const void *W2,
+                              const void *dy, float beta, float *dx, float *dW_gate,
+                              float *dW_mask, float *dW1, float *dW3, float *dW2,
+                              void *workspace, size_t workspace_bytes, void *stream);
+/* Kernel launches of one beam_moe_backward call (13; 0 for T = 0 or a bad
+ * descriptor). */
+int beam_moe_backward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last
  * call: BEAM_OK, BEAM_ERR_TIMEOUT (a bounded device wait expired, the kernel

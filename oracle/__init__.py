@@ -58,7 +58,7 @@ def _load():
         lib.oracle_max_threads.argtypes = []
         lib.oracle_shared_experts.argtypes = [i, i, i, i, i, p, p, p, p, i, i, p, i]
         lib.oracle_backward.argtypes = [i, i, i, i, i, i, i, d, d, i, p, p, p, p, p, p, p, i, p,
-                                        p, p, p, p, p, p, p, p, i]
+                                        p, p, p, p, p, p, p, p, p, p, i]
         for f in (lib.oracle_logits, lib.oracle_route, lib.oracle_route_f32,
                   lib.oracle_permutation, lib.oracle_experts, lib.oracle_max_threads,
                   lib.oracle_shared_experts, lib.oracle_backward):
@@ -197,10 +197,12 @@ def add_shared(y, x, W1s, W3s, W2s, dtype, t_begin=0, t_end=None, nthreads=0):
 
 
 def backward(x, W_gate, W_mask, W1, W3, W2, dy, K, renorm, dtype, beta=0.0, tau_logit=0.0,
-             ste=True, experts=None, nthreads=0):
+             ste=True, experts=None, logits=None, nthreads=0):
     """Training-mode gradients of L = sum <dy, y> + beta * sum of the candidates'
     sigmoid(z), with the straight-through estimator (ste=False drops its term).
     `experts`: ids whose weight gradients are returned (None: all, in order).
+    `logits`: [T, 2E] (r then z) to route with, e.g. another implementation's
+    fp32 logits (widened exactly); None computes them.
     Returns a dict of fp64 arrays: dx, dW_gate, dW_mask (None without a mask),
     dW1, dW3 [n_sel, I, d], dW2 [n_sel, d, I], u and dz [T, K]."""
     lib = _load()
@@ -210,6 +212,11 @@ def backward(x, W_gate, W_mask, W1, W3, W2, dy, K, renorm, dtype, beta=0.0, tau_
     T, d = x.shape
     E, I, _ = W1.shape
     sel = None if experts is None else np.ascontiguousarray(experts, dtype=np.int32)
+    r_in = z_in = None
+    if logits is not None:
+        lg = np.asarray(logits, dtype=np.float64)
+        r_in = np.ascontiguousarray(lg[:, :E])
+        z_in = np.ascontiguousarray(lg[:, E:2 * E]) if Wm is not None else None
     n_sel = E if sel is None else len(sel)
     out = dict(dx=np.empty((T, d)), dW_gate=np.empty((E, d)),
                dW_mask=np.zeros((E, d)) if Wm is not None else None,
@@ -218,7 +225,7 @@ def backward(x, W_gate, W_mask, W1, W3, W2, dy, K, renorm, dtype, beta=0.0, tau_
     _check(lib.oracle_backward(T, d, E, I, K, int(renorm), _code(dtype), float(tau_logit),
                                float(beta), int(bool(ste)), _ptr(x), _ptr(Wg), _ptr(Wm),
                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), n_sel, _ptr(sel),
-                               _ptr(out["dx"]), _ptr(out["dW_gate"]), _ptr(out["dW_mask"]),
+                               _ptr(r_in), _ptr(z_in), _ptr(out["dx"]), _ptr(out["dW_gate"]), _ptr(out["dW_mask"]),
                                _ptr(out["dW1"]), _ptr(out["dW3"]), _ptr(out["dW2"]),
                                _ptr(out["u"]), _ptr(out["dz"]), int(nthreads)), "backward")
     return out

@@ -316,8 +316,9 @@ static double sigmoid_d(double v) { return 1.0 / (1.0 + exp(-v)); }
 int oracle_backward(int T, int d, int E, int I, int K, int renorm, int dtype, double tau_logit,
                     double beta, int ste, const void *x, const void *W_gate, const void *W_mask,
                     const void *W1, const void *W3, const void *W2, const void *dy, int n_sel,
-                    const int32_t *sel, double *dx, double *dWg, double *dWm, double *dW1,
-                    double *dW3, double *dW2, double *u, double *dz, int nthreads) {
+                    const int32_t *sel, const double *r_in, const double *z_in, double *dx,
+                    double *dWg, double *dWm, double *dW1, double *dW3, double *dW2, double *u,
+                    double *dz, int nthreads) {
     if (T < 0 || d <= 0 || E <= 0 || I <= 0 || K <= 0 || K > E) return -1;
     if (!x || !W_gate || !W1 || !W3 || !W2 || !dy || !dx || !dWg) return -1;
     if (dtype != ORACLE_BF16 && dtype != ORACLE_F32) return -1;
@@ -348,8 +349,14 @@ int oracle_backward(int T, int d, int E, int I, int K, int renorm, int dtype, do
         rc = -1;
         goto done;
     }
-    rc = oracle_logits(T, d, E, dtype, x, W_gate, W_mask, r, W_mask ? zl : NULL);
-    if (rc) goto done;
+    if (r_in) {
+        memcpy(r, r_in, sizeof(double) * TE);
+        if (W_mask && z_in) memcpy(zl, z_in, sizeof(double) * TE);
+        else if (W_mask) { rc = -1; goto done; }
+    } else {
+        rc = oracle_logits(T, d, E, dtype, x, W_gate, W_mask, r, W_mask ? zl : NULL);
+        if (rc) goto done;
+    }
     rc = oracle_route(T, E, K, renorm, tau_logit, r, W_mask ? zl : NULL, cand, g, idx, w, NULL,
                       NULL);
     if (rc) goto done;

@@ -97,12 +97,15 @@ int oracle_shared_experts(int T, int d, int n_shared, int Is, int dtype, const v
  * no penalty).  Outputs fp64, overwritten: dx [T,d]; dWg, dWm [E,d] (dWm
  * untouched without a mask); u, dz [T,K] or NULL; the expert gradients of the
  * n_sel experts listed in sel (sel NULL: all E in order), each NULL-able:
- * dW1, dW3 [n_sel,I,d], dW2 [n_sel,d,I].  Returns -2 on a non-finite value. */
+ * dW1, dW3 [n_sel,I,d], dW2 [n_sel,d,I].  Returns -2 on a non-finite value.
+ * r_in, z_in [T,E]: logits to route with instead of computing them (another
+ * implementation's, widened), or NULL; z_in is used only with a mask. */
 int oracle_backward(int T, int d, int E, int I, int K, int renorm, int dtype, double tau_logit,
                     double beta, int ste, const void *x, const void *W_gate, const void *W_mask,
                     const void *W1, const void *W3, const void *W2, const void *dy, int n_sel,
-                    const int32_t *sel, double *dx, double *dWg, double *dWm, double *dW1,
-                    double *dW3, double *dW2, double *u, double *dz, int nthreads);
+                    const int32_t *sel, const double *r_in, const double *z_in, double *dx,
+                    double *dWg, double *dWm, double *dW1, double *dW3, double *dW2, double *u,
+                    double *dz, int nthreads);
 
 /* Threads the OpenMP runtime would use by default (for reporting). */
 int oracle_max_threads(void);

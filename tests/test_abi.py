@@ -137,3 +137,23 @@ def test_shared_expert_descriptor_rules():
     vp = ctypes.c_void_p
     ptrs = [vp(4096 * (i + 1)) for i in range(8)]
     assert L.beam_moe_forward(ctypes.byref(ok), *ptrs, ctypes.c_size_t(1 << 40), None) == 1
+
+
+def test_backward_descriptor_and_argument_checks():
+    dsc = abi.desc(8, 2048, 128, 768, 8, "bf16", 1)
+    assert abi.backward_workspace_size(dsc) > abi.workspace_size(dsc)
+    assert abi.backward_kernel_count(dsc) == 13
+    assert abi.backward_kernel_count(abi.desc(0, 2048, 128, 768, 8, "bf16", 1)) == 0
+    shared = abi.desc(8, 2048, 64, 1408, 6, "bf16", 1, n_shared=2, I_shared=1408)
+    assert abi.backward_workspace_size(shared) == 0  # shared experts: forward only
+    L = abi.lib()
+    p = [ctypes.c_void_p(4096 * (i + 1)) for i in range(13)]
+    big = ctypes.c_size_t(1 << 40)
+
+    def call(desc, beta, dWm):
+        return L.beam_moe_backward(ctypes.byref(desc), p[0], p[1], p[2], p[3], p[4], p[5], p[6],
+                                   ctypes.c_float(beta), p[7], p[8], dWm, p[9], p[10], p[11],
+                                   p[12], big, None)
+    assert call(dsc, 0.1, None) == 1            # W_mask given, dW_mask missing
+    assert call(dsc, float("nan"), p[0]) == 1   # beta must be finite
+    assert call(shared, 0.1, p[0]) == 2         # unsupported: shared experts
