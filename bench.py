@@ -51,7 +51,7 @@ def flush_l2(buf, i):
     flush's own write-backs."""
     import torch
     buf.fill_(i & 255)
-    buf.view(-1, 1 << 20).sum(dtype=torch.int64)
+    buf.view(torch.int32).amax()  # one read pass, no conversion copy
 
 
 # ----------------------------------------------------------- distributed --

@@ -149,113 +149,164 @@ __global__ void __launch_bounds__(256) bw_token_kernel(const BwArgs a, const TIn
     }
 }
 
-// ------------------------------------------------- kept-row tile products --
-// For one tile of the candidate grouping and a 256-column slice, the kept rows
-// r get C[r][n] = sum_k A[r][k] B_e[k][n] (+ A2 B2_e), where B_e is row-major
-// [Kdim][N] at B + e * Kdim * N.  Threads: 4 row groups x 64 column groups,
-// 4 x 4 outputs each; kept rows are compacted into groups of 16 first.
-//   DH: A = dyp (dtype), B = W2 (Kdim = d, N = I); with dh = w C:
-//       da = dh b SiLU'(a), db = dh SiLU(a) (a, b from the forward buffers)
-//   DX: A = da, A2 = db (f32), B = W1, B2 = W3 (Kdim = I, N = d); dxp = C
-enum { TG_DH = 0, TG_DX = 1 };
-constexpr int kTgCols = 256, kTgKc = 16;
-
-template <int MODE, typename TA, typename TB>
-__global__ void __launch_bounds__(256) tile_product_kernel(const BwArgs a, const TA *A,
-                                                           const TA *A2, const TB *B,
-                                                           const TB *B2, int Kdim, int N) {
-    __shared__ int s_rows[kMaxTileRows];
-    __shared__ float s_w[kMaxTileRows];
-    __shared__ int s_n;
-    __shared__ float As[16][kTgKc + 1];
-    __shared__ __align__(16) float Bs[kTgKc][kTgCols];
-    griddep_wait();
-    griddep_launch_dependents();
-    const int ti = blockIdx.x;
-    if (ti >= a.meta[0]) return;
-    const int4 tile = a.tiles[ti];
-    const int e = tile.x, row0 = tile.y, rows = tile.z;
-    const int n0 = blockIdx.y * kTgCols;
-    const int tid = threadIdx.x, tr = tid >> 6, tc = tid & 63;
-    if (tid == 0) {
-        int n = 0;
-        for (int r = 0; r < rows; ++r) {
-            const int pr = a.pair[row0 + r];
-            if (pr >= 0 && a.idx[pr] >= 0) {  // kept candidate
-                s_rows[n] = row0 + r;
-                s_w[n] = a.w[pr];
-                ++n;
-            }
-        }
-        s_n = n;
+// Kept rows of one tile of the candidate grouping, compacted in order into
+// s_row / s_w (row index, w = g m).  rows <= kMaxTileRows.
+__device__ int stage_kept_rows(const BwArgs &a, int row0, int rows, int *s_flag, float *s_fw,
+                               int *s_row, float *s_w, int *s_n) {
+    for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+        const int pr = a.pair[row0 + r];
+        const bool kept = pr >= 0 && a.idx[pr] >= 0;
+        s_flag[r] = kept ? row0 + r : -1;
+        s_fw[r] = kept ? a.w[pr] : 0.0f;
     }
     __syncthreads();
-    const int nk = s_n;
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int r = 0; r < rows; ++r)
+            if (s_flag[r] >= 0) {
+                s_row[n] = s_flag[r];
+                s_w[n] = s_fw[r];
+                ++n;
+            }
+        *s_n = n;
+    }
+    __syncthreads();
+    return *s_n;
+}
+
+// Eight consecutive elements as fp32 (16-byte aligned for bf16, 32 for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+    const float4 x = *reinterpret_cast<const float4 *>(p);
+    const float4 y = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+
+// ------------------------------------------------- kept-row products (split) --
+// For one tile and one split s of the reduction range, the kept rows r get
+//   part[s][r][n] = sum_{k in split s} A[r][k] B_e[k][n]  (+ A2[r][k] B2_e[k][n])
+// with B_e row-major [Kdim][N] at B + e * Kdim * N.  Each thread owns 8
+// consecutive columns and streams them with one 16-byte load per k; the A rows
+// (4 kept rows at a time) are staged in shared memory 512 k at a time.
+//   DH: A = dyp, B = W2 (Kdim = d, N = I)
+//   DX: A = da, A2 = db, B = W1, B2 = W3 (Kdim = I, N = d)
+enum { TG_DH = 0, TG_DX = 1 };
+constexpr int kRgKch = 512;
+
+template <int MODE, typename TA, typename TB>
+__global__ void __launch_bounds__(256) rowgemm_kernel(const BwArgs a, const TA *A, const TA *A2,
+                                                      const TB *B, const TB *B2, int Kdim, int N,
+                                                      int S) {
+    __shared__ int s_flag[kMaxTileRows], s_row[kMaxTileRows], s_n;
+    __shared__ float s_fw[kMaxTileRows], s_w[kMaxTileRows];
+    __shared__ __align__(16) float As[4][kRgKch];
+    __shared__ __align__(16) float A2s[MODE == TG_DX ? 4 : 1][MODE == TG_DX ? kRgKch : 4];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int ti = blockIdx.x, sp = blockIdx.y;
+    if (ti >= a.meta[0]) return;
+    const int4 tile = a.tiles[ti];
+    const int e = tile.x;
+    const int nk = stage_kept_rows(a, tile.y, tile.z, s_flag, s_fw, s_row, s_w, &s_n);
+    if (nk == 0) return;
+    const int kc = Kdim / S, k0 = sp * kc;
+    const int NG = N / 8;
     const long long bstride = (long long)Kdim * N;
-    for (int g0 = 0; g0 < nk; g0 += 16) {
-        const int gn = min(16, nk - g0);
-        const bool active = tr * 4 < gn;  // warp-uniform: 2 warps per row group
-        float c[4][4];
+    const TB *Be = B + (long long)e * bstride;
+    const TB *B2e = (MODE == TG_DX) ? B2 + (long long)e * bstride : nullptr;
+    float *part = a.part + (long long)sp * a.p_cap * N;
+    for (int g0 = 0; g0 < nk; g0 += 4) {
+        const int gn = min(4, nk - g0);
+        for (int cgb = 0; cgb < NG; cgb += blockDim.x) {
+            const int cg = cgb + threadIdx.x;
+            const bool active = cg < NG;
+            float acc[4][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) c[i][j] = 0.0f;
-        for (int pass = 0; pass < (MODE == TG_DX ? 2 : 1); ++pass) {
-            const TA *Ap = pass ? A2 : A;
-            const TB *Bp = (pass ? B2 : B) + (long long)e * bstride;
-            for (int k0 = 0; k0 < Kdim; k0 += kTgKc) {
-                {   // A: 16 rows x 16 k, one element per thread
-                    const int rr = tid >> 4, kk = tid & 15;
-                    As[rr][kk] = (rr < gn && k0 + kk < Kdim)
-                                     ? load_f(Ap, (long long)s_rows[g0 + rr] * Kdim + k0 + kk)
-                                     : 0.0f;
-                }
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {  // B: 16 k x 256 columns
-                    const int idx = q * 256 + tid, kk = idx >> 8, nn = idx & 255;
-                    Bs[kk][nn] = (n0 + nn < N && k0 + kk < Kdim)
-                                     ? load_f(Bp, (long long)(k0 + kk) * N + n0 + nn)
-                                     : 0.0f;
+                for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
+            for (int kb = k0; kb < k0 + kc; kb += kRgKch) {
+                const int kn = min(kRgKch, k0 + kc - kb);
+                for (int q = threadIdx.x; q < 4 * kn; q += blockDim.x) {
+                    const int r = q / kn, k = q - r * kn;
+                    const long long ro = (r < gn) ? (long long)s_row[g0 + r] * Kdim : 0;
+                    As[r][k] = (r < gn) ? load_f(A, ro + kb + k) : 0.0f;
+                    if (MODE == TG_DX) A2s[r][k] = (r < gn) ? load_f(A2, ro + kb + k) : 0.0f;
                 }
                 __syncthreads();
                 if (active) {
+                    const TB *bp = Be + (long long)kb * N + cg * 8;
+                    const TB *bp2 = (MODE == TG_DX) ? B2e + (long long)kb * N + cg * 8 : nullptr;
+#pragma unroll 4
+                    for (int k = 0; k < kn; ++k) {
+                        float bv[8];
+                        load8(bp + (long long)k * N, bv);
 #pragma unroll
-                    for (int kk = 0; kk < kTgKc; ++kk) {
-                        const float4 bv = *reinterpret_cast<const float4 *>(&Bs[kk][tc * 4]);
+                        for (int r = 0; r < 4; ++r) {
+                            const float av = As[r][k];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float av = As[tr * 4 + i][kk];
-                            c[i][0] = fmaf(av, bv.x, c[i][0]);
-                            c[i][1] = fmaf(av, bv.y, c[i][1]);
-                            c[i][2] = fmaf(av, bv.z, c[i][2]);
-                            c[i][3] = fmaf(av, bv.w, c[i][3]);
+                            for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av, bv[c], acc[r][c]);
+                        }
+                        if (MODE == TG_DX) {
+                            load8(bp2 + (long long)k * N, bv);
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                const float av = A2s[r][k];
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av, bv[c], acc[r][c]);
+                            }
                         }
                     }
                 }
                 __syncthreads();
             }
-        }
-        if (active) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int lr = tr * 4 + i;
-                if (lr >= gn) continue;
-                const long long row = s_rows[g0 + lr];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int n = n0 + tc * 4 + j;
-                    if (n >= N) continue;
-                    const long long o = row * N + n;
-                    if (MODE == TG_DH) {
-                        const float dh = s_w[g0 + lr] * c[i][j];
-                        const float av = a.A[o], bv = a.B[o], sa = sigm(av);
-                        a.da[o] = dh * bv * sa * (1.0f + av * (1.0f - sa));
-                        a.db[o] = dh * av * sa;
-                    } else {
-                        a.dxp[o] = c[i][j];
-                    }
+            if (active) {
+                for (int r = 0; r < gn; ++r) {
+                    float *o = part + (long long)s_row[g0 + r] * N + cg * 8;
+                    *reinterpret_cast<float4 *>(o) =
+                        make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+                    *reinterpret_cast<float4 *>(o + 4) =
+                        make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
                 }
             }
+        }
+    }
+}
+
+// dh = w * (sum of the splits, in order); da = dh b SiLU'(a), db = dh SiLU(a),
+// and h = SiLU(a) b in fp32, for the kept rows of a tile.
+__global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S) {
+    __shared__ int s_flag[kMaxTileRows], s_row[kMaxTileRows], s_n;
+    __shared__ float s_fw[kMaxTileRows], s_w[kMaxTileRows];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int ti = blockIdx.x;
+    if (ti >= a.meta[0]) return;
+    const int4 tile = a.tiles[ti];
+    const int nk = stage_kept_rows(a, tile.y, tile.z, s_flag, s_fw, s_row, s_w, &s_n);
+    const int I = a.I;
+    const long long split = (long long)a.p_cap * I;
+    for (int q = 0; q < nk; ++q) {
+        const long long row = s_row[q];
+        for (int i = threadIdx.x; i < I; i += blockDim.x) {
+            const long long o = row * I + i;
+            float c = 0.0f;
+            for (int sp = 0; sp < S; ++sp) c += a.part[sp * split + o];
+            const float dh = s_w[q] * c;
+            const float av = a.A[o], bv = a.B[o], sa = sigm(av);
+            a.da[o] = dh * bv * sa * (1.0f + av * (1.0f - sa));
+            a.db[o] = dh * av * sa;
+            a.h[o] = av * sa * bv;
         }
     }
 }
@@ -263,7 +314,7 @@ __global__ void __launch_bounds__(256) tile_product_kernel(const BwArgs a, const
 // ---------------------------------------------------------------------- dx --
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *Wg,
-                                                    const TIn *Wm) {
+                                                    const TIn *Wm, int S) {
     __shared__ float s_dr[kMaxE];
     __shared__ int s_pos[kMaxK], s_cand[kMaxK];
     __shared__ float s_dz[kMaxK];
@@ -271,6 +322,7 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *W
     griddep_wait();
     griddep_launch_dependents();
     const int K = a.K, E = a.E, d = a.d;
+    const long long split = (long long)a.p_cap * d;
     for (int t = blockIdx.x; t < a.T; t += gridDim.x) {
         for (int e = threadIdx.x; e < E; e += blockDim.x) s_dr[e] = a.dr[(long long)t * E + e];
         if (threadIdx.x < K) {
@@ -283,8 +335,12 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *W
         __syncthreads();
         for (int j = threadIdx.x; j < d; j += blockDim.x) {
             float acc = 0.0f;
-            for (int k = 0; k < K; ++k)  // expert part, kept slots in order
-                if (s_kept[k]) acc += a.dxp[(long long)s_pos[k] * d + j];
+            for (int k = 0; k < K; ++k)  // expert part: kept slots in order, splits in order
+                if (s_kept[k]) {
+                    float c = 0.0f;
+                    for (int sp = 0; sp < S; ++sp) c += a.part[sp * split + (long long)s_pos[k] * d + j];
+                    acc += c;
+                }
             for (int e = 0; e < E; ++e) {  // W_gate^T dr
                 const float c = s_dr[e];
                 if (c != 0.0f) acc = fmaf(c, load_f(Wg, (long long)e * d + j), acc);
@@ -299,12 +355,34 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *W
 }
 
 // -------------------------------------------------------- weight gradients --
-// dW1_e[i] += sum over kept rows r of e (in order) da[r][i] x_r, likewise dW3
-// with db.  Block (expert, 4 rows of I); threads over d.
+// Kept rows of expert e (rows [first, first + n) of the candidate grouping),
+// chunk [r0, r0 + cnt): compacted row indices into s_kr (returns how many).
+constexpr int kWgChunk = 256;
+__device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, int *s_flag,
+                                  int *s_kr, int *s_n) {
+    for (int q = threadIdx.x; q < cnt; q += blockDim.x) {
+        const int r = first + r0 + q;
+        s_flag[q] = a.idx[a.pair[r]] >= 0 ? r : -1;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int q = 0; q < cnt; ++q)
+            if (s_flag[q] >= 0) s_kr[n++] = s_flag[q];
+        *s_n = n;
+    }
+    __syncthreads();
+    return *s_n;
+}
+
+// dW1_e[i] += sum over kept rows (in order) da[r][i] x_r, dW3 likewise with db.
+// Block (expert, 4 rows of I); each thread owns 8 consecutive columns of d.
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn *xp, float *dW1,
                                                       float *dW3) {
-    __shared__ int s_first;
+    __shared__ int s_first, s_n;
+    __shared__ int s_flag[kWgChunk], s_kr[kWgChunk];
+    __shared__ float s_da[kWgChunk][4], s_db[kWgChunk][4];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
@@ -313,54 +391,67 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
     const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
     const int n = a.counts_all[e];
     const int d = a.d, I = a.I;
-    constexpr int kCols = 8;  // d <= 2048 per pass of 256 threads
-    for (int jb = 0; jb < d; jb += 256 * kCols) {
-        float g1[4][kCols], g3[4][kCols];
+    for (int jb = 0; jb < d; jb += 8 * blockDim.x) {
+        const int j = jb + threadIdx.x * 8;
+        const bool active = j < d;
+        float g1[4][8], g3[4][8];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) g1[i][c] = g3[i][c] = 0.0f;
-        for (int r = first; r < first + n; ++r) {
-            const int pr = a.pair[r];
-            if (a.idx[pr] < 0) continue;  // masked candidate: no weight gradient
-            float va[4], vb[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int c = 0; c < 8; ++c) g1[i][c] = g3[i][c] = 0.0f;
+        for (int r0 = 0; r0 < n; r0 += kWgChunk) {
+            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_flag, s_kr,
+                                              &s_n);
+            for (int q = threadIdx.x; q < 4 * nk; q += blockDim.x) {
+                const int kq = q >> 2, i = q & 3;
                 const bool ok = i0 + i < I;
-                va[i] = ok ? a.da[(long long)r * I + i0 + i] : 0.0f;
-                vb[i] = ok ? a.db[(long long)r * I + i0 + i] : 0.0f;
+                s_da[kq][i] = ok ? a.da[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
+                s_db[kq][i] = ok ? a.db[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
             }
+            __syncthreads();
+            if (active) {
+#pragma unroll 2
+                for (int kq = 0; kq < nk; ++kq) {
+                    float xv[8];
+                    load8(xp + (long long)s_kr[kq] * d + j, xv);
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-                const int j = jb + c * 256 + threadIdx.x;
-                const float xv = j < d ? load_f(xp, (long long)r * d + j) : 0.0f;
+                    for (int i = 0; i < 4; ++i) {
+                        const float va = s_da[kq][i], vb = s_db[kq][i];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    g1[i][c] = fmaf(va[i], xv, g1[i][c]);
-                    g3[i][c] = fmaf(vb[i], xv, g3[i][c]);
+                        for (int c = 0; c < 8; ++c) {
+                            g1[i][c] = fmaf(va, xv[c], g1[i][c]);
+                            g3[i][c] = fmaf(vb, xv[c], g3[i][c]);
+                        }
+                    }
                 }
             }
+            __syncthreads();
         }
+        if (active) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (i0 + i >= I) continue;
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-                const int j = jb + c * 256 + threadIdx.x;
-                if (j >= d) continue;
+            for (int i = 0; i < 4; ++i) {
+                if (i0 + i >= I) continue;
                 const long long o = ((long long)e * I + i0 + i) * d + j;
-                dW1[o] += g1[i][c];
-                dW3[o] += g3[i][c];
+                float4 *p1 = reinterpret_cast<float4 *>(dW1 + o);
+                float4 *p3 = reinterpret_cast<float4 *>(dW3 + o);
+                float4 u0 = p1[0], u1 = p1[1], v0 = p3[0], v1 = p3[1];
+                u0.x += g1[i][0]; u0.y += g1[i][1]; u0.z += g1[i][2]; u0.w += g1[i][3];
+                u1.x += g1[i][4]; u1.y += g1[i][5]; u1.z += g1[i][6]; u1.w += g1[i][7];
+                v0.x += g3[i][0]; v0.y += g3[i][1]; v0.z += g3[i][2]; v0.w += g3[i][3];
+                v1.x += g3[i][4]; v1.y += g3[i][5]; v1.z += g3[i][6]; v1.w += g3[i][7];
+                p1[0] = u0; p1[1] = u1; p3[0] = v0; p3[1] = v1;
             }
         }
     }
 }
 
-// dW2_e[j] += sum over kept rows r of e (in order) w_r dy_r[j] h_r, with
-// h = SiLU(a) b in fp32.  Block (expert, 8 rows of d); threads over I.
+// dW2_e[j] += sum over kept rows (in order) w_r dy_r[j] h_r (h fp32 from the
+// finalize step).  Block (expert, 8 rows of d); each thread owns 4 columns of I.
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *dyp, float *dW2) {
-    __shared__ int s_first;
+    __shared__ int s_first, s_n;
+    __shared__ int s_flag[kWgChunk], s_kr[kWgChunk];
+    __shared__ float s_dy[kWgChunk][8];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
@@ -369,40 +460,48 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
     const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
     const int n = a.counts_all[e];
     const int d = a.d, I = a.I;
-    constexpr int kCols = 8;  // I <= 2048 per pass
-    for (int ib = 0; ib < I; ib += 256 * kCols) {
-        float g[8][kCols];
+    for (int ib = 0; ib < I; ib += 4 * blockDim.x) {
+        const int i = ib + threadIdx.x * 4;
+        const bool active = i < I;
+        float g[8][4];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj)
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) g[jj][c] = 0.0f;
-        for (int r = first; r < first + n; ++r) {
-            const int pr = a.pair[r];
-            if (a.idx[pr] < 0) continue;
-            const float wk = a.w[pr];
-            float dv[8];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                dv[jj] = (j0 + jj < d) ? wk * load_f(dyp, (long long)r * d + j0 + jj) : 0.0f;
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-                const int i = ib + c * 256 + threadIdx.x;
-                float h = 0.0f;
-                if (i < I) {
-                    const float av = a.A[(long long)r * I + i], bv = a.B[(long long)r * I + i];
-                    h = av * sigm(av) * bv;
-                }
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) g[jj][c] = fmaf(dv[jj], h, g[jj][c]);
+            for (int c = 0; c < 4; ++c) g[jj][c] = 0.0f;
+        for (int r0 = 0; r0 < n; r0 += kWgChunk) {
+            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_flag, s_kr,
+                                              &s_n);
+            for (int q = threadIdx.x; q < 8 * nk; q += blockDim.x) {
+                const int kq = q >> 3, jj = q & 7;
+                const int r = s_kr[kq];
+                const float wk = a.w[a.pair[r]];
+                s_dy[kq][jj] = (j0 + jj < d) ? wk * load_f(dyp, (long long)r * d + j0 + jj) : 0.0f;
             }
+            __syncthreads();
+            if (active) {
+#pragma unroll 2
+                for (int kq = 0; kq < nk; ++kq) {
+                    const float4 hv = *reinterpret_cast<const float4 *>(a.h + (long long)s_kr[kq] * I + i);
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const float dv = s_dy[kq][jj];
+                        g[jj][0] = fmaf(dv, hv.x, g[jj][0]);
+                        g[jj][1] = fmaf(dv, hv.y, g[jj][1]);
+                        g[jj][2] = fmaf(dv, hv.z, g[jj][2]);
+                        g[jj][3] = fmaf(dv, hv.w, g[jj][3]);
+                    }
+                }
+            }
+            __syncthreads();
         }
+        if (active) {
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            if (j0 + jj >= d) continue;
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-                const int i = ib + c * 256 + threadIdx.x;
-                if (i < I) dW2[((long long)e * d + j0 + jj) * I + i] += g[jj][c];
+            for (int jj = 0; jj < 8; ++jj) {
+                if (j0 + jj >= d) continue;
+                float4 *p = reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
+                float4 v = *p;
+                v.x += g[jj][0]; v.y += g[jj][1]; v.z += g[jj][2]; v.w += g[jj][3];
+                *p = v;
             }
         }
     }
@@ -418,7 +517,7 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
     griddep_launch_dependents();
     const int e = blockIdx.x;
     const int j = blockIdx.y * 256 + threadIdx.x;
-    const int d = a.d, E = a.E, K = a.K;
+    const int d = a.d, E = a.E;
     float gg = 0.0f;
     for (int t = 0; t < a.T; ++t) {
         const float c = a.dr[(long long)t * E + e];
@@ -428,12 +527,10 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
     if (dWm) {
         const int first = a.counts_all[e] ? expert_first_row(a.tiles, a.meta[0], e, &s_first) : 0;
         for (int r = first; r < first + a.counts_all[e]; ++r) {
-            const int pr = a.pair[r];
-            const float c = a.dz[pr];
+            const float c = a.dz[a.pair[r]];
             if (j < d) gm = fmaf(c, load_f(xp, (long long)r * d + j), gm);
         }
     }
-    (void)K;
     if (j < d) {
         dWg[(long long)e * d + j] += gg;
         if (dWm) dWm[(long long)e * d + j] += gm;
@@ -449,8 +546,7 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
                                    float *dW3, float *dW2, int n_sm, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
     const int tb = a.T < 8 * n_sm ? a.T : 8 * n_sm;
-    const dim3 g_dh(a.tiles_cap, (a.I + kTgCols - 1) / kTgCols);
-    const dim3 g_dx(a.tiles_cap, (a.d + kTgCols - 1) / kTgCols);
+    const dim3 g_dh(a.tiles_cap, a.S), g_fin(a.tiles_cap);
     const dim3 g_w13(a.E, (a.I + 3) / 4), g_w2(a.E, (a.d + 7) / 8), g_r(a.E, (a.d + 255) / 256);
     cudaError_t e;
     if (dtype == BEAM_BF16) {
@@ -458,16 +554,16 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
         const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
         const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
         if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-        if ((e = launch_pdl(tile_product_kernel<TG_DH, T, T>, g_dh, dim3(256), 0, st, a, dypb,
-                            dypb, static_cast<const T *>(W2), static_cast<const T *>(W2), a.d,
-                            a.I)))
+        if ((e = launch_pdl(rowgemm_kernel<TG_DH, T, T>, g_dh, dim3(256), 0, st, a, dypb, dypb,
+                            static_cast<const T *>(W2), static_cast<const T *>(W2), a.d, a.I, a.S)))
             return e;
-        if ((e = launch_pdl(tile_product_kernel<TG_DX, float, T>, g_dx, dim3(256), 0, st, a,
+        if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.S))) return e;
+        if ((e = launch_pdl(rowgemm_kernel<TG_DX, float, T>, g_dh, dim3(256), 0, st, a,
                             static_cast<const float *>(a.da), static_cast<const float *>(a.db),
-                            static_cast<const T *>(W1), static_cast<const T *>(W3), a.I, a.d)))
+                            static_cast<const T *>(W1), static_cast<const T *>(W3), a.I, a.d, a.S)))
             return e;
         if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a,
-                            static_cast<const T *>(Wg), static_cast<const T *>(Wm))))
+                            static_cast<const T *>(Wg), static_cast<const T *>(Wm), a.S)))
             return e;
         if ((e = launch_pdl(bw_dw13_kernel<T>, g_w13, dim3(256), 0, st, a, xpb, dW1, dW3)))
             return e;
@@ -478,15 +574,16 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
     const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
     const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
     if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-    if ((e = launch_pdl(tile_product_kernel<TG_DH, T, T>, g_dh, dim3(256), 0, st, a, dypb, dypb,
-                        static_cast<const T *>(W2), static_cast<const T *>(W2), a.d, a.I)))
+    if ((e = launch_pdl(rowgemm_kernel<TG_DH, T, T>, g_dh, dim3(256), 0, st, a, dypb, dypb,
+                        static_cast<const T *>(W2), static_cast<const T *>(W2), a.d, a.I, a.S)))
         return e;
-    if ((e = launch_pdl(tile_product_kernel<TG_DX, float, T>, g_dx, dim3(256), 0, st, a,
+    if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.S))) return e;
+    if ((e = launch_pdl(rowgemm_kernel<TG_DX, float, T>, g_dh, dim3(256), 0, st, a,
                         static_cast<const float *>(a.da), static_cast<const float *>(a.db),
-                        static_cast<const T *>(W1), static_cast<const T *>(W3), a.I, a.d)))
+                        static_cast<const T *>(W1), static_cast<const T *>(W3), a.I, a.d, a.S)))
         return e;
     if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a,
-                        static_cast<const T *>(Wg), static_cast<const T *>(Wm))))
+                        static_cast<const T *>(Wg), static_cast<const T *>(Wm), a.S)))
         return e;
     if ((e = launch_pdl(bw_dw13_kernel<T>, g_w13, dim3(256), 0, st, a, xpb, dW1, dW3))) return e;
     if ((e = launch_pdl(bw_dw2_kernel<T>, g_w2, dim3(256), 0, st, a, dypb, dW2))) return e;

@@ -450,8 +450,9 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
 // The backward workspace is the forward plan (its grouping now holds every
 // candidate: T*K pairs fit p_cap) followed by the training-only arrays.
 struct BwdPlan {
+    int S;  // reduction splits of the kept-row products
     size_t off_cand, off_gk, off_counts_all, off_logits, off_dyp, off_A, off_B, off_da, off_db,
-        off_dxp, off_u, off_dz, off_dr, bytes;
+        off_h, off_part, off_u, off_dz, off_dr, bytes;
 };
 
 beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan *B) {
@@ -476,7 +477,11 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     B->off_B = take(4 * pc * I);
     B->off_da = take(4 * pc * I);
     B->off_db = take(4 * pc * I);
-    B->off_dxp = take(4 * pc * dd);
+    B->off_h = take(4 * pc * I);
+    // Thin decode tiles leave most SMs idle with one block per tile: split the
+    // reduction of the kept-row products four ways (d and I are multiples of 8).
+    B->S = P->BN < 128 ? 4 : 1;
+    B->off_part = take(4 * size_t(B->S) * pc * (dd > I ? dd : I));
     B->off_u = take(4 * T * K);
     B->off_dz = take(4 * T * K);
     B->off_dr = take(4 * T * E);
@@ -606,6 +611,8 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
     a.renorm = d->renorm_topk;
     a.has_mask = Wm != nullptr;
     a.tiles_cap = P.tiles_cap;
+    a.p_cap = P.p_cap;
+    a.S = B.S;
     a.beta = beta;
     a.Y = y;
     a.logits = logits;
@@ -623,7 +630,8 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
     a.B = Bv;
     a.da = reinterpret_cast<float *>(ws + B.off_da);
     a.db = reinterpret_cast<float *>(ws + B.off_db);
-    a.dxp = reinterpret_cast<float *>(ws + B.off_dxp);
+    a.h = reinterpret_cast<float *>(ws + B.off_h);
+    a.part = reinterpret_cast<float *>(ws + B.off_part);
     a.u = reinterpret_cast<float *>(ws + B.off_u);
     a.dz = reinterpret_cast<float *>(ws + B.off_dz);
     a.dr = reinterpret_cast<float *>(ws + B.off_dr);
@@ -705,9 +713,10 @@ int beam_moe_backward_kernel_count(const beam_moe_desc *desc) {
     beam_moe_plan_info P;
     BwdPlan B;
     if (make_bwd_plan(desc, &P, &B) != BEAM_OK || desc->T == 0) return 0;
-    // router, top-K, grouping, dy gather, gate/up, down, then the seven
-    // CUDA-core stages (token, dh, dxp, dx, dW1/dW3, dW2, router weights)
-    return 13;
+    // router, top-K, grouping, dy gather, gate/up, down, then the eight
+    // CUDA-core stages (token, dh product, dh finalize, dx product, dx,
+    // dW1/dW3, dW2, router weights)
+    return 14;
 }
 
 size_t beam_moe_workspace_size(const beam_moe_desc *desc) {

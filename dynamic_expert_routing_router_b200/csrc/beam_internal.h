@@ -147,7 +147,8 @@ cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const floa
 // Training-mode backward (backward.cu).  Rows are those of the grouping of all
 // candidates (masked ones included); every array lives in the workspace.
 struct BwArgs {
-    int T, d, E, I, K, renorm, has_mask, tiles_cap;
+    int T, d, E, I, K, renorm, has_mask, tiles_cap, p_cap;
+    int S;                   // splits of the reduction in the kept-row products
     float beta;
     const float *Y;          // [p_cap][d] every candidate's expert output
     const float *logits;     // [T][2E] router logits (r, then z)
@@ -163,7 +164,8 @@ struct BwArgs {
     const int *counts_all;   // [E] candidates per expert
     const float *A, *B;      // [p_cap][I] gate / up pre-activations
     float *da, *db;          // [p_cap][I]
-    float *dxp;              // [p_cap][d] expert part of dx per kept row
+    float *h;                // [p_cap][I] SiLU(a) b in fp32 (kept rows)
+    float *part;             // [S][p_cap][max(d, I)] split partial products
     float *u, *dz;           // [T][K]
     float *dr;               // [T][E]
     float *dx;               // [T][d]

@@ -260,7 +260,7 @@ beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const vo
                               const void *dy, float beta, float *dx, float *dW_gate,
                               float *dW_mask, float *dW1, float *dW3, float *dW2,
                               void *workspace, size_t workspace_bytes, void *stream);
-/* Kernel launches of one beam_moe_backward call (13; 0 for T = 0 or a bad
+/* Kernel launches of one beam_moe_backward call (14; 0 for T = 0 or a bad
  * descriptor). */
 int beam_moe_backward_kernel_count(const beam_moe_desc *desc);
 
