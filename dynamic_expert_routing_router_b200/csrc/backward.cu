@@ -193,24 +193,44 @@ __device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
 }
 
 // ------------------------------------------------- kept-row products (split) --
-// For one tile and one split s of the reduction range, the kept rows r get
-//   part[s][r][n] = sum_{k in split s} A[r][k] B_e[k][n]  (+ A2[r][k] B2_e[k][n])
-// with B_e row-major [Kdim][N] at B + e * Kdim * N.  Each thread owns 8
-// consecutive columns and streams them with one 16-byte load per k; the A rows
-// (4 kept rows at a time) are staged in shared memory 512 k at a time.
+// For one tile and one split sp of the reduction range, the kept rows r get
+//   part[sp][r][n] = sum_{k in split} A[r][k] B_e[k][n]  (+ A2[r][k] B2_e[k][n])
+// with B_e row-major [Kdim][N] at B + e * Kdim * N.
 //   DH: A = dyp, B = W2 (Kdim = d, N = I)
 //   DX: A = da, A2 = db, B = W1, B2 = W3 (Kdim = I, N = d)
+// The weight rows stream through a 4-stage shared-memory ring of 16-byte
+// cp.async copies issued by every thread, so the copies in flight do not
+// depend on how many threads compute.  A stage is 16 KB: 8 k-rows (DH) or 4
+// k-rows of each matrix (DX) of one column pass of 2 KB of row (1024 bf16 /
+// 512 fp32 columns, 8 per computing thread).  Kept rows go in groups of 4,
+// whose A values sit in shared memory for the whole split.
 enum { TG_DH = 0, TG_DX = 1 };
-constexpr int kRgKch = 512;
+constexpr int kRgStages = 4;
+template <int MODE>
+struct RgCfg {
+    static constexpr int KCH = MODE == TG_DX ? 4 : 8;  // k-rows per stage
+    static constexpr int NMAT = MODE == TG_DX ? 2 : 1;
+};
+template <int MODE, typename TB>
+__host__ __device__ constexpr int rg_cols() { return 2048 / int(sizeof(TB)); }  // columns per pass
+template <int MODE, typename TB>
+size_t rg_smem_bytes(int kc) {
+    return size_t(kRgStages) * RgCfg<MODE>::KCH * rg_cols<MODE, TB>() * sizeof(TB) *
+               RgCfg<MODE>::NMAT +
+           size_t(4) * kc * sizeof(float) * RgCfg<MODE>::NMAT;
+}
 
 template <int MODE, typename TA, typename TB>
-__global__ void __launch_bounds__(256) rowgemm_kernel(const BwArgs a, const TA *A, const TA *A2,
-                                                      const TB *B, const TB *B2, int Kdim, int N,
-                                                      int S) {
+__global__ void __launch_bounds__(256, 1) rowgemm_kernel(const BwArgs a, const TA *A,
+                                                         const TA *A2, const TB *B, const TB *B2,
+                                                         int Kdim, int N, int S) {
+    constexpr int KCH = RgCfg<MODE>::KCH, NMAT = RgCfg<MODE>::NMAT;
+    constexpr int CPB = rg_cols<MODE, TB>();
+    constexpr size_t MAT_BYTES = size_t(KCH) * CPB * sizeof(TB);  // one matrix, one stage
+    constexpr size_t STAGE_BYTES = MAT_BYTES * NMAT;
+    extern __shared__ __align__(128) unsigned char rg_smem[];
     __shared__ int s_flag[kMaxTileRows], s_row[kMaxTileRows], s_n;
     __shared__ float s_fw[kMaxTileRows], s_w[kMaxTileRows];
-    __shared__ __align__(16) float As[4][kRgKch];
-    __shared__ __align__(16) float A2s[MODE == TG_DX ? 4 : 1][MODE == TG_DX ? kRgKch : 4];
     griddep_wait();
     griddep_launch_dependents();
     const int ti = blockIdx.x, sp = blockIdx.y;
@@ -220,65 +240,109 @@ __global__ void __launch_bounds__(256) rowgemm_kernel(const BwArgs a, const TA *
     const int nk = stage_kept_rows(a, tile.y, tile.z, s_flag, s_fw, s_row, s_w, &s_n);
     if (nk == 0) return;
     const int kc = Kdim / S, k0 = sp * kc;
-    const int NG = N / 8;
+    const int nchunks = (kc + KCH - 1) / KCH;
+    float *As = reinterpret_cast<float *>(rg_smem + kRgStages * STAGE_BYTES);  // [4][kc]
+    float *A2s = As + 4 * kc;                                                   // DX only
     const long long bstride = (long long)Kdim * N;
     const TB *Be = B + (long long)e * bstride;
-    const TB *B2e = (MODE == TG_DX) ? B2 + (long long)e * bstride : nullptr;
+    const TB *B2e = NMAT == 2 ? B2 + (long long)e * bstride : nullptr;
     float *part = a.part + (long long)sp * a.p_cap * N;
     for (int g0 = 0; g0 < nk; g0 += 4) {
         const int gn = min(4, nk - g0);
-        for (int cgb = 0; cgb < NG; cgb += blockDim.x) {
-            const int cg = cgb + threadIdx.x;
-            const bool active = cg < NG;
+        // A rows of the group for the whole split (batches of 8 independent loads).
+        for (int q0 = threadIdx.x; q0 < 4 * kc; q0 += 8 * blockDim.x) {
+            float v[8], v2[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int q = q0 + u * blockDim.x;
+                const int r = q / kc, k = q - r * kc;
+                const bool ok = q < 4 * kc && r < gn;
+                const long long o = ok ? (long long)s_row[g0 + r] * Kdim + k0 + k : 0;
+                v[u] = ok ? load_f(A, o) : 0.0f;
+                v2[u] = (NMAT == 2 && ok) ? load_f(A2, o) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int q = q0 + u * blockDim.x;
+                if (q < 4 * kc) {
+                    As[q] = v[u];
+                    if (NMAT == 2) A2s[q] = v2[u];
+                }
+            }
+        }
+        __syncthreads();
+        for (int c0 = 0; c0 < N; c0 += CPB) {
+            const int ncol = min(CPB, N - c0);
+            const int cg = threadIdx.x;  // 8 columns each
+            const bool active = cg * 8 < ncol;
+            // Copy k-rows [k0 + c*KCH, +kn) x columns [c0, c0 + ncol) into stage c.
+            auto issue = [&](int c) {
+                if (c < nchunks) {
+                    const int kb = k0 + c * KCH, kn = min(KCH, k0 + kc - kb);
+                    unsigned char *dst = rg_smem + (c % kRgStages) * STAGE_BYTES;
+                    const int per_row = ncol * int(sizeof(TB)) / 16;
+                    for (int q = threadIdx.x; q < kn * per_row; q += blockDim.x) {
+                        const int u = q / per_row, v = q - u * per_row;
+                        const long long go = (long long)(kb + u) * N + c0;
+                        cp_async_16(dst + size_t(u) * CPB * sizeof(TB) + size_t(v) * 16,
+                                    reinterpret_cast<const unsigned char *>(Be + go) + size_t(v) * 16);
+                        if (NMAT == 2)
+                            cp_async_16(dst + MAT_BYTES + size_t(u) * CPB * sizeof(TB) + size_t(v) * 16,
+                                        reinterpret_cast<const unsigned char *>(B2e + go) + size_t(v) * 16);
+                    }
+                }
+                cp_async_commit();  // every thread, every call: uniform group counts
+            };
             float acc[4][8];
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
-            for (int kb = k0; kb < k0 + kc; kb += kRgKch) {
-                const int kn = min(kRgKch, k0 + kc - kb);
-                for (int q = threadIdx.x; q < 4 * kn; q += blockDim.x) {
-                    const int r = q / kn, k = q - r * kn;
-                    const long long ro = (r < gn) ? (long long)s_row[g0 + r] * Kdim : 0;
-                    As[r][k] = (r < gn) ? load_f(A, ro + kb + k) : 0.0f;
-                    if (MODE == TG_DX) A2s[r][k] = (r < gn) ? load_f(A2, ro + kb + k) : 0.0f;
-                }
-                __syncthreads();
+                for (int cc = 0; cc < 8; ++cc) acc[r][cc] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < kRgStages - 1; ++c) issue(c);
+            for (int c = 0; c < nchunks; ++c) {
+                issue(c + kRgStages - 1);
+                cp_async_wait<kRgStages - 1>();  // this thread's copies of chunk c landed
+                __syncthreads();                   // everyone's did
                 if (active) {
-                    const TB *bp = Be + (long long)kb * N + cg * 8;
-                    const TB *bp2 = (MODE == TG_DX) ? B2e + (long long)kb * N + cg * 8 : nullptr;
+                    const unsigned char *st = rg_smem + (c % kRgStages) * STAGE_BYTES;
+                    const int kn = min(KCH, kc - c * KCH);
+                    const float *ar = As + c * KCH;
+                    const float *ar2 = A2s + c * KCH;
 #pragma unroll 4
-                    for (int k = 0; k < kn; ++k) {
+                    for (int u = 0; u < kn; ++u) {
                         float bv[8];
-                        load8(bp + (long long)k * N, bv);
+                        load8(reinterpret_cast<const TB *>(st + size_t(u) * CPB * sizeof(TB)) + cg * 8, bv);
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
-                            const float av = As[r][k];
+                            const float av = ar[r * kc + u];
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av, bv[c], acc[r][c]);
+                            for (int cc = 0; cc < 8; ++cc) acc[r][cc] = fmaf(av, bv[cc], acc[r][cc]);
                         }
-                        if (MODE == TG_DX) {
-                            load8(bp2 + (long long)k * N, bv);
+                        if (NMAT == 2) {
+                            load8(reinterpret_cast<const TB *>(st + MAT_BYTES + size_t(u) * CPB * sizeof(TB)) + cg * 8, bv);
 #pragma unroll
                             for (int r = 0; r < 4; ++r) {
-                                const float av = A2s[r][k];
+                                const float av = ar2[r * kc + u];
 #pragma unroll
-                                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av, bv[c], acc[r][c]);
+                                for (int cc = 0; cc < 8; ++cc) acc[r][cc] = fmaf(av, bv[cc], acc[r][cc]);
                             }
                         }
                     }
                 }
-                __syncthreads();
+                __syncthreads();  // stage c is refilled by the next issue
             }
+            cp_async_wait<0>();
             if (active) {
                 for (int r = 0; r < gn; ++r) {
-                    float *o = part + (long long)s_row[g0 + r] * N + cg * 8;
+                    float *o = part + (long long)s_row[g0 + r] * N + c0 + cg * 8;
                     *reinterpret_cast<float4 *>(o) =
                         make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
                     *reinterpret_cast<float4 *>(o + 4) =
                         make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
                 }
             }
+            __syncthreads();
         }
     }
 }
@@ -312,13 +376,18 @@ __global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S)
 }
 
 // ---------------------------------------------------------------------- dx --
+// Block per token; each thread owns 8 consecutive columns, so every term is
+// one 16-byte load and the loads of all terms are independent.  The router
+// terms (nonzero dr in expert order, then the K dz in slot order) are listed
+// in shared memory first.
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *Wg,
                                                     const TIn *Wm, int S) {
     __shared__ float s_dr[kMaxE];
-    __shared__ int s_pos[kMaxK], s_cand[kMaxK];
-    __shared__ float s_dz[kMaxK];
-    __shared__ int s_kept[kMaxK];
+    __shared__ float s_c[kMaxE + kMaxK];  // coefficients
+    __shared__ int s_row[kMaxE + kMaxK];  // their weight rows
+    __shared__ int s_pos[kMaxK];
+    __shared__ int s_ng, s_nr, s_nk;
     griddep_wait();
     griddep_launch_dependents();
     const int K = a.K, E = a.E, d = a.d;
@@ -327,28 +396,58 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *W
         for (int e = threadIdx.x; e < E; e += blockDim.x) s_dr[e] = a.dr[(long long)t * E + e];
         if (threadIdx.x < K) {
             const long long o = (long long)t * K + threadIdx.x;
-            s_pos[threadIdx.x] = a.pair_pos[o];
-            s_cand[threadIdx.x] = a.cand[o];
-            s_dz[threadIdx.x] = a.dz[o];
-            s_kept[threadIdx.x] = a.idx[o] >= 0;
+            s_c[kMaxE + threadIdx.x] = Wm ? a.dz[o] : 0.0f;
+            s_row[kMaxE + threadIdx.x] = a.cand[o];
+            s_pos[threadIdx.x] = a.idx[o] >= 0 ? a.pair_pos[o] : -1;
         }
         __syncthreads();
-        for (int j = threadIdx.x; j < d; j += blockDim.x) {
-            float acc = 0.0f;
-            for (int k = 0; k < K; ++k)  // expert part: kept slots in order, splits in order
-                if (s_kept[k]) {
-                    float c = 0.0f;
-                    for (int sp = 0; sp < S; ++sp) c += a.part[sp * split + (long long)s_pos[k] * d + j];
-                    acc += c;
+        if (threadIdx.x == 0) {
+            int n = 0;
+            for (int e = 0; e < E; ++e)
+                if (s_dr[e] != 0.0f) {
+                    s_c[n] = s_dr[e];
+                    s_row[n] = e;
+                    ++n;
                 }
-            for (int e = 0; e < E; ++e) {  // W_gate^T dr
-                const float c = s_dr[e];
-                if (c != 0.0f) acc = fmaf(c, load_f(Wg, (long long)e * d + j), acc);
-            }
+            s_ng = n;
+            int nk = 0;
+            for (int k = 0; k < K; ++k)
+                if (s_pos[k] >= 0) s_pos[nk++] = s_pos[k];
+            s_nk = nk;
             if (Wm)
-                for (int k = 0; k < K; ++k)  // W_mask^T dz
-                    acc = fmaf(s_dz[k], load_f(Wm, (long long)s_cand[k] * d + j), acc);
-            a.dx[(long long)t * d + j] = acc;
+                for (int k = 0; k < K; ++k) {  // n <= E, so the dz block moves down
+                    s_c[n] = s_c[kMaxE + k];
+                    s_row[n] = s_row[kMaxE + k];
+                    ++n;
+                }
+            s_nr = n;
+        }
+        __syncthreads();
+        const int ng = s_ng, nr = s_nr, nk = s_nk;
+        for (int j = threadIdx.x * 8; j < d; j += blockDim.x * 8) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int q = 0; q < nk; ++q) {  // expert part: kept slots in order, splits in order
+                float c[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int sp = 0; sp < S; ++sp) {
+                    float v[8];
+                    load8(a.part + sp * split + (long long)s_pos[q] * d + j, v);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) c[i] += v[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] += c[i];
+            }
+#pragma unroll 4
+            for (int q = 0; q < nr; ++q) {  // W_gate^T dr, then W_mask^T dz
+                float v[8];
+                load8((q < ng ? Wg : Wm) + (long long)s_row[q] * d + j, v);
+                const float cq = s_c[q];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(cq, v[i], acc[i]);
+            }
+            float *o = a.dx + (long long)t * d + j;
+            *reinterpret_cast<float4 *>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            *reinterpret_cast<float4 *>(o + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         }
         __syncthreads();
     }
@@ -376,34 +475,36 @@ __device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, i
 }
 
 // dW1_e[i] += sum over kept rows (in order) da[r][i] x_r, dW3 likewise with db.
-// Block (expert, 4 rows of I); each thread owns 8 consecutive columns of d.
+// Block (expert, 2 rows of I); each thread owns 8 consecutive columns of d.
+constexpr int kW13Rows = 2;
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn *xp, float *dW1,
                                                       float *dW3) {
+    constexpr int R = kW13Rows;
     __shared__ int s_first, s_n;
     __shared__ int s_flag[kWgChunk], s_kr[kWgChunk];
-    __shared__ float s_da[kWgChunk][4], s_db[kWgChunk][4];
+    __shared__ float s_da[kWgChunk][R], s_db[kWgChunk][R];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
     if (a.counts_kept[e] == 0) return;  // no kept pair: no gradient, rows untouched
-    const int i0 = blockIdx.y * 4;
+    const int i0 = blockIdx.y * R;
     const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
     const int n = a.counts_all[e];
     const int d = a.d, I = a.I;
     for (int jb = 0; jb < d; jb += 8 * blockDim.x) {
         const int j = jb + threadIdx.x * 8;
         const bool active = j < d;
-        float g1[4][8], g3[4][8];
+        float g1[R][8], g3[R][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < R; ++i)
 #pragma unroll
             for (int c = 0; c < 8; ++c) g1[i][c] = g3[i][c] = 0.0f;
         for (int r0 = 0; r0 < n; r0 += kWgChunk) {
             const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_flag, s_kr,
                                               &s_n);
-            for (int q = threadIdx.x; q < 4 * nk; q += blockDim.x) {
-                const int kq = q >> 2, i = q & 3;
+            for (int q = threadIdx.x; q < R * nk; q += blockDim.x) {
+                const int kq = q / R, i = q - kq * R;
                 const bool ok = i0 + i < I;
                 s_da[kq][i] = ok ? a.da[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
                 s_db[kq][i] = ok ? a.db[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
@@ -415,7 +516,7 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
                     float xv[8];
                     load8(xp + (long long)s_kr[kq] * d + j, xv);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < R; ++i) {
                         const float va = s_da[kq][i], vb = s_db[kq][i];
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
@@ -428,13 +529,26 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
             __syncthreads();
         }
         if (active) {
+            // Read-modify-write: every read issued before any add or store.
+            float4 old[R][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < R; ++i) {
+                if (i0 + i >= I) continue;
+                const long long o = ((long long)e * I + i0 + i) * d + j;
+                const float4 *p1 = reinterpret_cast<const float4 *>(dW1 + o);
+                const float4 *p3 = reinterpret_cast<const float4 *>(dW3 + o);
+                old[i][0] = p1[0];
+                old[i][1] = p1[1];
+                old[i][2] = p3[0];
+                old[i][3] = p3[1];
+            }
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
                 if (i0 + i >= I) continue;
                 const long long o = ((long long)e * I + i0 + i) * d + j;
                 float4 *p1 = reinterpret_cast<float4 *>(dW1 + o);
                 float4 *p3 = reinterpret_cast<float4 *>(dW3 + o);
-                float4 u0 = p1[0], u1 = p1[1], v0 = p3[0], v1 = p3[1];
+                float4 u0 = old[i][0], u1 = old[i][1], v0 = old[i][2], v1 = old[i][3];
                 u0.x += g1[i][0]; u0.y += g1[i][1]; u0.z += g1[i][2]; u0.w += g1[i][3];
                 u1.x += g1[i][4]; u1.y += g1[i][5]; u1.z += g1[i][6]; u1.w += g1[i][7];
                 v0.x += g3[i][0]; v0.y += g3[i][1]; v0.z += g3[i][2]; v0.w += g3[i][3];
@@ -495,49 +609,111 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
             __syncthreads();
         }
         if (active) {
+            float4 old[8];  // all reads issued before any add or store
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                if (j0 + jj < d)
+                    old[jj] = *reinterpret_cast<const float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
                 if (j0 + jj >= d) continue;
-                float4 *p = reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
-                float4 v = *p;
+                float4 v = old[jj];
                 v.x += g[jj][0]; v.y += g[jj][1]; v.z += g[jj][2]; v.w += g[jj][3];
-                *p = v;
+                *reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i) = v;
             }
         }
     }
 }
 
-// dW_gate[e] += sum_t dr[t][e] x_t; dW_mask[e] += sum over the candidate rows
-// of e (token order) dz x.  Block (expert, 256 columns of d).
+// dW_gate[e] += sum_t dr[t][e] x_t (tokens ascending); dW_mask[e] += sum over
+// the candidate rows of e (token order) dz x.  Block (expert, 2048 columns);
+// each thread owns 8 columns; coefficients are staged in shared memory.
+constexpr int kDrChunk = 512;
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const TIn *x,
                                                          const TIn *xp, float *dWg, float *dWm) {
     __shared__ int s_first;
+    __shared__ float s_c[kDrChunk];
+    __shared__ int s_r[kDrChunk];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
-    const int j = blockIdx.y * 256 + threadIdx.x;
+    const int j = blockIdx.y * 2048 + threadIdx.x * 8;
+    const bool active = j < a.d;
     const int d = a.d, E = a.E;
-    float gg = 0.0f;
-    for (int t = 0; t < a.T; ++t) {
-        const float c = a.dr[(long long)t * E + e];
-        if (c != 0.0f && j < d) gg = fmaf(c, load_f(x, (long long)t * d + j), gg);
+    float gg[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float gm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int t0 = 0; t0 < a.T; t0 += kDrChunk) {
+        const int cnt = min(kDrChunk, a.T - t0);
+        for (int q = threadIdx.x; q < cnt; q += blockDim.x) s_c[q] = a.dr[(long long)(t0 + q) * E + e];
+        __syncthreads();
+        if (active) {
+#pragma unroll 4
+            for (int q = 0; q < cnt; ++q) {
+                const float c = s_c[q];
+                if (c == 0.0f) continue;  // same branch for the whole block
+                float v[8];
+                load8(x + (long long)(t0 + q) * d + j, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) gg[i] = fmaf(c, v[i], gg[i]);
+            }
+        }
+        __syncthreads();
     }
-    float gm = 0.0f;
-    if (dWm) {
-        const int first = a.counts_all[e] ? expert_first_row(a.tiles, a.meta[0], e, &s_first) : 0;
-        for (int r = first; r < first + a.counts_all[e]; ++r) {
-            const float c = a.dz[a.pair[r]];
-            if (j < d) gm = fmaf(c, load_f(xp, (long long)r * d + j), gm);
+    const int n = a.counts_all[e];
+    if (dWm && n > 0) {
+        const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
+        for (int r0 = 0; r0 < n; r0 += kDrChunk) {
+            const int cnt = min(kDrChunk, n - r0);
+            for (int q = threadIdx.x; q < cnt; q += blockDim.x) {
+                const int r = first + r0 + q;
+                s_r[q] = r;
+                s_c[q] = a.dz[a.pair[r]];
+            }
+            __syncthreads();
+            if (active) {
+#pragma unroll 4
+                for (int q = 0; q < cnt; ++q) {
+                    float v[8];
+                    load8(xp + (long long)s_r[q] * d + j, v);
+                    const float c = s_c[q];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) gm[i] = fmaf(c, v[i], gm[i]);
+                }
+            }
+            __syncthreads();
         }
     }
-    if (j < d) {
-        dWg[(long long)e * d + j] += gg;
-        if (dWm) dWm[(long long)e * d + j] += gm;
+    if (active) {
+        float4 *pg = reinterpret_cast<float4 *>(dWg + (long long)e * d + j);
+        float4 u0 = pg[0], u1 = pg[1];
+        u0.x += gg[0]; u0.y += gg[1]; u0.z += gg[2]; u0.w += gg[3];
+        u1.x += gg[4]; u1.y += gg[5]; u1.z += gg[6]; u1.w += gg[7];
+        pg[0] = u0;
+        pg[1] = u1;
+        if (dWm) {
+            float4 *pm = reinterpret_cast<float4 *>(dWm + (long long)e * d + j);
+            float4 v0 = pm[0], v1 = pm[1];
+            v0.x += gm[0]; v0.y += gm[1]; v0.z += gm[2]; v0.w += gm[3];
+            v1.x += gm[4]; v1.y += gm[5]; v1.z += gm[6]; v1.w += gm[7];
+            pm[0] = v0;
+            pm[1] = v1;
+        }
     }
 }
 
 }  // namespace
+
+template <int MODE, typename TA, typename TB>
+cudaError_t launch_rowgemm(const BwArgs &a, const TA *A, const TA *A2, const TB *B, const TB *B2,
+                           int Kdim, int N, cudaStream_t st) {
+    const size_t smem = rg_smem_bytes<MODE, TB>(Kdim / a.S);
+    auto kern = rowgemm_kernel<MODE, TA, TB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(a.tiles_cap, a.S), dim3(256), smem, st, a, A, A2, B, B2, Kdim, N,
+                      a.S);
+}
 
 cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
                                    const void *dy, const void *dyp, const void *Wg,
@@ -546,21 +722,21 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
                                    float *dW3, float *dW2, int n_sm, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
     const int tb = a.T < 8 * n_sm ? a.T : 8 * n_sm;
-    const dim3 g_dh(a.tiles_cap, a.S), g_fin(a.tiles_cap);
-    const dim3 g_w13(a.E, (a.I + 3) / 4), g_w2(a.E, (a.d + 7) / 8), g_r(a.E, (a.d + 255) / 256);
+    const dim3 g_fin(a.tiles_cap);
+    const dim3 g_w13(a.E, (a.I + kW13Rows - 1) / kW13Rows), g_w2(a.E, (a.d + 7) / 8),
+        g_r(a.E, (a.d + 2047) / 2048);
     cudaError_t e;
     if (dtype == BEAM_BF16) {
         using T = __nv_bfloat16;
         const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
         const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
         if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-        if ((e = launch_pdl(rowgemm_kernel<TG_DH, T, T>, g_dh, dim3(256), 0, st, a, dypb, dypb,
-                            static_cast<const T *>(W2), static_cast<const T *>(W2), a.d, a.I, a.S)))
+        if ((e = launch_rowgemm<TG_DH, T, T>(a, dypb, dypb, static_cast<const T *>(W2),
+                                             static_cast<const T *>(W2), a.d, a.I, st)))
             return e;
         if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.S))) return e;
-        if ((e = launch_pdl(rowgemm_kernel<TG_DX, float, T>, g_dh, dim3(256), 0, st, a,
-                            static_cast<const float *>(a.da), static_cast<const float *>(a.db),
-                            static_cast<const T *>(W1), static_cast<const T *>(W3), a.I, a.d, a.S)))
+        if ((e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, static_cast<const T *>(W1),
+                                                 static_cast<const T *>(W3), a.I, a.d, st)))
             return e;
         if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a,
                             static_cast<const T *>(Wg), static_cast<const T *>(Wm), a.S)))
@@ -574,13 +750,12 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
     const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
     const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
     if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-    if ((e = launch_pdl(rowgemm_kernel<TG_DH, T, T>, g_dh, dim3(256), 0, st, a, dypb, dypb,
-                        static_cast<const T *>(W2), static_cast<const T *>(W2), a.d, a.I, a.S)))
+    if ((e = launch_rowgemm<TG_DH, T, T>(a, dypb, dypb, static_cast<const T *>(W2),
+                                         static_cast<const T *>(W2), a.d, a.I, st)))
         return e;
     if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.S))) return e;
-    if ((e = launch_pdl(rowgemm_kernel<TG_DX, float, T>, g_dh, dim3(256), 0, st, a,
-                        static_cast<const float *>(a.da), static_cast<const float *>(a.db),
-                        static_cast<const T *>(W1), static_cast<const T *>(W3), a.I, a.d, a.S)))
+    if ((e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, static_cast<const T *>(W1),
+                                             static_cast<const T *>(W3), a.I, a.d, st)))
         return e;
     if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a,
                         static_cast<const T *>(Wg), static_cast<const T *>(Wm), a.S)))

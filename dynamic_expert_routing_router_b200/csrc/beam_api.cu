@@ -479,8 +479,8 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     B->off_db = take(4 * pc * I);
     B->off_h = take(4 * pc * I);
     // Thin decode tiles leave most SMs idle with one block per tile: split the
-    // reduction of the kept-row products four ways (d and I are multiples of 8).
-    B->S = P->BN < 128 ? 4 : 1;
+    // reduction of the kept-row products eight ways (d and I are multiples of 8).
+    B->S = P->BN < 128 ? 8 : 1;
     B->off_part = take(4 * size_t(B->S) * pc * (dd > I ? dd : I));
     B->off_u = take(4 * T * K);
     B->off_dz = take(4 * T * K);

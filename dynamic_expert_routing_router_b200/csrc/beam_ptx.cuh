@@ -103,6 +103,23 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *t
         : "memory");
 }
 
+// ----------------------------------------------------- cp.async (16 B) --
+// Asynchronous global -> shared copies for CUDA-core pipelines.  Both
+// addresses 16-byte aligned.  Completion by groups: commit, then wait until at
+// most N groups of this thread are pending (a hardware wait, not a spin).
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+                 "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // -------------------------------------------------------------- tcgen05 --
 
 __device__ __forceinline__ void tc_fence_before_sync() {
