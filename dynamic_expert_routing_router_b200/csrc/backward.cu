@@ -475,36 +475,34 @@ __device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, i
 }
 
 // dW1_e[i] += sum over kept rows (in order) da[r][i] x_r, dW3 likewise with db.
-// Block (expert, 2 rows of I); each thread owns 8 consecutive columns of d.
-constexpr int kW13Rows = 2;
+// Block (expert, 4 rows of I); each thread owns 8 consecutive columns of d.
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn *xp, float *dW1,
                                                       float *dW3) {
-    constexpr int R = kW13Rows;
     __shared__ int s_first, s_n;
     __shared__ int s_flag[kWgChunk], s_kr[kWgChunk];
-    __shared__ float s_da[kWgChunk][R], s_db[kWgChunk][R];
+    __shared__ float s_da[kWgChunk][4], s_db[kWgChunk][4];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
     if (a.counts_kept[e] == 0) return;  // no kept pair: no gradient, rows untouched
-    const int i0 = blockIdx.y * R;
+    const int i0 = blockIdx.y * 4;
     const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
     const int n = a.counts_all[e];
     const int d = a.d, I = a.I;
     for (int jb = 0; jb < d; jb += 8 * blockDim.x) {
         const int j = jb + threadIdx.x * 8;
         const bool active = j < d;
-        float g1[R][8], g3[R][8];
+        float g1[4][8], g3[4][8];
 #pragma unroll
-        for (int i = 0; i < R; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int c = 0; c < 8; ++c) g1[i][c] = g3[i][c] = 0.0f;
         for (int r0 = 0; r0 < n; r0 += kWgChunk) {
             const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_flag, s_kr,
                                               &s_n);
-            for (int q = threadIdx.x; q < R * nk; q += blockDim.x) {
-                const int kq = q / R, i = q - kq * R;
+            for (int q = threadIdx.x; q < 4 * nk; q += blockDim.x) {
+                const int kq = q >> 2, i = q & 3;
                 const bool ok = i0 + i < I;
                 s_da[kq][i] = ok ? a.da[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
                 s_db[kq][i] = ok ? a.db[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
@@ -516,7 +514,7 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
                     float xv[8];
                     load8(xp + (long long)s_kr[kq] * d + j, xv);
 #pragma unroll
-                    for (int i = 0; i < R; ++i) {
+                    for (int i = 0; i < 4; ++i) {
                         const float va = s_da[kq][i], vb = s_db[kq][i];
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
@@ -529,26 +527,13 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
             __syncthreads();
         }
         if (active) {
-            // Read-modify-write: every read issued before any add or store.
-            float4 old[R][4];
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-                if (i0 + i >= I) continue;
-                const long long o = ((long long)e * I + i0 + i) * d + j;
-                const float4 *p1 = reinterpret_cast<const float4 *>(dW1 + o);
-                const float4 *p3 = reinterpret_cast<const float4 *>(dW3 + o);
-                old[i][0] = p1[0];
-                old[i][1] = p1[1];
-                old[i][2] = p3[0];
-                old[i][3] = p3[1];
-            }
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 if (i0 + i >= I) continue;
                 const long long o = ((long long)e * I + i0 + i) * d + j;
                 float4 *p1 = reinterpret_cast<float4 *>(dW1 + o);
                 float4 *p3 = reinterpret_cast<float4 *>(dW3 + o);
-                float4 u0 = old[i][0], u1 = old[i][1], v0 = old[i][2], v1 = old[i][3];
+                float4 u0 = p1[0], u1 = p1[1], v0 = p3[0], v1 = p3[1];
                 u0.x += g1[i][0]; u0.y += g1[i][1]; u0.z += g1[i][2]; u0.w += g1[i][3];
                 u1.x += g1[i][4]; u1.y += g1[i][5]; u1.z += g1[i][6]; u1.w += g1[i][7];
                 v0.x += g3[i][0]; v0.y += g3[i][1]; v0.z += g3[i][2]; v0.w += g3[i][3];
@@ -609,53 +594,58 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
             __syncthreads();
         }
         if (active) {
-            float4 old[8];  // all reads issued before any add or store
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                if (j0 + jj < d)
-                    old[jj] = *reinterpret_cast<const float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
                 if (j0 + jj >= d) continue;
-                float4 v = old[jj];
+                float4 *p = reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
+                float4 v = *p;
                 v.x += g[jj][0]; v.y += g[jj][1]; v.z += g[jj][2]; v.w += g[jj][3];
-                *reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i) = v;
+                *p = v;
             }
         }
     }
 }
 
 // dW_gate[e] += sum_t dr[t][e] x_t (tokens ascending); dW_mask[e] += sum over
-// the candidate rows of e (token order) dz x.  Block (expert, 2048 columns);
-// each thread owns 8 columns; coefficients are staged in shared memory.
+// the candidate rows of e (token order) dz x.  Block (expert, 256 columns):
+// 64 threads x 4 columns; coefficients are staged in shared memory.
 constexpr int kDrChunk = 512;
+__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+}
+__device__ __forceinline__ void load4(const float *p, float (&v)[4]) {
+    const float4 x = *reinterpret_cast<const float4 *>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
 template <typename TIn>
-__global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const TIn *x,
-                                                         const TIn *xp, float *dWg, float *dWm) {
+__global__ void __launch_bounds__(64) bw_drouter_kernel(const BwArgs a, const TIn *x,
+                                                        const TIn *xp, float *dWg, float *dWm) {
     __shared__ int s_first;
     __shared__ float s_c[kDrChunk];
     __shared__ int s_r[kDrChunk];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
-    const int j = blockIdx.y * 2048 + threadIdx.x * 8;
+    const int j = blockIdx.y * 256 + threadIdx.x * 4;
     const bool active = j < a.d;
     const int d = a.d, E = a.E;
-    float gg[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float gm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float gg[4] = {0.f, 0.f, 0.f, 0.f}, gm[4] = {0.f, 0.f, 0.f, 0.f};
     for (int t0 = 0; t0 < a.T; t0 += kDrChunk) {
         const int cnt = min(kDrChunk, a.T - t0);
         for (int q = threadIdx.x; q < cnt; q += blockDim.x) s_c[q] = a.dr[(long long)(t0 + q) * E + e];
         __syncthreads();
         if (active) {
-#pragma unroll 4
+#pragma unroll 8
             for (int q = 0; q < cnt; ++q) {
                 const float c = s_c[q];
                 if (c == 0.0f) continue;  // same branch for the whole block
-                float v[8];
-                load8(x + (long long)(t0 + q) * d + j, v);
+                float v[4];
+                load4(x + (long long)(t0 + q) * d + j, v);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) gg[i] = fmaf(c, v[i], gg[i]);
+                for (int i = 0; i < 4; ++i) gg[i] = fmaf(c, v[i], gg[i]);
             }
         }
         __syncthreads();
@@ -672,13 +662,13 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
             }
             __syncthreads();
             if (active) {
-#pragma unroll 4
+#pragma unroll 8
                 for (int q = 0; q < cnt; ++q) {
-                    float v[8];
-                    load8(xp + (long long)s_r[q] * d + j, v);
+                    float v[4];
+                    load4(xp + (long long)s_r[q] * d + j, v);
                     const float c = s_c[q];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) gm[i] = fmaf(c, v[i], gm[i]);
+                    for (int i = 0; i < 4; ++i) gm[i] = fmaf(c, v[i], gm[i]);
                 }
             }
             __syncthreads();
@@ -686,18 +676,14 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
     }
     if (active) {
         float4 *pg = reinterpret_cast<float4 *>(dWg + (long long)e * d + j);
-        float4 u0 = pg[0], u1 = pg[1];
-        u0.x += gg[0]; u0.y += gg[1]; u0.z += gg[2]; u0.w += gg[3];
-        u1.x += gg[4]; u1.y += gg[5]; u1.z += gg[6]; u1.w += gg[7];
-        pg[0] = u0;
-        pg[1] = u1;
+        float4 u = *pg;
+        u.x += gg[0]; u.y += gg[1]; u.z += gg[2]; u.w += gg[3];
+        *pg = u;
         if (dWm) {
             float4 *pm = reinterpret_cast<float4 *>(dWm + (long long)e * d + j);
-            float4 v0 = pm[0], v1 = pm[1];
-            v0.x += gm[0]; v0.y += gm[1]; v0.z += gm[2]; v0.w += gm[3];
-            v1.x += gm[4]; v1.y += gm[5]; v1.z += gm[6]; v1.w += gm[7];
-            pm[0] = v0;
-            pm[1] = v1;
+            float4 v = *pm;
+            v.x += gm[0]; v.y += gm[1]; v.z += gm[2]; v.w += gm[3];
+            *pm = v;
         }
     }
 }
@@ -723,8 +709,7 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
     if (a.T <= 0) return cudaSuccess;
     const int tb = a.T < 8 * n_sm ? a.T : 8 * n_sm;
     const dim3 g_fin(a.tiles_cap);
-    const dim3 g_w13(a.E, (a.I + kW13Rows - 1) / kW13Rows), g_w2(a.E, (a.d + 7) / 8),
-        g_r(a.E, (a.d + 2047) / 2048);
+    const dim3 g_w13(a.E, (a.I + 3) / 4), g_w2(a.E, (a.d + 7) / 8), g_r(a.E, (a.d + 255) / 256);
     cudaError_t e;
     if (dtype == BEAM_BF16) {
         using T = __nv_bfloat16;
@@ -744,7 +729,7 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
         if ((e = launch_pdl(bw_dw13_kernel<T>, g_w13, dim3(256), 0, st, a, xpb, dW1, dW3)))
             return e;
         if ((e = launch_pdl(bw_dw2_kernel<T>, g_w2, dim3(256), 0, st, a, dypb, dW2))) return e;
-        return launch_pdl(bw_drouter_kernel<T>, g_r, dim3(256), 0, st, a, xb, xpb, dWg, dWm);
+        return launch_pdl(bw_drouter_kernel<T>, g_r, dim3(64), 0, st, a, xb, xpb, dWg, dWm);
     }
     using T = float;
     const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
@@ -762,7 +747,7 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
         return e;
     if ((e = launch_pdl(bw_dw13_kernel<T>, g_w13, dim3(256), 0, st, a, xpb, dW1, dW3))) return e;
     if ((e = launch_pdl(bw_dw2_kernel<T>, g_w2, dim3(256), 0, st, a, dypb, dW2))) return e;
-    return launch_pdl(bw_drouter_kernel<T>, g_r, dim3(256), 0, st, a, xb, xpb, dWg, dWm);
+    return launch_pdl(bw_drouter_kernel<T>, g_r, dim3(64), 0, st, a, xb, xpb, dWg, dWm);
 }
 
 }  // namespace beam

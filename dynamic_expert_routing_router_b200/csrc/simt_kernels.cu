@@ -353,23 +353,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
                                                       const float *w, const int *pair_pos, int T,
                                                       int K, int d, const float *Ys, int n_shared,
                                                       Tout *out) {
-    __shared__ int s_row[kMaxK];
-    __shared__ float s_w[kMaxK];
+    __shared__ int s_row[kMaxK], s_slot[kMaxK];
+    __shared__ float s_w[kMaxK], s_slotw[kMaxK];
     __shared__ int s_n;
     const int nvec = d / 8;
     griddep_wait();
     griddep_launch_dependents();
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < K) {  // slot metadata, one thread per slot
+            const long long o = (long long)t * K + threadIdx.x;
+            s_slot[threadIdx.x] = idx[o] >= 0 ? pair_pos[o] : -1;
+            s_slotw[threadIdx.x] = w[o];
+        }
+        __syncthreads();
         if (threadIdx.x == 0) {  // kept candidates of token t, in slot order
             int n = 0;
-            for (int k = 0; k < K; ++k) {
-                const long long o = (long long)t * K + k;
-                if (idx[o] >= 0) {
-                    s_row[n] = pair_pos[o];
-                    s_w[n] = w[o];
+            for (int k = 0; k < K; ++k)
+                if (s_slot[k] >= 0) {
+                    s_row[n] = s_slot[k];
+                    s_w[n] = s_slotw[k];
                     ++n;
                 }
-            }
             s_n = n;
         }
         __syncthreads();
