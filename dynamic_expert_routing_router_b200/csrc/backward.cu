@@ -690,12 +690,20 @@ __global__ void __launch_bounds__(64) bw_drouter_kernel(const BwArgs a, const TI
 
 }  // namespace
 
+// Longest split reduction each product supports (its A rows for a whole split
+// sit in shared memory): d <= 7168 for DH, I <= 4096 for DX at one split.
+template <int MODE>
+constexpr int rg_max_kc() { return MODE == TG_DX ? 4096 : 7168; }
+
 template <int MODE, typename TA, typename TB>
 cudaError_t launch_rowgemm(const BwArgs &a, const TA *A, const TA *A2, const TB *B, const TB *B2,
                            int Kdim, int N, cudaStream_t st) {
     const size_t smem = rg_smem_bytes<MODE, TB>(Kdim / a.S);
+    if (Kdim / a.S > rg_max_kc<MODE>()) return cudaErrorInvalidValue;
     auto kern = rowgemm_kernel<MODE, TA, TB>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    // The largest size this kernel is ever launched with; set once per device.
+    static std::atomic<unsigned long long> attr_set{0};  // this instantiation only
+    cudaError_t e = set_smem_once(kern, int(rg_smem_bytes<MODE, TB>(rg_max_kc<MODE>())), attr_set);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(a.tiles_cap, a.S), dim3(256), smem, st, a, A, A2, B, B2, Kdim, N,
                       a.S);

@@ -150,8 +150,51 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2D bf16 tensor map over a row-major [rows, inner] matrix, box = 64 x box_rows,
 // 128-byte swizzle (matches the UMMA descriptors in tc_gemm.cu), zero fill.
+// A tensor map holds only the address, shape, strides and box it was made
+// from, so an encoded map is cached under exactly those values: repeated
+// calls with the same buffers skip the driver call (host time per forward).
+struct TmapKey {
+    const void *base;
+    unsigned long long inner, rows;
+    unsigned box_rows;
+    bool operator==(const TmapKey &o) const {
+        return base == o.base && inner == o.inner && rows == o.rows && box_rows == o.box_rows;
+    }
+};
+struct TmapCache {
+    static constexpr int kSets = 64, kWays = 4;
+    struct Entry {
+        TmapKey key;
+        CUtensorMap map;
+        bool valid;
+    };
+    std::mutex mu;
+    Entry e[kSets][kWays] = {};
+    int next[kSets] = {};
+    static int set_of(const TmapKey &k) {
+        unsigned long long h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+        h ^= k.inner * 0xC2B2AE3D27D4EB4Full ^ k.rows * 0x165667B19E3779F9ull ^ k.box_rows;
+        return int((h >> 29) % kSets);
+    }
+};
+TmapCache &tmap_cache() {
+    static TmapCache c;
+    return c;
+}
+
 bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
                unsigned long long rows, unsigned box_rows) {
+    const TmapKey key{base, inner, rows, box_rows};
+    TmapCache &c = tmap_cache();
+    const int set = TmapCache::set_of(key);
+    {
+        std::lock_guard<std::mutex> lk(c.mu);
+        for (auto &en : c.e[set])
+            if (en.valid && en.key == key) {
+                *m = en.map;
+                return true;
+            }
+    }
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn || rows == 0) return false;
     cuuint64_t dims[2] = {inner, rows};
@@ -161,7 +204,14 @@ bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> lk(c.mu);
+    auto &slot = c.e[set][c.next[set]];
+    c.next[set] = (c.next[set] + 1) % TmapCache::kWays;
+    slot.key = key;
+    slot.map = *m;
+    slot.valid = true;
+    return true;
 }
 
 // Records the caller's timing events between stages.  External records
@@ -481,6 +531,8 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     // Thin decode tiles leave most SMs idle with one block per tile: split the
     // reduction of the kept-row products eight ways (d and I are multiples of 8).
     B->S = P->BN < 128 ? 8 : 1;
+    // The kept-row products hold a split's A rows in shared memory.
+    if (dd / B->S > 7168 || I / B->S > 4096) return BEAM_ERR_UNSUPPORTED_SHAPE;
     B->off_part = take(4 * size_t(B->S) * pc * (dd > I ? dd : I));
     B->off_u = take(4 * T * K);
     B->off_dz = take(4 * T * K);

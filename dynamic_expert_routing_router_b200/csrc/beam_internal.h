@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "beam_moe.h"
 
 namespace beam {
@@ -41,6 +43,23 @@ constexpr int kMaxTileRows = 128;     // largest token tile (BN)
 // Launch with programmatic stream serialization (PDL): the kernel may begin
 // its prologue while the previous kernel in the stream finishes; every kernel
 // of this library waits (griddep_wait) before touching global memory.
+// cudaFuncSetAttribute(kern, MaxDynamicSharedMemorySize, bytes) once per
+// kernel and device (the attribute persists; repeating it costs host time on
+// every launch).  `done` is the caller's flag word for this one kernel (one
+// bit per device); `bytes` must be the same on every call for that kernel.
+template <typename... KArgs>
+cudaError_t set_smem_once(void (*kern)(KArgs...), int bytes,
+                          std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args &&...args) {

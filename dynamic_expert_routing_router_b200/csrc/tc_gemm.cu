@@ -535,8 +535,8 @@ cudaError_t launch_cfg(const TcMaps &maps, const TcGemmArgs &args, int grid,
                        cudaStream_t stream) {
     using C = TcCfg<ModeTraits<MODE>::NUM_A, BN, ModeTraits<MODE>::XCH>;
     auto kern = tc_gemm_kernel<MODE, BN>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM_BYTES));
+    static std::atomic<unsigned long long> attr_set{0};  // this instantiation only
+    cudaError_t e = set_smem_once(kern, int(C::SMEM_BYTES), attr_set);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM_BYTES, stream, maps, args);
 }

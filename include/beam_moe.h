@@ -252,8 +252,10 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
  *                                  touched (zero them once per step)
  * Every sum runs in a fixed order: the gradients are bitwise repeatable.
  * Workspace: beam_moe_backward_workspace_size bytes, 256-byte aligned; the
- * caller owns it and every output.  Errors as for beam_moe_forward (shared
- * experts: BEAM_ERR_UNSUPPORTED_SHAPE). */
+ * caller owns it and every output.  Errors as for beam_moe_forward; also
+ * BEAM_ERR_UNSUPPORTED_SHAPE for shared experts, and for d > 7168 or I > 4096
+ * at 128-token tiles (8x larger at decode tile sizes), beyond which a split
+ * of the kept-row products no longer fits in shared memory. */
 size_t beam_moe_backward_workspace_size(const beam_moe_desc *desc);
 beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const void *W_gate,
                               const void *W_mask, const void *W1, const void *W3, const void *W2,
