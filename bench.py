@@ -311,33 +311,77 @@ def time_steps(layer, f, steps, warmup, profiled=False, only=None):
 
 
 def e2e_rate(layer, f, steps, warmup):
-    """Tokens/s through the C ABI with the batch in pinned host memory: H2D copy,
-    forward, D2H copy of the output, every step inside the timed region."""
+    """Tokens/s through the C ABI with the batch in pinned host memory: the H2D
+    copy of each step's tokens, the forward, and the D2H copy of its output,
+    every step inside the timed region.
+
+    Pipelined as a serving loop would run it: the input copy of step i+1 and the
+    output copy of step i-1 run on two copy streams while step i computes
+    (device and pinned buffers double-buffered, events order every reuse).
+    `serial_value` is the same loop with everything on one stream."""
     torch = layer.torch
+    abi = layer.abi
     hx = [x.cpu().pin_memory() for x in layer.xs]
-    hout = torch.empty((layer.T, layer.sh.d), dtype=torch.bfloat16).pin_memory()
-    xdev = torch.empty_like(layer.xs[0])
     Wm = layer.mask(f)
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    xdev = [torch.empty_like(layer.xs[0]) for _ in range(2)]
+    outd = [torch.empty_like(layer.out) for _ in range(2)]
+    hout = [torch.empty(tuple(layer.out.shape), dtype=layer.out.dtype).pin_memory()
+            for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_done + ev_out:
+        e.record(comp)
 
     def step(i):
-        xdev.copy_(hx[i % N_BATCHES], non_blocking=True)
-        layer.abi.forward(layer.dsc, xdev, layer.Wg, Wm, layer.W1, layer.W3, layer.W2,
-                          layer.out, layer.ws)
-        hout.copy_(layer.out, non_blocking=True)
+        b = i & 1
+        h2d.wait_event(ev_done[b])  # forward i-2 has finished reading xdev[b]
+        with torch.cuda.stream(h2d):
+            xdev[b].copy_(hx[i % N_BATCHES], non_blocking=True)
+        ev_in[b].record(h2d)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])  # output copy i-2 has finished reading outd[b]
+        abi.forward(layer.dsc, xdev[b], layer.Wg, Wm, layer.W1, layer.W3, layer.W2, outd[b],
+                    layer.ws, stream=comp)
+        ev_done[b].record(comp)
+        d2h.wait_event(ev_done[b])
+        with torch.cuda.stream(d2h):
+            hout[b].copy_(outd[b], non_blocking=True)
+        ev_out[b].record(d2h)
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(comp)
+        h2d.wait_stream(comp)
+        d2h.wait_stream(comp)
+        for i in range(n):
+            fn(i)
+        comp.wait_stream(h2d)
+        comp.wait_stream(d2h)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e-3
+
+    def serial_step(i):
+        xdev[0].copy_(hx[i % N_BATCHES], non_blocking=True)
+        abi.forward(layer.dsc, xdev[0], layer.Wg, Wm, layer.W1, layer.W3, layer.W2, outd[0],
+                    layer.ws)
+        hout[0].copy_(outd[0], non_blocking=True)
 
     for i in range(warmup):
         step(i)
+        serial_step(i)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(steps):
-        step(i)
-    e1.record()
-    torch.cuda.synchronize()
-    sec = e0.elapsed_time(e1) * 1e-3
+    sec = timed(step, steps)
+    sec_serial = timed(serial_step, steps)
     nbytes = layer.T * layer.sh.d * 2
     return dict(value=layer.T * steps / sec, unit="tokens/s", h2d_bytes_per_step=nbytes,
-                d2h_bytes_per_step=nbytes)
+                d2h_bytes_per_step=nbytes, serial_value=layer.T * steps / sec_serial,
+                note=("pipelined: input copy of step i+1 and output copy of step i-1 on two "
+                      "copy streams during step i; serial_value: one stream"))
 
 
 def cpu_baseline(layer, f, seconds, max_batches=None):
