@@ -77,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     for (uint32_t spin = 1; spin < (1u << 28); ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((spin & 127u) == 0) {
-            if (*abort_flag) return false;
+            if (abort_flag && *abort_flag) return false;
             if (globaltimer_ns() - t0 > timeout_ns) return false;
         }
     }

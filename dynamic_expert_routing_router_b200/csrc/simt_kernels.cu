@@ -12,6 +12,7 @@
 
 #include "beam_internal.h"
 #include "beam_ptx.cuh"
+#include "topk_token.cuh"
 
 namespace beam {
 
@@ -44,7 +45,6 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
     griddep_wait();
     griddep_launch_dependents();
 
-    const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int E2 = 2 * a.E;
     const int cols = a.has_mask ? E2 : a.E;  // columns that hold logits
@@ -86,79 +86,10 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
         __syncthreads();
         // ---- phase 2: one warp per token
         if (warp < nt) {
-            const int t = t0 + warp;
-            float r[EPL], z[EPL];
-            unsigned taken = 0;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int j = lane + 32 * i;
-                r[i] = -INFINITY;
-                z[i] = 0.0f;
-                if (j < a.E) {
-                    const float rs = s_logit[warp][j];
-                    r[i] = (rs != rs) ? -INFINITY : rs;  // NaN never wins a slot
-                    if (a.has_mask) z[i] = s_logit[warp][a.E + j];
-                } else {
-                    taken |= 1u << i;
-                }
-            }
-
-            int my_cand = -1;
-            float my_e = 0.0f, my_z = 0.0f, rmax = 0.0f, denom = 0.0f;
-            for (int k = 0; k < a.K; ++k) {
-                float bv = -INFINITY, bz = 0.0f;
-                int bi = INT_MAX;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i) {
-                    const int j = lane + 32 * i;
-                    if (!((taken >> i) & 1u) && (r[i] > bv || (r[i] == bv && j < bi))) {
-                        bv = r[i];
-                        bi = j;
-                        bz = z[i];
-                    }
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float ov = __shfl_xor_sync(kFull, bv, off);
-                    const int oi = __shfl_xor_sync(kFull, bi, off);
-                    const float oz = __shfl_xor_sync(kFull, bz, off);
-                    if (ov > bv || (ov == bv && oi < bi)) {
-                        bv = ov;
-                        bi = oi;
-                        bz = oz;
-                    }
-                }
-                if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
-                if (k == 0) rmax = bv;
-                const float ek = expf(bv - rmax);
-                denom += ek;
-                if (lane == k) {
-                    my_cand = bi;
-                    my_e = ek;
-                    my_z = bz;
-                }
-            }
-            if (!a.renorm) {
-                float part = 0.0f;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i)
-                    if (lane + 32 * i < a.E) part += expf(r[i] - rmax);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
-                denom = part;  // identical on every lane (pairwise sums commute exactly)
-            }
-            const bool kept = (lane < a.K) && (!a.has_mask || my_z >= a.thr);
-            if (lane < a.K) {
-                const float g = my_e / denom;
-                a.idx[(long long)t * a.K + lane] = kept ? my_cand : -1;
-                a.w[(long long)t * a.K + lane] = kept ? g : 0.0f;
-                if (kept) atomicAdd(&s_counts[my_cand], 1);
-                if (a.cand) a.cand[(long long)t * a.K + lane] = my_cand;
-                if (a.gk) a.gk[(long long)t * a.K + lane] = g;
-                if (a.counts_all) atomicAdd(&s_counts_all[my_cand], 1);
-            }
-            const int nkept = __popc(__ballot_sync(kFull, kept));
-            if (lane == 0) atomicAdd(&s_hist[nkept], 1);
+            const long long o = (long long)(t0 + warp) * a.K;
+            topk_token<EPL>(s_logit[warp], a.E, a.K, a.renorm, a.has_mask, a.thr, a.idx + o,
+                            a.w + o, a.cand ? a.cand + o : nullptr, a.gk ? a.gk + o : nullptr,
+                            s_counts, a.counts_all ? s_counts_all : nullptr, s_hist);
         }
         __syncthreads();  // s_logit is rewritten by the next tokens
     }

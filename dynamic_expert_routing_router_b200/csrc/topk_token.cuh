@@ -1,0 +1,98 @@
+// topk_token.cuh -- top-K, softmax, binary mask and aggregation of one token
+// by one warp (BEAM §3.2 Eq. 4-7).  The calling warp must be converged (every
+// shuffle below is full-mask).
+#pragma once
+
+#include <climits>
+
+namespace beam {
+
+// lg: the token's logits in shared memory, gate logits [0, E), mask
+// pre-activations [E, 2E) (read only with a mask).  Lane l holds experts l,
+// l+32, ...; K rounds of a warp arg-max (ties -> lower expert id) give the
+// candidates in descending order.  renorm: softmax over the candidates
+// (Eq. 4); else over all E.  Candidate k is kept iff its z >= thr = logit(tau)
+// (Eq. 6; NaN is not kept); w = g * m (Eq. 7).  Writes idx_t[k] / w_t[k] and,
+// when given, cand_t[k] / gk_t[k]; adds to the shared counters.
+template <int EPL>
+__device__ __forceinline__ void topk_token(const float *lg, int E, int K, int renorm,
+                                           int has_mask, float thr, int *idx_t, float *w_t,
+                                           int *cand_t, float *gk_t, int *s_counts,
+                                           int *s_counts_all, int *s_hist) {
+    constexpr unsigned kAll = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    float r[EPL], z[EPL];
+    unsigned taken = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int j = lane + 32 * i;
+        r[i] = -INFINITY;
+        z[i] = 0.0f;
+        if (j < E) {
+            const float rs = lg[j];
+            r[i] = (rs != rs) ? -INFINITY : rs;  // NaN never wins a slot
+            if (has_mask) z[i] = lg[E + j];
+        } else {
+            taken |= 1u << i;
+        }
+    }
+
+    int my_cand = -1;
+    float my_e = 0.0f, my_z = 0.0f, rmax = 0.0f, denom = 0.0f;
+    for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY, bz = 0.0f;
+        int bi = INT_MAX;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int j = lane + 32 * i;
+            if (!((taken >> i) & 1u) && (r[i] > bv || (r[i] == bv && j < bi))) {
+                bv = r[i];
+                bi = j;
+                bz = z[i];
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(kAll, bv, off);
+            const int oi = __shfl_xor_sync(kAll, bi, off);
+            const float oz = __shfl_xor_sync(kAll, bz, off);
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+                bz = oz;
+            }
+        }
+        if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
+        if (k == 0) rmax = bv;
+        const float ek = expf(bv - rmax);
+        denom += ek;
+        if (lane == k) {
+            my_cand = bi;
+            my_e = ek;
+            my_z = bz;
+        }
+    }
+    if (!renorm) {
+        float part = 0.0f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (lane + 32 * i < E) part += expf(r[i] - rmax);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kAll, part, off);
+        denom = part;  // identical on every lane (pairwise sums commute exactly)
+    }
+    const bool kept = (lane < K) && (!has_mask || my_z >= thr);
+    if (lane < K) {
+        const float g = my_e / denom;
+        idx_t[lane] = kept ? my_cand : -1;
+        w_t[lane] = kept ? g : 0.0f;
+        if (kept) atomicAdd(&s_counts[my_cand], 1);
+        if (cand_t) cand_t[lane] = my_cand;
+        if (gk_t) gk_t[lane] = g;
+        if (s_counts_all) atomicAdd(&s_counts_all[my_cand], 1);
+    }
+    const int nkept = __popc(__ballot_sync(kAll, kept));
+    if (lane == 0) atomicAdd(&s_hist[nkept], 1);
+}
+
+}  // namespace beam
