@@ -455,23 +455,33 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *W
 
 // -------------------------------------------------------- weight gradients --
 // Kept rows of expert e (rows [first, first + n) of the candidate grouping),
-// chunk [r0, r0 + cnt): compacted row indices into s_kr (returns how many).
+// chunk [r0, r0 + cnt): compacted row indices, in ascending order, into s_kr
+// (returns how many).  One thread per row of the chunk: blockDim.x ==
+// kWgChunk; s_wc holds the per-warp counts.
 constexpr int kWgChunk = 256;
-__device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, int *s_flag,
-                                  int *s_kr, int *s_n) {
-    for (int q = threadIdx.x; q < cnt; q += blockDim.x) {
-        const int r = first + r0 + q;
-        s_flag[q] = a.idx[a.pair[r]] >= 0 ? r : -1;
-    }
+// Bring the line holding p into L2 (the gradient rows a block will read back,
+// issued before its kept rows are staged so that the read overlaps them).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+__device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, int *s_wc,
+                                  int *s_kr) {
+    const int q = threadIdx.x, lane = q & 31, warp = q >> 5;
+    const int r = first + r0 + q;
+    const bool kept = q < cnt && a.idx[a.pair[r]] >= 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, kept);
+    if (lane == 0) s_wc[warp] = __popc(bal);
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int n = 0;
-        for (int q = 0; q < cnt; ++q)
-            if (s_flag[q] >= 0) s_kr[n++] = s_flag[q];
-        *s_n = n;
+    int base = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWgChunk / 32; ++w) {
+        const int c = s_wc[w];
+        base += w < warp ? c : 0;
+        total += c;
     }
+    if (kept) s_kr[base + __popc(bal & ((1u << lane) - 1u))] = r;
     __syncthreads();
-    return *s_n;
+    return total;
 }
 
 // dW1_e[i] += sum over kept rows (in order) da[r][i] x_r, dW3 likewise with db.
@@ -479,8 +489,8 @@ __device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, i
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn *xp, float *dW1,
                                                       float *dW3) {
-    __shared__ int s_first, s_n;
-    __shared__ int s_flag[kWgChunk], s_kr[kWgChunk];
+    __shared__ int s_first;
+    __shared__ int s_wc[kWgChunk / 32], s_kr[kWgChunk];
     __shared__ float s_da[kWgChunk][4], s_db[kWgChunk][4];
     griddep_wait();
     griddep_launch_dependents();
@@ -493,14 +503,21 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
     for (int jb = 0; jb < d; jb += 8 * blockDim.x) {
         const int j = jb + threadIdx.x * 8;
         const bool active = j < d;
+        if (active)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i0 + i < I) {
+                    const long long o = ((long long)e * I + i0 + i) * d + j;
+                    prefetch_l2(dW1 + o);
+                    prefetch_l2(dW3 + o);
+                }
         float g1[4][8], g3[4][8];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int c = 0; c < 8; ++c) g1[i][c] = g3[i][c] = 0.0f;
         for (int r0 = 0; r0 < n; r0 += kWgChunk) {
-            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_flag, s_kr,
-                                              &s_n);
+            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_wc, s_kr);
             for (int q = threadIdx.x; q < 4 * nk; q += blockDim.x) {
                 const int kq = q >> 2, i = q & 3;
                 const bool ok = i0 + i < I;
@@ -509,7 +526,7 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
             }
             __syncthreads();
             if (active) {
-#pragma unroll 2
+#pragma unroll 4
                 for (int kq = 0; kq < nk; ++kq) {
                     float xv[8];
                     load8(xp + (long long)s_kr[kq] * d + j, xv);
@@ -548,8 +565,8 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
 // finalize step).  Block (expert, 8 rows of d); each thread owns 4 columns of I.
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *dyp, float *dW2) {
-    __shared__ int s_first, s_n;
-    __shared__ int s_flag[kWgChunk], s_kr[kWgChunk];
+    __shared__ int s_first;
+    __shared__ int s_wc[kWgChunk / 32], s_kr[kWgChunk];
     __shared__ float s_dy[kWgChunk][8];
     griddep_wait();
     griddep_launch_dependents();
@@ -562,14 +579,17 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
     for (int ib = 0; ib < I; ib += 4 * blockDim.x) {
         const int i = ib + threadIdx.x * 4;
         const bool active = i < I;
+        if (active && (threadIdx.x & 1) == 0)  // one request per 32-byte sector
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                if (j0 + jj < d) prefetch_l2(dW2 + ((long long)e * d + j0 + jj) * I + i);
         float g[8][4];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj)
 #pragma unroll
             for (int c = 0; c < 4; ++c) g[jj][c] = 0.0f;
         for (int r0 = 0; r0 < n; r0 += kWgChunk) {
-            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_flag, s_kr,
-                                              &s_n);
+            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_wc, s_kr);
             for (int q = threadIdx.x; q < 8 * nk; q += blockDim.x) {
                 const int kq = q >> 3, jj = q & 7;
                 const int r = s_kr[kq];
@@ -578,7 +598,7 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
             }
             __syncthreads();
             if (active) {
-#pragma unroll 2
+#pragma unroll 4
                 for (int kq = 0; kq < nk; ++kq) {
                     const float4 hv = *reinterpret_cast<const float4 *>(a.h + (long long)s_kr[kq] * I + i);
 #pragma unroll
