@@ -729,6 +729,66 @@ cudaError_t launch_rowgemm(const BwArgs &a, const TA *A, const TA *A2, const TB 
                       a.S);
 }
 
+namespace {
+// One block of 256 threads walks the grouping's tiles in order; the first
+// tile of an expert with a kept pair emits that expert's row tiles.  Output
+// positions are an exclusive prefix over the tiles, so the list is in expert
+// order.
+__global__ void __launch_bounds__(256) expert_tiles_kernel(const int4 *tiles, const int *meta,
+                                                           const int *counts_kept,
+                                                           const int *counts_all,
+                                                           int rows_per_tile, int4 *xtiles,
+                                                           int *xmeta) {
+    __shared__ int s_warp[8];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int n = meta[0];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int base = 0;  // block-uniform
+    for (int b0 = 0; b0 < n; b0 += 256) {
+        const int ti = b0 + threadIdx.x;
+        int nt = 0, e = 0, row0 = 0, cnt = 0;
+        if (ti < n) {
+            const int4 t = tiles[ti];
+            e = t.x;
+            row0 = t.y;
+            if ((ti == 0 || tiles[ti - 1].x != e) && counts_kept[e] > 0) {
+                cnt = counts_all[e];
+                nt = (cnt + rows_per_tile - 1) / rows_per_tile;
+            }
+        }
+        int incl = nt;  // inclusive prefix within the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) s_warp[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            before += w < warp ? s_warp[w] : 0;
+            total += s_warp[w];
+        }
+        const int pos = base + before + incl - nt;
+        for (int j = 0; j < nt; ++j)
+            xtiles[pos + j] = make_int4(e, row0 + j * rows_per_tile,
+                                        min(rows_per_tile, cnt - j * rows_per_tile), 0);
+        base += total;
+        __syncthreads();  // s_warp is rewritten by the next round
+    }
+    if (threadIdx.x == 0) xmeta[0] = base;
+}
+}  // namespace
+
+cudaError_t launch_expert_tiles(const int4 *tiles, const int *meta, const int *counts_kept,
+                                const int *counts_all, int rows_per_tile, int4 *xtiles,
+                                int *xmeta, cudaStream_t st) {
+    return launch_pdl(expert_tiles_kernel, dim3(1), dim3(256), 0, st, tiles, meta, counts_kept,
+                      counts_all, rows_per_tile, xtiles, xmeta);
+}
+
 cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
                                    const void *dy, const void *dyp, const void *Wg,
                                    const void *Wm, const void *W1, const void *W3,
@@ -744,10 +804,12 @@ cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, co
         const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
         const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
         if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-        if ((e = launch_rowgemm<TG_DH, T, T>(a, dypb, dypb, static_cast<const T *>(W2),
+        if (!a.dh_tc &&
+            (e = launch_rowgemm<TG_DH, T, T>(a, dypb, dypb, static_cast<const T *>(W2),
                                              static_cast<const T *>(W2), a.d, a.I, st)))
             return e;
-        if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.S))) return e;
+        if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.dh_tc ? 1 : a.S)))
+            return e;
         if ((e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, static_cast<const T *>(W1),
                                                  static_cast<const T *>(W3), a.I, a.d, st)))
             return e;

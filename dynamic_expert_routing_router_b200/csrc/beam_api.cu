@@ -502,7 +502,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
 struct BwdPlan {
     int S;  // reduction splits of the kept-row products
     size_t off_cand, off_gk, off_counts_all, off_logits, off_dyp, off_A, off_B, off_da, off_db,
-        off_h, off_part, off_u, off_dz, off_dr, bytes;
+        off_h, off_part, off_u, off_dz, off_dr, off_xtiles, off_xmeta, bytes;
 };
 
 beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan *B) {
@@ -537,6 +537,10 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     B->off_u = take(4 * T * K);
     B->off_dz = take(4 * T * K);
     B->off_dr = take(4 * T * E);
+    // bf16: per-expert row tiles of the tensor-core dh product (at most one
+    // per grouping tile) and their count
+    B->off_xtiles = take(16 * size_t(P->tiles_cap));
+    B->off_xmeta = take(4);
     B->bytes = o;
     return BEAM_OK;
 }
@@ -646,6 +650,26 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
         g.out_ld = d->d;
         units = (long long)P.tiles_cap * g.n_mb;
         BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, P.BN, m2, g, int(units < n_sm ? units : n_sm), st));
+        // dh = dy W2_e for the kept experts on the tensor cores, one pass per
+        // expert (its candidate rows as 128-row tiles), into the first split
+        // of the partials; dh_finalize then sums a single split.
+        int4 *xtiles = reinterpret_cast<int4 *>(ws + B.off_xtiles);
+        int *xmeta = reinterpret_cast<int *>(ws + B.off_xmeta);
+        BEAM_TRY_CUDA(launch_expert_tiles(tiles, meta, counts, counts_all, kBlockM, xtiles, xmeta, st));
+        TcMaps m3;
+        if (!make_tmap(&m3.a0, W2, d->I, (unsigned long long)d->E * d->d, kBlockK)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&m3.b, dyp, d->d, P.p_cap, kBlockM)) return BEAM_ERR_CUDA;
+        m3.a1 = m3.a2 = m3.a0;
+        m3.b2 = m3.b;
+        g.meta = xmeta;
+        g.tiles = xtiles;
+        g.n_mb = d->I / kBlockM;
+        g.nk = d->d / kBlockK;
+        g.a_rows_per_expert = d->d;
+        g.out = ws + B.off_part;
+        g.out_ld = d->I;
+        units = (long long)P.tiles_cap * g.n_mb;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2T, kBlockM, m3, g, int(units < n_sm ? units : n_sm), st));
     } else {
         BEAM_TRY_CUDA(launch_gemm1_f32(static_cast<const float *>(xp), static_cast<const float *>(W1),
                                        static_cast<const float *>(W3), tiles, meta, P.tiles_cap,
@@ -684,6 +708,7 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
     a.db = reinterpret_cast<float *>(ws + B.off_db);
     a.h = reinterpret_cast<float *>(ws + B.off_h);
     a.part = reinterpret_cast<float *>(ws + B.off_part);
+    a.dh_tc = d->dtype == BEAM_BF16 ? 1 : 0;
     a.u = reinterpret_cast<float *>(ws + B.off_u);
     a.dz = reinterpret_cast<float *>(ws + B.off_dz);
     a.dr = reinterpret_cast<float *>(ws + B.off_dr);
@@ -767,8 +792,9 @@ int beam_moe_backward_kernel_count(const beam_moe_desc *desc) {
     if (make_bwd_plan(desc, &P, &B) != BEAM_OK || desc->T == 0) return 0;
     // router, top-K, grouping, dy gather, gate/up, down, then the eight
     // CUDA-core stages (token, dh product, dh finalize, dx product, dx,
-    // dW1/dW3, dW2, router weights)
-    return 14;
+    // dW1/dW3, dW2, router weights); bf16 runs the dh product on the tensor
+    // cores after building its expert tiles (one launch more).
+    return desc->dtype == BEAM_BF16 ? 15 : 14;
 }
 
 size_t beam_moe_workspace_size(const beam_moe_desc *desc) {

@@ -21,7 +21,8 @@ enum TcMode : int {
     MODE_GEMM1 = 1,   // SiLU(W1 x) * (W3 x) per kept pair  -> H
     MODE_GEMM2 = 2,   // W2 h per kept pair                  -> Y
     MODE_GEMM1_IL = 3, // GEMM1 with 64 rows of W1 and 64 of W3 interleaved in one tile
-    MODE_EXPERTS = 4   // MODE_GEMM1_IL units then MODE_GEMM2 units in one launch
+    MODE_EXPERTS = 4,  // MODE_GEMM1_IL units then MODE_GEMM2 units in one launch
+    MODE_GEMM2T = 5    // dy W2_e (training): W2_e read transposed (MN-major A) -> fp32 rows
 };
 
 // Tensor maps of one tensor-core launch.  a0/a1/b: the (first) GEMM's weight
@@ -185,10 +186,18 @@ struct BwArgs {
     float *da, *db;          // [p_cap][I]
     float *h;                // [p_cap][I] SiLU(a) b in fp32 (kept rows)
     float *part;             // [S][p_cap][max(d, I)] split partial products
+    int dh_tc;               // 1: dy W2_e is already in part (one split, tensor cores)
     float *u, *dz;           // [T][K]
     float *dr;               // [T][E]
     float *dx;               // [T][d]
 };
+// Kept experts' candidate rows as tiles of at most rows_per_tile rows (one
+// block): from the grouping's tile list, each expert with a kept pair gives
+// ceil(candidates / rows_per_tile) tiles starting at its first row.  xmeta[0]
+// = how many.  Never more than the grouping's tiles when rows_per_tile >= BN.
+cudaError_t launch_expert_tiles(const int4 *tiles, const int *meta, const int *counts_kept,
+                                const int *counts_all, int rows_per_tile, int4 *xtiles,
+                                int *xmeta, cudaStream_t st);
 cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
                                    const void *dy, const void *dyp, const void *Wg,
                                    const void *Wm, const void *W1, const void *W3,

@@ -161,6 +161,24 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
     return desc;
 }
 
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle:
+// each 128-byte row holds 64 consecutive M (or N) elements of one k, eight
+// k-rows form a 1024-byte atom (TMA SWIZZLE_128B boxes of 64 x rows).  The
+// leading byte offset steps between 64-element MN halves (mn_stride bytes);
+// the stride byte offset between 8-row k groups (1024).  A 16-deep k step
+// advances the start address by 2048 bytes.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint32_t mn_stride) {
+    uint64_t desc = 0;
+    desc |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+    desc |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;
+    desc |= static_cast<uint64_t>(1024u >> 4) << 32;
+    desc |= static_cast<uint64_t>(1u) << 46;
+    desc |= static_cast<uint64_t>(2u) << 61;
+    return desc;
+}
+// Instruction-descriptor bit marking A as MN-major (transposed).
+constexpr uint32_t kIdescAMajorMN = 1u << 15;
+
 // Instruction descriptor of tcgen05.mma.kind::f16: D fp32 [4,6), A bf16
 // [7,10), B bf16 [10,13), both K-major (bits 15, 16 clear), N >> 3 [17,23),
 // M >> 4 [24,29).

@@ -262,8 +262,9 @@ beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const vo
                               const void *dy, float beta, float *dx, float *dW_gate,
                               float *dW_mask, float *dW1, float *dW3, float *dW2,
                               void *workspace, size_t workspace_bytes, void *stream);
-/* Kernel launches of one beam_moe_backward call (14; 0 for T = 0 or a bad
- * descriptor). */
+/* Kernel launches of one beam_moe_backward call: 15 for bf16 (its dh = dy W2_e
+ * product runs on the tensor cores, after a launch that lists each kept
+ * expert's candidate rows), 14 for fp32; 0 for T = 0 or a bad descriptor. */
 int beam_moe_backward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last

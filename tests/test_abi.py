@@ -142,7 +142,8 @@ def test_shared_expert_descriptor_rules():
 def test_backward_descriptor_and_argument_checks():
     dsc = abi.desc(8, 2048, 128, 768, 8, "bf16", 1)
     assert abi.backward_workspace_size(dsc) > abi.workspace_size(dsc)
-    assert abi.backward_kernel_count(dsc) == 14
+    assert abi.backward_kernel_count(dsc) == 15  # bf16: dy W2 on the tensor cores
+    assert abi.backward_kernel_count(abi.desc(8, 128, 8, 256, 2, "f32", 0)) == 14
     assert abi.backward_kernel_count(abi.desc(0, 2048, 128, 768, 8, "bf16", 1)) == 0
     shared = abi.desc(8, 2048, 64, 1408, 6, "bf16", 1, n_shared=2, I_shared=1408)
     assert abi.backward_workspace_size(shared) == 0  # shared experts: forward only
