@@ -371,6 +371,10 @@ __global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S)
             a.da[o] = dh * bv * sa * (1.0f + av * (1.0f - sa));
             a.db[o] = dh * av * sa;
             a.h[o] = av * sa * bv;
+            if (a.da_bf) {  // operands of the tensor-core dx product
+                static_cast<__nv_bfloat16 *>(a.da_bf)[o] = __float2bfloat16_rn(a.da[o]);
+                static_cast<__nv_bfloat16 *>(a.db_bf)[o] = __float2bfloat16_rn(a.db[o]);
+            }
         }
     }
 }
@@ -789,55 +793,56 @@ cudaError_t launch_expert_tiles(const int4 *tiles, const int *meta, const int *c
                       counts_all, rows_per_tile, xtiles, xmeta);
 }
 
+namespace {
+template <typename T>
+cudaError_t backward_stages(const BwArgs &a, const T *x, const T *xp, const T *dy, const T *dyp,
+                            const T *Wg, const T *Wm, const T *W1, const T *W3, const T *W2,
+                            float *dWg, float *dWm, float *dW1, float *dW3, float *dW2, int n_sm,
+                            cudaStream_t st, int phase) {
+    const int tb = a.T < 8 * n_sm ? a.T : 8 * n_sm;
+    cudaError_t e;
+    if (phase == 0) {
+        if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dy))) return e;
+        if (!a.dh_tc && (e = launch_rowgemm<TG_DH, T, T>(a, dyp, dyp, W2, W2, a.d, a.I, st)))
+            return e;
+        return launch_pdl(dh_finalize_kernel, dim3(a.tiles_cap), dim3(256), 0, st, a,
+                          a.dh_tc ? 1 : a.S);
+    }
+    if (!a.dx_tc && (e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, W1, W3, a.I, a.d, st)))
+        return e;
+    if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a, Wg, Wm, a.dx_tc ? 1 : a.S)))
+        return e;
+    if ((e = launch_pdl(bw_dw13_kernel<T>, dim3(a.E, (a.I + 3) / 4), dim3(256), 0, st, a, xp, dW1,
+                        dW3)))
+        return e;
+    if ((e = launch_pdl(bw_dw2_kernel<T>, dim3(a.E, (a.d + 7) / 8), dim3(256), 0, st, a, dyp, dW2)))
+        return e;
+    return launch_pdl(bw_drouter_kernel<T>, dim3(a.E, (a.d + 255) / 256), dim3(64), 0, st, a, x, xp,
+                      dWg, dWm);
+}
+}  // namespace
+
 cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
                                    const void *dy, const void *dyp, const void *Wg,
                                    const void *Wm, const void *W1, const void *W3,
                                    const void *W2, float *dWg, float *dWm, float *dW1,
-                                   float *dW3, float *dW2, int n_sm, cudaStream_t st) {
+                                   float *dW3, float *dW2, int n_sm, cudaStream_t st, int phase) {
     if (a.T <= 0) return cudaSuccess;
-    const int tb = a.T < 8 * n_sm ? a.T : 8 * n_sm;
-    const dim3 g_fin(a.tiles_cap);
-    const dim3 g_w13(a.E, (a.I + 3) / 4), g_w2(a.E, (a.d + 7) / 8), g_r(a.E, (a.d + 255) / 256);
-    cudaError_t e;
     if (dtype == BEAM_BF16) {
         using T = __nv_bfloat16;
-        const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
-        const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
-        if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-        if (!a.dh_tc &&
-            (e = launch_rowgemm<TG_DH, T, T>(a, dypb, dypb, static_cast<const T *>(W2),
-                                             static_cast<const T *>(W2), a.d, a.I, st)))
-            return e;
-        if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.dh_tc ? 1 : a.S)))
-            return e;
-        if ((e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, static_cast<const T *>(W1),
-                                                 static_cast<const T *>(W3), a.I, a.d, st)))
-            return e;
-        if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a,
-                            static_cast<const T *>(Wg), static_cast<const T *>(Wm), a.S)))
-            return e;
-        if ((e = launch_pdl(bw_dw13_kernel<T>, g_w13, dim3(256), 0, st, a, xpb, dW1, dW3)))
-            return e;
-        if ((e = launch_pdl(bw_dw2_kernel<T>, g_w2, dim3(256), 0, st, a, dypb, dW2))) return e;
-        return launch_pdl(bw_drouter_kernel<T>, g_r, dim3(64), 0, st, a, xb, xpb, dWg, dWm);
+        return backward_stages<T>(a, static_cast<const T *>(x), static_cast<const T *>(xp),
+                                  static_cast<const T *>(dy), static_cast<const T *>(dyp),
+                                  static_cast<const T *>(Wg), static_cast<const T *>(Wm),
+                                  static_cast<const T *>(W1), static_cast<const T *>(W3),
+                                  static_cast<const T *>(W2), dWg, dWm, dW1, dW3, dW2, n_sm, st,
+                                  phase);
     }
-    using T = float;
-    const T *xb = static_cast<const T *>(x), *xpb = static_cast<const T *>(xp);
-    const T *dyb = static_cast<const T *>(dy), *dypb = static_cast<const T *>(dyp);
-    if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dyb))) return e;
-    if ((e = launch_rowgemm<TG_DH, T, T>(a, dypb, dypb, static_cast<const T *>(W2),
-                                         static_cast<const T *>(W2), a.d, a.I, st)))
-        return e;
-    if ((e = launch_pdl(dh_finalize_kernel, g_fin, dim3(256), 0, st, a, a.S))) return e;
-    if ((e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, static_cast<const T *>(W1),
-                                             static_cast<const T *>(W3), a.I, a.d, st)))
-        return e;
-    if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a,
-                        static_cast<const T *>(Wg), static_cast<const T *>(Wm), a.S)))
-        return e;
-    if ((e = launch_pdl(bw_dw13_kernel<T>, g_w13, dim3(256), 0, st, a, xpb, dW1, dW3))) return e;
-    if ((e = launch_pdl(bw_dw2_kernel<T>, g_w2, dim3(256), 0, st, a, dypb, dW2))) return e;
-    return launch_pdl(bw_drouter_kernel<T>, g_r, dim3(64), 0, st, a, xb, xpb, dWg, dWm);
+    return backward_stages<float>(a, static_cast<const float *>(x), static_cast<const float *>(xp),
+                                  static_cast<const float *>(dy), static_cast<const float *>(dyp),
+                                  static_cast<const float *>(Wg), static_cast<const float *>(Wm),
+                                  static_cast<const float *>(W1), static_cast<const float *>(W3),
+                                  static_cast<const float *>(W2), dWg, dWm, dW1, dW3, dW2, n_sm, st,
+                                  phase);
 }
 
 }  // namespace beam

@@ -502,7 +502,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
 struct BwdPlan {
     int S;  // reduction splits of the kept-row products
     size_t off_cand, off_gk, off_counts_all, off_logits, off_dyp, off_A, off_B, off_da, off_db,
-        off_h, off_part, off_u, off_dz, off_dr, off_xtiles, off_xmeta, bytes;
+        off_h, off_part, off_u, off_dz, off_dr, off_xtiles, off_xmeta, off_dab, off_dbb, bytes;
 };
 
 beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan *B) {
@@ -541,6 +541,9 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     // per grouping tile) and their count
     B->off_xtiles = take(16 * size_t(P->tiles_cap));
     B->off_xmeta = take(4);
+    // bf16: da, db rounded once more as the tensor-core dx product's operands
+    B->off_dab = take(d->dtype == BEAM_BF16 ? 2 * pc * I : 0);
+    B->off_dbb = take(d->dtype == BEAM_BF16 ? 2 * pc * I : 0);
     B->bytes = o;
     return BEAM_OK;
 }
@@ -709,12 +712,40 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
     a.h = reinterpret_cast<float *>(ws + B.off_h);
     a.part = reinterpret_cast<float *>(ws + B.off_part);
     a.dh_tc = d->dtype == BEAM_BF16 ? 1 : 0;
+    a.dx_tc = a.dh_tc;
+    a.da_bf = a.dx_tc ? ws + B.off_dab : nullptr;
+    a.db_bf = a.dx_tc ? ws + B.off_dbb : nullptr;
     a.u = reinterpret_cast<float *>(ws + B.off_u);
     a.dz = reinterpret_cast<float *>(ws + B.off_dz);
     a.dr = reinterpret_cast<float *>(ws + B.off_dr);
     a.dx = dx;
     BEAM_TRY_CUDA(launch_backward_stages(a, d->dtype, x, xp, dy, dyp, Wg, Wm, W1, W3, W2, dWg,
-                                         dWm, dW1, dW3, dW2, n_sm, st));
+                                         dWm, dW1, dW3, dW2, n_sm, st, 0));
+    if (a.dx_tc) {
+        // dxp = da W1_e + db W3_e on the tensor cores over the same expert
+        // tiles: 2I k-rows per unit (W1_e with da, then W3_e with db).
+        TcMaps m4;
+        if (!make_tmap(&m4.a0, W1, d->d, (unsigned long long)d->E * d->I, kBlockK)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&m4.a1, W3, d->d, (unsigned long long)d->E * d->I, kBlockK)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&m4.b, a.da_bf, d->I, P.p_cap, kBlockM)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&m4.b2, a.db_bf, d->I, P.p_cap, kBlockM)) return BEAM_ERR_CUDA;
+        m4.a2 = m4.a0;
+        TcGemmArgs g;
+        std::memset(&g, 0, sizeof(g));
+        g.meta = reinterpret_cast<int *>(ws + B.off_xmeta);
+        g.tiles = reinterpret_cast<int4 *>(ws + B.off_xtiles);
+        g.err = err;
+        g.timeout_ns = kWaitTimeoutNs;
+        g.n_mb = d->d / kBlockM;
+        g.nk = 2 * (d->I / kBlockK);
+        g.a_rows_per_expert = d->I;
+        g.out = a.part;
+        g.out_ld = d->d;
+        const long long units = (long long)P.tiles_cap * g.n_mb;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1T, kBlockM, m4, g, int(units < n_sm ? units : n_sm), st));
+    }
+    BEAM_TRY_CUDA(launch_backward_stages(a, d->dtype, x, xp, dy, dyp, Wg, Wm, W1, W3, W2, dWg,
+                                         dWm, dW1, dW3, dW2, n_sm, st, 1));
     return BEAM_OK;
 }
 

@@ -22,7 +22,8 @@ enum TcMode : int {
     MODE_GEMM2 = 2,   // W2 h per kept pair                  -> Y
     MODE_GEMM1_IL = 3, // GEMM1 with 64 rows of W1 and 64 of W3 interleaved in one tile
     MODE_EXPERTS = 4,  // MODE_GEMM1_IL units then MODE_GEMM2 units in one launch
-    MODE_GEMM2T = 5    // dy W2_e (training): W2_e read transposed (MN-major A) -> fp32 rows
+    MODE_GEMM2T = 5,   // dy W2_e (training): W2_e read transposed (MN-major A) -> fp32 rows
+    MODE_GEMM1T = 6    // da W1_e + db W3_e (training): W1_e, W3_e read transposed -> fp32 rows
 };
 
 // Tensor maps of one tensor-core launch.  a0/a1/b: the (first) GEMM's weight
@@ -187,6 +188,9 @@ struct BwArgs {
     float *h;                // [p_cap][I] SiLU(a) b in fp32 (kept rows)
     float *part;             // [S][p_cap][max(d, I)] split partial products
     int dh_tc;               // 1: dy W2_e is already in part (one split, tensor cores)
+    int dx_tc;               // 1: da W1_e + db W3_e runs on the tensor cores between the
+                             //    two stage phases, into part (one split)
+    void *da_bf, *db_bf;     // [p_cap][I] bf16 copies of da, db (kept rows) or null
     float *u, *dz;           // [T][K]
     float *dr;               // [T][E]
     float *dx;               // [T][d]
@@ -198,11 +202,13 @@ struct BwArgs {
 cudaError_t launch_expert_tiles(const int4 *tiles, const int *meta, const int *counts_kept,
                                 const int *counts_all, int rows_per_tile, int4 *xtiles,
                                 int *xmeta, cudaStream_t st);
+// phase 0: token stage, dh product (unless dh_tc), dh finalize; phase 1: dx
+// product (unless dx_tc), dx, dW1/dW3, dW2, router weights.
 cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
                                    const void *dy, const void *dyp, const void *Wg,
                                    const void *Wm, const void *W1, const void *W3,
                                    const void *W2, float *dWg, float *dWm, float *dW1,
-                                   float *dW3, float *dW2, int n_sm, cudaStream_t st);
+                                   float *dW3, float *dW2, int n_sm, cudaStream_t st, int phase);
 
 // fp32 SIMT path (BEAM_F32).
 cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,

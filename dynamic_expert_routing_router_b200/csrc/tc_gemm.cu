@@ -12,6 +12,9 @@
 //   MODE_GEMM2T   dh = dy W2_e (training): the A tile is 128 columns of W2_e
 //                 over 64 of its rows, i.e. W2_e read transposed (MN-major,
 //                 two 64-column TMA boxes per stage); fp32 out
+//   MODE_GEMM1T   dxp = da W1_e + db W3_e (training): one reduction of 2I
+//                 k-rows, W1_e with da rows then W3_e with db rows, the weights
+//                 read transposed as in MODE_GEMM2T; fp32 out
 //   MODE_EXPERTS  MODE_GEMM1_IL units followed by MODE_GEMM2 units in one
 //                 launch: a down-projection unit of a token tile starts once
 //                 every gate/up unit of that tile has published its rows of H
@@ -125,7 +128,8 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs
     }
     int v = u, n_mb = p.n_mb, rows_per_mb = kBlockM, a_rows = p.a_rows_per_expert;
     if (MODE == MODE_GEMM1_IL) rows_per_mb = kBlockM / 2;
-    if (MODE == MODE_GEMM2T) rows_per_mb = 0;  // a_row: the expert's first k-row; mb picks columns
+    if (MODE == MODE_GEMM2T || MODE == MODE_GEMM1T)
+        rows_per_mb = 0;  // a_row: the expert's first k-row; mb picks columns
     if (MODE == MODE_EXPERTS) {
         if (u < n_first) {
             rows_per_mb = kBlockM / 2;
@@ -311,8 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
-                    const int kx = (w.kb0 + kb) * kBlockK;
-                    if (MODE == MODE_GEMM2T) {
+                    int kx = (w.kb0 + kb) * kBlockK;
+                    if (MODE == MODE_GEMM1T && 2 * kb >= w.nk) {  // second half: W3_e with db
+                        am = &maps.a1;
+                        bm = &maps.b2;
+                        kx -= (w.nk / 2) * kBlockK;
+                    }
+                    if (MODE == MODE_GEMM2T || MODE == MODE_GEMM1T) {
                         // W2_e rows [kx, kx + 64) x columns [mb 128, + 128): two boxes
                         tma_load_2d(st, am, w.mb * kBlockM, w.a_row + kx, &full_bar[s]);
                         tma_load_2d(st + C::A_BYTES / 2, am, w.mb * kBlockM + kBlockM / 2,
@@ -342,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------- MMA issuer --
         if (lane == 0) {
             constexpr uint32_t IDESC =
-                umma_idesc_bf16_f32(kBlockM, BN) | (MODE == MODE_GEMM2T ? kIdescAMajorMN : 0u);
+                umma_idesc_bf16_f32(kBlockM, BN) |
+                ((MODE == MODE_GEMM2T || MODE == MODE_GEMM1T) ? kIdescAMajorMN : 0u);
             uint32_t it = 0;
             bool ok = true;
             for (uint32_t lu = 0;; ++lu) {
@@ -384,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = umma_desc_sw128(sb + kk * 32);
                         const uint64_t adesc =
-                            MODE == MODE_GEMM2T
+                            (MODE == MODE_GEMM2T || MODE == MODE_GEMM1T)
                                 ? umma_desc_sw128_mn(sa + kk * (kUmmaK / 8) * 1024, C::A_BYTES / 2)
                                 : umma_desc_sw128(sa + kk * 32);
                         umma_bf16(d0, adesc, bdesc, IDESC, acc);
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + a * C::ACC_COLS;
             const bool gate_up_il =
                 MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
-            const bool down = MODE == MODE_GEMM2 || MODE == MODE_GEMM2T ||
+            const bool down = MODE == MODE_GEMM2 || MODE == MODE_GEMM2T || MODE == MODE_GEMM1T ||
                               (MODE == MODE_EXPERTS && w.phase == 1);
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -580,6 +590,7 @@ cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArg
         case MODE_GEMM1_IL: return launch_bn<MODE_GEMM1_IL>(bn, maps, args, grid, stream);
         case MODE_EXPERTS: return launch_bn<MODE_EXPERTS>(bn, maps, args, grid, stream);
         case MODE_GEMM2T: return launch_bn<MODE_GEMM2T>(bn, maps, args, grid, stream);
+        case MODE_GEMM1T: return launch_bn<MODE_GEMM1T>(bn, maps, args, grid, stream);
         default: return cudaErrorInvalidValue;
     }
 }
