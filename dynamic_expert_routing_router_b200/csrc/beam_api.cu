@@ -531,8 +531,10 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     // Thin decode tiles leave most SMs idle with one block per tile: split the
     // reduction of the kept-row products eight ways (d and I are multiples of 8).
     B->S = P->BN < 128 ? 8 : 1;
-    // The kept-row products hold a split's A rows in shared memory.
-    if (dd / B->S > 7168 || I / B->S > 4096) return BEAM_ERR_UNSUPPORTED_SHAPE;
+    // fp32: the CUDA-core kept-row products hold a split's A rows in shared
+    // memory (bf16 runs both products on the tensor cores).
+    if (d->dtype != BEAM_BF16 && (dd / B->S > 7168 || I / B->S > 4096))
+        return BEAM_ERR_UNSUPPORTED_SHAPE;
     B->off_part = take(4 * size_t(B->S) * pc * (dd > I ? dd : I));
     B->off_u = take(4 * T * K);
     B->off_dz = take(4 * T * K);

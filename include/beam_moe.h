@@ -253,9 +253,14 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
  * Every sum runs in a fixed order: the gradients are bitwise repeatable.
  * Workspace: beam_moe_backward_workspace_size bytes, 256-byte aligned; the
  * caller owns it and every output.  Errors as for beam_moe_forward; also
- * BEAM_ERR_UNSUPPORTED_SHAPE for shared experts, and for d > 7168 or I > 4096
- * at 128-token tiles (8x larger at decode tile sizes), beyond which a split
- * of the kept-row products no longer fits in shared memory. */
+ * BEAM_ERR_UNSUPPORTED_SHAPE for shared experts, and for fp32 layers with
+ * d > 7168 or I > 4096 at 128-token tiles (8x larger at decode tile sizes),
+ * beyond which a split of the CUDA-core kept-row products no longer fits in
+ * shared memory.
+ * Precision (bf16): both kept-row products (dh = dy W2_e and
+ * dxp = da W1_e + db W3_e) run on the tensor cores with bf16 operands and fp32
+ * accumulation; their da, db operands are da, db rounded once to bf16, while
+ * dW1, dW3 use da, db in fp32. */
 size_t beam_moe_backward_workspace_size(const beam_moe_desc *desc);
 beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const void *W_gate,
                               const void *W_mask, const void *W1, const void *W3, const void *W2,
