@@ -734,63 +734,82 @@ cudaError_t launch_rowgemm(const BwArgs &a, const TA *A, const TA *A2, const TB 
 }
 
 namespace {
-// One block of 256 threads walks the grouping's tiles in order; the first
-// tile of an expert with a kept pair emits that expert's row tiles.  Output
-// positions are an exclusive prefix over the tiles, so the list is in expert
-// order.
+// Exclusive prefix of v over the block's 256 threads (in thread order) and
+// the block total; s_warp holds 8 ints and is free again on return.
+__device__ __forceinline__ int block_excl_prefix(int v, int *s_warp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        before += w < warp ? s_warp[w] : 0;
+        tot += s_warp[w];
+    }
+    __syncthreads();
+    *total = tot;
+    return before + incl - v;
+}
+
+// One block of 256 threads walks the grouping's tiles in order.  The first
+// tile of each expert emits that expert's row tiles into list 0 (every
+// candidate expert) and, when the expert has a kept pair, into list 1.
+// Positions are exclusive prefixes over the tiles, so both lists are in
+// expert order.
 __global__ void __launch_bounds__(256) expert_tiles_kernel(const int4 *tiles, const int *meta,
                                                            const int *counts_kept,
                                                            const int *counts_all,
-                                                           int rows_per_tile, int4 *xtiles,
-                                                           int *xmeta) {
+                                                           int rows_per_tile, int4 *xt_all,
+                                                           int4 *xt_kept, int *xmeta) {
     __shared__ int s_warp[8];
     griddep_wait();
     griddep_launch_dependents();
     const int n = meta[0];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int base = 0;  // block-uniform
+    int base_all = 0, base_kept = 0;  // block-uniform
     for (int b0 = 0; b0 < n; b0 += 256) {
         const int ti = b0 + threadIdx.x;
         int nt = 0, e = 0, row0 = 0, cnt = 0;
+        bool kept = false;
         if (ti < n) {
             const int4 t = tiles[ti];
             e = t.x;
             row0 = t.y;
-            if ((ti == 0 || tiles[ti - 1].x != e) && counts_kept[e] > 0) {
+            if (ti == 0 || tiles[ti - 1].x != e) {
                 cnt = counts_all[e];
                 nt = (cnt + rows_per_tile - 1) / rows_per_tile;
+                kept = counts_kept[e] > 0;
             }
         }
-        int incl = nt;  // inclusive prefix within the warp
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
+        int tot_all, tot_kept;
+        const int pa = base_all + block_excl_prefix(nt, s_warp, &tot_all);
+        const int pk = base_kept + block_excl_prefix(kept ? nt : 0, s_warp, &tot_kept);
+        for (int j = 0; j < nt; ++j) {
+            const int4 v = make_int4(e, row0 + j * rows_per_tile,
+                                     min(rows_per_tile, cnt - j * rows_per_tile), 0);
+            xt_all[pa + j] = v;
+            if (kept) xt_kept[pk + j] = v;
         }
-        if (lane == 31) s_warp[warp] = incl;
-        __syncthreads();
-        int before = 0, total = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            before += w < warp ? s_warp[w] : 0;
-            total += s_warp[w];
-        }
-        const int pos = base + before + incl - nt;
-        for (int j = 0; j < nt; ++j)
-            xtiles[pos + j] = make_int4(e, row0 + j * rows_per_tile,
-                                        min(rows_per_tile, cnt - j * rows_per_tile), 0);
-        base += total;
-        __syncthreads();  // s_warp is rewritten by the next round
+        base_all += tot_all;
+        base_kept += tot_kept;
     }
-    if (threadIdx.x == 0) xmeta[0] = base;
+    if (threadIdx.x == 0) {
+        xmeta[0] = base_all;
+        xmeta[1] = base_kept;
+    }
 }
 }  // namespace
 
 cudaError_t launch_expert_tiles(const int4 *tiles, const int *meta, const int *counts_kept,
-                                const int *counts_all, int rows_per_tile, int4 *xtiles,
-                                int *xmeta, cudaStream_t st) {
+                                const int *counts_all, int rows_per_tile, int4 *xt_all,
+                                int4 *xt_kept, int *xmeta, cudaStream_t st) {
     return launch_pdl(expert_tiles_kernel, dim3(1), dim3(256), 0, st, tiles, meta, counts_kept,
-                      counts_all, rows_per_tile, xtiles, xmeta);
+                      counts_all, rows_per_tile, xt_all, xt_kept, xmeta);
 }
 
 namespace {

@@ -502,7 +502,8 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
 struct BwdPlan {
     int S;  // reduction splits of the kept-row products
     size_t off_cand, off_gk, off_counts_all, off_logits, off_dyp, off_A, off_B, off_da, off_db,
-        off_h, off_part, off_u, off_dz, off_dr, off_xtiles, off_xmeta, off_dab, off_dbb, bytes;
+        off_h, off_part, off_u, off_dz, off_dr, off_xt_all, off_xt_kept, off_xmeta, off_dab, off_dbb,
+        bytes;
 };
 
 beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan *B) {
@@ -539,10 +540,11 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     B->off_u = take(4 * T * K);
     B->off_dz = take(4 * T * K);
     B->off_dr = take(4 * T * E);
-    // bf16: per-expert row tiles of the tensor-core dh product (at most one
-    // per grouping tile) and their count
-    B->off_xtiles = take(16 * size_t(P->tiles_cap));
-    B->off_xmeta = take(4);
+    // bf16: per-expert row tiles of the tensor-core GEMMs (at most one per
+    // grouping tile): every candidate expert's, the kept experts', two counts
+    B->off_xt_all = take(16 * size_t(P->tiles_cap));
+    B->off_xt_kept = take(16 * size_t(P->tiles_cap));
+    B->off_xmeta = take(8);
     // bf16: da, db rounded once more as the tensor-core dx product's operands
     B->off_dab = take(d->dtype == BEAM_BF16 ? 2 * pc * I : 0);
     B->off_dbb = take(d->dtype == BEAM_BF16 ? 2 * pc * I : 0);
@@ -620,16 +622,23 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
 
     // Forward of every candidate: a, b (fp32), H, and Y = H W2^T.
     if (d->dtype == BEAM_BF16) {
+        // Each expert's candidate rows as 128-row tiles, so that every GEMM
+        // below reads an expert's weights once (not once per 16-row tile).
+        int4 *xt_all = reinterpret_cast<int4 *>(ws + B.off_xt_all);
+        int4 *xt_kept = reinterpret_cast<int4 *>(ws + B.off_xt_kept);
+        int *xmeta = reinterpret_cast<int *>(ws + B.off_xmeta);
+        BEAM_TRY_CUDA(launch_expert_tiles(tiles, meta, counts, counts_all, kBlockM, xt_all, xt_kept,
+                                          xmeta, st));
         TcMaps maps;
         if (!make_tmap(&maps.a0, W1, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.a1, W3, d->d, (unsigned long long)d->E * d->I, kBlockM)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, kBlockM)) return BEAM_ERR_CUDA;
         maps.a2 = maps.a0;
         maps.b2 = maps.b;
         TcGemmArgs g;
         std::memset(&g, 0, sizeof(g));
-        g.meta = meta;
-        g.tiles = tiles;
+        g.meta = xmeta;  // [0]: tiles of every candidate expert
+        g.tiles = xt_all;
         g.err = err;
         g.timeout_ns = kWaitTimeoutNs;
         g.n_mb = d->I / kBlockM;
@@ -640,10 +649,10 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
         g.a_out = A;
         g.b_out = Bv;
         long long units = (long long)P.tiles_cap * g.n_mb;
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, maps, g, int(units < n_sm ? units : n_sm), st));
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, kBlockM, maps, g, int(units < n_sm ? units : n_sm), st));
         TcMaps m2;
         if (!make_tmap(&m2.a0, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&m2.b, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&m2.b, h, d->I, P.p_cap, kBlockM)) return BEAM_ERR_CUDA;
         m2.a1 = m2.a0;
         m2.a2 = m2.a0;
         m2.b2 = m2.b;
@@ -654,20 +663,16 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
         g.out = y;
         g.out_ld = d->d;
         units = (long long)P.tiles_cap * g.n_mb;
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, P.BN, m2, g, int(units < n_sm ? units : n_sm), st));
-        // dh = dy W2_e for the kept experts on the tensor cores, one pass per
-        // expert (its candidate rows as 128-row tiles), into the first split
-        // of the partials; dh_finalize then sums a single split.
-        int4 *xtiles = reinterpret_cast<int4 *>(ws + B.off_xtiles);
-        int *xmeta = reinterpret_cast<int *>(ws + B.off_xmeta);
-        BEAM_TRY_CUDA(launch_expert_tiles(tiles, meta, counts, counts_all, kBlockM, xtiles, xmeta, st));
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, kBlockM, m2, g, int(units < n_sm ? units : n_sm), st));
+        // dh = dy W2_e for the kept experts on the tensor cores, into the
+        // first split of the partials; dh_finalize then sums a single split.
         TcMaps m3;
         if (!make_tmap(&m3.a0, W2, d->I, (unsigned long long)d->E * d->d, kBlockK)) return BEAM_ERR_CUDA;
         if (!make_tmap(&m3.b, dyp, d->d, P.p_cap, kBlockM)) return BEAM_ERR_CUDA;
         m3.a1 = m3.a2 = m3.a0;
         m3.b2 = m3.b;
-        g.meta = xmeta;
-        g.tiles = xtiles;
+        g.meta = xmeta + 1;  // [1]: tiles of the kept experts
+        g.tiles = xt_kept;
         g.n_mb = d->I / kBlockM;
         g.nk = d->d / kBlockK;
         g.a_rows_per_expert = d->d;
@@ -734,8 +739,8 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
         m4.a2 = m4.a0;
         TcGemmArgs g;
         std::memset(&g, 0, sizeof(g));
-        g.meta = reinterpret_cast<int *>(ws + B.off_xmeta);
-        g.tiles = reinterpret_cast<int4 *>(ws + B.off_xtiles);
+        g.meta = reinterpret_cast<int *>(ws + B.off_xmeta) + 1;  // kept experts' tiles
+        g.tiles = reinterpret_cast<int4 *>(ws + B.off_xt_kept);
         g.err = err;
         g.timeout_ns = kWaitTimeoutNs;
         g.n_mb = d->d / kBlockM;

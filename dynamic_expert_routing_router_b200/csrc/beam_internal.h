@@ -195,13 +195,15 @@ struct BwArgs {
     float *dr;               // [T][E]
     float *dx;               // [T][d]
 };
-// Kept experts' candidate rows as tiles of at most rows_per_tile rows (one
-// block): from the grouping's tile list, each expert with a kept pair gives
-// ceil(candidates / rows_per_tile) tiles starting at its first row.  xmeta[0]
-// = how many.  Never more than the grouping's tiles when rows_per_tile >= BN.
+// Each expert's candidate rows as tiles of at most rows_per_tile rows (one
+// block): from the grouping's tile list, an expert gives
+// ceil(candidates / rows_per_tile) tiles starting at its first row.  xt_all
+// lists every candidate expert's (count in xmeta[0]); xt_kept only those of
+// experts with a kept pair (xmeta[1]).  Neither is longer than the grouping's
+// tile list when rows_per_tile >= BN.
 cudaError_t launch_expert_tiles(const int4 *tiles, const int *meta, const int *counts_kept,
-                                const int *counts_all, int rows_per_tile, int4 *xtiles,
-                                int *xmeta, cudaStream_t st);
+                                const int *counts_all, int rows_per_tile, int4 *xt_all,
+                                int4 *xt_kept, int *xmeta, cudaStream_t st);
 // phase 0: token stage, dh product (unless dh_tc), dh finalize; phase 1: dx
 // product (unless dx_tc), dx, dW1/dW3, dW2, router weights.
 cudaError_t launch_backward_stages(const BwArgs &a, int dtype, const void *x, const void *xp,
