@@ -185,6 +185,17 @@ __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
         v[2 * i + 1] = f.y;
     }
 }
+// Four consecutive elements as fp32 (8-byte aligned for bf16, 16 for fp32).
+__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+}
+__device__ __forceinline__ void load4(const float *p, float (&v)[4]) {
+    const float4 x = *reinterpret_cast<const float4 *>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
 __device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
     const float4 x = *reinterpret_cast<const float4 *>(p);
     const float4 y = *reinterpret_cast<const float4 *>(p + 4);
@@ -360,10 +371,12 @@ __global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S)
     const int nk = stage_kept_rows(a, tile.y, tile.z, s_flag, s_fw, s_row, s_w, &s_n);
     const int I = a.I;
     const long long split = (long long)a.p_cap * I;
-    for (int q = 0; q < nk; ++q) {
-        const long long row = s_row[q];
-        for (int i = threadIdx.x; i < I; i += blockDim.x) {
-            const long long o = row * I + i;
+    // Every (kept row, column) of the tile in one loop: the loads of all rows
+    // are independent.
+    for (int qi = threadIdx.x; qi < nk * I; qi += blockDim.x) {
+        const int q = qi / I, i = qi - q * I;
+        {
+            const long long o = (long long)s_row[q] * I + i;
             float c = 0.0f;
             for (int sp = 0; sp < S; ++sp) c += a.part[sp * split + o];
             const float dh = s_w[q] * c;
@@ -379,6 +392,29 @@ __global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S)
     }
 }
 
+// Exclusive prefix of v over the block's 256 threads (in thread order) and
+// the block total; s_warp holds 8 ints and is free again on return.
+__device__ __forceinline__ int block_excl_prefix(int v, int *s_warp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        before += w < warp ? s_warp[w] : 0;
+        tot += s_warp[w];
+    }
+    __syncthreads();
+    *total = tot;
+    return before + incl - v;
+}
+
 // ---------------------------------------------------------------------- dx --
 // Block per token; each thread owns 8 consecutive columns, so every term is
 // one 16-byte load and the loads of all terms are independent.  The router
@@ -387,49 +423,46 @@ __global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S)
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *Wg,
                                                     const TIn *Wm, int S) {
-    __shared__ float s_dr[kMaxE];
     __shared__ float s_c[kMaxE + kMaxK];  // coefficients
     __shared__ int s_row[kMaxE + kMaxK];  // their weight rows
     __shared__ int s_pos[kMaxK];
-    __shared__ int s_ng, s_nr, s_nk;
+    __shared__ int s_warp[8], s_nk;
     griddep_wait();
     griddep_launch_dependents();
     const int K = a.K, E = a.E, d = a.d;
     const long long split = (long long)a.p_cap * d;
     for (int t = blockIdx.x; t < a.T; t += gridDim.x) {
-        for (int e = threadIdx.x; e < E; e += blockDim.x) s_dr[e] = a.dr[(long long)t * E + e];
-        if (threadIdx.x < K) {
-            const long long o = (long long)t * K + threadIdx.x;
-            s_c[kMaxE + threadIdx.x] = Wm ? a.dz[o] : 0.0f;
-            s_row[kMaxE + threadIdx.x] = a.cand[o];
-            s_pos[threadIdx.x] = a.idx[o] >= 0 ? a.pair_pos[o] : -1;
+        // Router terms: the nonzero dr[t][e] in expert order (block prefix),
+        // then the K dz in slot order; kept slots' rows in slot order (warp 0).
+        int ng = 0;  // block-uniform
+        for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+            const int e = e0 + threadIdx.x;
+            const float c = e < E ? a.dr[(long long)t * E + e] : 0.0f;
+            int tot;
+            const int pos = block_excl_prefix(c != 0.0f ? 1 : 0, s_warp, &tot);
+            if (c != 0.0f) {
+                s_c[ng + pos] = c;
+                s_row[ng + pos] = e;
+            }
+            ng += tot;
+        }
+        if (threadIdx.x < 32) {
+            const int k = threadIdx.x;
+            const long long o = (long long)t * K + k;
+            const bool kept = k < K && a.idx[o] >= 0;
+            const unsigned bal = __ballot_sync(0xffffffffu, kept);
+            if (kept) s_pos[__popc(bal & ((1u << k) - 1u))] = a.pair_pos[o];
+            if (k == 0) s_nk = __popc(bal);
+            if (Wm && k < K) {
+                s_c[ng + k] = a.dz[o];
+                s_row[ng + k] = a.cand[o];
+            }
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int n = 0;
-            for (int e = 0; e < E; ++e)
-                if (s_dr[e] != 0.0f) {
-                    s_c[n] = s_dr[e];
-                    s_row[n] = e;
-                    ++n;
-                }
-            s_ng = n;
-            int nk = 0;
-            for (int k = 0; k < K; ++k)
-                if (s_pos[k] >= 0) s_pos[nk++] = s_pos[k];
-            s_nk = nk;
-            if (Wm)
-                for (int k = 0; k < K; ++k) {  // n <= E, so the dz block moves down
-                    s_c[n] = s_c[kMaxE + k];
-                    s_row[n] = s_row[kMaxE + k];
-                    ++n;
-                }
-            s_nr = n;
-        }
-        __syncthreads();
-        const int ng = s_ng, nr = s_nr, nk = s_nk;
+        const int nr = ng + (Wm ? K : 0), nk = s_nk;
         for (int j = threadIdx.x * 8; j < d; j += blockDim.x * 8) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
             for (int q = 0; q < nk; ++q) {  // expert part: kept slots in order, splits in order
                 float c[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int sp = 0; sp < S; ++sp) {
@@ -456,6 +489,7 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const BwArgs a, const TIn *W
         __syncthreads();
     }
 }
+
 
 // -------------------------------------------------------- weight gradients --
 // Kept rows of expert e (rows [first, first + n) of the candidate grouping),
@@ -631,45 +665,48 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
 }
 
 // dW_gate[e] += sum_t dr[t][e] x_t (tokens ascending); dW_mask[e] += sum over
-// the candidate rows of e (token order) dz x.  Block (expert, 256 columns):
-// 64 threads x 4 columns; coefficients are staged in shared memory.
-constexpr int kDrChunk = 512;
-__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4]) {
-    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
-    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
-}
-__device__ __forceinline__ void load4(const float *p, float (&v)[4]) {
-    const float4 x = *reinterpret_cast<const float4 *>(p);
-    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-}
+// the candidate rows of e (token order) dz x.  Block (expert, 1024 columns):
+// 256 threads x 4 columns.  Each round of 256 tokens first lists the nonzero
+// dr[t][e] in token order (with renorm only the tokens that have e as a
+// candidate), so the sums run without branches and keep four row loads in
+// flight; zero terms add nothing, so the order of the others is unchanged.
+constexpr int kDrChunk = 256;
+constexpr int kDrCols = 1024;
 template <typename TIn>
-__global__ void __launch_bounds__(64) bw_drouter_kernel(const BwArgs a, const TIn *x,
-                                                        const TIn *xp, float *dWg, float *dWm) {
-    __shared__ int s_first;
+__global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const TIn *x,
+                                                         const TIn *xp, float *dWg, float *dWm) {
+    __shared__ int s_first, s_warp[8];
     __shared__ float s_c[kDrChunk];
     __shared__ int s_r[kDrChunk];
     griddep_wait();
     griddep_launch_dependents();
     const int e = blockIdx.x;
-    const int j = blockIdx.y * 256 + threadIdx.x * 4;
+    const int j = blockIdx.y * kDrCols + threadIdx.x * 4;
     const bool active = j < a.d;
     const int d = a.d, E = a.E;
+    if (active) {
+        prefetch_l2(dWg + (long long)e * d + j);
+        if (dWm) prefetch_l2(dWm + (long long)e * d + j);
+    }
     float gg[4] = {0.f, 0.f, 0.f, 0.f}, gm[4] = {0.f, 0.f, 0.f, 0.f};
     for (int t0 = 0; t0 < a.T; t0 += kDrChunk) {
-        const int cnt = min(kDrChunk, a.T - t0);
-        for (int q = threadIdx.x; q < cnt; q += blockDim.x) s_c[q] = a.dr[(long long)(t0 + q) * E + e];
+        const int t = t0 + threadIdx.x;
+        const float c = t < a.T ? a.dr[(long long)t * E + e] : 0.0f;
+        int nz;
+        const int pos = block_excl_prefix(c != 0.0f ? 1 : 0, s_warp, &nz);
+        if (c != 0.0f) {
+            s_c[pos] = c;
+            s_r[pos] = t;
+        }
         __syncthreads();
         if (active) {
-#pragma unroll 8
-            for (int q = 0; q < cnt; ++q) {
-                const float c = s_c[q];
-                if (c == 0.0f) continue;  // same branch for the whole block
+#pragma unroll 4
+            for (int q = 0; q < nz; ++q) {
                 float v[4];
-                load4(x + (long long)(t0 + q) * d + j, v);
+                load4(x + (long long)s_r[q] * d + j, v);
+                const float cq = s_c[q];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) gg[i] = fmaf(c, v[i], gg[i]);
+                for (int i = 0; i < 4; ++i) gg[i] = fmaf(cq, v[i], gg[i]);
             }
         }
         __syncthreads();
@@ -686,7 +723,7 @@ __global__ void __launch_bounds__(64) bw_drouter_kernel(const BwArgs a, const TI
             }
             __syncthreads();
             if (active) {
-#pragma unroll 8
+#pragma unroll 4
                 for (int q = 0; q < cnt; ++q) {
                     float v[4];
                     load4(xp + (long long)s_r[q] * d + j, v);
@@ -734,28 +771,6 @@ cudaError_t launch_rowgemm(const BwArgs &a, const TA *A, const TA *A2, const TB 
 }
 
 namespace {
-// Exclusive prefix of v over the block's 256 threads (in thread order) and
-// the block total; s_warp holds 8 ints and is free again on return.
-__device__ __forceinline__ int block_excl_prefix(int v, int *s_warp, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += u;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    int before = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        before += w < warp ? s_warp[w] : 0;
-        tot += s_warp[w];
-    }
-    __syncthreads();
-    *total = tot;
-    return before + incl - v;
-}
 
 // One block of 256 threads walks the grouping's tiles in order.  The first
 // tile of each expert emits that expert's row tiles into list 0 (every
@@ -836,8 +851,8 @@ cudaError_t backward_stages(const BwArgs &a, const T *x, const T *xp, const T *d
         return e;
     if ((e = launch_pdl(bw_dw2_kernel<T>, dim3(a.E, (a.d + 7) / 8), dim3(256), 0, st, a, dyp, dW2)))
         return e;
-    return launch_pdl(bw_drouter_kernel<T>, dim3(a.E, (a.d + 255) / 256), dim3(64), 0, st, a, x, xp,
-                      dWg, dWm);
+    return launch_pdl(bw_drouter_kernel<T>, dim3(a.E, (a.d + kDrCols - 1) / kDrCols), dim3(256), 0,
+                      st, a, x, xp, dWg, dWm);
 }
 }  // namespace
 
