@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(256) bw_token_kernel(const BwArgs a, const TIn
         float acc[kMaxK];
 #pragma unroll
         for (int k = 0; k < kMaxK; ++k) acc[k] = 0.0f;
+#pragma unroll 4
         for (int j = tid; j < d; j += blockDim.x) {
             const float g = load_f(dy, (long long)t * d + j);
 #pragma unroll
