@@ -117,6 +117,34 @@ def test_bf16_decode_backward_matches_oracle(T, f, renorm):
         assert torch.equal(g2[k], 2 * v), k
 
 
+def test_bf16_backward_hot_expert_spans_several_row_tiles():
+    """An expert that is the top candidate of all T = 300 tokens and kept for
+    nearly all of them: its candidate (and kept) rows span three 128-row tiles
+    of the tensor-core GEMMs and two 256-row chunks of the weight-gradient
+    kernels, paths a decode batch of 128 tokens never reaches."""
+    T, hot = 300, 3
+    sh = inputs.Shape(256, 16, 4, 256, 1, "bf16")
+    x = inputs.make_tokens(sh, T, seed=31, device=DEV)  # last feature = 1
+    Wg = inputs.make_gate(sh, seed=4, device=DEV)
+    Wm = inputs.make_mask(sh, 0.35, seed=4, device=DEV)
+    Wg[hot, sh.d - 1] = 6.0  # a candidate of every token
+    Wm[hot, sh.d - 1] = 3.0  # and kept unless x . W_mask[hot] < -3
+    W1, W3, W2 = inputs.make_experts(sh, seed=4, device=DEV)
+    dy = inputs.make_upstream_grad(sh, T, seed=9, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm)
+    beta = 0.01
+    g, _ = gpu_backward(dsc, x, Wg, Wm, W1, W3, W2, dy, beta)
+    rt = gpu_route(dsc, x, Wg, Wm)
+    kept = np.bincount(rt["idx"][rt["idx"] >= 0], minlength=sh.E)
+    assert kept[hot] > 2 * 128, kept[hot]
+    touched = np.flatnonzero(kept)
+    sel = sorted({hot, int(touched[0]), int(touched[-1])})
+    ref = oracle.backward(host(x), host(Wg), host(Wm), host(W1), host(W3), host(W2), host(dy),
+                          sh.K, sh.renorm, "bf16", beta=beta, experts=sel, logits=rt["logits"])
+    _compare(g, ref, torch.as_tensor(sel, device=DEV), 1e-2, 1e-3)
+    assert torch.count_nonzero(g["dW2"][hot]) > 0
+
+
 def test_bf16_backward_without_mask_and_repeatable():
     T = 16
     sh = inputs.QWEN3
