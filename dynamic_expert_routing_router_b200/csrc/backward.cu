@@ -19,6 +19,8 @@
 // Every sum runs in a fixed order, so the gradients are bitwise repeatable.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include <climits>
 
 #include "beam_internal.h"
@@ -669,10 +671,36 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
 // the candidate rows of e (token order) dz x.  Block (expert, 1024 columns):
 // 256 threads x 4 columns.  Each round of 256 tokens first lists the nonzero
 // dr[t][e] in token order (with renorm only the tokens that have e as a
-// candidate), so the sums run without branches and keep four row loads in
-// flight; zero terms add nothing, so the order of the others is unchanged.
+// candidate), so the sums run without branches and load eight rows at a time
+// (a popular expert has a term for nearly every token); zero terms add
+// nothing, so the order of the others is unchanged.
 constexpr int kDrChunk = 256;
 constexpr int kDrCols = 1024;
+// g[0..3] += sum over q < n (in order) c[q] * X[r[q]][j .. j+3]: the rows are
+// loaded eight at a time before their terms are added.
+template <typename TIn>
+__device__ __forceinline__ void sum_rows(const TIn *X, int d, int j, const int *r, const float *c,
+                                         int n, float (&g)[4]) {
+    int q = 0;
+    for (; q + 8 <= n; q += 8) {
+        float v[8][4];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) load4(X + (long long)r[q + b] * d + j, v[b]);
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const float cq = c[q + b];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) g[i] = fmaf(cq, v[b][i], g[i]);
+        }
+    }
+    for (; q < n; ++q) {
+        float v[4];
+        load4(X + (long long)r[q] * d + j, v);
+        const float cq = c[q];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) g[i] = fmaf(cq, v[i], g[i]);
+    }
+}
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const TIn *x,
                                                          const TIn *xp, float *dWg, float *dWm) {
@@ -700,16 +728,7 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
             s_r[pos] = t;
         }
         __syncthreads();
-        if (active) {
-#pragma unroll 4
-            for (int q = 0; q < nz; ++q) {
-                float v[4];
-                load4(x + (long long)s_r[q] * d + j, v);
-                const float cq = s_c[q];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) gg[i] = fmaf(cq, v[i], gg[i]);
-            }
-        }
+        if (active) sum_rows(x, d, j, s_r, s_c, nz, gg);
         __syncthreads();
     }
     const int n = a.counts_all[e];
@@ -723,16 +742,7 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
                 s_c[q] = a.dz[a.pair[r]];
             }
             __syncthreads();
-            if (active) {
-#pragma unroll 4
-                for (int q = 0; q < cnt; ++q) {
-                    float v[4];
-                    load4(xp + (long long)s_r[q] * d + j, v);
-                    const float c = s_c[q];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) gm[i] = fmaf(c, v[i], gm[i]);
-                }
-            }
+            if (active) sum_rows(xp, d, j, s_r, s_c, cnt, gm);
             __syncthreads();
         }
     }
@@ -838,13 +848,21 @@ cudaError_t backward_stages(const BwArgs &a, const T *x, const T *xp, const T *d
     cudaError_t e;
     if (phase == 0) {
         if ((e = launch_pdl(bw_token_kernel<T>, dim3(tb), dim3(256), 0, st, a, dy))) return e;
-        if (!a.dh_tc && (e = launch_rowgemm<TG_DH, T, T>(a, dyp, dyp, W2, W2, a.d, a.I, st)))
-            return e;
+        if constexpr (std::is_same<T, float>::value) {
+            if (!a.dh_tc && (e = launch_rowgemm<TG_DH, T, T>(a, dyp, dyp, W2, W2, a.d, a.I, st)))
+                return e;
+        } else if (!a.dh_tc) {
+            return cudaErrorInvalidValue;  // bf16 runs dy W2_e on the tensor cores
+        }
         return launch_pdl(dh_finalize_kernel, dim3(a.tiles_cap), dim3(256), 0, st, a,
                           a.dh_tc ? 1 : a.S);
     }
-    if (!a.dx_tc && (e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, W1, W3, a.I, a.d, st)))
-        return e;
+    if constexpr (std::is_same<T, float>::value) {
+        if (!a.dx_tc && (e = launch_rowgemm<TG_DX, float, T>(a, a.da, a.db, W1, W3, a.I, a.d, st)))
+            return e;
+    } else if (!a.dx_tc) {
+        return cudaErrorInvalidValue;  // bf16 runs da W1_e + db W3_e on the tensor cores
+    }
     if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a, Wg, Wm, a.dx_tc ? 1 : a.S)))
         return e;
     if ((e = launch_pdl(bw_dw13_kernel<T>, dim3(a.E, (a.I + 3) / 4), dim3(256), 0, st, a, xp, dW1,
