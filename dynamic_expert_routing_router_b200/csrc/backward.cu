@@ -1,4 +1,7 @@
-// backward.cu -- CUDA-core stages of the training-mode backward pass.
+// backward.cu -- CUDA-core stages of the training-mode backward pass (the bf16
+// layer runs its two kept-row products, dh and dxp, on the tensor cores:
+// MODE_GEMM2T and MODE_GEMM1T in tc_gemm.cu, over the per-expert row tiles
+// listed here; the fp32 layer runs them with rowgemm_kernel below).
 //
 // Objective (news article on BEAM, §4, readings in the C ABI header):
 //   L = sum_t <dy_t, y_t> + beta * sum_t sum_k sigmoid(z_{t,c_k}),

@@ -529,9 +529,10 @@ beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan
     B->off_da = take(4 * pc * I);
     B->off_db = take(4 * pc * I);
     B->off_h = take(4 * pc * I);
-    // Thin decode tiles leave most SMs idle with one block per tile: split the
-    // reduction of the kept-row products eight ways (d and I are multiples of 8).
-    B->S = P->BN < 128 ? 8 : 1;
+    // fp32 runs the kept-row products on CUDA cores, one block per tile: at
+    // thin decode tiles split their reduction eight ways (d and I are
+    // multiples of 8).  bf16 runs them on the tensor cores: one split.
+    B->S = (d->dtype != BEAM_BF16 && P->BN < 128) ? 8 : 1;
     // fp32: the CUDA-core kept-row products hold a split's A rows in shared
     // memory (bf16 runs both products on the tensor cores).
     if (d->dtype != BEAM_BF16 && (dd / B->S > 7168 || I / B->S > 4096))
@@ -828,10 +829,9 @@ int beam_moe_backward_kernel_count(const beam_moe_desc *desc) {
     beam_moe_plan_info P;
     BwdPlan B;
     if (make_bwd_plan(desc, &P, &B) != BEAM_OK || desc->T == 0) return 0;
-    // router, top-K, grouping, dy gather, gate/up, down, then the eight
-    // CUDA-core stages (token, dh product, dh finalize, dx product, dx,
-    // dW1/dW3, dW2, router weights); bf16 runs the dh product on the tensor
-    // cores after building its expert tiles (one launch more).
+    // Both: router, top-K, grouping, dy gather, gate/up, down, token, dh
+    // product, dh finalize, dx product, dx, dW1/dW3, dW2, router weights (14).
+    // bf16 also lists the per-expert row tiles its tensor-core GEMMs run over.
     return desc->dtype == BEAM_BF16 ? 15 : 14;
 }
 
