@@ -139,6 +139,19 @@ def test_shared_expert_descriptor_rules():
     assert L.beam_moe_forward(ctypes.byref(ok), *ptrs, ctypes.c_size_t(1 << 40), None) == 1
 
 
+def test_backward_split_limit_applies_to_fp32_only():
+    """The CUDA-core kept-row products (fp32) hold a split of their A rows in
+    shared memory, so an fp32 layer with d > 7168 at 128-token tiles has no
+    backward; the bf16 layer runs them on the tensor cores and has one."""
+    big_bf16 = abi.desc(1024, 8192, 8, 256, 2, "bf16", 1)
+    big_f32 = abi.desc(1024, 8192, 8, 256, 2, "f32", 1)
+    assert abi.plan(big_bf16)["BN"] == 128 and abi.workspace_size(big_f32) > 0
+    assert abi.backward_workspace_size(big_bf16) > abi.workspace_size(big_bf16)
+    assert abi.backward_kernel_count(big_bf16) == 15
+    assert abi.backward_workspace_size(big_f32) == 0
+    assert abi.backward_kernel_count(big_f32) == 0
+
+
 def test_backward_descriptor_and_argument_checks():
     dsc = abi.desc(8, 2048, 128, 768, 8, "bf16", 1)
     assert abi.backward_workspace_size(dsc) > abi.workspace_size(dsc)
