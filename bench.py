@@ -34,6 +34,38 @@ import sys
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+
+# ncu records of DRAM traffic per launch of a dominant kernel (key=value text
+# under profiles/): reported only for the same kernel and workload, and only
+# while the sources that define the kernel hash to the recorded value.
+TRAFFIC_RECORDS = ["profiles/experts_fused_decode_T128_kept15.traffic.txt"]
+
+
+def recorded_traffic(kernel: str, T: int, kept: float):
+    """(bytes per launch, source) from a matching ncu record, else (None, why)."""
+    import hashlib
+    why = "no ncu record of this kernel and workload"
+    for rel in TRAFFIC_RECORDS:
+        path = os.path.join(ROOT, rel)
+        if not os.path.exists(path):
+            continue
+        rec = {}
+        for line in open(path):
+            line = line.strip()
+            if line and not line.startswith("#") and "=" in line:
+                k, v = line.split("=", 1)
+                rec[k.strip()] = v.strip()
+        if rec.get("kernel") != kernel or int(rec.get("T", -1)) != T or \
+                abs(float(rec.get("kept", -1)) - kept) > 1e-9:
+            continue
+        h = hashlib.sha256()
+        for f in rec["kernel_sources"].split():
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != rec["kernel_sources_sha256"]:
+            return None, "kernel sources changed since the ncu record (" + rel + ")"
+        return float(rec["dram_bytes_per_launch"]), rel
+    return None, why
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
@@ -681,8 +713,13 @@ def run_beam(args):
         achieved, peak, unit, bound = a_flops / t_dom / 1e12, pk["bf16"], "TFLOP/s", "tensor"
     else:
         achieved, peak, unit, bound = a_bytes / t_dom / 1e9, pk["hbm"], "GB/s", "hbm"
+    try:
+        traffic, traffic_source = recorded_traffic(names[dom], T, f_head)
+    except (OSError, ValueError, KeyError) as exc:  # a reporting field: never fail the run
+        traffic, traffic_source = None, f"ncu record unreadable: {exc}"
     roofline = dict(kernel=names[dom], bound=bound, achieved=achieved, peak=peak, unit=unit,
-                    frac=achieved / peak, traffic=None, peak_source=pk["source"],
+                    frac=achieved / peak, traffic=traffic, traffic_source=traffic_source,
+                    peak_source=pk["source"],
                     us_per_launch=t_dom * 1e6,
                     algorithmic_bytes_per_launch=a_bytes, algorithmic_flops_per_launch=a_flops)
     t_roof = sum(layer_roofline_seconds(layer, st[i % N_BATCHES], True, pk)
