@@ -81,6 +81,12 @@ def lib():
         L.beam_moe_backward.restype = i32
         L.beam_moe_backward_kernel_count.argtypes = [pd]
         L.beam_moe_backward_kernel_count.restype = i32
+        L.beam_moe_route_noalloc_check.argtypes = [vp]
+        L.beam_moe_route_noalloc_check.restype = i32
+        L.beam_moe_tau_to_logit.argtypes = [ctypes.c_float]
+        L.beam_moe_tau_to_logit.restype = ctypes.c_float
+        L.beam_moe_set_fault_injection.argtypes = [i32, ctypes.c_ulonglong]
+        L.beam_moe_set_fault_injection.restype = i32
         L.beam_status_str.argtypes = [i32]
         L.beam_status_str.restype = ctypes.c_char_p
         L.beam_moe_stage_name.argtypes = [i32]
@@ -93,10 +99,8 @@ def lib():
 
 
 def tau_logit(tau: float) -> float:
-    """The descriptor's mask threshold for sigmoid(z) >= tau, as stored (fp32)."""
-    import math
-    import numpy as np
-    return float(np.float32(math.log(tau / (1.0 - tau))))
+    """The descriptor's mask threshold for sigmoid(z) >= tau (beam_moe_tau_to_logit)."""
+    return float(lib().beam_moe_tau_to_logit(ctypes.c_float(tau)))
 
 
 def desc(T, d, E, I, K, dtype="bf16", renorm=1, tau=0.5, n_shared=0, I_shared=0) -> Desc:
@@ -104,7 +108,7 @@ def desc(T, d, E, I, K, dtype="bf16", renorm=1, tau=0.5, n_shared=0, I_shared=0)
     n_shared always-on shared experts of width I_shared."""
     code = dtype if isinstance(dtype, int) else (BEAM_BF16 if dtype == "bf16" else BEAM_F32)
     return Desc(int(T), int(d), int(E), int(I), int(K), int(code), int(renorm),
-                tau_logit(tau) if tau != 0.5 else 0.0, int(n_shared), int(I_shared))
+                tau_logit(tau), int(n_shared), int(I_shared))
 
 
 def _ptr(t):
@@ -213,6 +217,21 @@ def route_noalloc(dsc, x, W_gate, W_mask, topk_idx, topk_w, counts, hist=None, l
                                      _ptr(logits), _stream(stream)), "beam_moe_route_noalloc")
 
 
+def route_noalloc_check(stream=None):
+    """Synchronise and read the error word of the last route_noalloc call."""
+    _ok(lib().beam_moe_route_noalloc_check(_stream(stream)), "beam_moe_route_noalloc_check")
+
+
+FAULT_NONE, FAULT_EXPERT_STAGE, FAULT_ROUTER_STAGE = 0, 1, 2
+
+
+def set_fault_injection(mode: int, wait_limit_ns: int = 0):
+    """Testing aid (beam_moe_set_fault_injection): make a bounded device wait
+    expire in later calls; mode 0 and wait_limit_ns 0 restore the defaults."""
+    _ok(lib().beam_moe_set_fault_injection(int(mode), int(wait_limit_ns)),
+        "beam_moe_set_fault_injection")
+
+
 def forward(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, stream=None):
     _ok(lib().beam_moe_forward(ctypes.byref(dsc), _ptr(x), _ptr(W_gate), _ptr(W_mask),
                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out), _ptr(workspace),
@@ -269,5 +288,7 @@ def workspace_views(dsc, workspace) -> dict:
         xp=view(P["off_xp"], P["p_cap"] * dsc.d, dt, es).view(P["p_cap"], dsc.d),
         h=view(P["off_h"], P["p_cap"] * dsc.I, dt, es).view(P["p_cap"], dsc.I),
         y=view(P["off_y"], P["p_cap"] * dsc.d, torch.float32, 4).view(P["p_cap"], dsc.d),
+        ys=view(P["off_ys"], dsc.n_shared * T * dsc.d, torch.float32, 4).view(
+            dsc.n_shared * T, dsc.d),
         plan=P,
     )

@@ -23,6 +23,16 @@ namespace {
 constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s per bounded wait
 constexpr int kMaxDevices = 64;
 
+// Test hooks (beam_moe_set_fault_injection): off unless a test sets them.
+std::atomic<int> g_fault{FAULT_NONE};
+std::atomic<unsigned long long> g_wait_limit_ns{0};
+
+unsigned long long wait_limit_ns() {
+    const unsigned long long v = g_wait_limit_ns.load(std::memory_order_relaxed);
+    return v ? v : kWaitTimeoutNs;
+}
+int fault_mode() { return g_fault.load(std::memory_order_relaxed); }
+
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -249,8 +259,10 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
                          const void *Wg, const void *Wm, const RouteOut &ro, char *ws,
                          cudaStream_t st, const Recorder &rec, int n_sm) {
     float *partial = reinterpret_cast<float *>(ws + P.off_partial);
-    int *hdr = reinterpret_cast<int *>(ws);  // err + meta (8 ints)
-    ZeroRegion zero[3] = {{hdr, 8}, {ro.counts, d->E}, {ro.hist, ro.hist ? d->K + 1 : 0}};
+    // The router clears meta, counts and the histogram for the later kernels,
+    // never the error words (see kRouterTimeoutTag).
+    int *hdr = reinterpret_cast<int *>(ws);
+    ZeroRegion zero[3] = {{hdr + kHdrMeta, 4}, {ro.counts, d->E}, {ro.hist, ro.hist ? d->K + 1 : 0}};
     BEAM_TRY_CUDA(rec.rec(0));
     if (d->dtype == BEAM_BF16) {
         TcMaps maps;
@@ -272,11 +284,13 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
         a.out = partial;
         a.out_ld = 2LL * d->E;
         a.out_split_stride = (long long)d->T * 2 * d->E;
-        a.err = hdr;
+        a.err = hdr + kHdrErrRouter;
+        a.err_code = kRouterTimeoutTag;
+        a.fault_skip = fault_mode() == FAULT_ROUTER_STAGE;
         a.zero[0] = zero[0];
         a.zero[1] = zero[1];
         a.zero[2] = zero[2];
-        a.timeout_ns = kWaitTimeoutNs;
+        a.timeout_ns = wait_limit_ns();
         const int grid = a.n_units < n_sm ? a.n_units : n_sm;
         BEAM_TRY_CUDA(launch_tc_gemm(MODE_ROUTER, P.router_bn, maps, a, grid, st));
     } else {
@@ -294,6 +308,7 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
     t.renorm = d->renorm_topk;
     t.has_mask = Wm != nullptr;
     t.thr = d->mask_logit_threshold;
+    t.hdr = hdr;
     t.logits = ro.logits;
     t.idx = ro.idx;
     t.w = ro.w;
@@ -396,7 +411,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         g.meta = meta;
         g.tiles = tiles;
         g.err = err;
-        g.timeout_ns = kWaitTimeoutNs;
+        g.timeout_ns = wait_limit_ns();
         g.n_mb = d->I / int(wbox);
         g.nk = d->d / kBlockK;
         g.a_rows_per_expert = d->I;
@@ -404,6 +419,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         g.out_ld = d->I;
 
         BEAM_TRY_CUDA(rec.rec(4));
+        g.fault_skip = fault_mode() == FAULT_EXPERT_STAGE;  // tests only
         if (fused) {
             g.n_mb2 = d->d / kBlockM;
             g.nk2 = d->I / kBlockK;
@@ -421,6 +437,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
             BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, maps, g,
                                          int(units < n_sm ? units : n_sm), st));
             BEAM_TRY_CUDA(rec.rec(5));
+            g.fault_skip = 0;
             TcMaps m2 = maps;
             m2.a0 = maps.a2;
             m2.a1 = maps.a2;
@@ -468,7 +485,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         TcGemmArgs g;
         std::memset(&g, 0, sizeof(g));
         g.err = err;
-        g.timeout_ns = kWaitTimeoutNs;
+        g.timeout_ns = wait_limit_ns();
         g.dense = 1;
         g.dense_ntt = ntt;
         g.dense_T = d->T;
@@ -641,7 +658,7 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
         g.meta = xmeta;  // [0]: tiles of every candidate expert
         g.tiles = xt_all;
         g.err = err;
-        g.timeout_ns = kWaitTimeoutNs;
+        g.timeout_ns = wait_limit_ns();
         g.n_mb = d->I / kBlockM;
         g.nk = d->d / kBlockK;
         g.a_rows_per_expert = d->I;
@@ -743,7 +760,7 @@ beam_status backward_impl(const beam_moe_desc *d, const void *x, const void *Wg,
         g.meta = reinterpret_cast<int *>(ws + B.off_xmeta) + 1;  // kept experts' tiles
         g.tiles = reinterpret_cast<int4 *>(ws + B.off_xt_kept);
         g.err = err;
-        g.timeout_ns = kWaitTimeoutNs;
+        g.timeout_ns = wait_limit_ns();
         g.n_mb = d->d / kBlockM;
         g.nk = 2 * (d->I / kBlockK);
         g.a_rows_per_expert = d->I;
@@ -917,6 +934,23 @@ beam_status beam_moe_check(const beam_moe_desc *desc, void *workspace, void *str
         return BEAM_ERR_CUDA;
     if (err == DEV_ERR_TIMEOUT) return BEAM_ERR_TIMEOUT;
     if (err != 0) return BEAM_ERR_INTERNAL;
+    return BEAM_OK;
+}
+
+float beam_moe_tau_to_logit(float tau) {
+    if (!(tau >= 0.0f && tau <= 1.0f)) return NAN;  // NaN and values outside [0, 1]
+    // ln(tau / (1 - tau)) in double, rounded once to the descriptor's float;
+    // the limits tau = 0 and 1 give -inf (keep every candidate whose z is not
+    // NaN) and +inf (keep none).
+    const double t = double(tau);
+    return float(std::log(t / (1.0 - t)));
+}
+
+beam_status beam_moe_set_fault_injection(int mode, unsigned long long wait_limit_ns) {
+    if (mode != FAULT_NONE && mode != FAULT_EXPERT_STAGE && mode != FAULT_ROUTER_STAGE)
+        return BEAM_ERR_INVALID_ARG;
+    g_fault.store(mode, std::memory_order_relaxed);
+    g_wait_limit_ns.store(wait_limit_ns, std::memory_order_relaxed);
     return BEAM_OK;
 }
 

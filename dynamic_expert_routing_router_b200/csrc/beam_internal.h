@@ -15,6 +15,20 @@ namespace beam {
 // Device error word values (workspace `err`).
 enum : int { DEV_OK = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_INTERNAL = 2 };
 
+// The router kernel never writes the error word itself: its CTAs would race
+// with the clear that starts a call.  A router CTA whose bounded wait expires
+// writes this tag into the header's second word instead; the top-K kernel,
+// which runs after the whole router grid, folds it into the error word (and
+// resets it), so the word it leaves is exactly this call's router status.  A
+// tag, not a small code, so that a fresh workspace's leftover bytes are not
+// taken for a timeout.
+constexpr int kRouterTimeoutTag = 0x5EA71AB5;
+constexpr int kHdrErr = 0, kHdrErrRouter = 1, kHdrMeta = 4;  // int offsets in the header
+
+// Fault injection for tests (beam_moe_set_fault_injection): which launch skips
+// one stage load in CTA 0 so that its MMA issuer's bounded wait expires.
+enum : int { FAULT_NONE = 0, FAULT_EXPERT_STAGE = 1, FAULT_ROUTER_STAGE = 2 };
+
 // Roles of the tensor-core GEMM kernel.
 enum TcMode : int {
     MODE_ROUTER = 0,  // logits: [W_gate | W_mask] rows x token rows, split over d
@@ -97,7 +111,9 @@ struct TcGemmArgs {
     void *out;           // router: f32 partial [S][T][2E]; GEMM1: H (bf16); GEMM2: Y (f32)
     long long out_ld;    // elements per output row
     long long out_split_stride;  // router: elements per split slab
-    int *err;            // device error word
+    int *err;            // device error word (router: the header's router word)
+    int err_code;        // value written on a wait expiry (0 = DEV_ERR_TIMEOUT)
+    int fault_skip;      // 1: CTA 0 skips the first stage load of its first unit (tests)
     ZeroRegion zero[3];  // router: regions CTA 0 clears for the later kernels
     unsigned long long timeout_ns;
     // MODE_EXPERTS: the down projection that follows the gate/up units
@@ -121,6 +137,7 @@ struct TopkArgs {
     const float *partial;  // [S][T][2E]
     int S, T, E, K, renorm, has_mask;
     float thr;             // keep iff z >= thr (logit of the threshold tau)
+    int *hdr;              // workspace header: block 0 sets err from the router word
     float *logits;         // [T][2E] or NULL
     int *idx;              // [T][K]
     float *w;              // [T][K]

@@ -2,13 +2,13 @@
 // that cannot allocate device memory, with its scratch in a fixed device
 // array that this file owns.
 //
-// Who cannot allocate: code that runs while a stream is being captured into
-// a CUDA graph in the global or thread-local capture mode, where cudaMalloc
-// is an illegal call that invalidates the capture; and plugins embedded in a
-// host runtime whose memory pool owns the device memory and does not let its
-// extensions allocate on their own.  Such callers still own their inputs and
-// outputs; only the library's scratch (the router's split-K partial logits
-// and the error/counter header) moves into the array below.
+// Who cannot allocate: plugins embedded in a host runtime whose memory pool
+// owns all of the device's memory and gives its extensions none of their own
+// (a serving engine that reserves the GPU up front, for example), and callers
+// working inside a fixed memory budget where any allocation may fail or
+// fragment the pool.  Such callers still own their inputs and outputs; only
+// the library's scratch (the router's split-K partial logits and the
+// error/counter header) moves into the array below.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -64,4 +64,18 @@ extern "C" beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const v
     return beam::route_into_scratch(desc, x, W_gate, W_mask, topk_idx, topk_w, expert_counts,
                                     kept_hist, logits, scratch, kScratchBytes,
                                     static_cast<cudaStream_t>(stream));
+}
+
+extern "C" beam_status beam_moe_route_noalloc_check(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BEAM_ERR_CUDA;
+    void *scratch = nullptr;
+    beam_status s = scratch_for_current_device(&scratch);
+    if (s != BEAM_OK) return s;
+    int err = 0;  // the header's error word (offset 0 of the scratch)
+    if (cudaMemcpy(&err, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return BEAM_ERR_CUDA;
+    if (err == beam::DEV_ERR_TIMEOUT) return BEAM_ERR_TIMEOUT;
+    if (err != beam::DEV_OK) return BEAM_ERR_INTERNAL;
+    return BEAM_OK;
 }

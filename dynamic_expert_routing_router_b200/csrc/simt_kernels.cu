@@ -44,6 +44,13 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
     __syncthreads();
     griddep_wait();
     griddep_launch_dependents();
+    if (a.hdr && blockIdx.x == 0 && threadIdx.x == 0) {
+        // The whole router grid has finished: this call's error word starts
+        // from the router's status, and the router word is reset.
+        const int rs = a.hdr[kHdrErrRouter];
+        a.hdr[kHdrErr] = rs == kRouterTimeoutTag ? DEV_ERR_TIMEOUT : DEV_OK;
+        a.hdr[kHdrErrRouter] = 0;
+    }
 
     const int warp = threadIdx.x >> 5;
     const int E2 = 2 * a.E;

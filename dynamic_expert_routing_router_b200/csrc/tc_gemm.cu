@@ -159,8 +159,10 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs
     return w;
 }
 
-__device__ __forceinline__ void signal_abort(int *err, int *abort_flag) {
-    atomicExch(err, DEV_ERR_TIMEOUT);
+// A bounded wait expired: record it (DEV_ERR_TIMEOUT, or the router's tag)
+// and tell the CTA's other roles to stop.
+__device__ __forceinline__ void signal_abort(const TcGemmArgs &p, int *abort_flag) {
+    atomicExch(p.err, p.err_code ? p.err_code : int(DEV_ERR_TIMEOUT));
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
 }
 
@@ -313,6 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (p.fault_skip && blockIdx.x == 0 && lu == 0 && kb == 0)
+                        continue;  // test hook: this stage never fills (its MMA wait expires)
                     uint8_t *st = smem + size_t(s) * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
                     int kx = (w.kb0 + kb) * kBlockK;
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
             }
             if (!ok) {
-                signal_abort(p.err, &abort_sh);
+                signal_abort(p, &abort_sh);
                 // Let this CTA's own copies land before it can exit.
                 for (uint32_t j = (it > uint32_t(STAGES) ? it - STAGES : 0u); j < it; ++j)
                     mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1u, nullptr,
@@ -408,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&tfull_bar[a]);  // accumulator complete
             }
             if (!ok) {
-                signal_abort(p.err, &abort_sh);
+                signal_abort(p, &abort_sh);
                 umma_commit(&drain_bar);  // wait for the MMAs already issued
                 mbar_wait_bounded(&drain_bar, 0u, nullptr, p.timeout_ns);
             }
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 epilogue_sync();
                 const int v0 = uvote[0], v1 = uvote[1], v2 = uvote[2], v3 = uvote[3];
                 if (!(v0 && v1 && v2 && v3)) {
-                    if (lane == 0) signal_abort(p.err, &abort_sh);
+                    if (lane == 0) signal_abort(p, &abort_sh);
                     break;
                 }
                 if (v0 == 2 || v1 == 2 || v2 == 2 || v3 == 2) break;
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = xvote[0] && xvote[1] && xvote[2] && xvote[3];
             }
             if (!ok) {
-                if (lane == 0) signal_abort(p.err, &abort_sh);
+                if (lane == 0) signal_abort(p, &abort_sh);
                 break;
             }
             tc_fence_after_sync();

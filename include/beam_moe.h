@@ -71,7 +71,8 @@ typedef enum { BEAM_BF16 = 0, BEAM_F32 = 1 } beam_dtype;
  *   pre-activation z >= mask_logit_threshold (i.e. sigmoid(z) >= tau).
  *   0 is the paper's tau = 0.5, so a zero-initialised descriptor keeps the
  *   method's default; other values reproduce the threshold ablation (news
- *   article on BEAM, §8).  Must not be NaN.
+ *   article on BEAM, §8); beam_moe_tau_to_logit converts a tau.  Must not
+ *   be NaN.
  * n_shared, I_shared: always-on shared experts (news article on BEAM, §5:
  *   models such as Qwen1.5-MoE and DeepSeek-V2-Lite keep running them for
  *   every token, all-masked tokens included), n_shared SwiGLU experts of
@@ -155,10 +156,13 @@ beam_status beam_moe_route(const beam_moe_desc *desc, const void *x, const void 
 
 /* The whole layer, Eq. (4)-(8): out [T,d] = sum of kept experts' outputs
  * weighted by g * m.  W_mask NULL runs the same kernels with the mask test
- * off (vanilla Top-K MoE).  Launches BEAM_MOE_FORWARD_STAGES kernels:
- * router GEMM, top-K + mask, grouping, row gather, gate/up GEMM + SwiGLU,
- * down GEMM, weighted combine.  No host synchronisation; capturable into a
- * CUDA graph. */
+ * off (vanilla Top-K MoE).  Launches beam_moe_forward_kernel_count(desc)
+ * kernels: with 128-row token tiles (bf16 prefill batches, and BEAM_F32) all
+ * seven stages -- router GEMM, top-K + mask, grouping, row gather, gate/up
+ * GEMM + SwiGLU, down GEMM, weighted combine; with thinner tiles (bf16 decode
+ * batches) five, because the grouping copies the token rows and both expert
+ * GEMMs run as one launch.  No host synchronisation; capturable into a CUDA
+ * graph. */
 beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const void *W_gate,
                              const void *W_mask, const void *W1, const void *W3,
                              const void *W2, void *out, void *workspace,
@@ -196,30 +200,37 @@ beam_status beam_moe_forward_profiled(const beam_moe_desc *desc, const void *x,
 /* beam_moe_route for callers that cannot allocate device memory.  The paper
  * has no counterpart: this is a service of this library.
  *
- * Who needs it: code running while a stream is captured into a CUDA graph in
- * the global or thread-local capture mode (cudaMalloc is illegal there and
- * breaks the capture), and plugins inside a runtime whose memory pool owns
- * the device memory and does not let extensions allocate.  The caller still
- * passes every input and output exactly as for beam_moe_route; the scratch
- * (router partial logits, error word, counters) lives in a file-scope device
- * array of BEAM_MOE_ROUTE_NOALLOC_SCRATCH_BYTES that every GPU loading the
- * library holds until the process exits.  Nothing here calls cudaMalloc,
- * cudaFree or any allocating routine.
+ * Who needs it: plugins inside a host runtime whose memory pool owns all of
+ * the device memory and lets its extensions allocate none (a serving engine
+ * that reserves the GPU when it starts, for example), and callers inside a
+ * fixed memory budget, where a new allocation may fail or fragment the pool.
+ * The caller still passes every input and output exactly as for
+ * beam_moe_route; the scratch (router partial logits, error words, counters)
+ * lives in a file-scope device array of BEAM_MOE_ROUTE_NOALLOC_SCRATCH_BYTES
+ * that every GPU loading the library holds until the process exits.  Nothing
+ * here calls cudaMalloc, cudaFree or any allocating routine.
  *  - Size limit: the call needs beam_moe_plan(desc)->off_idx bytes of
  *    scratch; larger batches return BEAM_ERR_WORKSPACE before any launch (for
  *    d=2048, E=128 every T up to 8192 fits).
  *  - The first call on a device looks the array's address up on that device
  *    (cudaGetSymbolAddress, with that device current); make that first call
  *    before any stream capture.
- *  - All calls share the one array: calls whose kernels may overlap on the GPU
- *    (different streams, or concurrent host threads) race on it and must be
- *    ordered by the caller.  Each call clears what must start at zero.
- *  - Same kernels and results as beam_moe_route; beam_moe_check does not
- *    apply (there is no caller workspace to read). */
+ *  - All calls share the one array, which keeps the last call's contents:
+ *    calls whose kernels may overlap on the GPU (different streams, or
+ *    concurrent host threads) race on it and must be ordered by the caller.
+ *    Each call clears what must start at zero.
+ *  - Same kernels and results as beam_moe_route.  Its device error word is in
+ *    the array: read it with beam_moe_route_noalloc_check. */
 beam_status beam_moe_route_noalloc(const beam_moe_desc *desc, const void *x,
                                    const void *W_gate, const void *W_mask, int32_t *topk_idx,
                                    float *topk_w, int32_t *expert_counts, int32_t *kept_hist,
                                    float *logits, void *stream);
+
+/* Synchronise `stream`, then read the error word of the last
+ * beam_moe_route_noalloc call on the current device: BEAM_OK, or
+ * BEAM_ERR_TIMEOUT when a bounded device wait of the router expired (its
+ * outputs are then not valid).  Allocates nothing. */
+beam_status beam_moe_route_noalloc_check(void *stream);
 
 /* Kernel launches one forward call makes for `desc`: 5 (bf16 with
  * decode-sized token tiles) or 7, plus 2 with shared experts; 0 for T = 0 or
@@ -274,8 +285,36 @@ int beam_moe_backward_kernel_count(const beam_moe_desc *desc);
 
 /* Synchronise `stream`, then read the workspace error word written by the last
  * call: BEAM_OK, BEAM_ERR_TIMEOUT (a bounded device wait expired, the kernel
- * returned early) or BEAM_ERR_INTERNAL (a device consistency check failed). */
+ * returned early; that call's outputs are not valid) or BEAM_ERR_INTERNAL (a
+ * device consistency check failed).  Every call resets the word, so it
+ * describes the last call made on the workspace.  After a timeout the
+ * workspace and the context stay usable: the next call starts clean. */
 beam_status beam_moe_check(const beam_moe_desc *desc, void *workspace, void *stream);
+
+/* The descriptor's mask_logit_threshold for a threshold tau of Eq. (6):
+ * ln(tau / (1 - tau)) evaluated in double and rounded once to float, so that
+ * a candidate is kept iff sigmoid(z) >= tau <=> z >= the returned value.
+ * tau = 0.5 gives 0 exactly; tau = 0 gives -inf, tau = 1 gives +inf; NaN for
+ * tau outside [0, 1] (which beam_moe_plan rejects). */
+float beam_moe_tau_to_logit(float tau);
+
+/* Testing aid, off by default; the paper has no counterpart.  It lets a test
+ * observe the bounded-wait path without faulting or hanging the GPU:
+ *   mode 0  off;
+ *   mode 1  in every later forward call, CTA 0 of the expert GEMM launch (the
+ *           fused expert kernel at decode tile sizes, the gate/up GEMM
+ *           otherwise; bf16 only) skips the first shared-memory stage of its
+ *           first unit: it issues neither the copy nor the transaction count,
+ *           so the MMA issuer's bounded wait on that stage expires;
+ *   mode 2  the same in CTA 0 of the router GEMM of every later route or
+ *           forward call (bf16 only).
+ * The kernels then record the timeout, let their own copies and MMAs land,
+ * free their tensor memory and return: beam_moe_check reports
+ * BEAM_ERR_TIMEOUT and the context stays usable.  wait_limit_ns replaces the
+ * 1 s limit of every bounded device wait (0 restores it).  Process-wide; set
+ * it while no other thread is calling the library.  BEAM_ERR_INVALID_ARG for
+ * an unknown mode. */
+beam_status beam_moe_set_fault_injection(int mode, unsigned long long wait_limit_ns);
 
 /* Static, NUL-terminated name of a status code. */
 const char *beam_status_str(beam_status status);

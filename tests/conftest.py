@@ -1,3 +1,4 @@
+import json
 import os
 import sys
 
@@ -20,3 +21,14 @@ def _build_libraries():
     from dynamic_expert_routing_router_b200 import build
     oracle.build()
     build.build()
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With BEAM_PARITY_REPORT=<path>, write what the parity tests observed
+    (router logit error, decision flip rate, worst value errors) as JSON."""
+    path = os.environ.get("BEAM_PARITY_REPORT")
+    mod = sys.modules.get("_parity")
+    if not path or mod is None:
+        return
+    with open(path, "w") as f:
+        json.dump(mod.REPORT, f, indent=1)

@@ -171,3 +171,28 @@ def test_backward_descriptor_and_argument_checks():
     assert call(dsc, 0.1, None) == 1            # W_mask given, dW_mask missing
     assert call(dsc, float("nan"), p[0]) == 1   # beta must be finite
     assert call(shared, 0.1, p[0]) == 2         # unsupported: shared experts
+
+
+def test_tau_to_logit_behind_the_abi():
+    """beam_moe_tau_to_logit: ln(tau / (1 - tau)) rounded once to float32; the
+    paper's tau = 0.5 is exactly 0 (sigmoid(0) = 1/2)."""
+    import math
+
+    import numpy as np
+    f = abi.lib().beam_moe_tau_to_logit
+    assert f(0.5) == 0.0
+    for tau in (0.1, 0.3, 0.7, 0.9):
+        t = float(np.float32(tau))  # the value the float argument carries
+        assert f(tau) == float(np.float32(math.log(t / (1.0 - t))))
+        assert f(tau) == -f(float(np.float32(1.0 - t))) or abs(f(tau) + f(1.0 - t)) < 1e-6
+    assert f(0.0) == -math.inf and f(1.0) == math.inf
+    for bad in (-0.1, 1.5, float("nan")):
+        assert math.isnan(f(bad))
+    assert abi.desc(4, 2048, 128, 768, 8, tau=0.3).mask_logit_threshold == f(0.3)
+
+
+def test_fault_injection_switch_checks_its_mode():
+    with pytest.raises(abi.BeamError) as ei:
+        abi.set_fault_injection(7)
+    assert ei.value.status == 1
+    abi.set_fault_injection(abi.FAULT_NONE, 0)  # the default, idempotent

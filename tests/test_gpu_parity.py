@@ -16,9 +16,11 @@ import torch
 import oracle
 from dynamic_expert_routing_router_b200 import abi, inputs
 
-from _parity import (BF16_TOL_RMS, assert_grouping_bitexact, assert_routing_bitexact,
-                     assert_values, bf16_excess, compact_experts, gpu_forward, gpu_route, host,
-                     oracle_from_logits, oracle_values)
+from _parity import (BF16_TOL_RMS, assert_combine, assert_expert_rows,
+                     assert_grouping_bitexact, assert_logits, assert_routing_bitexact,
+                     assert_token_sample, assert_values, bf16_excess, compact_experts,
+                     gpu_forward, gpu_route, host, oracle_from_logits, oracle_values,
+                     pick_experts, report, strided_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +57,7 @@ def test_tiny_f32_layer_matches_oracle():
     # GPU fp32 logits against the oracle's fp64 logits
     r, z = oracle.logits(host(L["x"]), host(L["W_gate"]), host(L["W_mask"]), "f32")
     np.testing.assert_allclose(g["logits"], np.concatenate([r, z], 1), rtol=0, atol=1e-5)
+    assert_logits(g, L["x"], L["W_gate"], L["W_mask"], "f32", sh.K, sh.renorm, name="tiny_f32")
     kept = (g["idx"] >= 0).mean()
     assert 0.35 <= kept <= 0.65, kept
     out, ws = gpu_forward(dsc, L["x"], L["W_gate"], L["W_mask"], L["W1"], L["W3"], L["W2"])
@@ -63,6 +66,8 @@ def test_tiny_f32_layer_matches_oracle():
     assert_grouping_bitexact(dsc, views, g["idx"])
     ref = oracle_values(L["x"], L["W1"], L["W3"], L["W2"], g["idx"], o["w"], "f32")
     assert_values(out, ref, g["idx"], "f32")
+    assert_combine(out, views, "f32")
+    assert_expert_rows(views, L["x"], L["W1"], L["W3"], L["W2"], "f32", range(sh.E))
 
 
 def test_tiny_f32_zero_mask_is_vanilla_topk_bitwise():
@@ -96,15 +101,19 @@ def test_qwen3_decode_matches_oracle(T, f, qwen3_experts, qwen3_experts_host):
     g = gpu_route(dsc, x, Wg, Wm)
     o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
     assert_routing_bitexact(g, o)
+    assert_logits(g, x, Wg, Wm, "bf16", sh.K, sh.renorm, name=f"decode_T{T}_f{f}")
     out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
     views = abi.workspace_views(dsc, ws)
     assert np.array_equal(views["idx"].cpu().numpy(), g["idx"])
     assert np.array_equal(views["w"].cpu().numpy(), g["w"])
     assert_grouping_bitexact(dsc, views, g["idx"])
-    n = min(T, 32)
     h1, h3, h2 = qwen3_experts_host
-    ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16", 0, n)
-    assert_values(out, ref, g["idx"], "bf16", rows=slice(0, n))
+    ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16")  # every token
+    worst = assert_values(out, ref, g["idx"], "bf16")
+    assert_combine(out, views, "bf16")
+    nrow, wrow = assert_expert_rows(views, x, W1, W3, W2, "bf16", pick_experts(g["counts"]))
+    report(name=f"decode_T{T}_f{f}", kind="values", tokens=T, worst_token_excess=worst,
+           expert_rows=nrow, worst_expert_row=wrow)
     if f >= 1.0:
         assert (g["idx"] >= 0).all()
 
@@ -135,10 +144,18 @@ def test_qwen3_prefill_matches_oracle(f, qwen3_experts, qwen3_experts_host):
     views = abi.workspace_views(dsc, ws)
     assert np.array_equal(views["idx"].cpu().numpy(), g["idx"])
     assert_grouping_bitexact(dsc, views, g["idx"])
+    assert_logits(g, x, Wg, Wm, "bf16", sh.K, sh.renorm, name=f"prefill_T{T}_f{f}")
     h1, h3, h2 = qwen3_experts_host
-    for t0 in (0, T - 40):  # first rows and the ragged end
-        ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16", t0, t0 + 40)
-        assert_values(out, ref, g["idx"], "bf16", rows=slice(t0, t0 + 40))
+    # every 32nd token plus both ends: each expert's rows are in token order,
+    # so the sample reaches the middle tiles of every expert's row range
+    rows = strided_rows(T, 32)
+    worst = assert_token_sample(out, x, h1, h3, h2, g["idx"], o["w"], "bf16", rows)
+    assert_combine(out, views, "bf16")
+    # whole experts: the hottest spans many 128-row tiles
+    nrow, wrow = assert_expert_rows(views, x, W1, W3, W2, "bf16", pick_experts(g["counts"]))
+    report(name=f"prefill_T{T}_f{f}", kind="values", tokens=len(rows),
+           worst_token_excess=worst, expert_rows=nrow, worst_expert_row=wrow,
+           hottest_expert_rows=int(g["counts"].max()))
 
 
 # ------------------------------------------------------------ invariants --
@@ -258,14 +275,17 @@ def test_mask_threshold_tau_matches_oracle(tau, qwen3_experts, qwen3_experts_hos
     g = gpu_route(dsc, x, Wg, Wm)
     o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True, tau_logit=thr)
     assert_routing_bitexact(g, o)
+    assert_logits(g, x, Wg, Wm, "bf16", sh.K, sh.renorm, tau_logit=thr, name=f"tau_{tau}")
     base = gpu_route(abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm), x, Wg, Wm)
     kept, kept05 = (g["idx"] >= 0).sum(), (base["idx"] >= 0).sum()
     assert (kept < kept05) if tau > 0.5 else (kept > kept05)
     out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
-    assert_grouping_bitexact(dsc, abi.workspace_views(dsc, ws), g["idx"])
+    views = abi.workspace_views(dsc, ws)
+    assert_grouping_bitexact(dsc, views, g["idx"])
     h1, h3, h2 = qwen3_experts_host
-    ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16", 0, 24)
-    assert_values(out, ref, g["idx"], "bf16", rows=slice(0, 24))
+    ref = oracle.experts(host(x), h1, h3, h2, g["idx"], o["w"], "bf16")  # every token
+    assert_values(out, ref, g["idx"], "bf16")
+    assert_combine(out, views, "bf16")
 
 
 # ----------------------------------------------------------- edge shapes --
@@ -294,11 +314,14 @@ def test_edge_shapes_match_oracle(name, T, d, E, I, K, renorm, f):
     g = gpu_route(dsc, x, Wg, Wm)
     o = oracle_from_logits(g["logits"], E, K, renorm, True)
     assert_routing_bitexact(g, o)
+    assert_logits(g, x, Wg, Wm, "bf16", K, renorm, name=f"edge_{name}")
     out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
     views = abi.workspace_views(dsc, ws)
     assert_grouping_bitexact(dsc, views, g["idx"])
     ref = oracle_values(x, W1, W3, W2, g["idx"], o["w"], "bf16")
     assert_values(out, ref, g["idx"], "bf16")
+    assert_combine(out, views, "bf16")
+    assert_expert_rows(views, x, W1, W3, W2, "bf16", pick_experts(g["counts"]))
 
 
 def test_empty_batch_is_a_no_op():
@@ -324,14 +347,19 @@ def test_large_layer_matches_oracle(T, f, large_layer):
     g = gpu_route(dsc, x, Wg, Wm)
     o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
     assert_routing_bitexact(g, o)
+    assert_logits(g, x, Wg, Wm, "bf16", sh.K, sh.renorm, name=f"large_T{T}_f{f}")
     out, ws = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2)
     views = abi.workspace_views(dsc, ws)
     assert_grouping_bitexact(dsc, views, g["idx"])
-    n = 6
-    c1, c3, c2, cidx = compact_experts(W1, W3, W2, g["idx"][:n])
-    xs = host(x[:n])
-    ref = oracle.experts(xs, c1, c3, c2, cidx, o["w"][:n], "bf16")
-    assert_values(out, ref, g["idx"], "bf16", rows=slice(0, n))
+    # tokens spread over the batch (oracle on the experts they use only)
+    rows = strided_rows(T, max(1, T // 4), ends=2)
+    worst = assert_token_sample(out, x, W1, W3, W2, g["idx"], o["w"], "bf16", rows,
+                                compact=True)
+    assert_combine(out, views, "bf16")
+    nrow, wrow = assert_expert_rows(views, x, W1, W3, W2, "bf16",
+                                    pick_experts(g["counts"], n_random=1), max_rows=96)
+    report(name=f"large_T{T}_f{f}", kind="values", tokens=len(rows), worst_token_excess=worst,
+           expert_rows=nrow, worst_expert_row=wrow)
 
 
 @pytest.fixture(scope="module")
@@ -365,12 +393,12 @@ def test_48_layer_decode_stack_matches_oracle():
         g = gpu_route(dsc, x, Wg, Wm)
         o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
         assert_routing_bitexact(g, o)
+        assert_logits(g, x, Wg, Wm, "bf16", sh.K, sh.renorm, name=f"stack_layer{layer}")
         out, _ = gpu_forward(dsc, x, Wg, Wm, W1, W3, W2, ws=ws)
+        assert_combine(out, abi.workspace_views(dsc, ws), "bf16")
         if layer % 8 == 7:
-            n = 4
-            c1, c3, c2, cidx = compact_experts(W1, W3, W2, g["idx"][:n])
-            ref = oracle.experts(host(x[:n]), c1, c3, c2, cidx, o["w"][:n], "bf16")
-            assert_values(out, ref, g["idx"], "bf16", rows=slice(0, n))
+            assert_token_sample(out, x, W1, W3, W2, g["idx"], o["w"], "bf16",
+                                strided_rows(T, 16, ends=1), compact=True)
         kept.append((g["idx"] >= 0).mean())
         x = inputs.stack_next_input(out, layer)
         del W1, W3, W2
@@ -403,17 +431,20 @@ def test_shared_experts_match_oracle(name, sh, S, T, f):
     g = gpu_route(dsc, x, Wg, Wm)
     o = oracle_from_logits(g["logits"], E, K, renorm, True)
     assert_routing_bitexact(g, o)
+    assert_logits(g, x, Wg, Wm, "bf16", K, renorm, name=f"shared_{name}")
     ws = abi.alloc_workspace(dsc, DEV)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
     abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, out, ws)
     abi.check(dsc, ws)
-    n = min(T, 24)
-    for t0 in sorted({0, T - n}):
-        ref = oracle.experts(host(x), host(W1), host(W3), host(W2), g["idx"], o["w"], "bf16",
-                             t0, t0 + n)
-        oracle.add_shared(ref, host(x), host(W1s), host(W3s), host(W2s), "bf16", t0, t0 + n)
-        o_rows = out.float().cpu().numpy().astype(np.float64)[t0:t0 + n]
-        assert (bf16_excess(o_rows, ref) <= BF16_TOL_RMS).all()
+    # every 16th token and both ends, end to end (routed sum + shared experts)
+    rows = strided_rows(T, 16)
+    xr = host(x[torch.as_tensor(rows, device=DEV)])
+    ref = oracle.experts(xr, host(W1), host(W3), host(W2), g["idx"][rows], o["w"][rows], "bf16")
+    oracle.add_shared(ref, xr, host(W1s), host(W3s), host(W2s), "bf16")
+    o_rows = out.float().cpu().numpy().astype(np.float64)[rows]
+    assert (bf16_excess(o_rows, ref) <= BF16_TOL_RMS).all()
+    views = abi.workspace_views(dsc, ws)
+    assert_combine(out, views, "bf16", n_shared=S, ys=views["ys"])
 
 
 def test_shared_experts_serve_all_masked_tokens():

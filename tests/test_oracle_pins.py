@@ -377,3 +377,83 @@ def test_shared_experts_run_for_every_token_with_weight_one():
     ys, _, _, _ = oracle.forward(x, Wg, Wm, W1, W3, W2, K, 1, "f32", shared=(W1s, W3s, W2s))
     assert 0 < (rt2["idx"] >= 0).sum() < T * K
     np.testing.assert_allclose(ys - yr, ref, rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------------ bf16 storage decode --
+
+def _bf16_patterns_finite():
+    """Every finite bfloat16 bit pattern (exponent field not all ones), as int16."""
+    u = np.arange(1 << 16, dtype=np.uint32)
+    finite = ((u >> 7) & 0xFF) != 0xFF
+    return u[finite].astype(np.uint16).view(np.int16)
+
+
+def _torch_bf16_to_f64(bits):
+    """Independent decode: torch's own bfloat16 -> float64 conversion."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def test_oracle_bf16_decode_of_every_finite_pattern():
+    """The oracle widens bf16 storage (raw bits) to fp64 exactly as torch does,
+    for every finite pattern, through both operands of its logits: a one-hot
+    weight row picks one input element (x_tj * 1 + zeros is exact), and a
+    one-hot input row picks one weight element.
+
+    Catches: a wrong shift, byte order or sign handling in the decode, a
+    flushed subnormal, or the two operands decoded differently."""
+    pats = _bf16_patterns_finite()
+    d = 256
+    n = -(-len(pats) // d) * d
+    flat = np.zeros(n, np.int16)
+    flat[:len(pats)] = pats
+    X = flat.reshape(-1, d)
+    one = np.int16(0x3F80)  # bf16 1.0
+    eye = np.zeros((d, d), np.int16)
+    eye[np.arange(d), np.arange(d)] = one
+    want = _torch_bf16_to_f64(X)
+    r, _ = oracle.logits(X, eye, None, "bf16")   # r[t, e] = X[t, e]
+    assert np.array_equal(r, want + 0.0)         # -0.0 sums to +0.0: compare values
+    r2, _ = oracle.logits(eye, X, None, "bf16")  # r2[t, e] = X[e, t]
+    assert np.array_equal(r2, (want + 0.0).T)
+
+
+def test_oracle_bf16_layer_matches_numpy_on_torch_decode():
+    """Logits and the expert sum on bf16 storage equal numpy fp64 arithmetic on
+    torch's decode of the same bits: the logits bit for bit (sequential sums
+    of exact products, written as a cumulative sum in the same order), the
+    SwiGLU experts to 1e-12.
+
+    Catches: the bf16 path reading a wrong stride or operand, or mixing the
+    decode of x and of the weights."""
+    import torch
+    rng = np.random.default_rng(7)
+    T, d, E, I, K = 9, 64, 6, 48, 3
+    def b16(a):
+        return torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).view(
+            torch.int16).numpy()
+    x = b16(rng.standard_normal((T, d)))
+    Wg = b16(rng.standard_normal((E, d)) / 8)
+    Wm = b16(rng.standard_normal((E, d)) / 8)
+    W1 = b16(rng.standard_normal((E, I, d)) / 8)
+    W3 = b16(rng.standard_normal((E, I, d)) / 8)
+    W2 = b16(rng.standard_normal((E, d, I)) / 7)
+    xf, Wgf, Wmf = (_torch_bf16_to_f64(a) for a in (x, Wg, Wm))
+    r, z = oracle.logits(x, Wg, Wm, "bf16")
+    r_np = np.cumsum(xf[:, None, :] * Wgf[None, :, :], axis=2)[..., -1]
+    z_np = np.cumsum(xf[:, None, :] * Wmf[None, :, :], axis=2)[..., -1]
+    assert np.array_equal(r, r_np) and np.array_equal(z, z_np)
+    rt = oracle.route(r, z, K, renorm=1)
+    y = oracle.experts(x, W1, W3, W2, rt["idx"], rt["w"], "bf16")
+    W1f, W3f, W2f = (_torch_bf16_to_f64(a) for a in (W1, W3, W2))
+    want = np.zeros((T, d))
+    for t in range(T):
+        for k in range(K):
+            e = rt["idx"][t, k]
+            if e < 0:
+                continue
+            a = W1f[e] @ xf[t]
+            b = W3f[e] @ xf[t]
+            want[t] += rt["w"][t, k] * (W2f[e] @ (_silu(a) * b))
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
