@@ -195,11 +195,13 @@ class ClockSampler:
 class Layer:
     """The decode layer on one GPU: weights, token batches, mask routers."""
 
-    def __init__(self, T, device, rank, seed=0, share=None):
+    def __init__(self, T, device, rank, seed=0, share=None, shape=None, zipf=1.1):
         import torch
         from dynamic_expert_routing_router_b200 import abi, inputs
         self.torch, self.abi, self.inputs = torch, abi, inputs
-        self.sh = sh = inputs.QWEN3
+        if share is not None:
+            shape = share.sh
+        self.sh = sh = shape or inputs.QWEN3
         self.T = T
         self.device = device
         if share is not None:  # same layer weights, another batch size
@@ -207,7 +209,7 @@ class Layer:
             self.masks = share.masks
         else:
             self.W1, self.W3, self.W2 = inputs.make_experts(sh, seed=seed, device=device)
-            self.Wg = inputs.make_gate(sh, seed=seed, device=device)
+            self.Wg = inputs.make_gate(sh, seed=seed, device=device, zipf=zipf)
             self.masks = {}
         self.xs = [inputs.make_tokens(sh, T, seed=1000 * (rank + 1) + b, device=device)
                    for b in range(N_BATCHES)]
@@ -440,6 +442,44 @@ def cpu_baseline(layer, f, seconds, max_batches=None):
                        f"only), {el:.1f} s")
 
 
+def cpu_baseline_one_core(T, f, seconds):
+    """The same oracle on ONE host core: a child process with OMP_NUM_THREADS=1
+    (the thread count is fixed when the OpenMP runtime starts) times the whole
+    layer on CPU-drawn weights of the same recipe."""
+    env = dict(os.environ, OMP_NUM_THREADS="1", CUDA_VISIBLE_DEVICES="")
+    cmd = [sys.executable, os.path.abspath(__file__), "--cpu-child", "--T", str(T),
+           "--kept", str(f), "--cpu-seconds", str(seconds)]
+    try:
+        out = subprocess.run(cmd, env=env, capture_output=True, text=True,
+                             timeout=seconds * 4 + 120)
+        return json.loads(out.stdout.strip().splitlines()[-1])
+    except (subprocess.SubprocessError, ValueError, IndexError) as exc:
+        return dict(value=None, cores=1, kind="oracle", error=str(exc)[:200])
+
+
+def cpu_child(args):
+    import oracle
+    from dynamic_expert_routing_router_b200 import inputs
+    sh = inputs.QWEN3
+    W = [inputs.host_array(t) for t in inputs.make_experts(sh, seed=0, device="cpu")]
+    Wg = inputs.host_array(inputs.make_gate(sh, seed=0, device="cpu"))
+    Wm = inputs.host_array(inputs.make_mask(sh, args.kept, seed=0, device="cpu"))
+    xs = [inputs.host_array(inputs.make_tokens(sh, args.T, seed=1000 + b, device="cpu"))
+          for b in range(2)]
+    toks, n, t0 = 0, 0, time.perf_counter()
+    while True:
+        oracle.forward(xs[n % 2], Wg, Wm, *W, sh.K, sh.renorm, "bf16")
+        toks += args.T
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= args.cpu_seconds:
+            break
+    print(json.dumps(dict(value=toks / el, unit="tokens/s", cores=oracle.max_threads(),
+                          kind="oracle",
+                          sample=f"{n} batch(es) of T={args.T} tokens (whole layer, fp64, "
+                                 f"kept pairs only), {el:.1f} s, one thread")))
+
+
 def stack_bench(device, rank, Ts=(1, 64, 256), replays=5):
     """Decode through the 48-layer stack (one set of seeded weights per layer,
     ~58 GB of experts): per T, the stack time with each layer's mask router
@@ -652,6 +692,96 @@ def backward_bench(layer, f, steps, warmup, pk):
     return out
 
 
+def stage_times(layer, f, steps, warmup):
+    """Per-stage device time (us) of one configuration: one pass with every
+    stage event recorded, then each of the two longest stages alone between
+    its own two events (the least perturbed timing of those kernels)."""
+    abi = layer.abi
+    S = abi.FORWARD_STAGES
+    fused = abi.plan(layer.dsc)["BN"] < 128 and layer.sh.dtype == "bf16"
+    _, stage_s = time_steps(layer, f, steps, warmup, profiled=True)
+    mean = [sum(s[j] for s in stage_s) / len(stage_s) for j in range(S)]
+    names = [abi.stage_name(j) for j in range(S)]
+    if fused:
+        names[4] = "experts_fused_gate_up_down"
+    launched = [j for j in range(S) if not (fused and j in (3, 5))]
+    top = sorted(launched, key=lambda j: -mean[j])[:2]
+    alone = {}
+    for j in top:
+        _, only = time_steps(layer, f, steps, warmup, profiled=True, only=j)
+        alone[names[j]] = sum(only) / len(only)
+    return names, {names[j]: mean[j] * 1e6 for j in launched}, alone, fused
+
+
+def config_rows(layer, label, fs, pk, steps, warmup):
+    """One configuration (shape, T) at each kept fraction and with the mask
+    disabled: layer time, layer roofline, per-stage times, and the dominant
+    expert kernel against its own roofline (tensor-bound when its flops at the
+    measured bf16 peak take longer than its bytes at the measured HBM copy
+    rate, else HBM-bound)."""
+    rows, base = [], None
+    for f in fs:
+        sts = layer.routing_stats(f)
+        gs, _ = time_steps(layer, f, steps, warmup)
+        tm = sum(gs) / len(gs)
+        troof = sum(layer_roofline_seconds(layer, s_, f is not None, pk) for s_ in sts) / len(sts)
+        names, st_us, alone, fused = stage_times(layer, f, steps, warmup)
+        algs = [algorithmic(layer, s_, f is not None) for s_ in sts]
+        kern = {}
+        for key in ("gemm1_gate_up_swiglu", "gemm2_down", "experts_fused_gate_up_down"):
+            if key not in alone:
+                continue
+            if key == "experts_fused_gate_up_down":
+                by = sum(a["gemm1_gate_up_swiglu"]["bytes"] + a["gemm2_down"]["bytes"]
+                         for a in algs) / len(algs)
+                fl = sum(a["gemm1_gate_up_swiglu"]["flops"] + a["gemm2_down"]["flops"]
+                         for a in algs) / len(algs)
+            else:
+                by = sum(a[key]["bytes"] for a in algs) / len(algs)
+                fl = sum(a[key]["flops"] for a in algs) / len(algs)
+            t = alone[key]
+            if fl / (pk["bf16"] * 1e12) > by / (pk["hbm"] * 1e9):
+                kern[key] = dict(us=t * 1e6, bound="tensor", achieved=fl / t / 1e12,
+                                 unit="TFLOP/s", peak=pk["bf16"], frac=fl / t / 1e12 / pk["bf16"])
+            else:
+                kern[key] = dict(us=t * 1e6, bound="hbm", achieved=by / t / 1e9, unit="GB/s",
+                                 peak=pk["hbm"], frac=by / t / 1e9 / pk["hbm"])
+        kept = sum(s_["P"] for s_ in sts) / len(sts) / (layer.T * layer.sh.K)
+        row = dict(config=label, T=layer.T, kept_target=f if f is not None else "unmasked",
+                   kept_measured=round(kept, 4),
+                   experts_touched=sum(s_["U"] for s_ in sts) / len(sts),
+                   tokens_per_s=layer.T / tm, us_per_layer=tm * 1e6,
+                   roofline_us=troof * 1e6, roofline_frac=troof / tm,
+                   stages_us=st_us, expert_kernels=kern)
+        if f is None:
+            base = tm
+        elif base is not None:
+            row["speedup_vs_unmasked"] = base / tm
+        rows.append(row)
+    return rows
+
+
+def config_bench(device, rank, pk, steps, warmup):
+    """Prefill (T = 8192, Qwen3-30B-A3B shape, kept 15/35/100 %) and the large
+    fine-grained layer (d = 7168, E = 256, I = 2048, uniform router; T = 16
+    and 4096, kept 15/50 %), each next to the mask-disabled kernels."""
+    import torch
+    from dynamic_expert_routing_router_b200 import inputs
+    rows = []
+    pre = Layer(8192, device, rank)
+    rows += config_rows(pre, "prefill_qwen3_T8192", (None, 0.15, 0.35, 1.0), pk, steps, warmup)
+    del pre
+    torch.cuda.empty_cache()
+    big = Layer(16, device, rank, shape=inputs.LARGE, zipf=None)
+    rows += config_rows(big, "large_d7168_E256_T16", (None, 0.15, 0.5), pk, steps, warmup)
+    big4k = Layer(4096, device, rank, share=big)
+    rows += config_rows(big4k, "large_d7168_E256_T4096", (None, 0.15, 0.5), pk,
+                        max(5, steps // 4), warmup)
+    del big4k, big
+    torch.cuda.empty_cache()
+    return rows
+
+
 def run_beam(args):
     import torch
     rank, world, local = dist_env()
@@ -753,6 +883,10 @@ def run_beam(args):
             if lay is not layer:
                 del lay
 
+    per_config = None
+    if not args.no_config:
+        per_config = config_bench(device, rank, pk, args.sweep_steps // 2, 5)
+
     e2e = e2e_rate(layer, f_head, max(20, min(args.steps, 500)), 5)
 
     stack = None
@@ -770,6 +904,7 @@ def run_beam(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(layer, f_head, args.cpu_seconds)
+        cpu["single_core"] = cpu_baseline_one_core(T, f_head, args.cpu_seconds / 2)
 
     clocks = clk.summary()
     line = {
@@ -798,6 +933,7 @@ def run_beam(args):
                          f"graph: {prof_mean * 1e6:.1f} us/step vs {step_mean * 1e6:.1f} "
                          "without them)"),
         "per_kept_fraction": sweep,
+        "per_config": per_config,
         "stack_48_layers": stack,
         "shared_experts": shared,
         "backward": backward,
@@ -812,6 +948,23 @@ def run_beam(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def profile_forwards(args):
+    """A short, fixed launch sequence for a profiler: build the workload, then
+    `args.profile_forwards` eager forward calls, each after an L2 flush."""
+    import torch
+    from dynamic_expert_routing_router_b200 import inputs
+    torch.cuda.set_device(0)
+    sh = inputs.LARGE if args.shape == "large" else inputs.QWEN3
+    layer = Layer(args.T, "cuda:0", 0, shape=sh, zipf=None if args.shape == "large" else 1.1)
+    Wm = layer.mask(args.kept if args.kept < 1.0 else 1.0)
+    for i in range(args.profile_forwards):
+        flush_l2(layer.flush, i)
+        layer.abi.forward(layer.dsc, layer.xs[i % N_BATCHES], layer.Wg, Wm, layer.W1, layer.W3,
+                          layer.W2, layer.out, layer.ws)
+    layer.abi.check(layer.dsc, layer.ws)
+    torch.cuda.synchronize()
 
 
 def run_reference(args):
@@ -874,7 +1027,20 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=32)
+    ap.add_argument("--no-config", action="store_true",
+                    help="skip the prefill and large-layer configurations")
+    ap.add_argument("--cpu-child", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--profile-forwards", type=int, default=0,
+                    help="only run this many eager forwards (L2 flushed before each) of "
+                         "the --shape/--T/--kept workload, then exit: a target for ncu")
+    ap.add_argument("--shape", choices=["qwen3", "large"], default="qwen3")
     args = ap.parse_args(argv)
+    if args.cpu_child:
+        cpu_child(args)
+        return
+    if args.profile_forwards:
+        profile_forwards(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -81,6 +81,12 @@ def lib():
         L.beam_moe_backward.restype = i32
         L.beam_moe_backward_kernel_count.argtypes = [pd]
         L.beam_moe_backward_kernel_count.restype = i32
+        L.beam_moe_ep_dispatch.argtypes = [pd, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.beam_moe_ep_dispatch.restype = i32
+        L.beam_moe_expert_rows.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.beam_moe_expert_rows.restype = i32
+        L.beam_moe_ep_combine.argtypes = [pd, vp, vp, vp, vp, vp, vp]
+        L.beam_moe_ep_combine.restype = i32
         L.beam_moe_route_noalloc_check.argtypes = [vp]
         L.beam_moe_route_noalloc_check.restype = i32
         L.beam_moe_tau_to_logit.argtypes = [ctypes.c_float]
@@ -257,6 +263,30 @@ def forward_profiled(dsc, x, W_gate, W_mask, W1, W3, W2, out, workspace, events,
                                         _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out),
                                         _ptr(workspace), workspace.numel(), _stream(stream),
                                         arr), "beam_moe_forward_profiled")
+
+
+def ep_dispatch(dsc, n_ranks, x, topk_idx, counts, send_rows, send_pair, send_expert,
+                send_counts, pair_pos, workspace, stream=None):
+    """Kept pairs grouped by destination rank (expert-parallel dispatch)."""
+    _ok(lib().beam_moe_ep_dispatch(ctypes.byref(dsc), int(n_ranks), _ptr(x), _ptr(topk_idx),
+                                   _ptr(counts), _ptr(send_rows), _ptr(send_pair),
+                                   _ptr(send_expert), _ptr(send_counts), _ptr(pair_pos),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)),
+        "beam_moe_ep_dispatch")
+
+
+def expert_rows(dsc, x_rows, expert_id, W1, W3, W2, y_rows, workspace, stream=None):
+    """y_rows[i] = E_{expert_id[i]}(x_rows[i]) in fp32 (dsc.K == 1, dsc.T rows)."""
+    _ok(lib().beam_moe_expert_rows(ctypes.byref(dsc), _ptr(x_rows), _ptr(expert_id), _ptr(W1),
+                                   _ptr(W3), _ptr(W2), _ptr(y_rows), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "beam_moe_expert_rows")
+
+
+def ep_combine(dsc, y_rows, topk_idx, topk_w, pair_pos, out, stream=None):
+    """out_t = sum over kept k of topk_w[t,k] * y_rows[pair_pos[t,k]] (slot order)."""
+    _ok(lib().beam_moe_ep_combine(ctypes.byref(dsc), _ptr(y_rows), _ptr(topk_idx),
+                                  _ptr(topk_w), _ptr(pair_pos), _ptr(out), _stream(stream)),
+        "beam_moe_ep_combine")
 
 
 def check(dsc, workspace, stream=None):

@@ -328,37 +328,16 @@ beam_status check_ws(const beam_moe_plan_info &P, const void *ws, size_t bytes) 
     return BEAM_OK;
 }
 
-beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, const void *Wm,
-                         const void *W1, const void *W3, const void *W2, const void *W1s,
-                         const void *W3s, const void *W2s, void *out, void *workspace,
-                         size_t ws_bytes, void *stream, void *const *events) {
-    beam_moe_plan_info P;
-    beam_status s = make_plan(d, &P);
-    if (s != BEAM_OK) return s;
-    if (!x || !Wg || !W1 || !W3 || !W2 || !out) return BEAM_ERR_INVALID_ARG;
-    for (const void *p : {x, Wg, W1, W3, W2, static_cast<const void *>(out)})
-        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
-    if (d->n_shared > 0) {
-        if (!W1s || !W3s || !W2s) return BEAM_ERR_INVALID_ARG;
-        for (const void *p : {W1s, W3s, W2s})
-            if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
-    }
-    if (Wm && !aligned16(Wm)) return BEAM_ERR_INVALID_ARG;
-    s = check_ws(P, workspace, ws_bytes);
-    if (s != BEAM_OK) return s;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const Recorder rec{events, st};
-    if (d->T == 0) {  // nothing to compute; leave a clean error word and counters
-        BEAM_TRY_CUDA(cudaMemsetAsync(workspace, 0, P.off_partial, st));
-        for (int i = 0; i <= BEAM_MOE_FORWARD_STAGES; ++i) BEAM_TRY_CUDA(rec.rec(i));
-        return BEAM_OK;
-    }
-    const int n_sm = sm_count();
-    char *ws = static_cast<char *>(workspace);
+// Stages 2-6 of a call whose routing (idx, w, counts, hist, a clean header)
+// is already in the workspace: grouping, row copy, expert GEMMs, shared
+// experts, combine.  out_dtype is the combine's output type.
+beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, const void *x,
+                        const void *W1, const void *W3, const void *W2, const void *W1s,
+                        const void *W3s, const void *W2s, void *out, int out_dtype, char *ws,
+                        cudaStream_t st, const Recorder &rec, int n_sm) {
     int *err = reinterpret_cast<int *>(ws + P.off_err);
     int *meta = reinterpret_cast<int *>(ws + P.off_meta);
     int *counts = reinterpret_cast<int *>(ws + P.off_counts);
-    int *hist = reinterpret_cast<int *>(ws + P.off_hist);
     int *idx = reinterpret_cast<int *>(ws + P.off_idx);
     float *w = reinterpret_cast<float *>(ws + P.off_w);
     int *pair = reinterpret_cast<int *>(ws + P.off_pair);
@@ -368,10 +347,6 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     void *xp = ws + P.off_xp;
     void *h = ws + P.off_h;
     float *y = reinterpret_cast<float *>(ws + P.off_y);
-
-    const RouteOut ro{idx, w, counts, hist, nullptr};
-    s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
-    if (s != BEAM_OK) return s;
 
     // Thin token tiles (decode, bf16): the grouping kernel also copies the
     // token rows (no gather launch), gate and up rows are interleaved in one
@@ -507,11 +482,51 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     }
 
     BEAM_TRY_CUDA(rec.rec(6));
-    BEAM_TRY_CUDA(launch_combine(d->dtype, y, idx, w, pair_pos, d->T, d->K, d->d, ys,
+    BEAM_TRY_CUDA(launch_combine(out_dtype, y, idx, w, pair_pos, d->T, d->K, d->d, ys,
                                  d->n_shared, out, n_sm, st));
     BEAM_TRY_CUDA(rec.rec(7));
     return BEAM_OK;
 }
+
+beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, const void *Wm,
+                         const void *W1, const void *W3, const void *W2, const void *W1s,
+                         const void *W3s, const void *W2s, void *out, void *workspace,
+                         size_t ws_bytes, void *stream, void *const *events) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(d, &P);
+    if (s != BEAM_OK) return s;
+    if (!x || !Wg || !W1 || !W3 || !W2 || !out) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x, Wg, W1, W3, W2, static_cast<const void *>(out)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    if (d->n_shared > 0) {
+        if (!W1s || !W3s || !W2s) return BEAM_ERR_INVALID_ARG;
+        for (const void *p : {W1s, W3s, W2s})
+            if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    }
+    if (Wm && !aligned16(Wm)) return BEAM_ERR_INVALID_ARG;
+    s = check_ws(P, workspace, ws_bytes);
+    if (s != BEAM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Recorder rec{events, st};
+    if (d->T == 0) {  // nothing to compute; leave a clean error word and counters
+        BEAM_TRY_CUDA(cudaMemsetAsync(workspace, 0, P.off_partial, st));
+        for (int i = 0; i <= BEAM_MOE_FORWARD_STAGES; ++i) BEAM_TRY_CUDA(rec.rec(i));
+        return BEAM_OK;
+    }
+    const int n_sm = sm_count();
+    char *ws = static_cast<char *>(workspace);
+    int *counts = reinterpret_cast<int *>(ws + P.off_counts);
+    int *hist = reinterpret_cast<int *>(ws + P.off_hist);
+    int *idx = reinterpret_cast<int *>(ws + P.off_idx);
+    float *w = reinterpret_cast<float *>(ws + P.off_w);
+
+    const RouteOut ro{idx, w, counts, hist, nullptr};
+    s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
+    if (s != BEAM_OK) return s;
+
+    return launch_tail(d, P, x, W1, W3, W2, W1s, W3s, W2s, out, d->dtype, ws, st, rec, n_sm);
+}
+
 
 // ------------------------------------------------------------ backward --
 // The backward workspace is the forward plan (its grouping now holds every
@@ -934,6 +949,103 @@ beam_status beam_moe_check(const beam_moe_desc *desc, void *workspace, void *str
         return BEAM_ERR_CUDA;
     if (err == DEV_ERR_TIMEOUT) return BEAM_ERR_TIMEOUT;
     if (err != 0) return BEAM_ERR_INTERNAL;
+    return BEAM_OK;
+}
+
+beam_status beam_moe_ep_dispatch(const beam_moe_desc *desc, int n_ranks, const void *x,
+                                 const int32_t *topk_idx, const int32_t *expert_counts,
+                                 void *send_rows, int32_t *send_pair, int32_t *send_expert,
+                                 int32_t *send_counts, int32_t *pair_pos, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(desc, &P);
+    if (s != BEAM_OK) return s;
+    if (n_ranks < 1 || n_ranks > desc->E || desc->E % n_ranks != 0) return BEAM_ERR_INVALID_ARG;
+    if (desc->n_shared != 0) return BEAM_ERR_INVALID_ARG;
+    if (!x || !topk_idx || !expert_counts || !send_rows || !send_pair || !send_expert ||
+        !send_counts || !pair_pos)
+        return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x, static_cast<const void *>(topk_idx),
+                          static_cast<const void *>(expert_counts), static_cast<const void *>(send_rows),
+                          static_cast<const void *>(send_pair),
+                          static_cast<const void *>(send_expert),
+                          static_cast<const void *>(send_counts),
+                          static_cast<const void *>(pair_pos)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    s = check_ws(P, workspace, workspace_bytes);
+    if (s != BEAM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (desc->T == 0) {
+        BEAM_TRY_CUDA(cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * size_t(n_ranks), st));
+        return BEAM_OK;
+    }
+    const size_t es = desc->dtype == BEAM_BF16 ? 2 : 4;
+    EpDispatchArgs a;
+    a.idx = topk_idx;
+    a.counts = expert_counts;
+    a.T = desc->T;
+    a.K = desc->K;
+    a.E = desc->E;
+    a.G = n_ranks;
+    a.x = static_cast<const uint4 *>(x);
+    a.row_vec = int(es * size_t(desc->d) / 16);
+    a.R = kPermCopyBlocks;
+    a.send_rows = static_cast<uint4 *>(send_rows);
+    a.send_pair = send_pair;
+    a.send_expert = send_expert;
+    a.send_counts = send_counts;
+    a.pair_pos = pair_pos;
+    a.err = reinterpret_cast<int *>(static_cast<char *>(workspace) + P.off_err);
+    BEAM_TRY_CUDA(launch_ep_dispatch(a, st));
+    return BEAM_OK;
+}
+
+beam_status beam_moe_expert_rows(const beam_moe_desc *desc, const void *x_rows,
+                                 const int32_t *expert_id, const void *W1, const void *W3,
+                                 const void *W2, float *y_rows, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(desc, &P);
+    if (s != BEAM_OK) return s;
+    if (desc->K != 1 || desc->n_shared != 0) return BEAM_ERR_INVALID_ARG;
+    if (!x_rows || !expert_id || !W1 || !W3 || !W2 || !y_rows) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {x_rows, static_cast<const void *>(expert_id), W1, W3, W2,
+                          static_cast<const void *>(y_rows)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    s = check_ws(P, workspace, workspace_bytes);
+    if (s != BEAM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // header (error words, meta), counts and histogram start at zero
+    BEAM_TRY_CUDA(cudaMemsetAsync(workspace, 0, P.off_partial, st));
+    if (desc->T == 0) return BEAM_OK;
+    char *ws = static_cast<char *>(workspace);
+    const int n_sm = sm_count();
+    BEAM_TRY_CUDA(launch_set_routing(expert_id, desc->T, desc->E,
+                                     reinterpret_cast<int *>(ws + P.off_idx),
+                                     reinterpret_cast<float *>(ws + P.off_w),
+                                     reinterpret_cast<int *>(ws + P.off_counts),
+                                     reinterpret_cast<int *>(ws + P.off_hist),
+                                     reinterpret_cast<int *>(ws + P.off_err), n_sm, st));
+    return launch_tail(desc, P, x_rows, W1, W3, W2, nullptr, nullptr, nullptr, y_rows, BEAM_F32,
+                       ws, st, Recorder{nullptr, st}, n_sm);
+}
+
+beam_status beam_moe_ep_combine(const beam_moe_desc *desc, const float *y_rows,
+                                const int32_t *topk_idx, const float *topk_w,
+                                const int32_t *pair_pos, void *out, void *stream) {
+    beam_moe_plan_info P;
+    beam_status s = make_plan(desc, &P);
+    if (s != BEAM_OK) return s;
+    if (desc->n_shared != 0) return BEAM_ERR_INVALID_ARG;
+    if (desc->T == 0) return BEAM_OK;
+    if (!topk_idx || !topk_w || !pair_pos || !out || !y_rows) return BEAM_ERR_INVALID_ARG;
+    for (const void *p : {static_cast<const void *>(y_rows), static_cast<const void *>(topk_idx),
+                          static_cast<const void *>(topk_w), static_cast<const void *>(pair_pos),
+                          static_cast<const void *>(out)})
+        if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    BEAM_TRY_CUDA(launch_combine(desc->dtype, y_rows, topk_idx, topk_w, pair_pos, desc->T, desc->K,
+                                 desc->d, nullptr, 0, out, sm_count(), st));
     return BEAM_OK;
 }
 

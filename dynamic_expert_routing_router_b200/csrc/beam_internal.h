@@ -171,6 +171,28 @@ struct PermuteArgs {
 };
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 
+// Expert-parallel dispatch (ep_kernels.cu): kept pairs listed by expert
+// (ascending) then token, which groups them by destination rank r = e / (E/G).
+struct EpDispatchArgs {
+    const int *idx;      // [T][K] candidate or -1
+    const int *counts;   // [E] kept pairs per expert
+    int T, K, E, G;
+    const uint4 *x;      // token rows
+    int row_vec;         // 16-byte vectors per row
+    int R;               // blocks per expert (row copy)
+    uint4 *send_rows;    // [P][row_vec] kept pairs' token rows, in listed order
+    int *send_pair;      // [P] t*K + k of each send row
+    int *send_expert;    // [P] local expert id of each send row on its destination
+    int *send_counts;    // [G] send rows per destination rank
+    int *pair_pos;       // [T][K] send row of a kept pair
+    int *err;
+};
+cudaError_t launch_ep_dispatch(const EpDispatchArgs &a, cudaStream_t stream);
+// Received rows -> routing of a K = 1 layer call with weight 1 (counts, hist
+// zeroed by the caller).
+cudaError_t launch_set_routing(const int *expert_id, int N, int E, int *idx, float *w, int *counts,
+                               int *hist, int *err, int n_sm, cudaStream_t stream);
+
 // Gather token rows into expert order (row_bytes multiple of 16).
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
                           long long row_bytes, int p_cap, void *xp, int n_sm,

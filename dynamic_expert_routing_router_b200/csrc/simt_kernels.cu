@@ -12,13 +12,13 @@
 
 #include "beam_internal.h"
 #include "beam_ptx.cuh"
+#include "grouping.cuh"
 #include "topk_token.cuh"
 
 namespace beam {
 
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------ top-K + mask --
 //
@@ -118,28 +118,12 @@ __global__ void __launch_bounds__(256) topk_mask_kernel(const TopkArgs a, int tp
 // With a row copy (x, xp set), R blocks share an expert: each one repeats the
 // listing (identical values, so the duplicate writes agree) and then copies
 // every R-th group of its rows of x into xp, one warp per row.
-constexpr int kPermThreads = 256;
-
-__device__ __forceinline__ int block_sum_256(int v, int *s_red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-    __syncthreads();
-    if (lane == 0) s_red[warp] = v;
-    __syncthreads();
-    int total = 0;
-#pragma unroll
-    for (int i = 0; i < kPermThreads / 32; ++i) total += s_red[i];
-    return total;
-}
+constexpr int kPermThreads = kGroupThreads;
 
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs a) {
-    __shared__ int s_red[kPermThreads / 32];
-    __shared__ int s_wcnt[4 * (kPermThreads / 32)];
-    __shared__ int s_wpre[4 * (kPermThreads / 32)];
-    __shared__ int s_total;
+    __shared__ GroupSmem sm;
     const int e = blockIdx.x / a.R, replica = blockIdx.x % a.R;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
     griddep_wait();
     griddep_launch_dependents();
 
@@ -147,12 +131,12 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     if (tid < a.E) c = a.counts[tid];
     const int padded = (c + a.BN - 1) / a.BN * a.BN;
     const int ntile = (c + a.BN - 1) / a.BN;
-    const int off_e = block_sum_256(tid < e ? padded : 0, s_red);
-    const int toff_e = block_sum_256(tid < e ? ntile : 0, s_red);
+    const int off_e = group_block_sum(tid < e ? padded : 0, sm);
+    const int toff_e = group_block_sum(tid < e ? ntile : 0, sm);
     if (e == 0) {
-        const int tot_rows = block_sum_256(padded, s_red);
-        const int tot_tiles = block_sum_256(ntile, s_red);
-        const int tot_pairs = block_sum_256(c, s_red);
+        const int tot_rows = group_block_sum(padded, sm);
+        const int tot_tiles = group_block_sum(ntile, sm);
+        const int tot_pairs = group_block_sum(c, sm);
         if (tid == 0) {
             a.meta[0] = tot_tiles;
             a.meta[1] = tot_rows;
@@ -160,52 +144,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
         }
     }
     const int count_e = a.counts[e];
-
-    // Each pass covers kSub * 256 tokens as kSub coalesced sub-chunks (token
-    // base + q * 256 + tid); ranks follow (sub-chunk, warp, lane), i.e. token
-    // order.  A token matches expert e in at most one slot.
-    constexpr int kSub = 4;
-    constexpr int kWarps = kPermThreads / 32;
-    int running = 0;
-    for (int base = 0; base < a.T; base += kPermThreads * kSub) {
-        int km[kSub];
-        unsigned bal[kSub];
-#pragma unroll
-        for (int q = 0; q < kSub; ++q) {
-            const int t = base + q * kPermThreads + tid;
-            km[q] = -1;
-            if (t < a.T) {
-                const int *row = a.idx + (long long)t * a.K;
-                for (int k = 0; k < a.K; ++k)
-                    if (row[k] == e) km[q] = k;
-            }
-            bal[q] = __ballot_sync(kFull, km[q] >= 0);
-            if (lane == 0) s_wcnt[q * kWarps + warp] = __popc(bal[q]);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int acc = 0;
-            for (int i = 0; i < kSub * kWarps; ++i) {
-                s_wpre[i] = acc;
-                acc += s_wcnt[i];
-            }
-            s_total = acc;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int q = 0; q < kSub; ++q) {
-            if (km[q] >= 0) {
-                const int t = base + q * kPermThreads + tid;
-                const int pos = off_e + running + s_wpre[q * kWarps + warp] +
-                                __popc(bal[q] & ((1u << lane) - 1u));
-                a.pair[pos] = t * a.K + km[q];
-                a.pair_pos[(long long)t * a.K + km[q]] = pos;
-            }
-        }
-        running += s_total;
-        __syncthreads();
-    }
-    if (tid == 0 && running != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
+    const int listed = list_expert_pairs(a.idx, a.T, a.K, e, off_e, a.pair, a.pair_pos, sm);
+    if (tid == 0 && listed != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
 
     const int padded_e = (count_e + a.BN - 1) / a.BN * a.BN;
     for (int r = count_e + tid; r < padded_e; r += kPermThreads) a.pair[off_e + r] = -1;
@@ -217,23 +157,10 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     }
     if (a.xp == nullptr) return;
     // Row copy.  The pair entries read back were written by this block (the
-    // listing loop ends with a barrier); padding rows are not copied, they
-    // only feed padding columns of the GEMMs, which are never stored.
-    for (int r = replica * kWarps + warp; r < count_e; r += a.R * kWarps) {
-        const int pr = a.pair[off_e + r];
-        const uint4 *src = a.x + (long long)(pr / a.K) * a.row_vec;
-        uint4 *dst = a.xp + (long long)(off_e + r) * a.row_vec;
-        int v = lane;
-        for (; v + 96 < a.row_vec; v += 128) {  // four 16-byte loads in flight per lane
-            const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 32);
-            const uint4 a2 = __ldg(src + v + 64), a3 = __ldg(src + v + 96);
-            dst[v] = a0;
-            dst[v + 32] = a1;
-            dst[v + 64] = a2;
-            dst[v + 96] = a3;
-        }
-        for (; v < a.row_vec; v += 32) dst[v] = __ldg(src + v);
-    }
+    // listing ends with a barrier); padding rows are not copied, they only
+    // feed padding columns of the GEMMs, which are never stored.
+    copy_listed_rows(a.x, a.xp, a.pair, off_e, count_e, replica * kGroupWarps + warp,
+                     a.R * kGroupWarps, a.K, a.row_vec);
 }
 
 // ------------------------------------------------------------------ gather --

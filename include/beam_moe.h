@@ -283,6 +283,62 @@ beam_status beam_moe_backward(const beam_moe_desc *desc, const void *x, const vo
  * expert's candidate rows), 14 for fp32; 0 for T = 0 or a bad descriptor. */
 int beam_moe_backward_kernel_count(const beam_moe_desc *desc);
 
+/* ------------------------------------------------- expert parallelism --
+ * G ranks (one process per GPU), rank r owning experts [r E/G, (r+1) E/G).
+ * The pages describe the exchange only in general terms (the MoE tutorial
+ * page on "Beam", §4.2: tokens travel to the GPU that holds their expert by
+ * an all-to-all) and BEAM's own contribution to it in the news article on
+ * BEAM, §5: masked entries are left out of the expert-token grouping.  Here
+ * only KEPT pairs are dispatched, so the mask cuts the rows that cross the
+ * interconnect by the kept fraction.  A step, per rank:
+ *   beam_moe_route (own tokens) -> beam_moe_ep_dispatch -> all-to-all of the
+ *   send counts, rows and local expert ids -> beam_moe_expert_rows on the
+ *   received rows -> all-to-all of the fp32 rows back -> beam_moe_ep_combine.
+ * The exchanges are the caller's (NCCL through torch.distributed in the
+ * Python binding); these calls never touch another GPU's memory. */
+
+/* Dispatch of the kept pairs of one routed batch (desc, topk_idx and
+ * expert_counts as written by beam_moe_route on `workspace`).  Pairs are
+ * listed by expert (ascending) then token (ascending) -- the order of the
+ * layer's own grouping -- so the rows bound for rank r are contiguous and
+ * ranks appear in order.  Writes, with P = the number of kept pairs:
+ *   send_rows   [P, d] (desc dtype)  the pairs' token rows, in that order
+ *   send_pair   int32 [P]    t*K + k of each row
+ *   send_expert int32 [P]    the row's expert id local to its destination
+ *   send_counts int32 [n_ranks]  rows per destination rank
+ *   pair_pos    int32 [T,K]  send row of each kept pair (masked: unwritten)
+ * Capacity: send_rows/send_pair/send_expert hold T*K entries.  Needs
+ * E % n_ranks == 0, 1 <= n_ranks <= E and n_shared == 0.  A consistency
+ * failure sets the workspace error word (BEAM_ERR_INTERNAL through
+ * beam_moe_check), which this call never clears: check once after the step. */
+beam_status beam_moe_ep_dispatch(const beam_moe_desc *desc, int n_ranks, const void *x,
+                                 const int32_t *topk_idx, const int32_t *expert_counts,
+                                 void *send_rows, int32_t *send_pair, int32_t *send_expert,
+                                 int32_t *send_counts, int32_t *pair_pos, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/* Expert outputs of pre-routed rows: y_rows[i] = E_{expert_id[i]}(x_rows[i])
+ * (Eq. 3), fp32, computed by the layer's own grouping and expert GEMMs, so a
+ * row's value is the per-pair output the one-GPU layer combines.  desc: T =
+ * number of rows, E = the experts in W1/W3/W2, K = 1, n_shared = 0; the
+ * router fields are unused.  expert_id int32 [T]: an id in [0, E) or -1 (the
+ * row gets zeros); any other value sets BEAM_ERR_INTERNAL and is treated as
+ * -1.  Workspace: beam_moe_workspace_size(desc) bytes; errors through
+ * beam_moe_check on it. */
+beam_status beam_moe_expert_rows(const beam_moe_desc *desc, const void *x_rows,
+                                 const int32_t *expert_id, const void *W1, const void *W3,
+                                 const void *W2, float *y_rows, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/* Eq. (8) at the source rank: out_t = sum over kept k, in slot order, of
+ * topk_w[t,k] * y_rows[pair_pos[t,k]] (fp32 sums, one rounding to the desc
+ * dtype); 0 for a token with no kept candidate.  y_rows: the returned fp32
+ * rows in send order (non-NULL even when no pair is kept; nothing is then
+ * read).  T = 0 does nothing. */
+beam_status beam_moe_ep_combine(const beam_moe_desc *desc, const float *y_rows,
+                                const int32_t *topk_idx, const float *topk_w,
+                                const int32_t *pair_pos, void *out, void *stream);
+
 /* Synchronise `stream`, then read the workspace error word written by the last
  * call: BEAM_OK, BEAM_ERR_TIMEOUT (a bounded device wait expired, the kernel
  * returned early; that call's outputs are not valid) or BEAM_ERR_INTERNAL (a
