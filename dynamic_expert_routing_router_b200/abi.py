@@ -38,11 +38,12 @@ class Desc(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("BN", ctypes.c_int), ("router_bn", ctypes.c_int),
                 ("router_splits", ctypes.c_int), ("p_cap", ctypes.c_int),
-                ("tiles_cap", ctypes.c_int), ("reserved", ctypes.c_int)] + \
+                ("tiles_cap", ctypes.c_int), ("sub_bn", ctypes.c_int),
+                ("reserved", ctypes.c_int)] + \
                [(n, ctypes.c_size_t) for n in (
                    "off_err", "off_meta", "off_counts", "off_hist", "off_partial", "off_idx",
                    "off_w", "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h", "off_y",
-                   "off_tile_done", "off_hs", "off_ys", "workspace_bytes")]
+                   "off_tile_done", "off_hs", "off_ys", "off_tiles_sub", "workspace_bytes")]
 
 
 _lib = None

@@ -64,21 +64,27 @@ beam_status validate_desc(const beam_moe_desc *d) {
 int shared_bn(int T) { return T <= 16 ? 16 : T <= 256 ? 32 : 128; }
 
 // Token-tile height of the expert GEMMs from the mean kept-or-not pairs per
-// expert (T*K/E): decode batches use thin tiles, prefill batches 128 rows.
-int choose_bn(const beam_moe_desc *d) {
+// expert (T*K/E): decode batches use thin tiles, prefill batches 128 rows, and
+// large bf16 prefill batches 256 (the gate/up GEMM then moves 64 KB of
+// operands per 8.4 MFLOP stage instead of 48 KB per 4.2 MFLOP; the MMA's N
+// follows each tile's valid rows, so the wider padding costs no tensor work).
+int choose_bn(const beam_moe_desc *d, bool wide) {
     const long long avg = cdiv((long long)d->T * d->K, d->E);
     if (avg <= 16) return 16;
     if (avg <= 32) return 32;
     if (avg <= 64) return 64;
+    if (wide && avg >= 256) return 256;
     return 128;
 }
 
-beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
+// `backward`: the training call's plan (its per-expert 128-row tile lists
+// need token tiles of at most 128 rows).
+beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P, bool backward = false) {
     beam_status st = validate_desc(d);
     if (st != BEAM_OK) return st;
     std::memset(P, 0, sizeof(*P));
     const long long T = d->T, K = d->K, E = d->E;
-    P->BN = choose_bn(d);
+    P->BN = choose_bn(d, d->dtype == BEAM_BF16 && !backward);
     if (d->dtype == BEAM_BF16) {
         // Router: enough (token tile x row block x split) units to cover the
         // SMs at decode sizes, while the split partials stay smaller than the
@@ -122,7 +128,12 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
     const size_t srows = size_t(d->n_shared) * size_t(T);  // shared rows: every token
     P->off_hs = align256(P->off_tile_done + 4 * size_t(tiles_cap));
     P->off_ys = align256(P->off_hs + es * srows * size_t(d->n_shared > 0 ? d->I_shared : 0));
-    o = align256(P->off_ys + 4 * srows * size_t(d->d));
+    // 256-row token tiles: the gate/up GEMM runs over 128-row sub-tiles of
+    // them (two 128-row weight tiles and two accumulator buffers per unit).
+    P->sub_bn = P->BN > kBlockM ? kBlockM : P->BN;
+    P->off_tiles_sub = align256(P->off_ys + 4 * srows * size_t(d->d));
+    const size_t sub_cap = P->BN > kBlockM ? size_t(cdiv(T * K, kBlockM) + E) : 0;
+    o = align256(P->off_tiles_sub + 16 * sub_cap);
     P->workspace_bytes = o;
     return BEAM_OK;
 }
@@ -365,6 +376,11 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
                    fused ? static_cast<uint4 *>(xp) : nullptr,
                    row_vec,  fused ? kPermCopyBlocks : 1,
                    meta,     err};
+    int4 *tiles_sub = reinterpret_cast<int4 *>(ws + P.off_tiles_sub);
+    if (P.sub_bn < P.BN) {  // 128-row sub-tiles for the gate/up GEMM; count in meta[3]
+        pa.tiles_sub = tiles_sub;
+        pa.sub_bn = P.sub_bn;
+    }
     BEAM_TRY_CUDA(launch_permute(pa, st));
 
     BEAM_TRY_CUDA(rec.rec(3));
@@ -377,7 +393,7 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
         TcMaps maps;
         if (!make_tmap(&maps.a0, W1, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.a1, W3, d->d, (unsigned long long)d->E * d->I, wbox)) return BEAM_ERR_CUDA;
-        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
+        if (!make_tmap(&maps.b, xp, d->d, P.p_cap, P.sub_bn)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.a2, W2, d->I, (unsigned long long)d->E * d->d, kBlockM)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.b2, h, d->I, P.p_cap, P.BN)) return BEAM_ERR_CUDA;
 
@@ -408,11 +424,20 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
                                          int(units < n_sm ? units : n_sm), st));
             BEAM_TRY_CUDA(rec.rec(5));  // the down GEMM ran inside the fused launch
         } else {
-            long long units = (long long)P.tiles_cap * g.n_mb;
-            BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.BN, maps, g,
+            // gate/up over the 128-row sub-tiles when the tiles are 256 rows
+            const bool sub = P.sub_bn < P.BN;
+            long long units = (long long)(sub ? cdiv((long long)d->T * d->K, P.sub_bn) + d->E
+                                              : P.tiles_cap) * g.n_mb;
+            if (sub) {
+                g.meta = meta + 3;
+                g.tiles = tiles_sub;
+            }
+            BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, P.sub_bn, maps, g,
                                          int(units < n_sm ? units : n_sm), st));
             BEAM_TRY_CUDA(rec.rec(5));
             g.fault_skip = 0;
+            g.meta = meta;
+            g.tiles = tiles;
             TcMaps m2 = maps;
             m2.a0 = maps.a2;
             m2.a1 = maps.a2;
@@ -539,7 +564,7 @@ struct BwdPlan {
 };
 
 beam_status make_bwd_plan(const beam_moe_desc *d, beam_moe_plan_info *P, BwdPlan *B) {
-    beam_status s = make_plan(d, P);
+    beam_status s = make_plan(d, P, true);
     if (s != BEAM_OK) return s;
     if (d->n_shared != 0) return BEAM_ERR_UNSUPPORTED_SHAPE;  // shared experts: forward only
     const size_t T = size_t(d->T), K = size_t(d->K), E = size_t(d->E), I = size_t(d->I);

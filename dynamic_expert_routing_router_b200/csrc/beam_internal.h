@@ -56,6 +56,7 @@ constexpr int kMaxShared = 16;        // shared experts per layer
 constexpr int kPermCopyBlocks = 4;    // grouping blocks per expert when they copy rows
 constexpr int kMaxTileRows = 128;     // largest token tile (BN)
 
+
 // Launch with programmatic stream serialization (PDL): the kernel may begin
 // its prologue while the previous kernel in the stream finishes; every kernel
 // of this library waits (griddep_wait) before touching global memory.
@@ -123,6 +124,7 @@ struct TcGemmArgs {
     float *a_out, *b_out;     // MODE_GEMM1 (or null): fp32 pre-activations, like H
     int *tile_done;           // per tile: gate/up units whose H rows are published
     int *work_ctr;            // next unit to hand out (zeroed by the router kernel)
+
     // MODE_GEMM1 / MODE_GEMM2 over every token (shared experts): tile ti of
     // n_units / n_mb is (shared expert ti / dense_ntt, token tile ti % dense_ntt);
     // GEMM1 reads x rows, GEMM2 reads and both write rows s * T + token.
@@ -168,6 +170,8 @@ struct PermuteArgs {
     int R;        // blocks per expert (>= 1)
     int *meta;
     int *err;
+    int4 *tiles_sub;  // or null: the same rows as tiles of sub_bn rows (count -> meta[3])
+    int sub_bn;
 };
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 

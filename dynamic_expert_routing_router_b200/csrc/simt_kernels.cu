@@ -133,14 +133,19 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
     const int ntile = (c + a.BN - 1) / a.BN;
     const int off_e = group_block_sum(tid < e ? padded : 0, sm);
     const int toff_e = group_block_sum(tid < e ? ntile : 0, sm);
+    // sub-tiles (sub_bn < BN): the same rows, in tiles of sub_bn rows
+    const int nsub = a.tiles_sub ? (c + a.sub_bn - 1) / a.sub_bn : 0;
+    const int soff_e = a.tiles_sub ? group_block_sum(tid < e ? nsub : 0, sm) : 0;
     if (e == 0) {
         const int tot_rows = group_block_sum(padded, sm);
         const int tot_tiles = group_block_sum(ntile, sm);
         const int tot_pairs = group_block_sum(c, sm);
+        const int tot_sub = a.tiles_sub ? group_block_sum(nsub, sm) : 0;
         if (tid == 0) {
             a.meta[0] = tot_tiles;
             a.meta[1] = tot_rows;
             a.meta[2] = tot_pairs;
+            if (a.tiles_sub) a.meta[3] = tot_sub;
         }
     }
     const int count_e = a.counts[e];
@@ -155,6 +160,11 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
         a.tiles[toff_e + j] = make_int4(e, off_e + j * a.BN, rows, 0);
         a.tile_done[toff_e + j] = 0;
     }
+    if (a.tiles_sub)
+        for (int j = tid; j * a.sub_bn < count_e; j += kPermThreads)
+            a.tiles_sub[soff_e + j] =
+                make_int4(e, off_e + j * a.sub_bn, min(a.sub_bn, count_e - j * a.sub_bn), 0);
+
     if (a.xp == nullptr) return;
     // Row copy.  The pair entries read back were written by this block (the
     // listing ends with a barrier); padding rows are not copied, they only

@@ -70,7 +70,10 @@ struct TcCfg {
     static constexpr uint32_t SMEM_BYTES =
         STAGES * STAGE_BYTES + XCH_BYTES + 1024;  // + alignment slack
     static constexpr uint32_t ACC_COLS = NUM_A * BN;  // fp32 columns per accumulator
-    static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+    // Two accumulator buffers (one unit's epilogue overlaps the next unit's
+    // MMAs) when they fit the 512 TMEM columns, else one.
+    static constexpr uint32_t ACC_BUFS = 2 * ACC_COLS <= 512 ? 2 : 1;
+    static constexpr uint32_t TMEM_COLS = ACC_BUFS * ACC_COLS;
     static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
     static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
                   "TMEM allocation must be a power of two in [32, 512]");
@@ -161,6 +164,15 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs
 
 // A bounded wait expired: record it (DEV_ERR_TIMEOUT, or the router's tag)
 // and tell the CTA's other roles to stop.
+// Token columns a unit computes: its valid rows rounded up to the MMA's N
+// step of 16 (16 <= N <= BN for M = 128).
+template <int MODE, int BN>
+__device__ __forceinline__ int unit_cols(const Unit &w, const TcGemmArgs &p) {
+    const int rows = MODE == MODE_ROUTER ? min(BN, p.T - w.tt * BN) : w.rows;
+    const int n = (rows + 15) & ~15;
+    return n < 16 ? 16 : (n > BN ? BN : n);
+}
+
 __device__ __forceinline__ void signal_abort(const TcGemmArgs &p, int *abort_flag) {
     atomicExch(p.err, p.err_code ? p.err_code : int(DEV_ERR_TIMEOUT));
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
@@ -354,9 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer --
         if (lane == 0) {
-            constexpr uint32_t IDESC =
-                umma_idesc_bf16_f32(kBlockM, BN) |
-                ((MODE == MODE_GEMM2T || MODE == MODE_GEMM1T) ? kIdescAMajorMN : 0u);
+            constexpr uint32_t kAMajor =
+                (MODE == MODE_GEMM2T || MODE == MODE_GEMM1T) ? kIdescAMajorMN : 0u;
             uint32_t it = 0;
             bool ok = true;
             for (uint32_t lu = 0;; ++lu) {
@@ -374,9 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else if (u >= n_units) {
                     break;
                 }
-                const int nk = (MODE == MODE_EXPERTS && u >= n_first) ? p.nk2 : p.nk;
-                const uint32_t a = lu & 1u;
-                if (!mbar_wait_bounded(&tempty_bar[a], ((lu >> 1) & 1u) ^ 1u, abort_flag,
+                const Unit w = decode_unit<MODE, BN>(u, n_first, p);
+                const int nk = w.nk;
+                // MMA N = the unit's valid token rows rounded up to 16: the
+                // padding rows of an expert's last tile cost no tensor work
+                const uint32_t IDESC = umma_idesc_bf16_f32(kBlockM, unit_cols<MODE, BN>(w, p)) |
+                                       kAMajor;
+                const uint32_t a = lu % C::ACC_BUFS;
+                if (!mbar_wait_bounded(&tempty_bar[a], ((lu / C::ACC_BUFS) & 1u) ^ 1u, abort_flag,
                                        p.timeout_ns)) {
                     ok = false;
                     break;
@@ -452,8 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (v0 == 2 || v1 == 2 || v2 == 2 || v3 == 2) break;
             }
             const Unit w = decode_unit<MODE, BN>(u, n_first, p);
-            const uint32_t a = lu & 1u;
-            ok = mbar_wait_bounded(&tfull_bar[a], (lu >> 1) & 1u, abort_flag, p.timeout_ns);
+            const uint32_t a = lu % C::ACC_BUFS;
+            ok = mbar_wait_bounded(&tfull_bar[a], (lu / C::ACC_BUFS) & 1u, abort_flag,
+                                   p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (ModeTraits<MODE>::XCH) {
                 // The four warps meet at named barriers below: agree first.
@@ -471,8 +488,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
             const bool down = MODE == MODE_GEMM2 || MODE == MODE_GEMM2T || MODE == MODE_GEMM1T ||
                               (MODE == MODE_EXPERTS && w.phase == 1);
+            // Split unit (MODE_EXPERTS, few tiles): store this split's fp32
+            // partial, free the accumulator and count the arrival.  The split
+            // that arrives last sums the group's partials in split order and
+            // finishes the unit from that sum; the others are done.
+            const int ncol = unit_cols<MODE, BN>(w, p);  // same in the 4 epilogue warps
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = 0; c0 < ncol; c0 += 16) {
                 uint32_t g[16], v[16];
                 tmem_ld_16(tb + c0, g);
                 if (NUM_A == 2) tmem_ld_16(tb + BN + c0, v);
@@ -578,6 +600,11 @@ cudaError_t launch_bn(int bn, const TcMaps &maps, const TcGemmArgs &args, int gr
         case 32: return launch_cfg<MODE, 32>(maps, args, grid, stream);
         case 64: return launch_cfg<MODE, 64>(maps, args, grid, stream);
         case 128: return launch_cfg<MODE, 128>(maps, args, grid, stream);
+        case 256:  // prefill batches: the two expert GEMMs only
+            if constexpr (MODE == MODE_GEMM1 || MODE == MODE_GEMM2)
+                return launch_cfg<MODE, 256>(maps, args, grid, stream);
+            else
+                return cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
 }

@@ -122,8 +122,10 @@ class ExpertParallelLayer:
         return out
 
     def check(self):
-        """Device error words of this rank's calls (synchronises)."""
-        abi.check(self.dsc, self.ws)
+        """Device error words of this rank's calls (synchronises).  A rank
+        with no tokens launched nothing on its routing workspace."""
+        if self.T > 0:
+            abi.check(self.dsc, self.ws)
         if "dsc" in self._rows_ws:
             abi.check(self._rows_ws["dsc"], self._rows_ws["ws"])
 

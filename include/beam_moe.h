@@ -93,7 +93,8 @@ typedef struct {
  *   err       int32      device error word (0 = ok), read by beam_moe_check
  *   meta      int32[4]   [0] tiles in the tile list, [1] padded rows,
  *                        [2] kept pairs P, [3] work counter of the fused
- *                        expert kernel (units handed out so far)
+ *                        expert kernel (units handed out so far), or with
+ *                        256-row tiles the number of 128-row sub-tiles
  *   counts    int32[E]   kept pairs per expert
  *   hist      int32[K+1] tokens by number of kept candidates
  *   partial   f32[S][T][2E] router partial logits (S = router_splits)
@@ -109,17 +110,20 @@ typedef struct {
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
  *   y         f32[p_cap][d] expert output per pair
  *   hs        [n_shared*T][I_shared] shared experts' SwiGLU activations (dtype)
- *   ys        f32[n_shared*T][d] shared experts' outputs                    */
+ *   ys        f32[n_shared*T][d] shared experts' outputs
+ *   tiles_sub int32[][4] with 256-row tiles: the same rows as 128-row tiles,
+ *             the gate/up GEMM's units (their count in meta[3])            */
 typedef struct {
     int BN;            /* token rows per expert tile; the padding unit */
     int router_bn;     /* token rows per router tile */
     int router_splits; /* router split-K factor S */
     int p_cap;         /* rows of xp / h / y / pair */
     int tiles_cap;     /* entries of the tile list */
+    int sub_bn;        /* token rows of the gate/up GEMM's tiles (BN, or 128 when BN = 256) */
     int reserved;
     size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
         off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done, off_hs,
-        off_ys;
+        off_ys, off_tiles_sub;
     size_t workspace_bytes;
 } beam_moe_plan_info;
 

@@ -43,7 +43,7 @@ def test_plan_layout_is_consistent():
     for T in (0, 1, 8, 32, 128, 8192):
         dsc = abi.desc(T, 2048, 128, 768, 8, "bf16", 1)
         P = abi.plan(dsc)
-        assert P["BN"] in (16, 32, 64, 128)
+        assert P["BN"] in (16, 32, 64, 128, 256)
         assert P["p_cap"] == T * 8 + 128 * (P["BN"] - 1)
         offs = [P[k] for k in ("off_counts", "off_hist", "off_partial", "off_idx", "off_w",
                                "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h",
@@ -52,7 +52,9 @@ def test_plan_layout_is_consistent():
         assert P["off_y"] + 2 * P["p_cap"] * 2048 <= P["workspace_bytes"]
         assert abi.workspace_size(dsc) == P["workspace_bytes"]
         assert (2048 // 64) % P["router_splits"] == 0
-    assert abi.plan(abi.desc(8192, 2048, 128, 768, 8))["BN"] == 128
+    assert abi.plan(abi.desc(8192, 2048, 128, 768, 8))["BN"] == 256
+    assert abi.plan(abi.desc(2048, 2048, 128, 768, 8))["BN"] == 128
+    assert abi.plan(abi.desc(8192, 2048, 128, 768, 8, "f32"))["BN"] == 128
     assert abi.plan(abi.desc(128, 2048, 128, 768, 8))["BN"] == 16
 
 
@@ -145,7 +147,7 @@ def test_backward_split_limit_applies_to_fp32_only():
     backward; the bf16 layer runs them on the tensor cores and has one."""
     big_bf16 = abi.desc(1024, 8192, 8, 256, 2, "bf16", 1)
     big_f32 = abi.desc(1024, 8192, 8, 256, 2, "f32", 1)
-    assert abi.plan(big_bf16)["BN"] == 128 and abi.workspace_size(big_f32) > 0
+    assert abi.plan(big_bf16)["BN"] in (128, 256) and abi.workspace_size(big_f32) > 0
     assert abi.backward_workspace_size(big_bf16) > abi.workspace_size(big_bf16)
     assert abi.backward_kernel_count(big_bf16) == 15
     assert abi.backward_workspace_size(big_f32) == 0

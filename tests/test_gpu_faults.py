@@ -136,6 +136,7 @@ GUARD_SHAPES = [
     ("T600_E60", 600, 1024, 60, 256, 4, 0, 0.6, "bf16"),
     ("T37_qwen3", 37, 2048, 128, 768, 8, 1, 0.35, "bf16"),
     ("T2100_qwen3_prefill_tiles", 2100, 2048, 128, 768, 8, 1, 0.35, "bf16"),
+    ("T4100_qwen3_256row_tiles", 4100, 2048, 128, 768, 8, 1, 0.6, "bf16"),
     ("T37_tiny_f32", 37, 128, 8, 256, 2, 0, 0.5, "f32"),
 ]
 
