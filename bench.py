@@ -7,7 +7,7 @@ top-8, SwiGLU I=768, softmax renormalised over the Top-K, Zipf(1.1) expert
 skew, synthetic seeded data (dynamic_expert_routing_router_b200/inputs.py).
 The headline is T=128 tokens per step with the mask router keeping ~15% of the
 candidates (the paper's 1.23-of-8 operating point).  A step is one full layer
-forward (7 kernels) through the C ABI on one batch already resident in HBM;
+forward (5 kernels at decode sizes) through the C ABI on one batch already resident in HBM;
 8 distinct token batches are cycled and L2 is flushed (256 MiB write) before
 every timed step.  Each step is timed with CUDA events on the launch stream,
 recorded by the library between its kernels, so the per-kernel times come from
