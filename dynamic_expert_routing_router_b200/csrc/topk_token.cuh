@@ -12,7 +12,9 @@ namespace beam {
 // l+32, ...; K rounds of a warp arg-max (ties -> lower expert id) give the
 // candidates in descending order.  renorm: softmax over the candidates
 // (Eq. 4); else over all E.  Candidate k is kept iff its z >= thr = logit(tau)
-// (Eq. 6; NaN is not kept); w = g * m (Eq. 7).  Writes idx_t[k] / w_t[k] and,
+// (Eq. 6; NaN is not kept); w = g * m (Eq. 7).  A -inf gate logit weighs 0,
+// and a token whose candidates are all -inf gets weights 0 (its softmax is
+// 0/0; it then contributes nothing).  Writes idx_t[k] / w_t[k] and,
 // when given, cand_t[k] / gk_t[k]; adds to the shared counters.
 template <int EPL>
 __device__ __forceinline__ void topk_token(const float *lg, int E, int K, int renorm,
@@ -64,7 +66,9 @@ __device__ __forceinline__ void topk_token(const float *lg, int E, int K, int re
         }
         if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
         if (k == 0) rmax = bv;
-        const float ek = expf(bv - rmax);
+        // a -inf logit has weight 0 (Eq. 1); this also keeps a row whose
+        // every logit is -inf (rmax = -inf) free of inf - inf
+        const float ek = bv == -INFINITY ? 0.0f : expf(bv - rmax);
         denom += ek;
         if (lane == k) {
             my_cand = bi;
@@ -76,14 +80,14 @@ __device__ __forceinline__ void topk_token(const float *lg, int E, int K, int re
         float part = 0.0f;
 #pragma unroll
         for (int i = 0; i < EPL; ++i)
-            if (lane + 32 * i < E) part += expf(r[i] - rmax);
+            if (lane + 32 * i < E && r[i] != -INFINITY) part += expf(r[i] - rmax);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kAll, part, off);
         denom = part;  // identical on every lane (pairwise sums commute exactly)
     }
     const bool kept = (lane < K) && (!has_mask || my_z >= thr);
     if (lane < K) {
-        const float g = my_e / denom;
+        const float g = denom > 0.0f ? my_e / denom : 0.0f;  // every logit -inf: weights 0
         idx_t[lane] = kept ? my_cand : -1;
         w_t[lane] = kept ? g : 0.0f;
         if (kept) atomicAdd(&s_counts[my_cand], 1);

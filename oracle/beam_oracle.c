@@ -95,7 +95,9 @@ int oracle_route(int T, int E, int K, int renorm, double tau_logit, const double
     for (int t = 0; t < T && rc == 0; ++t) {
         const double *rt = r + (size_t)t * E;
         for (int e = 0; e < E; ++e) {
-            if (!isfinite(rt[e])) rc = -2;
+            /* -inf is a logit of weight 0 (Eq. 1 writes it for the experts
+             * outside the Top-K); NaN and +inf have no defined softmax. */
+            if (isnan(rt[e]) || rt[e] == INFINITY) rc = -2;
         }
         if (rc) break;
         /* Top-K: K rounds of "largest remaining logit, lowest index on ties". */
@@ -115,12 +117,19 @@ int oracle_route(int T, int E, int K, int renorm, double tau_logit, const double
          * candidates.  Shifted by the largest logit, which is rt[c[0]]. */
         double m = rt[c[0]];
         double denom = 0.0;
-        if (renorm) {
-            for (int k = 0; k < K; ++k) denom += exp(rt[c[k]] - m);
+        if (m == -INFINITY) {
+            /* READING: every candidate's logit is -inf, so Eq. (4) is 0/0; the
+             * candidates get weight 0 and the token contributes nothing, as an
+             * all-masked token does. */
+            for (int k = 0; k < K; ++k) gk[k] = 0.0;
         } else {
-            for (int e = 0; e < E; ++e) denom += exp(rt[e] - m);
+            if (renorm) {
+                for (int k = 0; k < K; ++k) denom += exp(rt[c[k]] - m);
+            } else {
+                for (int e = 0; e < E; ++e) denom += exp(rt[e] - m);
+            }
+            for (int k = 0; k < K; ++k) gk[k] = exp(rt[c[k]] - m) / denom;
         }
-        for (int k = 0; k < K; ++k) gk[k] = exp(rt[c[k]] - m) / denom;
         /* Binary mask on the candidates, then aggregation. */
         int kept = 0;
         for (int k = 0; k < K; ++k) {

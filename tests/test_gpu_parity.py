@@ -85,6 +85,36 @@ def test_tiny_f32_zero_mask_is_vanilla_topk_bitwise():
     assert_values(outn, ref, o["idx"], "f32")
 
 
+def test_tiny_f32_minus_inf_gate_row_gets_zero_weights():
+    """One token's gate logits overflow to -inf in fp32 (x[t,0] = 1e30 against
+    W_gate[:, 0] = -1e10): its softmax is 0/0, so its weights are 0 and its
+    output row is 0 -- no NaN anywhere.  Decisions bit-exact with the oracle
+    fed the same (partly -inf) logits; every other token as usual.  Feature 0
+    meets zero columns of W_mask, W1 and W3, so the rest of the layer stays
+    finite."""
+    gamma = json.load(open(os.path.join(HERE, "golden", "tiny_gamma.json")))["gamma"]
+    L = inputs.make_tiny(T=64, seed=0, gamma=gamma, device="cpu")
+    t0 = 17
+    L["x"][:, 0] = 0.0
+    L["x"][t0, 0] = 1e30
+    L["W_gate"][:, 0] = -1e10
+    L["W_mask"][:, 0] = 0.0
+    L["W1"][:, :, 0] = 0.0
+    L["W3"][:, :, 0] = 0.0
+    L = {k: v.to(DEV) for k, v in L.items()}
+    sh = inputs.TINY
+    dsc = abi.desc(64, sh.d, sh.E, sh.I, sh.K, "f32", sh.renorm)
+    g = gpu_route(dsc, L["x"], L["W_gate"], L["W_mask"])
+    assert np.isneginf(g["logits"][t0, :sh.E]).all()
+    assert np.isfinite(g["w"]).all() and (g["w"][t0] == 0).all()
+    o = oracle_from_logits(g["logits"], sh.E, sh.K, sh.renorm, True)
+    assert_routing_bitexact(g, o)
+    out, ws = gpu_forward(dsc, L["x"], L["W_gate"], L["W_mask"], L["W1"], L["W3"], L["W2"])
+    assert torch.isfinite(out).all() and (out[t0] == 0).all()
+    ref = oracle_values(L["x"], L["W1"], L["W3"], L["W2"], g["idx"], o["w"], "f32")
+    assert_values(out, ref, g["idx"], "f32")
+
+
 # ---------------------------------------------------------------- decode --
 
 DECODE = [(T, f) for T in (1, 8, 32, 128) for f in (0.15, 0.35, 0.6, 1.0)]

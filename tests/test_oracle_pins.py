@@ -457,3 +457,36 @@ def test_oracle_bf16_layer_matches_numpy_on_torch_decode():
             b = W3f[e] @ xf[t]
             want[t] += rt["w"][t, k] * (W2f[e] @ (_silu(a) * b))
     np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_minus_inf_gate_logits_weigh_zero():
+    """Eq. (1) writes -inf for the experts outside the Top-K, i.e. a -inf logit
+    has weight 0.  A row with some -inf logits: the finite ones follow
+    scipy's softmax as if the -inf entries were absent.  A row whose every
+    logit is -inf has no defined softmax (0/0): its weights are 0 (reading).
+    NaN and +inf are still rejected.
+
+    Catches: inf - inf reaching the weights, a NaN weight spreading into y."""
+    E, K = 6, 3
+    r = np.array([[1.0, -np.inf, 0.5, -np.inf, 2.0, -1.0],
+                  [-np.inf] * E,
+                  [0.3, 0.1, -0.2, 0.4, -np.inf, 0.0]])
+    for renorm in (0, 1):
+        out = oracle.route(r, None, K, renorm)
+        assert np.isfinite(out["w"]).all()
+        assert (out["w"][1] == 0).all() and list(out["cand"][1]) == [0, 1, 2]
+        for t in (0, 2):
+            fin = np.isfinite(r[t])
+            cand = out["cand"][t]
+            if renorm:
+                ref = softmax(r[t][cand])
+            else:
+                full = np.zeros(E)
+                full[fin] = softmax(r[t][fin])
+                ref = full[cand]
+            np.testing.assert_allclose(out["w"][t], ref, rtol=1e-15, atol=0)
+    for bad in (np.nan, np.inf):
+        rb = r.copy()
+        rb[0, 0] = bad
+        with pytest.raises(FloatingPointError):
+            oracle.route(rb, None, K, 1)
