@@ -351,71 +351,113 @@ def e2e_rate(layer, f, steps, warmup):
 
     Pipelined as a serving loop would run it: the input copy of step i+1 and the
     output copy of step i-1 run on two copy streams while step i computes
-    (device and pinned buffers double-buffered, events order every reuse).
-    `serial_value` is the same loop with everything on one stream."""
+    (device buffers double-buffered, events order every reuse).  Eight
+    consecutive steps (one per token batch) are captured into one CUDA graph,
+    which is replayed: each replay copies each of its eight steps' inputs from
+    pinned host memory and each step's output back, exactly as the eager loop
+    would, without the host's per-call launch time.  `eager_value` is the same
+    pipelined loop issued call by call from Python; `serial_value` the eager
+    loop on one stream."""
     torch = layer.torch
     abi = layer.abi
+    W = N_BATCHES
     hx = [x.cpu().pin_memory() for x in layer.xs]
     Wm = layer.mask(f)
-    comp = torch.cuda.current_stream()
-    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    comp, h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     xdev = [torch.empty_like(layer.xs[0]) for _ in range(2)]
     outd = [torch.empty_like(layer.out) for _ in range(2)]
     hout = [torch.empty(tuple(layer.out.shape), dtype=layer.out.dtype).pin_memory()
-            for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    for e in ev_done + ev_out:
-        e.record(comp)
+            for _ in range(W)]
 
-    def step(i):
-        b = i & 1
-        h2d.wait_event(ev_done[b])  # forward i-2 has finished reading xdev[b]
-        with torch.cuda.stream(h2d):
-            xdev[b].copy_(hx[i % N_BATCHES], non_blocking=True)
-        ev_in[b].record(h2d)
-        comp.wait_event(ev_in[b])
-        comp.wait_event(ev_out[b])  # output copy i-2 has finished reading outd[b]
-        abi.forward(layer.dsc, xdev[b], layer.Wg, Wm, layer.W1, layer.W3, layer.W2, outd[b],
-                    layer.ws, stream=comp)
-        ev_done[b].record(comp)
-        d2h.wait_event(ev_done[b])
-        with torch.cuda.stream(d2h):
-            hout[b].copy_(outd[b], non_blocking=True)
-        ev_out[b].record(d2h)
+    def pipelined(n, ev_done, ev_out):
+        """n steps; step i's buffers wait for step i-2's users (events)."""
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                h2d.wait_event(ev_done[i - 2])  # forward i-2 has finished reading xdev[b]
+            with torch.cuda.stream(h2d):
+                xdev[b].copy_(hx[i % W], non_blocking=True)
+            ev_in[i].record(h2d)
+            comp.wait_event(ev_in[i])
+            if i >= 2:
+                comp.wait_event(ev_out[i - 2])  # output copy i-2 has finished reading outd[b]
+            abi.forward(layer.dsc, xdev[b], layer.Wg, Wm, layer.W1, layer.W3, layer.W2, outd[b],
+                        layer.ws, stream=comp)
+            ev_done[i].record(comp)
+            d2h.wait_event(ev_done[i])
+            with torch.cuda.stream(d2h):
+                hout[i % W].copy_(outd[b], non_blocking=True)
+            ev_out[i].record(d2h)
 
-    def timed(fn, n):
+    def run_eager(n):
+        ev_done = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        h2d.wait_stream(comp)
+        d2h.wait_stream(comp)
+        pipelined(n, ev_done, ev_out)
+        comp.wait_stream(h2d)
+        comp.wait_stream(d2h)
+
+    # one graph of W pipelined steps (events recorded inside the capture only)
+    torch.cuda.synchronize()
+    for _ in range(2):  # warm-up outside the capture (tensor maps, attributes)
+        run_eager(W)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=comp):
+        fork = torch.cuda.Event()
+        fork.record(comp)
+        h2d.wait_event(fork)
+        d2h.wait_event(fork)
+        pipelined(W, [torch.cuda.Event() for _ in range(W)],
+                  [torch.cuda.Event() for _ in range(W)])
+        comp.wait_stream(h2d)
+        comp.wait_stream(d2h)
+    torch.cuda.synchronize()
+
+    def timed(fn):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record(comp)
-        h2d.wait_stream(comp)
-        d2h.wait_stream(comp)
-        for i in range(n):
-            fn(i)
-        comp.wait_stream(h2d)
-        comp.wait_stream(d2h)
+        fn()
         e1.record(comp)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) * 1e-3
 
-    def serial_step(i):
-        xdev[0].copy_(hx[i % N_BATCHES], non_blocking=True)
-        abi.forward(layer.dsc, xdev[0], layer.Wg, Wm, layer.W1, layer.W3, layer.W2, outd[0],
-                    layer.ws)
-        hout[0].copy_(outd[0], non_blocking=True)
+    replays = max(1, steps // W)
 
-    for i in range(warmup):
-        step(i)
-        serial_step(i)
-    torch.cuda.synchronize()
-    sec = timed(step, steps)
-    sec_serial = timed(serial_step, steps)
+    def run_graph():
+        with torch.cuda.stream(comp):
+            for _ in range(replays):
+                graph.replay()
+
+    for _ in range(max(1, warmup // W)):
+        run_graph()
+    sec = timed(run_graph)
+    n_steps = replays * W
+    sec_eager = timed(lambda: run_eager(n_steps))
+
+    def serial_loop():
+        with torch.cuda.stream(comp):
+            for i in range(n_steps):
+                xdev[0].copy_(hx[i % W], non_blocking=True)
+                abi.forward(layer.dsc, xdev[0], layer.Wg, Wm, layer.W1, layer.W3, layer.W2,
+                            outd[0], layer.ws, stream=comp)
+                hout[i % W].copy_(outd[0], non_blocking=True)
+
+    sec_serial = timed(serial_loop)
+    abi.check(layer.dsc, layer.ws, stream=comp)
+    del graph
     nbytes = layer.T * layer.sh.d * 2
-    return dict(value=layer.T * steps / sec, unit="tokens/s", h2d_bytes_per_step=nbytes,
-                d2h_bytes_per_step=nbytes, serial_value=layer.T * steps / sec_serial,
+    return dict(value=layer.T * n_steps / sec, unit="tokens/s", h2d_bytes_per_step=nbytes,
+                d2h_bytes_per_step=nbytes, steps=n_steps,
+                eager_value=layer.T * n_steps / sec_eager,
+                serial_value=layer.T * n_steps / sec_serial,
                 note=("pipelined: input copy of step i+1 and output copy of step i-1 on two "
-                      "copy streams during step i; serial_value: one stream"))
+                      "copy streams during step i; 8 consecutive steps per CUDA graph replay, "
+                      "every step's copies included; eager_value: the same loop issued from "
+                      "Python call by call; serial_value: one stream, eager"))
 
 
 def cpu_baseline(layer, f, seconds, max_batches=None):
