@@ -39,11 +39,11 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("BN", ctypes.c_int), ("router_bn", ctypes.c_int),
                 ("router_splits", ctypes.c_int), ("p_cap", ctypes.c_int),
                 ("tiles_cap", ctypes.c_int), ("sub_bn", ctypes.c_int),
-                ("reserved", ctypes.c_int)] + \
+                ("one_launch", ctypes.c_int)] + \
                [(n, ctypes.c_size_t) for n in (
                    "off_err", "off_meta", "off_counts", "off_hist", "off_partial", "off_idx",
                    "off_w", "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h", "off_y",
-                   "off_tile_done", "off_hs", "off_ys", "off_tiles_sub", "workspace_bytes")]
+                   "off_tile_done", "off_hs", "off_ys", "off_tiles_sub", "off_ctl", "workspace_bytes")]
 
 
 _lib = None
@@ -73,6 +73,8 @@ def lib():
         L.beam_moe_check.argtypes = [pd, vp, vp]
         L.beam_moe_route_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.beam_moe_route_noalloc.restype = i32
+        L.beam_moe_set_one_launch_tokens.argtypes = [i32]
+        L.beam_moe_set_one_launch_tokens.restype = i32
         L.beam_moe_forward_kernel_count.argtypes = [pd]
         L.beam_moe_forward_kernel_count.restype = i32
         L.beam_moe_backward_workspace_size.argtypes = [pd]
@@ -151,6 +153,11 @@ def stage_name(i: int):
 
 def workspace_size(dsc: Desc) -> int:
     return int(lib().beam_moe_workspace_size(ctypes.byref(dsc)))
+
+
+def set_one_launch_tokens(max_tokens: int) -> int:
+    """Largest batch run as one launch (0 = never); returns the previous value."""
+    return int(lib().beam_moe_set_one_launch_tokens(int(max_tokens)))
 
 
 def kernel_count(dsc: Desc) -> int:
@@ -311,6 +318,8 @@ def workspace_views(dsc, workspace) -> dict:
         meta=view(P["off_meta"], 4, torch.int32, 4),
         counts=view(P["off_counts"], E, torch.int32, 4),
         hist=view(P["off_hist"], K + 1, torch.int32, 4),
+        partial=view(P["off_partial"], P["router_splits"] * T * 2 * E, torch.float32, 4).view(
+            P["router_splits"], T, 2 * E),
         idx=view(P["off_idx"], T * K, torch.int32, 4).view(T, K),
         w=view(P["off_w"], T * K, torch.float32, 4).view(T, K),
         pair=view(P["off_pair"], P["p_cap"], torch.int32, 4),

@@ -33,6 +33,11 @@ unsigned long long wait_limit_ns() {
 }
 int fault_mode() { return g_fault.load(std::memory_order_relaxed); }
 
+// Largest batch that beam_moe_forward runs as one launch
+// (beam_moe_set_one_launch_tokens); the kernel itself takes up to kDlMaxT.
+constexpr int kOneLaunchDefaultTokens = 4;
+std::atomic<int> g_one_launch_tokens{kOneLaunchDefaultTokens};
+
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -77,6 +82,15 @@ int choose_bn(const beam_moe_desc *d, bool wide) {
     return 128;
 }
 
+// Small bf16 batches: the router logits come from the one-launch kernel's
+// router units (CUDA cores, one split) in every call -- forward, routing
+// only, backward -- so that all of them take the same decisions on the same
+// inputs.  `dl` receives the unit sizes for the call's mask and SM count.
+bool small_batch(const beam_moe_desc *d, int has_mask, int n_sm, DecodeLayerArgs *dl) {
+    return d->dtype == BEAM_BF16 &&
+           decode_layer_config(d->T, d->d, d->E, d->I, d->K, has_mask, n_sm, dl);
+}
+
 // `backward`: the training call's plan (its per-expert 128-row tile lists
 // need token tiles of at most 128 rows).
 beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P, bool backward = false) {
@@ -85,7 +99,14 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P, bool backwa
     std::memset(P, 0, sizeof(*P));
     const long long T = d->T, K = d->K, E = d->E;
     P->BN = choose_bn(d, d->dtype == BEAM_BF16 && !backward);
-    if (d->dtype == BEAM_BF16) {
+    DecodeLayerArgs dl;
+    const bool small = small_batch(d, 1, kNominalSMs, &dl);
+    P->one_launch = small && d->n_shared == 0 && !backward &&
+                    d->T <= g_one_launch_tokens.load(std::memory_order_relaxed);
+    if (small) {
+        P->router_bn = 16;  // unused: the router runs on CUDA cores
+        P->router_splits = 1;
+    } else if (d->dtype == BEAM_BF16) {
         // Router: enough (token tile x row block x split) units to cover the
         // SMs at decode sizes, while the split partials stay smaller than the
         // router weights; prefill needs no split.
@@ -133,7 +154,10 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P, bool backwa
     P->sub_bn = P->BN > kBlockM ? kBlockM : P->BN;
     P->off_tiles_sub = align256(P->off_ys + 4 * srows * size_t(d->d));
     const size_t sub_cap = P->BN > kBlockM ? size_t(cdiv(T * K, kBlockM) + E) : 0;
-    o = align256(P->off_tiles_sub + 16 * sub_cap);
+    // one-launch counters: per expert, then per (token, down row block)
+    P->off_ctl = align256(P->off_tiles_sub + 16 * sub_cap);
+    const size_t ctl = small ? size_t(E) + size_t(T) * size_t(d->d / dl.R2) : 0;
+    o = align256(P->off_ctl + 4 * ctl);
     P->workspace_bytes = o;
     return BEAM_OK;
 }
@@ -177,9 +201,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 struct TmapKey {
     const void *base;
     unsigned long long inner, rows;
-    unsigned box_rows;
+    unsigned box_rows, chunks;
     bool operator==(const TmapKey &o) const {
-        return base == o.base && inner == o.inner && rows == o.rows && box_rows == o.box_rows;
+        return base == o.base && inner == o.inner && rows == o.rows && box_rows == o.box_rows &&
+               chunks == o.chunks;
     }
 };
 struct TmapCache {
@@ -203,9 +228,12 @@ TmapCache &tmap_cache() {
     return c;
 }
 
+// chunks > 0: a 3D view [inner / 64][rows][64] of the same matrix whose box
+// is `chunks` consecutive 64-column chunks of box_rows rows: one copy lands
+// them as `chunks` swizzled 64-column boxes, one after another.
 bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
-               unsigned long long rows, unsigned box_rows) {
-    const TmapKey key{base, inner, rows, box_rows};
+               unsigned long long rows, unsigned box_rows, unsigned chunks = 0) {
+    const TmapKey key{base, inner, rows, box_rows, chunks};
     TmapCache &c = tmap_cache();
     const int set = TmapCache::set_of(key);
     {
@@ -218,13 +246,25 @@ bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
     }
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn || rows == 0) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * 2};
-    cuuint32_t box[2] = {unsigned(kBlockK), box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r;
+    if (chunks == 0) {
+        cuuint64_t dims[2] = {inner, rows};
+        cuuint64_t strides[1] = {inner * 2};
+        cuuint32_t box[2] = {unsigned(kBlockK), box_rows};
+        cuuint32_t estr[2] = {1, 1};
+        r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        if (inner % kBlockK != 0) return false;
+        cuuint64_t dims[3] = {unsigned(kBlockK), rows, inner / kBlockK};
+        cuuint64_t strides[2] = {inner * 2, kBlockK * 2};
+        cuuint32_t box[3] = {unsigned(kBlockK), box_rows, chunks};
+        cuuint32_t estr[3] = {1, 1, 1};
+        r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     if (r != CUDA_SUCCESS) return false;
     std::lock_guard<std::mutex> lk(c.mu);
     auto &slot = c.e[set][c.next[set]];
@@ -275,7 +315,23 @@ beam_status launch_route(const beam_moe_desc *d, const beam_moe_plan_info &P, co
     int *hdr = reinterpret_cast<int *>(ws);
     ZeroRegion zero[3] = {{hdr + kHdrMeta, 4}, {ro.counts, d->E}, {ro.hist, ro.hist ? d->K + 1 : 0}};
     BEAM_TRY_CUDA(rec.rec(0));
-    if (d->dtype == BEAM_BF16) {
+    DecodeLayerArgs dl;
+    if (small_batch(d, Wm != nullptr, n_sm, &dl)) {
+        dl.mode = DL_ROUTER_ONLY;
+        dl.x = x;
+        dl.Wg = Wg;
+        dl.Wm = Wm;
+        dl.partial = partial;
+        dl.hdr = hdr;
+        dl.zero[0] = zero[0];
+        dl.zero[1] = zero[1];
+        dl.zero[2] = zero[2];
+        dl.fault_skip = fault_mode() == FAULT_ROUTER_STAGE ? FAULT_ROUTER_STAGE : FAULT_NONE;
+        dl.timeout_ns = wait_limit_ns();
+        DlMaps none;
+        std::memset(&none, 0, sizeof(none));  // the router items read no tensor map
+        BEAM_TRY_CUDA(launch_decode_layer(none, dl, dl.n_ru < n_sm ? dl.n_ru : n_sm, st));
+    } else if (d->dtype == BEAM_BF16) {
         TcMaps maps;
         if (!make_tmap(&maps.a0, Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
         if (!make_tmap(&maps.a1, Wm ? Wm : Wg, d->d, d->E, kBlockM)) return BEAM_ERR_CUDA;
@@ -544,6 +600,51 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
     int *hist = reinterpret_cast<int *>(ws + P.off_hist);
     int *idx = reinterpret_cast<int *>(ws + P.off_idx);
     float *w = reinterpret_cast<float *>(ws + P.off_w);
+
+    if (P.one_launch) {
+        DecodeLayerArgs dl;
+        if (!small_batch(d, Wm != nullptr, n_sm, &dl)) return BEAM_ERR_INTERNAL;
+        dl.mode = DL_FORWARD;
+        dl.renorm = d->renorm_topk;
+        dl.thr = d->mask_logit_threshold;
+        dl.x = x;
+        dl.Wg = Wg;
+        dl.Wm = Wm;
+        dl.W1 = W1;
+        dl.W3 = W3;
+        dl.W2 = W2;
+        dl.out = out;
+        dl.partial = reinterpret_cast<float *>(ws + P.off_partial);
+        dl.idx = idx;
+        dl.w = w;
+        dl.counts = counts;
+        dl.hist = hist;
+        dl.pair = reinterpret_cast<int *>(ws + P.off_pair);
+        dl.pair_pos = reinterpret_cast<int *>(ws + P.off_pair_pos);
+        dl.tiles = reinterpret_cast<int4 *>(ws + P.off_tiles);
+        dl.BN = P.BN;
+        dl.H = ws + P.off_h;
+        dl.Y = reinterpret_cast<float *>(ws + P.off_y);
+        dl.hdr = reinterpret_cast<int *>(ws);
+        dl.e1_done = reinterpret_cast<int *>(ws + P.off_ctl);
+        dl.comb_cnt = dl.e1_done + d->E;
+        dl.fault_skip = fault_mode();
+        dl.timeout_ns = wait_limit_ns();
+        DlMaps maps;
+        // boxes: 8 rows x 4 chunks (W1, W3), 16 rows x 2 chunks (W2, H)
+        if (!make_tmap(&maps.w1, W1, d->d, (unsigned long long)d->E * d->I, 8, 4) ||
+            !make_tmap(&maps.w3, W3, d->d, (unsigned long long)d->E * d->I, 8, 4) ||
+            !make_tmap(&maps.w2, W2, d->I, (unsigned long long)d->E * d->d, 16, 2) ||
+            !make_tmap(&maps.h, ws + P.off_h, d->I, P.p_cap, 16, 2))
+            return BEAM_ERR_CUDA;
+        BEAM_TRY_CUDA(rec.rec(0));
+        // The kernel's counters start from zero: the header (error words,
+        // meta, router count) is cleared here; CTA 0 clears the rest.
+        BEAM_TRY_CUDA(cudaMemsetAsync(ws, 0, P.off_counts, st));
+        BEAM_TRY_CUDA(launch_decode_layer(maps, dl, n_sm, st));
+        for (int i = 1; i <= BEAM_MOE_FORWARD_STAGES; ++i) BEAM_TRY_CUDA(rec.rec(i));
+        return BEAM_OK;
+    }
 
     const RouteOut ro{idx, w, counts, hist, nullptr};
     s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
@@ -1104,10 +1205,16 @@ const char *beam_status_str(beam_status status) {
     return "BEAM_ERR_UNKNOWN";
 }
 
+int beam_moe_set_one_launch_tokens(int max_tokens) {
+    const int v = max_tokens < 0 ? 0 : max_tokens > kDlMaxT ? kDlMaxT : max_tokens;
+    return g_one_launch_tokens.exchange(v, std::memory_order_relaxed);
+}
+
 int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     beam_moe_plan_info P;
     if (make_plan(desc, &P) != BEAM_OK) return 0;
     if (desc->T == 0) return 0;
+    if (P.one_launch) return 1;
     const int shared = desc->n_shared > 0 ? 2 : 0;
     // Fused decode path: rows copied by the grouping kernel (no gather
     // launch) and one launch for both expert GEMMs.

@@ -197,6 +197,69 @@ cudaError_t launch_ep_dispatch(const EpDispatchArgs &a, cudaStream_t stream);
 cudaError_t launch_set_routing(const int *expert_id, int N, int E, int *idx, float *w, int *counts,
                                int *hist, int *err, int n_sm, cudaStream_t stream);
 
+// ---------------------------------------------------------------------------
+// The whole layer of a small decode batch in one launch (decode_layer.cu).
+// One persistent CTA per SM (15 consumer warps and one producer warp); the
+// phases hand off through counters in the workspace, never through a kernel
+// boundary:
+//   router items   2 rows of [W_gate; W_mask] against every token -> logits
+//   routing        every CTA reads all logits and takes the same top-K, mask
+//                  and grouping in shared memory (no second hand-off)
+//   gate/up items  one row of W1 and of W3 of one kept expert -> H[., i]
+//   down items     R2 rows of W2 of one kept expert -> columns of Y; the item
+//                  that completes a (token, row block) of the output sums the
+//                  token's kept rows of Y in slot order (the combine)
+// The producer streams each item's rows (bulk copies) into a ring of
+// shared-memory stages ahead of the consumer warps.
+constexpr int kDlThreads = 512;        // 15 consumer warps + 1 producer warp
+constexpr int kDlMaxT = 16;             // tokens per call on this path
+constexpr int kDlMaxStages = 32;
+constexpr int kDlSmemCap = 200 * 1024;  // dynamic shared memory budget
+constexpr int kHdrDlRouter = 8;         // header int: router units published
+
+enum : int { DL_FORWARD = 0, DL_ROUTER_ONLY = 1 };
+
+struct DecodeLayerArgs {
+    int mode;                    // DL_FORWARD, or DL_ROUTER_ONLY (logits only)
+    int T, d, E, I, K, renorm, has_mask;
+    float thr;                   // keep iff z >= thr
+    const void *x, *Wg, *Wm, *W1, *W3, *W2;  // bf16
+    void *out;                   // bf16 [T][d]
+    float *partial;              // [T][2E] logits (one split)
+    int *idx;                    // [T][K]
+    float *w;                    // [T][K]
+    int *counts, *hist;          // [E], [K+1]
+    int *pair, *pair_pos;        // grouping rows (BN-padded per expert)
+    int4 *tiles;
+    int BN;
+    void *H;                     // bf16 [rows][I]
+    float *Y;                    // [rows][d]
+    int *hdr;                    // workspace header (error words, meta, router counter)
+    int *e1_done;                // [E] gate/up units finished per expert
+    int *comb_cnt;               // [T][d / R2] down items finished per (token, row block)
+    ZeroRegion zero[3];          // router-only mode: regions CTA 0 clears
+    int rr, n_ru;                // rows per router item, router items
+    int R1, R2;                  // rows per gate/up item (of I), per down item (of d)
+    int n_stages, stage_bytes;
+    int sm_off_lg, sm_off_stage, smem_bytes;  // dynamic shared memory layout
+    int fault_skip;              // tests: FAULT_* of this call
+    unsigned long long timeout_ns;
+};
+
+// Shape limits and unit sizes of the one-launch path; false if the shape does
+// not fit it (the caller then takes the multi-kernel path).
+bool decode_layer_config(int T, int d, int E, int I, int K, int has_mask, int n_sm,
+                         DecodeLayerArgs *cfg);
+// Tensor maps of the expert weights and of H for the one-launch path's tiles
+// (128-byte swizzle, boxes of 64 columns): W1 and W3 [E*I, d] with boxes of
+// 8 rows, W2 [E*d, I] and H [rows, I] with boxes of 16 rows.  Router-only
+// launches do not read them.
+struct DlMaps {
+    CUtensorMap w1, w3, w2, h;
+};
+cudaError_t launch_decode_layer(const DlMaps &maps, const DecodeLayerArgs &a, int grid,
+                                cudaStream_t stream);
+
 // Gather token rows into expert order (row_bytes multiple of 16).
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
                           long long row_bytes, int p_cap, void *xp, int n_sm,

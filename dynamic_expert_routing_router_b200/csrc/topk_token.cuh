@@ -39,39 +39,46 @@ __device__ __forceinline__ void topk_token(const float *lg, int E, int K, int re
         }
     }
 
+    // Selection keys: larger logit -> larger unsigned key (-0 counts as +0,
+    // since the two compare equal); 0 marks an entry that can no longer win.
+    // Each round takes the largest key over the warp with one redux.sync and
+    // the lowest expert id holding it with another (ties -> lower id).
+    unsigned key[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const float v = r[i] == 0.0f ? 0.0f : r[i];
+        const unsigned b = __float_as_uint(v);
+        key[i] = ((taken >> i) & 1u) ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
+    }
     int my_cand = -1;
     float my_e = 0.0f, my_z = 0.0f, rmax = 0.0f, denom = 0.0f;
     for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY, bz = 0.0f;
+        unsigned bk = 0u;
         int bi = INT_MAX;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int j = lane + 32 * i;
-            if (!((taken >> i) & 1u) && (r[i] > bv || (r[i] == bv && j < bi))) {
-                bv = r[i];
-                bi = j;
-                bz = z[i];
+        for (int i = 0; i < EPL; ++i)
+            if (key[i] > bk) {  // i ascending: the lowest id among equal keys
+                bk = key[i];
+                bi = lane + 32 * i;
             }
-        }
+        const unsigned wk = __reduce_max_sync(kAll, bk);
+        const int wi = int(__reduce_min_sync(kAll, bk == wk ? unsigned(bi) : 0xffffffffu));
+        const float bv = __uint_as_float((wk & 0x80000000u) ? (wk & 0x7fffffffu) : ~wk);
+        float oz = 0.0f;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(kAll, bv, off);
-            const int oi = __shfl_xor_sync(kAll, bi, off);
-            const float oz = __shfl_xor_sync(kAll, bz, off);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-                bz = oz;
+        for (int i = 0; i < EPL; ++i)
+            if (lane + 32 * i == wi) {
+                oz = z[i];
+                key[i] = 0u;
             }
-        }
-        if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
+        const float bz = __shfl_sync(kAll, oz, wi & 31);
         if (k == 0) rmax = bv;
         // a -inf logit has weight 0 (Eq. 1); this also keeps a row whose
         // every logit is -inf (rmax = -inf) free of inf - inf
         const float ek = bv == -INFINITY ? 0.0f : expf(bv - rmax);
         denom += ek;
         if (lane == k) {
-            my_cand = bi;
+            my_cand = wi;
             my_e = ek;
             my_z = bz;
         }

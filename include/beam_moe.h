@@ -112,7 +112,12 @@ typedef struct {
  *   hs        [n_shared*T][I_shared] shared experts' SwiGLU activations (dtype)
  *   ys        f32[n_shared*T][d] shared experts' outputs
  *   tiles_sub int32[][4] with 256-row tiles: the same rows as 128-row tiles,
- *             the gate/up GEMM's units (their count in meta[3])            */
+ *             the gate/up GEMM's units (their count in meta[3])
+ *   ctl       int32[]     one-launch path: gate/up units finished per expert,
+ *                         down units finished per (token, output row block)
+ * With one_launch the layer runs as one kernel that writes err, meta,
+ * counts, hist, partial (one split), idx, w, pair, pair_pos, tiles, h and y
+ * as above; xp, tile_done, hs, ys and tiles_sub are not used.             */
 typedef struct {
     int BN;            /* token rows per expert tile; the padding unit */
     int router_bn;     /* token rows per router tile */
@@ -120,10 +125,10 @@ typedef struct {
     int p_cap;         /* rows of xp / h / y / pair */
     int tiles_cap;     /* entries of the tile list */
     int sub_bn;        /* token rows of the gate/up GEMM's tiles (BN, or 128 when BN = 256) */
-    int reserved;
+    int one_launch;    /* 1: beam_moe_forward runs the whole layer as one kernel */
     size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
         off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done, off_hs,
-        off_ys, off_tiles_sub;
+        off_ys, off_tiles_sub, off_ctl;
     size_t workspace_bytes;
 } beam_moe_plan_info;
 
@@ -240,6 +245,18 @@ beam_status beam_moe_route_noalloc_check(void *stream);
  * decode-sized token tiles) or 7, plus 2 with shared experts; 0 for T = 0 or
  * a bad descriptor. */
 int beam_moe_forward_kernel_count(const beam_moe_desc *desc);
+
+/* Tuning switch of the one-launch path (plan field one_launch): bf16 calls
+ * without shared experts and with at most max_tokens tokens (and at most 16,
+ * whose token rows, logits and weight stages fit one CTA's shared memory)
+ * run router, top-K + mask, grouping, both expert projections and the
+ * combine as ONE kernel whose phases hand off through counters in the
+ * workspace.  Larger batches take the multi-kernel path.  0 turns it off.
+ * Default 4: the batch sizes where it was measured faster.  Returns the
+ * previous value; process-wide, not per call.  Routing at those sizes (and
+ * only the routing) is the same in both paths: the router logits of every
+ * bf16 call with T <= 16 come from the same router code. */
+int beam_moe_set_one_launch_tokens(int max_tokens);
 
 /* ------------------------------------------------------------ training --
  * Backward pass of the layer for training the mask router (techwalker news

@@ -95,9 +95,11 @@ def assert_grouping_bitexact(dsc, views, idx):
 
 
 def bf16_half_ulp(a):
-    """Half a unit in the last place of bfloat16 (8 significant bits) at |a|."""
+    """Half a unit in the last place of bfloat16 (8 significant bits) at |a|;
+    below the smallest normal, 2^-126, the spacing stays that of the
+    subnormals, 2^-133."""
     a = np.abs(np.asarray(a, np.float64))
-    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), -126.0)
     return np.where(a > 0, np.exp2(e - 8), 0.0)
 
 
@@ -220,7 +222,12 @@ def assert_combine(out, views, dtype, n_shared=0, ys=None):
     if dtype == "bf16":
         tol = tol + bf16_half_ulp(np.maximum(np.abs(o), np.abs(ref)))
     bad = np.abs(o - ref) > tol
-    assert not bad.any(), f"combine differs at {np.argwhere(bad)[:5].tolist()}"
+    if bad.any():
+        at = np.argwhere(bad)[:5]
+        detail = [(int(i), int(j), float(o[i, j]), float(ref[i, j]), float(tol[i, j]))
+                  for i, j in at]
+        raise AssertionError(f"combine differs at {int(bad.sum())} elements, first "
+                             f"(t, j, out, ref, tol): {detail}")
     empty = (idx < 0).all(axis=1)
     if not n_shared:
         assert (o[empty] == 0).all()

@@ -115,6 +115,43 @@ def test_kernel_count_per_path():
     assert abi.kernel_count(abi.desc(4, 2000, 128, 768, 8, "bf16", 1)) == 0
 
 
+def test_one_launch_path_selection():
+    """bf16 batches of at most 16 tokens whose token rows, logits and weight
+    stages fit one CTA's shared memory can run the whole layer as one kernel
+    (by default up to 4 tokens: beam_moe_set_one_launch_tokens); the router of
+    every bf16 call at those sizes then runs unsplit (one partial)."""
+    prev = abi.set_one_launch_tokens(16)
+    try:
+        for T in (1, 8, 16):
+            dsc = abi.desc(T, 2048, 128, 768, 8, "bf16", 1)
+            P = abi.plan(dsc)
+            assert P["one_launch"] == 1 and abi.kernel_count(dsc) == 1
+            assert P["router_splits"] == 1
+            # counters: one per expert, one per (token, 16-row block of d)
+            assert P["off_ctl"] + 4 * (128 + T * 2048 // 16) <= P["workspace_bytes"]
+            assert P["off_ctl"] >= P["off_tiles_sub"] and P["off_ctl"] % 256 == 0
+        big = abi.plan(abi.desc(17, 2048, 128, 768, 8, "bf16", 1))
+        assert big["one_launch"] == 0 and big["off_ctl"] + 0 <= big["workspace_bytes"]
+        assert abi.kernel_count(abi.desc(17, 2048, 128, 768, 8, "bf16", 1)) == 5
+        # d = 7168, E = 256: one token fits, sixteen do not (their rows take 224 KB)
+        assert abi.plan(abi.desc(1, 7168, 256, 2048, 8, "bf16", 0))["one_launch"] == 1
+        assert abi.plan(abi.desc(16, 7168, 256, 2048, 8, "bf16", 0))["one_launch"] == 0
+        # the switch: 0 turns the path off; the default takes up to 4 tokens
+        abi.set_one_launch_tokens(0)
+        assert abi.plan(abi.desc(1, 2048, 128, 768, 8, "bf16", 1))["one_launch"] == 0
+        assert abi.plan(abi.desc(1, 2048, 128, 768, 8, "bf16", 1))["router_splits"] == 1
+        abi.set_one_launch_tokens(4)
+        assert abi.plan(abi.desc(4, 2048, 128, 768, 8, "bf16", 1))["one_launch"] == 1
+        assert abi.plan(abi.desc(5, 2048, 128, 768, 8, "bf16", 1))["one_launch"] == 0
+        assert abi.set_one_launch_tokens(99) == 4 and abi.set_one_launch_tokens(4) == 16
+    finally:
+        abi.set_one_launch_tokens(prev)
+    # fp32, shared experts and the backward's plan keep the multi-kernel path
+    assert abi.plan(abi.desc(4, 128, 8, 256, 2, "f32", 0))["one_launch"] == 0
+    sh = abi.desc(4, 2048, 64, 1408, 6, "bf16", 1, n_shared=2, I_shared=1408)
+    assert abi.plan(sh)["one_launch"] == 0 and abi.plan(sh)["router_splits"] == 1
+
+
 def test_nan_mask_threshold_is_rejected():
     dsc = abi.desc(4, 2048, 128, 768, 8, "bf16", 1)
     dsc.mask_logit_threshold = float("nan")

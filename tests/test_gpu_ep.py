@@ -118,9 +118,15 @@ def test_expert_parallel_matches_oracle_and_one_gpu(name, sh, G, Ts, f):
         # values: oracle at the bf16 bar, every token
         ref = oracle.experts(host(x), h1, h3, h2, idx, o["w"], "bf16")
         worst = assert_values(out, ref, idx, "bf16")
-        # and the one-GPU layer on the same tokens
+        # and the one-GPU layer on the same tokens, on the multi-kernel path
+        # (the one the expert-parallel steps distribute; the one-launch path
+        # of small batches computes the same values in another order)
         one = torch.empty_like(out)
-        abi.forward(dsc, x, R["Wg"], R["Wm"], W1, W3, W2, one, ws)
+        prev = abi.set_one_launch_tokens(0)
+        try:
+            abi.forward(dsc, x, R["Wg"], R["Wm"], W1, W3, W2, one, ws)
+        finally:
+            abi.set_one_launch_tokens(prev)
         abi.check(dsc, ws)
         report(name=f"ep_{name}_rank{r}", kind="ep", T=T, worst_token_excess=worst,
                bitwise_equal_to_one_gpu=bool(torch.equal(out, one)),

@@ -19,6 +19,15 @@ from dynamic_expert_routing_router_b200 import abi, inputs
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(autouse=True, scope="module")
+def one_launch_up_to_16_tokens():
+    """Every batch of at most 16 tokens takes the one-launch path here (the
+    library's default stops at 4)."""
+    prev = abi.set_one_launch_tokens(16)
+    yield
+    abi.set_one_launch_tokens(prev)
+
 DEV = "cuda"
 WAIT_LIMIT_NS = 50_000_000  # 50 ms instead of 1 s per bounded wait
 
@@ -45,7 +54,8 @@ def _layer(sh, T, f, seed=0):
     return x, Wg, Wm, W1, W3, W2
 
 
-@pytest.mark.parametrize("T", [32, 2048], ids=["decode_fused_experts", "prefill_gate_up_gemm"])
+@pytest.mark.parametrize("T", [4, 32, 2048],
+                         ids=["decode_one_launch", "decode_fused_experts", "prefill_gate_up_gemm"])
 def test_expert_wait_timeout_is_reported_then_recovers(T):
     sh = inputs.QWEN3
     x, Wg, Wm, W1, W3, W2 = _layer(sh, T, 0.35)
@@ -135,6 +145,8 @@ GUARD_SHAPES = [
     ("T37_E60", 37, 1024, 60, 256, 4, 1, 0.35, "bf16"),
     ("T600_E60", 600, 1024, 60, 256, 4, 0, 0.6, "bf16"),
     ("T37_qwen3", 37, 2048, 128, 768, 8, 1, 0.35, "bf16"),
+    ("T16_qwen3_one_launch", 16, 2048, 128, 768, 8, 1, 0.35, "bf16"),
+    ("T5_E60_one_launch", 5, 2048, 60, 1408, 4, 0, 0.35, "bf16"),
     ("T2100_qwen3_prefill_tiles", 2100, 2048, 128, 768, 8, 1, 0.35, "bf16"),
     ("T4100_qwen3_256row_tiles", 4100, 2048, 128, 768, 8, 1, 0.6, "bf16"),
     ("T37_tiny_f32", 37, 128, 8, 256, 2, 0, 0.5, "f32"),
