@@ -156,7 +156,8 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P, bool backwa
     const size_t sub_cap = P->BN > kBlockM ? size_t(cdiv(T * K, kBlockM) + E) : 0;
     // one-launch counters: per expert, then per (token, down row block)
     P->off_ctl = align256(P->off_tiles_sub + 16 * sub_cap);
-    const size_t ctl = small ? size_t(E) + size_t(T) * size_t(d->d / dl.R2) : 0;
+    const size_t ctl = small ? size_t(E) * size_t(d->I / 128) + size_t(T) * size_t(d->d / dl.R2)
+                             : 0;
     o = align256(P->off_ctl + 4 * ctl);
     P->workspace_bytes = o;
     return BEAM_OK;
@@ -627,7 +628,7 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         dl.Y = reinterpret_cast<float *>(ws + P.off_y);
         dl.hdr = reinterpret_cast<int *>(ws);
         dl.e1_done = reinterpret_cast<int *>(ws + P.off_ctl);
-        dl.comb_cnt = dl.e1_done + d->E;
+        dl.comb_cnt = dl.e1_done + d->E * (d->I / 128);
         dl.fault_skip = fault_mode();
         dl.timeout_ns = wait_limit_ns();
         DlMaps maps;

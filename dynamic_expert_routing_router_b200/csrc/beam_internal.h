@@ -214,7 +214,7 @@ cudaError_t launch_set_routing(const int *expert_id, int N, int E, int *idx, flo
 constexpr int kDlThreads = 512;        // 15 consumer warps + 1 producer warp
 constexpr int kDlMaxT = 16;             // tokens per call on this path
 constexpr int kDlMaxStages = 32;
-constexpr int kDlSmemCap = 200 * 1024;  // dynamic shared memory budget
+constexpr int kDlSmemCap = 196 * 1024;  // dynamic shared memory budget
 constexpr int kHdrDlRouter = 8;         // header int: router units published
 
 enum : int { DL_FORWARD = 0, DL_ROUTER_ONLY = 1 };
@@ -235,7 +235,7 @@ struct DecodeLayerArgs {
     void *H;                     // bf16 [rows][I]
     float *Y;                    // [rows][d]
     int *hdr;                    // workspace header (error words, meta, router counter)
-    int *e1_done;                // [E] gate/up units finished per expert
+    int *e1_done;                // [E][I / 128] gate/up units finished per block of H
     int *comb_cnt;               // [T][d / R2] down items finished per (token, row block)
     ZeroRegion zero[3];          // router-only mode: regions CTA 0 clears
     int rr, n_ru;                // rows per router item, router items

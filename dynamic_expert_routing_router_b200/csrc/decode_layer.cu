@@ -207,7 +207,7 @@ struct Routing {  // the routing and grouping of the call, in shared memory
 // of d for down) and number of k-tiles.
 struct Unit {
     bool up;
-    int e, row0, nkt;
+    int e, ti, row0, nkt;  // ti: the expert's index among the touched experts
 };
 
 }  // namespace
@@ -223,7 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ __align__(8) uint64_t x_bar;
     __shared__ Routing R;
     __shared__ int s_abort;
-    __shared__ int s_done[kMaxE];                   // gate/up units finished here, per expert
+    // gate/up units finished here per (touched expert, 128-column block of
+    // H): one byte each (at most 16), four blocks to a word
+    __shared__ unsigned s_done[kMaxE][4];
     __shared__ float s_rp[kConsumers][2][kDlMaxT];  // router partial sums, per warp
     // A unit's k-tiles are items of their own, taken by any warp; their partial
     // sums meet in the unit's slot (slot j % kSlots), added in k-tile order:
@@ -235,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int T = a.T, d = a.d, E = a.E, I = a.I, K = a.K, NS = a.n_stages;
     const int n_rows_router = a.has_mask ? 2 * E : E;
     const int U1 = I / 8, U2 = d / 16;                      // units per expert
+    const int NB = I / kKT2;  // 128-column blocks of H, 16 gate/up units each
     const int NKT1 = (d + kKT1 - 1) / kKT1, NKT2 = I / kKT2;  // k-tiles per unit
     const int XSP = d + 8;                                  // token row pitch, elements
     const size_t SB = size_t(a.stage_bytes);
@@ -265,7 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < E; i += kThreads) {
         R.cnt[i] = 0;
         R.tmask[i] = 0u;
-        s_done[i] = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) s_done[i][w] = 0u;
     }
     if (tid <= K) R.hist[tid] = 0;
     if (tid == 0) s_abort = 0;
@@ -278,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // barrier below, so every other CTA sees them cleared.
     if (b == 0) {
         if (forward) {
-            for (int i = tid; i < E; i += kThreads) a.e1_done[i] = 0;
+            for (int i = tid; i < E * NB; i += kThreads) a.e1_done[i] = 0;
             for (int i = tid; i < T * U2; i += kThreads) a.comb_cnt[i] = 0;
         } else {
 #pragma unroll
@@ -302,12 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         Unit u;
         u.up = h < n1u;
         if (u.up) {
-            u.e = R.te[h / U1];
+            u.ti = h / U1;
+            u.e = R.te[u.ti];
             u.row0 = (h % U1) * 8;
             u.nkt = NKT1;
         } else {
             const int v = h - n1u;
-            u.e = R.te[v / U2];
+            u.ti = v / U2;
+            u.e = R.te[u.ti];
             u.row0 = (v % U2) * 16;
             u.nkt = NKT2;
         }
@@ -383,16 +389,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the gate/up phase runs.  Down tiles waiting for their H
             // (`pend`, at most M) get it before this lane waits for a stage
             // to free up (it may be one of theirs) and at the end.
-            int waited_e = -1;  // the last expert whose H this lane saw complete
             int pend_s[2], pend_e[2], pend_k[2], pend_h[2], npend = 0;
             auto flush = [&]() -> bool {
                 for (int p = 0; p < npend; ++p) {
-                    if (pend_e[p] != waited_e) {
-                        if (!wait_count(a.e1_done + pend_e[p], U1, err, abort_flag, a.timeout_ns))
-                            return false;
-                        asm volatile("fence.proxy.async.global;" ::: "memory");  // H: async reads
-                        waited_e = pend_e[p];
-                    }
+                    // this tile's 128 columns of H: complete once the 16 gate/up
+                    // units that write them are published
+                    if (!wait_count(a.e1_done + pend_e[p] * NB + pend_k[p] / kKT2, 16, err,
+                                    abort_flag, a.timeout_ns))
+                        return false;
+                    asm volatile("fence.proxy.async.global;" ::: "memory");  // H: async reads
                     tma_load_3d(stage0 + size_t(pend_s[p]) * SB + 4096, &maps.h, 0, pend_h[p],
                                 pend_k[p] / 64, &full_bar[pend_s[p]]);
                 }
@@ -450,29 +455,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!forward) return;
         all_sync();
         if (*abort_flag) return;
-        const int NT = R.n_touched, n1u = NT * U1;
+        const int NT = R.n_touched, n1u = NT * U1, NBW = (NB + 3) / 4;
         const int my_e1u = b < n1u ? (n1u - 1 - b) / G + 1 : 0;
-        int pub[kMaxE / 32];
+        unsigned pub[kMaxE / 32][4];  // counts already published, same packing
 #pragma unroll
-        for (int k = 0; k < kMaxE / 32; ++k) pub[k] = 0;
+        for (int k = 0; k < kMaxE / 32; ++k)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) pub[k][w] = 0u;
         int published = 0;
         uint64_t t0 = globaltimer_ns();
         while (published < my_e1u) {
-            int dk[kMaxE / 32], mine = 0;
+            bool any = false;
 #pragma unroll
             for (int k = 0; k < kMaxE / 32; ++k) {
                 const int ti = lane + 32 * k;
-                dk[k] = ti < NT ? reinterpret_cast<volatile int *>(s_done)[R.te[ti]] - pub[k] : 0;
-                mine += dk[k];
+                if (ti < NT)
+                    for (int w = 0; w < NBW; ++w)
+                        any |= reinterpret_cast<volatile unsigned *>(s_done[ti])[w] != pub[k][w];
             }
-            if (__any_sync(kAll, mine > 0)) {
-                __threadfence();
+            if (__any_sync(kAll, any)) {
+                __threadfence();  // every row counted so far, before the adds
+                int mine = 0;
 #pragma unroll
-                for (int k = 0; k < kMaxE / 32; ++k)
-                    if (dk[k] > 0) {
-                        atomicAdd(a.e1_done + R.te[lane + 32 * k], dk[k]);
-                        pub[k] += dk[k];
+                for (int k = 0; k < kMaxE / 32; ++k) {
+                    const int ti = lane + 32 * k;
+                    if (ti >= NT) continue;
+                    for (int w = 0; w < NBW; ++w) {
+                        const unsigned now = reinterpret_cast<volatile unsigned *>(s_done[ti])[w];
+                        for (int q = 0; q < 4 && 4 * w + q < NB; ++q) {
+                            const int delta = int((now >> (8 * q)) & 255u) -
+                                              int((pub[k][w] >> (8 * q)) & 255u);
+                            if (delta > 0) {
+                                atomicAdd(a.e1_done + R.te[ti] * NB + 4 * w + q, delta);
+                                mine += delta;
+                            }
+                        }
+                        pub[k][w] = now;
                     }
+                }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(kAll, mine, off);
                 published += mine;
@@ -848,7 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u.up) {
             if (lane == 0) {
                 __threadfence_block();
-                atomicAdd(&s_done[u.e], 1);  // the publisher warp makes it visible
+                const int kb = u.row0 / kKT2;  // the publisher warp makes it visible
+                atomicAdd(&s_done[u.ti][kb >> 2], 1u << (8 * (kb & 3)));
             }
             continue;
         }

@@ -127,8 +127,9 @@ def test_one_launch_path_selection():
             P = abi.plan(dsc)
             assert P["one_launch"] == 1 and abi.kernel_count(dsc) == 1
             assert P["router_splits"] == 1
-            # counters: one per expert, one per (token, 16-row block of d)
-            assert P["off_ctl"] + 4 * (128 + T * 2048 // 16) <= P["workspace_bytes"]
+            # counters: one per (expert, 128 columns of H), one per (token, 16
+            # columns of the output)
+            assert P["off_ctl"] + 4 * (128 * 6 + T * 2048 // 16) <= P["workspace_bytes"]
             assert P["off_ctl"] >= P["off_tiles_sub"] and P["off_ctl"] % 256 == 0
         big = abi.plan(abi.desc(17, 2048, 128, 768, 8, "bf16", 1))
         assert big["one_launch"] == 0 and big["off_ctl"] + 0 <= big["workspace_bytes"]
