@@ -83,7 +83,7 @@ static_assert(kThreads == (kConsumers + 2) * 32, "a producer and a publisher war
 constexpr int kKT1 = 256, kKT2 = 128;
 constexpr int kStageMin = 8192;
 constexpr int kSlots = 8;  // units whose k-tiles may be in flight in one CTA
-constexpr int kTok = 4;  // tokens per pass of a router item (accumulators)
+constexpr int kTok = 2;  // tokens per pass of a router item (accumulators)
 
 // ------------------------------------------------------------ primitives --
 
@@ -226,6 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // gate/up units finished here per (touched expert, 128-column block of
     // H): one byte each (at most 16), four blocks to a word
     __shared__ unsigned s_done[kMaxE][4];
+    __shared__ unsigned s_pub[kMaxE * 4];  // the publisher's published counts, same packing
+    __shared__ int s_wtot[kMaxE / 32][4];   // expert scan: per-warp totals
     __shared__ float s_rp[kConsumers][2][kDlMaxT];  // router partial sums, per warp
     // A unit's k-tiles are items of their own, taken by any warp; their partial
     // sums meet in the unit's slot (slot j % kSlots), added in k-tile order:
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         R.cnt[i] = 0;
         R.tmask[i] = 0u;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) s_done[i][w] = 0u;
+        for (int w = 0; w < 4; ++w) s_done[i][w] = s_pub[4 * i + w] = 0u;
     }
     if (tid <= K) R.hist[tid] = 0;
     if (tid == 0) s_abort = 0;
@@ -457,41 +459,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag) return;
         const int NT = R.n_touched, n1u = NT * U1, NBW = (NB + 3) / 4;
         const int my_e1u = b < n1u ? (n1u - 1 - b) / G + 1 : 0;
-        unsigned pub[kMaxE / 32][4];  // counts already published, same packing
-#pragma unroll
-        for (int k = 0; k < kMaxE / 32; ++k)
-#pragma unroll
-            for (int w = 0; w < 4; ++w) pub[k][w] = 0u;
+        // Counts already published, in shared memory beside the live ones
+        // (the publisher's own; rolled loops: this warp runs beside the
+        // consumers, and its code competes with theirs for the instruction
+        // cache).
         int published = 0;
         uint64_t t0 = globaltimer_ns();
         while (published < my_e1u) {
             bool any = false;
-#pragma unroll
-            for (int k = 0; k < kMaxE / 32; ++k) {
-                const int ti = lane + 32 * k;
-                if (ti < NT)
-                    for (int w = 0; w < NBW; ++w)
-                        any |= reinterpret_cast<volatile unsigned *>(s_done[ti])[w] != pub[k][w];
-            }
+#pragma unroll 1
+            for (int i = lane; i < NT * NBW; i += 32)
+                any |= reinterpret_cast<volatile unsigned *>(&s_done[0][0])[(i / NBW) * 4 + i % NBW] !=
+                       s_pub[(i / NBW) * 4 + i % NBW];
             if (__any_sync(kAll, any)) {
-                __threadfence();  // every row counted so far, before the adds
+                __threadfence();  // every unit counted so far, before the adds
                 int mine = 0;
-#pragma unroll
-                for (int k = 0; k < kMaxE / 32; ++k) {
-                    const int ti = lane + 32 * k;
-                    if (ti >= NT) continue;
-                    for (int w = 0; w < NBW; ++w) {
-                        const unsigned now = reinterpret_cast<volatile unsigned *>(s_done[ti])[w];
-                        for (int q = 0; q < 4 && 4 * w + q < NB; ++q) {
-                            const int delta = int((now >> (8 * q)) & 255u) -
-                                              int((pub[k][w] >> (8 * q)) & 255u);
-                            if (delta > 0) {
-                                atomicAdd(a.e1_done + R.te[ti] * NB + 4 * w + q, delta);
-                                mine += delta;
-                            }
+#pragma unroll 1
+                for (int i = lane; i < NT * NBW; i += 32) {
+                    const int ti = i / NBW, w = i % NBW;
+                    const unsigned now =
+                        reinterpret_cast<volatile unsigned *>(&s_done[0][0])[ti * 4 + w];
+                    const unsigned was = s_pub[ti * 4 + w];
+#pragma unroll 1
+                    for (int q = 0; q < 4 && 4 * w + q < NB; ++q) {
+                        const int delta = int((now >> (8 * q)) & 255u) - int((was >> (8 * q)) & 255u);
+                        if (delta > 0) {
+                            atomicAdd(a.e1_done + R.te[ti] * NB + 4 * w + q, delta);
+                            mine += delta;
                         }
-                        pub[k][w] = now;
                     }
+                    s_pub[ti * 4 + w] = now;
                 }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(kAll, mine, off);
@@ -615,55 +612,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     consumers_sync();
-    if (warp == 0) {
-        // Lane l owns experts [8l, 8l + 8): padded rows, pairs, touched
-        // experts and tiles, summed along the lane, scanned across the warp
-        // (exclusive), then written along the lane again.  Rolled loops: this
-        // runs once per call, and unrolled straight-line code here cost ~5 us
-        // of instruction fetch.
+    // Thread e (of the first 8 warps) takes expert e: its padded rows, pairs,
+    // touched flag and tiles are scanned across the warp, then across the 8
+    // warp totals (exclusive prefixes, experts ascending).
+    if (warp < kMaxE / 32) {
         const int BN = a.BN, lbn = __ffs(BN) - 1;  // BN is a power of two
-        int tot[4] = {0, 0, 0, 0};  // rows, pairs, touched, tiles
-#pragma unroll 1
-        for (int q = 0; q < 8; ++q) {
-            const int e = lane * 8 + q;
-            const int c = (e < E && !*abort_flag) ? R.cnt[e] : 0;
-            const int nt = (c + BN - 1) >> lbn;
-            tot[0] += nt * BN;
-            tot[1] += c;
-            tot[2] += c > 0;
-            tot[3] += nt;
-        }
-        int pre[4];
+        const int e = tid;
+        const int c = (e < E && !*abort_flag) ? R.cnt[e] : 0;
+        const int nt = (c + BN - 1) >> lbn;
+        int v[4] = {nt * BN, c, c > 0, nt};  // rows, pairs, touched, tiles
+        int inc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            int v = tot[i];
-#pragma unroll 1
+            int x = v[i];
+#pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                const int o = __shfl_up_sync(kAll, v, off);
-                if (lane >= off) v += o;
+                const int o = __shfl_up_sync(kAll, x, off);
+                if (lane >= off) x += o;
             }
-            pre[i] = v - tot[i];  // exclusive
-            if (lane == 31) {
-                if (i == 0) R.n_rows = v;
-                if (i == 1) R.n_pairs = v;
-                if (i == 2) R.n_touched = v;  // 0 after a failure: no expert units
-                if (i == 3) R.n_tiles = v;
-            }
+            inc[i] = x;
+            if (lane == 31) s_wtot[warp][i] = x;
         }
-#pragma unroll 1
-        for (int q = 0; q < 8; ++q) {
-            const int e = lane * 8 + q;
-            if (e >= E) break;
-            const int c = !*abort_flag ? R.cnt[e] : 0;
-            const int nt = (c + BN - 1) >> lbn;
-            R.off[e] = pre[0];
-            R.coff[e] = pre[1];
-            R.toff[e] = pre[3];
-            if (c > 0) R.te[pre[2]] = e;
-            pre[0] += nt * BN;
-            pre[1] += c;
-            pre[2] += c > 0;
-            pre[3] += nt;
+        asm volatile("bar.sync 3, %0;" ::"n"(kMaxE) : "memory");  // the 8 scanning warps
+        int base[4] = {0, 0, 0, 0};
+        for (int w = 0; w < warp; ++w)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) base[i] += s_wtot[w][i];
+        if (e < E) {
+            R.off[e] = base[0] + inc[0] - v[0];
+            R.coff[e] = base[1] + inc[1] - v[1];
+            R.toff[e] = base[3] + inc[3] - v[3];
+            if (c > 0) R.te[base[2] + inc[2] - v[2]] = e;
+        }
+        if (tid == kMaxE - 1) {
+            R.n_rows = base[0] + inc[0];
+            R.n_pairs = base[1] + inc[1];
+            R.n_touched = base[2] + inc[2];  // 0 after a failure: no expert units
+            R.n_tiles = base[3] + inc[3];
         }
     }
     consumers_sync();
@@ -685,11 +670,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // as the multi-kernel path does, and zeroes the rows of tokens that keep
     // no expert (no down unit reaches them).
     if (b == G - 1) {
+#pragma unroll 1
         for (int i = tid; i < T * K; i += kConsumerThreads) {
             a.idx[i] = R.idx[i];
             a.w[i] = R.w[i];
             if (R.idx[i] >= 0) a.pair_pos[i] = R.pos[i];
         }
+#pragma unroll 1
         for (int i = tid; i < E; i += kConsumerThreads) a.counts[i] = R.cnt[i];
         if (tid <= K) a.hist[tid] = R.hist[tid];
         if (tid == 0) {
@@ -698,16 +685,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             a.hdr[kHdrMeta + 2] = R.n_pairs;
             a.hdr[kHdrMeta + 3] = 0;
         }
+#pragma unroll 1
         for (int q = warp; q < R.n_touched; q += kConsumers) {
             const int e = R.te[q], c = R.cnt[e], BN = a.BN;
             const int padded = (c + BN - 1) / BN * BN;
+#pragma unroll 1
             for (int j = lane; j < padded; j += 32)
                 a.pair[R.off[e] + j] = j < c ? R.pl[R.coff[e] + j] : -1;
+#pragma unroll 1
             for (int j = lane; j * BN < c; j += 32)
                 a.tiles[R.toff[e] + j] = make_int4(e, R.off[e] + j * BN, min(BN, c - j * BN), 0);
         }
+#pragma unroll 1
         for (int t = warp; t < T; t += kConsumers)
             if (R.nkept[t] == 0)
+#pragma unroll 1
                 for (int v = lane; v < nch; v += 32)
                     reinterpret_cast<uint4 *>(a.out)[size_t(t) * nch + v] = make_uint4(0, 0, 0, 0);
     }
@@ -753,6 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t pa = st + (a_row < 8 ? 0u : 4096u);
             const uint32_t pb0 = x_base + uint32_t((R.tok[coff + nA] * XSP + k0 + b_k) * 2);
             const uint32_t pb1 = x_base + uint32_t((R.tok[coff + nB] * XSP + k0 + b_k) * 2);
+#pragma unroll 1
             for (int ks = 0; ks < nks; ks += 2) {
                 uint32_t a0[4], a1[4], b0, b1, c0, c1;
                 const int jb = ks >> 2, ch = (ks & 3) * 2 + (a_col >> 3);
@@ -770,6 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         } else {
+#pragma unroll 1
             for (int ks = 0; ks < kKT2 / 16; ks += 2) {
                 uint32_t a0[4], a1[4], b0, b1, c0, c1;
                 const int jb = ks >> 2, ca = (ks & 3) * 2 + (a_col >> 3);
