@@ -39,11 +39,13 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("BN", ctypes.c_int), ("router_bn", ctypes.c_int),
                 ("router_splits", ctypes.c_int), ("p_cap", ctypes.c_int),
                 ("tiles_cap", ctypes.c_int), ("sub_bn", ctypes.c_int),
-                ("one_launch", ctypes.c_int)] + \
+                ("one_launch", ctypes.c_int), ("sh_bn", ctypes.c_int),
+                ("sh_split1", ctypes.c_int), ("sh_split2", ctypes.c_int)] + \
                [(n, ctypes.c_size_t) for n in (
                    "off_err", "off_meta", "off_counts", "off_hist", "off_partial", "off_idx",
                    "off_w", "off_pair", "off_pair_pos", "off_tiles", "off_xp", "off_h", "off_y",
-                   "off_tile_done", "off_hs", "off_ys", "off_tiles_sub", "off_ctl", "workspace_bytes")]
+                   "off_tile_done", "off_hs", "off_ys", "off_tiles_sub", "off_ctl", "off_sp",
+                   "workspace_bytes")]
 
 
 _lib = None
@@ -328,7 +330,7 @@ def workspace_views(dsc, workspace) -> dict:
         xp=view(P["off_xp"], P["p_cap"] * dsc.d, dt, es).view(P["p_cap"], dsc.d),
         h=view(P["off_h"], P["p_cap"] * dsc.I, dt, es).view(P["p_cap"], dsc.I),
         y=view(P["off_y"], P["p_cap"] * dsc.d, torch.float32, 4).view(P["p_cap"], dsc.d),
-        ys=view(P["off_ys"], dsc.n_shared * T * dsc.d, torch.float32, 4).view(
-            dsc.n_shared * T, dsc.d),
+        ys=view(P["off_ys"], max(1, P["sh_split2"]) * dsc.n_shared * T * dsc.d, torch.float32,
+                4).view(max(1, P["sh_split2"]) * dsc.n_shared * T, dsc.d),
         plan=P,
     )

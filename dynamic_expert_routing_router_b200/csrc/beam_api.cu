@@ -64,9 +64,28 @@ beam_status validate_desc(const beam_moe_desc *d) {
     return BEAM_OK;
 }
 
-// Token-tile height of the shared experts' GEMMs (every token, every shared
-// expert): thin tiles spread a decode batch's weight stream over more SMs.
-int shared_bn(int T) { return T <= 16 ? 16 : T <= 256 ? 32 : 128; }
+// Shared experts (every token, every shared expert): one token tile up to
+// 128 tokens (the MMA's N follows its valid rows), so their weights are read
+// once per 128 tokens, and the reductions split until about half the SMs
+// have a unit (the split partials are summed in split order).  Measured
+// (DeepSeekV2-Lite and Qwen1.5-MoE shapes, T = 1 and 128): half the SMs
+// beat a unit per SM (whose fp32 partials cost as much as the weights),
+// a quarter, and no split (T = 128, every candidate masked: 45.9 / 51.2
+// against 51.2 / 59.3, 46.9 / 63.4 and 61.0 / 63.4 us).
+void shared_plan(const beam_moe_desc *d, beam_moe_plan_info *P) {
+    const long long T = d->T, S = d->n_shared;
+    P->sh_bn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
+    const long long ntt = T > 0 ? cdiv(T, P->sh_bn) : 1;
+    const long long u1 = S * ntt * (d->I_shared / kBlockM), u2 = S * ntt * (d->d / kBlockM);
+    auto split = [](long long units, long long nk) {
+        long long k = cdiv(kNominalSMs / 2, units);
+        if (k > 8) k = 8;
+        if (k > nk) k = nk;
+        return int(k < 1 ? 1 : k);
+    };
+    P->sh_split1 = S > 0 ? split(u1, d->d / kBlockK) : 1;
+    P->sh_split2 = S > 0 ? split(u2, d->I_shared / kBlockK) : 1;
+}
 
 // Token-tile height of the expert GEMMs from the mean kept-or-not pairs per
 // expert (T*K/E): decode batches use thin tiles, prefill batches 128 rows, and
@@ -147,18 +166,21 @@ beam_status make_plan(const beam_moe_desc *d, beam_moe_plan_info *P, bool backwa
     P->off_y = align256(P->off_h + es * size_t(p_cap) * size_t(d->I));
     P->off_tile_done = align256(P->off_y + 4 * size_t(p_cap) * size_t(d->d));  // Y is fp32
     const size_t srows = size_t(d->n_shared) * size_t(T);  // shared rows: every token
+    shared_plan(d, P);
     P->off_hs = align256(P->off_tile_done + 4 * size_t(tiles_cap));
     P->off_ys = align256(P->off_hs + es * srows * size_t(d->n_shared > 0 ? d->I_shared : 0));
     // 256-row token tiles: the gate/up GEMM runs over 128-row sub-tiles of
     // them (two 128-row weight tiles and two accumulator buffers per unit).
     P->sub_bn = P->BN > kBlockM ? kBlockM : P->BN;
-    P->off_tiles_sub = align256(P->off_ys + 4 * srows * size_t(d->d));
+    P->off_tiles_sub = align256(P->off_ys + 4 * size_t(P->sh_split2) * srows * size_t(d->d));
     const size_t sub_cap = P->BN > kBlockM ? size_t(cdiv(T * K, kBlockM) + E) : 0;
     // one-launch counters: per expert, then per (token, down row block)
     P->off_ctl = align256(P->off_tiles_sub + 16 * sub_cap);
     const size_t ctl = small ? size_t(E) * size_t(d->I / 128) + size_t(T) * size_t(d->d / dl.R2)
                              : 0;
-    o = align256(P->off_ctl + 4 * ctl);
+    P->off_sp = align256(P->off_ctl + 4 * ctl);
+    const size_t sp = P->sh_split1 > 1 ? 2 * size_t(P->sh_split1) * srows * size_t(d->I_shared) : 0;
+    o = align256(P->off_sp + 4 * sp);
     P->workspace_bytes = o;
     return BEAM_OK;
 }
@@ -520,8 +542,11 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
 
     float *ys = reinterpret_cast<float *>(ws + P.off_ys);
     if (d->n_shared > 0) {
-        // Shared experts over every token (two dense launches; no grouping).
-        const int bn = shared_bn(d->T);
+        // Shared experts over every token (dense units; no grouping): the
+        // gate/up GEMM (its reduction split sh_split1 ways: partials, then a
+        // SwiGLU kernel), then the down GEMM (split sh_split2 ways: one slab
+        // of Ys per split, added by the combine).
+        const int bn = P.sh_bn;
         const int ntt = int(cdiv(d->T, bn));
         void *hs = ws + P.off_hs;
         const unsigned long long srows = (unsigned long long)d->n_shared * d->T;
@@ -546,18 +571,33 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
         g.dense = 1;
         g.dense_ntt = ntt;
         g.dense_T = d->T;
+        g.dense_slab_rows = int(srows);
         g.n_mb = d->I_shared / kBlockM;
         g.nk = d->d / kBlockK;
         g.a_rows_per_expert = d->I_shared;
-        g.n_units = d->n_shared * ntt * g.n_mb;
-        g.out = hs;
+        g.dense_ksplit = P.sh_split1;
+        g.n_units = d->n_shared * ntt * g.n_mb * P.sh_split1;
         g.out_ld = d->I_shared;
+        float *sp = reinterpret_cast<float *>(ws + P.off_sp);
+        const size_t slab1 = size_t(P.sh_split1) * srows * size_t(d->I_shared);
+        if (P.sh_split1 > 1) {  // fp32 partial pre-activations only
+            g.out = nullptr;
+            g.a_out = sp;
+            g.b_out = sp + slab1;
+        } else {
+            g.out = hs;
+        }
         BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, bn, m1, g, g.n_units < n_sm ? g.n_units : n_sm, st));
+        if (P.sh_split1 > 1)
+            BEAM_TRY_CUDA(launch_shared_swiglu(sp, sp + slab1, P.sh_split1,
+                                               (long long)srows * d->I_shared, hs, st));
+        g.a_out = g.b_out = nullptr;
         g.dense_gemm2 = 1;
         g.n_mb = d->d / kBlockM;
         g.nk = d->I_shared / kBlockK;
         g.a_rows_per_expert = d->d;
-        g.n_units = d->n_shared * ntt * g.n_mb;
+        g.dense_ksplit = P.sh_split2;
+        g.n_units = d->n_shared * ntt * g.n_mb * P.sh_split2;
         g.out = ys;
         g.out_ld = d->d;
         BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, bn, m2, g, g.n_units < n_sm ? g.n_units : n_sm, st));
@@ -565,7 +605,7 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
 
     BEAM_TRY_CUDA(rec.rec(6));
     BEAM_TRY_CUDA(launch_combine(out_dtype, y, idx, w, pair_pos, d->T, d->K, d->d, ys,
-                                 d->n_shared, out, n_sm, st));
+                                 d->n_shared * P.sh_split2, out, n_sm, st));
     BEAM_TRY_CUDA(rec.rec(7));
     return BEAM_OK;
 }
@@ -1216,7 +1256,7 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     if (make_plan(desc, &P) != BEAM_OK) return 0;
     if (desc->T == 0) return 0;
     if (P.one_launch) return 1;
-    const int shared = desc->n_shared > 0 ? 2 : 0;
+    const int shared = desc->n_shared > 0 ? (P.sh_split1 > 1 ? 3 : 2) : 0;
     // Fused decode path: rows copied by the grouping kernel (no gather
     // launch) and one launch for both expert GEMMs.
     return shared + ((desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 2

@@ -129,6 +129,12 @@ struct TcGemmArgs {
     // n_units / n_mb is (shared expert ti / dense_ntt, token tile ti % dense_ntt);
     // GEMM1 reads x rows, GEMM2 reads and both write rows s * T + token.
     int dense, dense_ntt, dense_T, dense_gemm2;
+    // Split reduction of dense units: unit u is (tile, m-block, split u % ksplit)
+    // over k-blocks [split * nk / ksplit, (split + 1) * nk / ksplit); its output
+    // rows move by split * dense_slab_rows (one slab per split).  GEMM1 with a
+    // null `out` writes only the fp32 pre-activations (a_out, b_out).
+    int dense_ksplit;
+    int dense_slab_rows;
 };
 
 cudaError_t launch_tc_gemm(int mode, int bn, const TcMaps &maps, const TcGemmArgs &args, int grid,
@@ -259,6 +265,11 @@ struct DlMaps {
 };
 cudaError_t launch_decode_layer(const DlMaps &maps, const DecodeLayerArgs &a, int grid,
                                 cudaStream_t stream);
+
+// Shared experts with a split gate/up reduction: H = SiLU(sum of the gate
+// partials) * (sum of the up partials), summed in split order, rounded to bf16.
+cudaError_t launch_shared_swiglu(const float *A, const float *B, int splits, long long n,
+                                 void *H, cudaStream_t stream);
 
 // Gather token rows into expert order (row_bytes multiple of 16).
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,

@@ -286,6 +286,38 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
     }
 }
 
+// --------------------------------------------- shared experts: SwiGLU ----
+// H[i] = SiLU(sum_j A[j][i]) * (sum_j B[j][i]), splits j in order, one bf16
+// rounding: the shared experts' gate/up GEMM with its reduction split.  The
+// same expression as the tensor-core epilogue's.
+__global__ void __launch_bounds__(256) shared_swiglu_kernel(const float4 *A, const float4 *B,
+                                                            int splits, long long n4,
+                                                            uint2 *H) {
+    griddep_wait();
+    griddep_launch_dependents();
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += 256ll * gridDim.x) {
+        float4 a = __ldg(A + i), b = __ldg(B + i);
+        for (int j = 1; j < splits; ++j) {
+            const float4 aj = __ldg(A + j * n4 + i), bj = __ldg(B + j * n4 + i);
+            a.x += aj.x;
+            a.y += aj.y;
+            a.z += aj.z;
+            a.w += aj.w;
+            b.x += bj.x;
+            b.y += bj.y;
+            b.z += bj.z;
+            b.w += bj.w;
+        }
+        const auto sm = [](float g, float u) { return g / (1.0f + __expf(-g)) * u; };
+        const __nv_bfloat162 h0 = __floats2bfloat162_rn(sm(a.x, b.x), sm(a.y, b.y));
+        const __nv_bfloat162 h1 = __floats2bfloat162_rn(sm(a.z, b.z), sm(a.w, b.w));
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t *>(&h0);
+        o.y = *reinterpret_cast<const uint32_t *>(&h1);
+        H[i] = o;
+    }
+}
+
 // ---------------------------------------------------------- fp32 path -----
 // Plain shared-memory tiled SIMT kernels for BEAM_F32 (small layers).  Each
 // output is one fp32 accumulator summed over the reduction index in order.
@@ -451,6 +483,17 @@ cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const floa
                           static_cast<__nv_bfloat16 *>(out));
     return launch_pdl(combine_kernel<float>, dim3(blocks), dim3(threads), 0, stream, Y, idx, w,
                       pair_pos, T, K, d, Ys, n_shared, static_cast<float *>(out));
+}
+
+cudaError_t launch_shared_swiglu(const float *A, const float *B, int splits, long long n,
+                                 void *H, cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    const long long n4 = n / 4;  // n: a multiple of 128 (I_shared)
+    long long blocks = (n4 + 255) / 256;
+    if (blocks > 4 * kNominalSMs) blocks = 4 * kNominalSMs;
+    return launch_pdl(shared_swiglu_kernel, dim3(unsigned(blocks)), dim3(256), 0, stream,
+                      reinterpret_cast<const float4 *>(A), reinterpret_cast<const float4 *>(B),
+                      splits, n4, static_cast<uint2 *>(H));
 }
 
 cudaError_t launch_router_f32(const float *x, const float *Wg, const float *Wm, int T, int d,

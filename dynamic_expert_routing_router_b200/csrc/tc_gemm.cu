@@ -147,10 +147,16 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_first, const TcGemmArgs
     w.mb = v % n_mb;
     w.ti = v / n_mb;
     if ((MODE == MODE_GEMM1 || MODE == MODE_GEMM2) && p.dense) {
+        const int ks = p.dense_ksplit > 1 ? p.dense_ksplit : 1;
+        const int js = u % ks, vv = u / ks;
+        w.mb = vv % n_mb;
+        w.ti = vv / n_mb;
+        w.kb0 = js * p.nk / ks;
+        w.nk = (js + 1) * p.nk / ks - w.kb0;
         const int sx = w.ti / p.dense_ntt, t0 = (w.ti % p.dense_ntt) * BN;
         w.a_row = sx * a_rows + w.mb * rows_per_mb;
-        w.out_row = sx * p.dense_T + t0;
-        w.b_row = p.dense_gemm2 ? w.out_row : t0;
+        w.out_row = js * p.dense_slab_rows + sx * p.dense_T + t0;
+        w.b_row = p.dense_gemm2 ? sx * p.dense_T + t0 : t0;
         w.rows = min(BN, p.dense_T - t0);
         return w;
     }
@@ -531,14 +537,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     epilogue_sync();
                 } else if (MODE == MODE_GEMM1) {
-                    // H (bf16): the next GEMM's operand.
-                    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
-                                         (long long)w.out_row * p.out_ld + w.mb * kBlockM + row;
+                    // H (bf16): the next GEMM's operand (none when the
+                    // reduction is split: the partials are summed later).
+                    if (p.out) {
+                        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) +
+                                             (long long)w.out_row * p.out_ld + w.mb * kBlockM + row;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        if (c0 + c < w.rows)
-                            out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(
-                                silu_mul(__uint_as_float(g[c]), __uint_as_float(v[c])));
+                        for (int c = 0; c < 16; ++c)
+                            if (c0 + c < w.rows)
+                                out[(long long)(c0 + c) * p.out_ld] = __float2bfloat16_rn(
+                                    silu_mul(__uint_as_float(g[c]), __uint_as_float(v[c])));
+                    }
                     if (p.a_out) {  // training: both pre-activations in fp32
                         const long long o = (long long)w.out_row * p.out_ld + w.mb * kBlockM + row;
 #pragma unroll

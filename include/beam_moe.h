@@ -110,7 +110,10 @@ typedef struct {
  *   h         [p_cap][I]  SiLU(x W1^T) * (x W3^T) per pair (dtype)
  *   y         f32[p_cap][d] expert output per pair
  *   hs        [n_shared*T][I_shared] shared experts' SwiGLU activations (dtype)
- *   ys        f32[n_shared*T][d] shared experts' outputs
+ *   ys        f32[sh_split2][n_shared*T][d] shared experts' outputs, one slab per
+ *             split of their down reduction (the combine adds every slab)
+ *   sp        f32[2][sh_split1][n_shared*T][I_shared] partial gate and up
+ *             pre-activations of the shared experts' split reduction
  *   tiles_sub int32[][4] with 256-row tiles: the same rows as 128-row tiles,
  *             the gate/up GEMM's units (their count in meta[3])
  *   ctl       int32[]     one-launch path: gate/up units finished per expert,
@@ -126,9 +129,12 @@ typedef struct {
     int tiles_cap;     /* entries of the tile list */
     int sub_bn;        /* token rows of the gate/up GEMM's tiles (BN, or 128 when BN = 256) */
     int one_launch;    /* 1: beam_moe_forward runs the whole layer as one kernel */
+    int sh_bn;         /* shared experts: token rows per tile */
+    int sh_split1;     /* shared experts: splits of the gate/up reduction (over d) */
+    int sh_split2;     /* shared experts: splits of the down reduction (over I_shared) */
     size_t off_err, off_meta, off_counts, off_hist, off_partial, off_idx, off_w,
         off_pair, off_pair_pos, off_tiles, off_xp, off_h, off_y, off_tile_done, off_hs,
-        off_ys, off_tiles_sub, off_ctl;
+        off_ys, off_tiles_sub, off_ctl, off_sp;
     size_t workspace_bytes;
 } beam_moe_plan_info;
 

@@ -164,7 +164,15 @@ def test_shared_expert_descriptor_rules():
     ok = abi.desc(64, 2048, 64, 1408, 6, "bf16", 1, n_shared=2, I_shared=1408)
     P = abi.plan(ok)
     assert P["off_ys"] > P["off_hs"] > P["off_tile_done"]
-    assert abi.kernel_count(ok) == abi.kernel_count(abi.desc(64, 2048, 64, 1408, 6)) + 2
+    # one token tile of 64 rows; the gate/up reduction (32 k-blocks) split 4
+    # ways over 22 units, the down reduction (22 k-blocks) 3 ways over 32 units
+    # (about half the SMs): gate/up GEMM, SwiGLU of the partials, down GEMM
+    assert (P["sh_bn"], P["sh_split1"], P["sh_split2"]) == (64, 4, 3)
+    assert P["off_sp"] + 4 * 2 * 4 * 2 * 64 * 1408 <= P["workspace_bytes"]
+    assert P["off_tiles_sub"] >= P["off_ys"] + 4 * 3 * 2 * 64 * 2048
+    assert abi.kernel_count(ok) == abi.kernel_count(abi.desc(64, 2048, 64, 1408, 6)) + 3
+    big = abi.plan(abi.desc(8192, 2048, 64, 1408, 6, "bf16", 1, n_shared=2, I_shared=1408))
+    assert (big["sh_bn"], big["sh_split1"], big["sh_split2"]) == (128, 1, 1)
     for bad, code in ((dict(n_shared=17, I_shared=128), 1), (dict(n_shared=2, I_shared=0), 1),
                       (dict(n_shared=2, I_shared=100), 2), (dict(n_shared=-1), 1)):
         with pytest.raises(abi.BeamError) as ei:

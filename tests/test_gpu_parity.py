@@ -474,7 +474,8 @@ def test_shared_experts_match_oracle(name, sh, S, T, f):
     o_rows = out.float().cpu().numpy().astype(np.float64)[rows]
     assert (bf16_excess(o_rows, ref) <= BF16_TOL_RMS).all()
     views = abi.workspace_views(dsc, ws)
-    assert_combine(out, views, "bf16", n_shared=S, ys=views["ys"])
+    # one slab of the shared experts' rows per split of their down reduction
+    assert_combine(out, views, "bf16", n_shared=S * views["plan"]["sh_split2"], ys=views["ys"])
 
 
 def test_shared_experts_serve_all_masked_tokens():
