@@ -238,7 +238,7 @@ def route_noalloc_check(stream=None):
     _ok(lib().beam_moe_route_noalloc_check(_stream(stream)), "beam_moe_route_noalloc_check")
 
 
-FAULT_NONE, FAULT_EXPERT_STAGE, FAULT_ROUTER_STAGE = 0, 1, 2
+FAULT_NONE, FAULT_EXPERT_STAGE, FAULT_ROUTER_STAGE, FAULT_SHARED_STAGE = 0, 1, 2, 3
 
 
 def set_fault_injection(mode: int, wait_limit_ns: int = 0):

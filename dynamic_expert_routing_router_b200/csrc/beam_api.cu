@@ -298,6 +298,48 @@ bool make_tmap(CUtensorMap *m, const void *base, unsigned long long inner,
     return true;
 }
 
+// A second stream per device for the shared experts, with the events that
+// fork it from the caller's stream and join it back.  Created on first use
+// outside a stream capture; held under a lock from the fork to the end of
+// the call's enqueue, so concurrent callers never interleave their events.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[kMaxDevices];
+
+// The current device's second stream, locked into *lock; null (the shared
+// experts then run on the caller's stream) when it does not exist yet and
+// `st` is being captured, or cannot be created.
+SideStream *side_stream(cudaStream_t st, std::unique_lock<std::mutex> *lock) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::unique_lock<std::mutex> lk(g_side_mu);
+    SideStream &ss = g_side[dev];
+    if (!ss.s) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+            return nullptr;
+        cudaStream_t s = nullptr;
+        cudaEvent_t f = nullptr, j = nullptr;
+        if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+            if (j) cudaEventDestroy(j);
+            if (f) cudaEventDestroy(f);
+            if (s) cudaStreamDestroy(s);
+            cudaGetLastError();
+            return nullptr;
+        }
+        ss.s = s;
+        ss.fork = f;
+        ss.join = j;
+    }
+    *lock = std::move(lk);
+    return &ss;
+}
+
 // Records the caller's timing events between stages.  External records
 // become event nodes when the call is captured into a CUDA graph, so the
 // per-kernel times can also be read from graph replays.
@@ -418,13 +460,90 @@ beam_status check_ws(const beam_moe_plan_info &P, const void *ws, size_t bytes) 
     return BEAM_OK;
 }
 
+// Shared experts over every token (dense units; no grouping), Ys = the
+// shared experts' outputs: on `st`, which may be a second stream beside the
+// routed experts' (nothing here reads the routing).  Timeouts go to the
+// header's shared-expert word (kSharedTimeoutTag), folded in by the combine.
+beam_status launch_shared_experts(const beam_moe_desc *d, const beam_moe_plan_info &P,
+                                  const void *x, const void *W1s, const void *W3s,
+                                  const void *W2s, char *ws, cudaStream_t st, int n_sm) {
+    float *ys = reinterpret_cast<float *>(ws + P.off_ys);
+    {
+        // Shared experts over every token (dense units; no grouping): the
+        // gate/up GEMM (its reduction split sh_split1 ways: partials, then a
+        // SwiGLU kernel), then the down GEMM (split sh_split2 ways: one slab
+        // of Ys per split, added by the combine).
+        const int bn = P.sh_bn;
+        const int ntt = int(cdiv(d->T, bn));
+        void *hs = ws + P.off_hs;
+        const unsigned long long srows = (unsigned long long)d->n_shared * d->T;
+        TcMaps m1, m2;
+        if (!make_tmap(&m1.a0, W1s, d->d, (unsigned long long)d->n_shared * d->I_shared, kBlockM))
+            return BEAM_ERR_CUDA;
+        if (!make_tmap(&m1.a1, W3s, d->d, (unsigned long long)d->n_shared * d->I_shared, kBlockM))
+            return BEAM_ERR_CUDA;
+        if (!make_tmap(&m1.b, x, d->d, d->T, bn)) return BEAM_ERR_CUDA;
+        m1.a2 = m1.a0;
+        m1.b2 = m1.b;
+        if (!make_tmap(&m2.a0, W2s, d->I_shared, (unsigned long long)d->n_shared * d->d, kBlockM))
+            return BEAM_ERR_CUDA;
+        if (!make_tmap(&m2.b, hs, d->I_shared, srows, bn)) return BEAM_ERR_CUDA;
+        m2.a1 = m2.a0;
+        m2.a2 = m2.a0;
+        m2.b2 = m2.b;
+        TcGemmArgs g;
+        std::memset(&g, 0, sizeof(g));
+        g.err = reinterpret_cast<int *>(ws) + kHdrErrShared;
+        g.err_code = kSharedTimeoutTag;
+        g.fault_skip = fault_mode() == FAULT_SHARED_STAGE;  // tests only
+        g.timeout_ns = wait_limit_ns();
+        g.dense = 1;
+        g.dense_ntt = ntt;
+        g.dense_T = d->T;
+        g.dense_slab_rows = int(srows);
+        g.n_mb = d->I_shared / kBlockM;
+        g.nk = d->d / kBlockK;
+        g.a_rows_per_expert = d->I_shared;
+        g.dense_ksplit = P.sh_split1;
+        g.n_units = d->n_shared * ntt * g.n_mb * P.sh_split1;
+        g.out_ld = d->I_shared;
+        float *sp = reinterpret_cast<float *>(ws + P.off_sp);
+        const size_t slab1 = size_t(P.sh_split1) * srows * size_t(d->I_shared);
+        if (P.sh_split1 > 1) {  // fp32 partial pre-activations only
+            g.out = nullptr;
+            g.a_out = sp;
+            g.b_out = sp + slab1;
+        } else {
+            g.out = hs;
+        }
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, bn, m1, g, g.n_units < n_sm ? g.n_units : n_sm, st));
+        if (P.sh_split1 > 1)
+            BEAM_TRY_CUDA(launch_shared_swiglu(sp, sp + slab1, P.sh_split1,
+                                               (long long)srows * d->I_shared, hs, st));
+        g.a_out = g.b_out = nullptr;
+        g.fault_skip = 0;
+        g.dense_gemm2 = 1;
+        g.n_mb = d->d / kBlockM;
+        g.nk = d->I_shared / kBlockK;
+        g.a_rows_per_expert = d->d;
+        g.dense_ksplit = P.sh_split2;
+        g.n_units = d->n_shared * ntt * g.n_mb * P.sh_split2;
+        g.out = ys;
+        g.out_ld = d->d;
+        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, bn, m2, g, g.n_units < n_sm ? g.n_units : n_sm, st));
+    }
+
+    return BEAM_OK;
+}
+
 // Stages 2-6 of a call whose routing (idx, w, counts, hist, a clean header)
 // is already in the workspace: grouping, row copy, expert GEMMs, shared
 // experts, combine.  out_dtype is the combine's output type.
 beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, const void *x,
                         const void *W1, const void *W3, const void *W2, const void *W1s,
                         const void *W3s, const void *W2s, void *out, int out_dtype, char *ws,
-                        cudaStream_t st, const Recorder &rec, int n_sm) {
+                        cudaStream_t st, const Recorder &rec, int n_sm,
+                        cudaEvent_t join = nullptr) {
     int *err = reinterpret_cast<int *>(ws + P.off_err);
     int *meta = reinterpret_cast<int *>(ws + P.off_meta);
     int *counts = reinterpret_cast<int *>(ws + P.off_counts);
@@ -541,71 +660,18 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
     }
 
     float *ys = reinterpret_cast<float *>(ws + P.off_ys);
-    if (d->n_shared > 0) {
-        // Shared experts over every token (dense units; no grouping): the
-        // gate/up GEMM (its reduction split sh_split1 ways: partials, then a
-        // SwiGLU kernel), then the down GEMM (split sh_split2 ways: one slab
-        // of Ys per split, added by the combine).
-        const int bn = P.sh_bn;
-        const int ntt = int(cdiv(d->T, bn));
-        void *hs = ws + P.off_hs;
-        const unsigned long long srows = (unsigned long long)d->n_shared * d->T;
-        TcMaps m1, m2;
-        if (!make_tmap(&m1.a0, W1s, d->d, (unsigned long long)d->n_shared * d->I_shared, kBlockM))
-            return BEAM_ERR_CUDA;
-        if (!make_tmap(&m1.a1, W3s, d->d, (unsigned long long)d->n_shared * d->I_shared, kBlockM))
-            return BEAM_ERR_CUDA;
-        if (!make_tmap(&m1.b, x, d->d, d->T, bn)) return BEAM_ERR_CUDA;
-        m1.a2 = m1.a0;
-        m1.b2 = m1.b;
-        if (!make_tmap(&m2.a0, W2s, d->I_shared, (unsigned long long)d->n_shared * d->d, kBlockM))
-            return BEAM_ERR_CUDA;
-        if (!make_tmap(&m2.b, hs, d->I_shared, srows, bn)) return BEAM_ERR_CUDA;
-        m2.a1 = m2.a0;
-        m2.a2 = m2.a0;
-        m2.b2 = m2.b;
-        TcGemmArgs g;
-        std::memset(&g, 0, sizeof(g));
-        g.err = err;
-        g.timeout_ns = wait_limit_ns();
-        g.dense = 1;
-        g.dense_ntt = ntt;
-        g.dense_T = d->T;
-        g.dense_slab_rows = int(srows);
-        g.n_mb = d->I_shared / kBlockM;
-        g.nk = d->d / kBlockK;
-        g.a_rows_per_expert = d->I_shared;
-        g.dense_ksplit = P.sh_split1;
-        g.n_units = d->n_shared * ntt * g.n_mb * P.sh_split1;
-        g.out_ld = d->I_shared;
-        float *sp = reinterpret_cast<float *>(ws + P.off_sp);
-        const size_t slab1 = size_t(P.sh_split1) * srows * size_t(d->I_shared);
-        if (P.sh_split1 > 1) {  // fp32 partial pre-activations only
-            g.out = nullptr;
-            g.a_out = sp;
-            g.b_out = sp + slab1;
-        } else {
-            g.out = hs;
-        }
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM1, bn, m1, g, g.n_units < n_sm ? g.n_units : n_sm, st));
-        if (P.sh_split1 > 1)
-            BEAM_TRY_CUDA(launch_shared_swiglu(sp, sp + slab1, P.sh_split1,
-                                               (long long)srows * d->I_shared, hs, st));
-        g.a_out = g.b_out = nullptr;
-        g.dense_gemm2 = 1;
-        g.n_mb = d->d / kBlockM;
-        g.nk = d->I_shared / kBlockK;
-        g.a_rows_per_expert = d->d;
-        g.dense_ksplit = P.sh_split2;
-        g.n_units = d->n_shared * ntt * g.n_mb * P.sh_split2;
-        g.out = ys;
-        g.out_ld = d->d;
-        BEAM_TRY_CUDA(launch_tc_gemm(MODE_GEMM2, bn, m2, g, g.n_units < n_sm ? g.n_units : n_sm, st));
+    if (d->n_shared > 0 && join == nullptr) {
+        const beam_status ss = launch_shared_experts(d, P, x, W1s, W3s, W2s, ws, st, n_sm);
+        if (ss != BEAM_OK) return ss;
     }
+    // The shared experts ran on a second stream: wait for them.
+    if (join) BEAM_TRY_CUDA(cudaStreamWaitEvent(st, join, 0));
 
     BEAM_TRY_CUDA(rec.rec(6));
     BEAM_TRY_CUDA(launch_combine(out_dtype, y, idx, w, pair_pos, d->T, d->K, d->d, ys,
-                                 d->n_shared * P.sh_split2, out, n_sm, st));
+                                 d->n_shared * P.sh_split2, out,
+                                 d->n_shared > 0 ? reinterpret_cast<int *>(ws) : nullptr, n_sm,
+                                 st));
     BEAM_TRY_CUDA(rec.rec(7));
     return BEAM_OK;
 }
@@ -687,11 +753,38 @@ beam_status forward_impl(const beam_moe_desc *d, const void *x, const void *Wg, 
         return BEAM_OK;
     }
 
+    // Shared experts read no routing: unless the caller times the stages,
+    // they run on a second stream from the start of the call, beside the
+    // router, top-K, grouping and routed experts, and the combine waits for
+    // both.  A captured call records the fork and the join as graph edges.
+    SideStream *side = nullptr;
+    std::unique_lock<std::mutex> side_lock;
+    if (d->n_shared > 0 && events == nullptr) {
+        side = side_stream(st, &side_lock);
+        if (side && (cudaEventRecord(side->fork, st) != cudaSuccess ||
+                     cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess))
+            return BEAM_ERR_CUDA;
+    }
+    if (side) {
+        s = launch_shared_experts(d, P, x, W1s, W3s, W2s, ws, side->s, n_sm);
+        // The join is recorded whatever happened, so that the caller's
+        // stream (or its capture) never leaves the second stream behind.
+        if (cudaEventRecord(side->join, side->s) != cudaSuccess) return BEAM_ERR_CUDA;
+        if (s != BEAM_OK) {
+            cudaStreamWaitEvent(st, side->join, 0);
+            return s;
+        }
+    }
+
     const RouteOut ro{idx, w, counts, hist, nullptr};
     s = launch_route(d, P, x, Wg, Wm, ro, ws, st, rec, n_sm);
-    if (s != BEAM_OK) return s;
-
-    return launch_tail(d, P, x, W1, W3, W2, W1s, W3s, W2s, out, d->dtype, ws, st, rec, n_sm);
+    // launch_tail waits for the join before the combine; on an earlier exit
+    // the caller's stream still joins the second stream here.
+    if (s == BEAM_OK)
+        s = launch_tail(d, P, x, W1, W3, W2, W1s, W3s, W2s, out, d->dtype, ws, st, rec, n_sm,
+                        side ? side->join : nullptr);
+    if (side && s != BEAM_OK) cudaStreamWaitEvent(st, side->join, 0);
+    return s;
 }
 
 
@@ -1212,7 +1305,7 @@ beam_status beam_moe_ep_combine(const beam_moe_desc *desc, const float *y_rows,
         if (!aligned16(p)) return BEAM_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     BEAM_TRY_CUDA(launch_combine(desc->dtype, y_rows, topk_idx, topk_w, pair_pos, desc->T, desc->K,
-                                 desc->d, nullptr, 0, out, sm_count(), st));
+                                 desc->d, nullptr, 0, out, nullptr, sm_count(), st));
     return BEAM_OK;
 }
 
@@ -1226,7 +1319,8 @@ float beam_moe_tau_to_logit(float tau) {
 }
 
 beam_status beam_moe_set_fault_injection(int mode, unsigned long long wait_limit_ns) {
-    if (mode != FAULT_NONE && mode != FAULT_EXPERT_STAGE && mode != FAULT_ROUTER_STAGE)
+    if (mode != FAULT_NONE && mode != FAULT_EXPERT_STAGE && mode != FAULT_ROUTER_STAGE &&
+        mode != FAULT_SHARED_STAGE)
         return BEAM_ERR_INVALID_ARG;
     g_fault.store(mode, std::memory_order_relaxed);
     g_wait_limit_ns.store(wait_limit_ns, std::memory_order_relaxed);

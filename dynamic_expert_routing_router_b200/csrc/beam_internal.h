@@ -23,11 +23,15 @@ enum : int { DEV_OK = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_INTERNAL = 2 };
 // tag, not a small code, so that a fresh workspace's leftover bytes are not
 // taken for a timeout.
 constexpr int kRouterTimeoutTag = 0x5EA71AB5;
-constexpr int kHdrErr = 0, kHdrErrRouter = 1, kHdrMeta = 4;  // int offsets in the header
+// The shared experts' GEMMs may run on a second stream, beside the router and
+// top-K kernels, so they do the same through the header's third word; the
+// combine, which runs after both streams have joined, folds and resets it.
+constexpr int kSharedTimeoutTag = 0x5EA75E0D;
+constexpr int kHdrErr = 0, kHdrErrRouter = 1, kHdrErrShared = 2, kHdrMeta = 4;  // int offsets
 
 // Fault injection for tests (beam_moe_set_fault_injection): which launch skips
 // one stage load in CTA 0 so that its MMA issuer's bounded wait expires.
-enum : int { FAULT_NONE = 0, FAULT_EXPERT_STAGE = 1, FAULT_ROUTER_STAGE = 2 };
+enum : int { FAULT_NONE = 0, FAULT_EXPERT_STAGE = 1, FAULT_ROUTER_STAGE = 2, FAULT_SHARED_STAGE = 3 };
 
 // Roles of the tensor-core GEMM kernel.
 enum TcMode : int {
@@ -277,10 +281,11 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
                           cudaStream_t stream);
 
 // out[t] = sum_k w[t,k] * Y[pair_pos[t,k]] over kept k; Y fp32, fp32 sums,
-// one rounding to the output dtype.
+// one rounding to the output dtype.  hdr (or null): the call's header, whose
+// shared-expert timeout tag is folded into its error word.
 cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
                            const int *pair_pos, int T, int K, int d, const float *Ys,
-                           int n_shared, void *out, int n_sm, cudaStream_t stream);
+                           int n_shared, void *out, int *hdr, int n_sm, cudaStream_t stream);
 
 // Training-mode backward (backward.cu).  Rows are those of the grouping of all
 // candidates (masked ones included); every array lives in the workspace.

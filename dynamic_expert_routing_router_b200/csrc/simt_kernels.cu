@@ -227,13 +227,19 @@ template <typename Tout>
 __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int *idx,
                                                       const float *w, const int *pair_pos, int T,
                                                       int K, int d, const float *Ys, int n_shared,
-                                                      Tout *out) {
+                                                      Tout *out, int *hdr) {
     __shared__ int s_row[kMaxK], s_slot[kMaxK];
     __shared__ float s_w[kMaxK], s_slotw[kMaxK];
     __shared__ int s_n;
     const int nvec = d / 8;
     griddep_wait();
     griddep_launch_dependents();
+    if (hdr && blockIdx.x == 0 && threadIdx.x == 0) {
+        // Every kernel of the call has finished (both streams joined before
+        // this launch): fold the shared experts' timeout tag, reset the word.
+        if (hdr[kHdrErrShared] == kSharedTimeoutTag) atomicExch(hdr + kHdrErr, DEV_ERR_TIMEOUT);
+        hdr[kHdrErrShared] = 0;
+    }
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < K) {  // slot metadata, one thread per slot
             const long long o = (long long)t * K + threadIdx.x;
@@ -472,7 +478,7 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
 
 cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
                            const int *pair_pos, int T, int K, int d, const float *Ys,
-                           int n_shared, void *out, int n_sm, cudaStream_t stream) {
+                           int n_shared, void *out, int *hdr, int n_sm, cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     int threads = d / 8;
     threads = threads >= 256 ? 256 : ((threads + 31) / 32) * 32;
@@ -480,9 +486,9 @@ cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const floa
     if (dtype == BEAM_BF16)
         return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), 0, stream,
                           Y, idx, w, pair_pos, T, K, d, Ys, n_shared,
-                          static_cast<__nv_bfloat16 *>(out));
+                          static_cast<__nv_bfloat16 *>(out), hdr);
     return launch_pdl(combine_kernel<float>, dim3(blocks), dim3(threads), 0, stream, Y, idx, w,
-                      pair_pos, T, K, d, Ys, n_shared, static_cast<float *>(out));
+                      pair_pos, T, K, d, Ys, n_shared, static_cast<float *>(out), hdr);
 }
 
 cudaError_t launch_shared_swiglu(const float *A, const float *B, int splits, long long n,

@@ -390,7 +390,9 @@ float beam_moe_tau_to_logit(float tau);
  *           first unit: it issues neither the copy nor the transaction count,
  *           so the MMA issuer's bounded wait on that stage expires;
  *   mode 2  the same in CTA 0 of the router GEMM of every later route or
- *           forward call (bf16 only).
+ *           forward call (bf16 only);
+ *   mode 3  the same in CTA 0 of the shared experts' gate/up GEMM of every
+ *           later forward call with shared experts (bf16 only).
  * The kernels then record the timeout, let their own copies and MMAs land,
  * free their tensor memory and return: beam_moe_check reports
  * BEAM_ERR_TIMEOUT and the context stays usable.  wait_limit_ns replaces the

@@ -101,6 +101,30 @@ def test_router_wait_timeout_reaches_the_error_word_then_recovers():
         abi.check(dsc, ws)  # the next call starts clean
 
 
+def test_shared_expert_wait_timeout_reaches_the_error_word_then_recovers():
+    """The shared experts' GEMMs run on a second stream beside the router and
+    top-K; their expiry goes through a tagged header word that the combine
+    folds into the error word."""
+    sh, S, T = inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED, 40
+    x, Wg, Wm, W1, W3, W2 = _layer(sh, T, 0.35, seed=4)
+    W1s, W3s, W2s = inputs.make_shared_experts(sh, S, seed=4, device=DEV)
+    dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm, n_shared=S, I_shared=sh.I)
+    ws = abi.alloc_workspace(dsc, DEV)
+    out = torch.empty((T, sh.d), dtype=torch.bfloat16, device=DEV)
+    with fault(abi.FAULT_SHARED_STAGE):
+        abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, out, ws)
+        with pytest.raises(abi.BeamError) as ei:
+            abi.check(dsc, ws)
+    assert ei.value.status == 5  # BEAM_ERR_TIMEOUT
+    abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, out, ws)
+    abi.check(dsc, ws)
+    ref = torch.empty_like(out)
+    ws2 = abi.alloc_workspace(dsc, DEV)
+    abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, ref, ws2)
+    abi.check(dsc, ws2)
+    assert torch.equal(out, ref)
+
+
 # ------------------------------------------------------------ guard bands --
 
 GUARD = 1024  # bytes of canary on each side (a multiple of 256: keeps alignment)

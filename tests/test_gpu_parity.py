@@ -496,3 +496,42 @@ def test_shared_experts_serve_all_masked_tokens():
     ref = np.zeros((T, d))
     oracle.add_shared(ref, host(x), host(W1s), host(W3s), host(W2s), "bf16")
     assert (bf16_excess(out.float().cpu().numpy().astype(np.float64), ref) <= BF16_TOL_RMS).all()
+
+
+def test_shared_experts_second_stream_graph_replay_and_dirty_workspace():
+    """The shared experts run on a second stream forked from the caller's and
+    joined before the combine.  Repeated calls, a CUDA-graph capture of the
+    call (fork and join become graph edges) and a workspace left dirty give
+    bitwise the same output; no call is left unjoined (the capture ends)."""
+    sh, S, T = inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED, 64
+    d, E, K, I = sh.d, sh.E, sh.K, sh.I
+    x = inputs.make_tokens(sh, T, seed=21, device=DEV)
+    Wg = inputs.make_gate(sh, seed=3, device=DEV)
+    Wm = inputs.make_mask(sh, 0.15, seed=3, device=DEV)
+    W1, W3, W2 = inputs.make_experts(sh, seed=3, device=DEV)
+    W1s, W3s, W2s = inputs.make_shared_experts(sh, S, seed=3, device=DEV)
+    dsc = abi.desc(T, d, E, I, K, "bf16", sh.renorm, n_shared=S, I_shared=I)
+    ws = abi.alloc_workspace(dsc, DEV)
+    ws.fill_(0xA5)
+    ref = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, ref, ws)
+    abi.check(dsc, ws)
+    out = torch.empty_like(ref)
+    for _ in range(3):
+        out.zero_()
+        abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, out, ws)
+        abi.check(dsc, ws)
+        assert torch.equal(out, ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    gout = torch.zeros_like(ref)
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, gout, ws, stream=s)
+    for _ in range(3):
+        gout.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        abi.check(dsc, ws)
+        assert torch.equal(gout, ref)
