@@ -579,7 +579,10 @@ beam_status launch_tail(const beam_moe_desc *d, const beam_moe_plan_info &P, con
         pa.tiles_sub = tiles_sub;
         pa.sub_bn = P.sub_bn;
     }
-    BEAM_TRY_CUDA(launch_permute(pa, st));
+    if (!fused && group_chunked_fits(d->T))  // large batches: chunked grouping (Y as scratch)
+        BEAM_TRY_CUDA(launch_group_chunked(pa, reinterpret_cast<int *>(y), st));
+    else
+        BEAM_TRY_CUDA(launch_permute(pa, st));
 
     BEAM_TRY_CUDA(rec.rec(3));
     if (!fused)
@@ -1353,8 +1356,9 @@ int beam_moe_forward_kernel_count(const beam_moe_desc *desc) {
     const int shared = desc->n_shared > 0 ? (P.sh_split1 > 1 ? 3 : 2) : 0;
     // Fused decode path: rows copied by the grouping kernel (no gather
     // launch) and one launch for both expert GEMMs.
-    return shared + ((desc->dtype == BEAM_BF16 && fused_experts(P)) ? BEAM_MOE_FORWARD_STAGES - 2
-                                                                     : BEAM_MOE_FORWARD_STAGES);
+    // Other batches: the grouping is two launches (chunked) up to 65536 tokens.
+    if (desc->dtype == BEAM_BF16 && fused_experts(P)) return shared + BEAM_MOE_FORWARD_STAGES - 2;
+    return shared + BEAM_MOE_FORWARD_STAGES + (group_chunked_fits(desc->T) ? 1 : 0);
 }
 
 const char *beam_moe_stage_name(int stage) {

@@ -185,6 +185,13 @@ struct PermuteArgs {
 };
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 
+// The same grouping (R = 1, no row copy) as two launches over token chunks:
+// per-chunk counts into chunk_cnt (at most 256 * E ints of scratch, 16-byte
+// aligned), then the placement.  Identical pair, pair_pos, tiles, tiles_sub and meta.
+// Only for T <= 65536 (group_chunked_fits).
+bool group_chunked_fits(int T);
+cudaError_t launch_group_chunked(const PermuteArgs &a, int *chunk_cnt, cudaStream_t stream);
+
 // Expert-parallel dispatch (ep_kernels.cu): kept pairs listed by expert
 // (ascending) then token, which groups them by destination rank r = e / (E/G).
 struct EpDispatchArgs {

@@ -173,6 +173,173 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermuteArgs
                      a.R * kGroupWarps, a.K, a.row_vec);
 }
 
+// ---------------------------------------------------- chunked grouping --
+//
+// The same grouping for large batches without a row copy, in two launches
+// over chunks of CT consecutive tokens (the per-expert listing above scans
+// every token once per expert).  Count: per chunk, the kept pairs of each
+// expert.  Place: a chunk's pairs of expert e start at off_e plus the pairs
+// of e in earlier chunks; within the chunk they follow token order (a bit per
+// token and expert, ranks by popcount).  Same rows, same order, same tiles as
+// the listing: every pair of expert e sits at off_e + (its token's rank among
+// e's tokens).
+constexpr int kChunkThreads = 256;
+
+// Tokens per chunk: 64, 128 or 256 (the chunk's token bits fit 8 words), at
+// most 256 chunks; 0 when T is too large for that.
+int group_chunk_tokens(int T) {
+    for (int ct = 64; ct <= 256; ct *= 2)
+        if ((T + ct - 1) / ct <= 256) return ct;
+    return 0;
+}
+
+__global__ void __launch_bounds__(kChunkThreads) group_count_kernel(const int *idx, int T, int K,
+                                                                  int E, int CT,
+                                                                  int *chunk_cnt) {
+    __shared__ int s_cnt[kMaxE];
+    for (int e = threadIdx.x; e < E; e += kChunkThreads) s_cnt[e] = 0;
+    __syncthreads();
+    griddep_wait();
+    griddep_launch_dependents();
+    const int t0 = blockIdx.x * CT, t1 = min(T, t0 + CT);
+    for (long long i = (long long)t0 * K + threadIdx.x; i < (long long)t1 * K; i += kChunkThreads) {
+        const int e = idx[i];
+        if (e >= 0) atomicAdd(&s_cnt[e], 1);
+    }
+    __syncthreads();
+    // expert-major: expert e's chunk counts are contiguous (pitch ncp)
+    const int ncp = (gridDim.x + 3) & ~3;
+    for (int e = threadIdx.x; e < E; e += kChunkThreads)
+        chunk_cnt[(long long)e * ncp + blockIdx.x] = s_cnt[e];
+}
+
+// Exclusive prefixes over the threads of the block (kChunkThreads) of N
+// values at once; tot[i] gets the sum of v[i].  Uses s_tmp[N][8].
+template <int N>
+__device__ __forceinline__ void chunk_block_scan(const int (&v)[N], int (&pre)[N], int (&tot)[N],
+                                                 int (*s_tmp)[kChunkThreads / 32]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        x[i] = v[i];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, x[i], off);
+            if (lane >= off) x[i] += o;
+        }
+    }
+    __syncthreads();
+    if (lane == 31)
+#pragma unroll
+        for (int i = 0; i < N; ++i) s_tmp[i][warp] = x[i];
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        int base = 0, all = 0;
+#pragma unroll
+        for (int w = 0; w < kChunkThreads / 32; ++w) {
+            if (w < warp) base += s_tmp[i][w];
+            all += s_tmp[i][w];
+        }
+        pre[i] = base + x[i] - v[i];
+        tot[i] = all;
+    }
+}
+
+__global__ void __launch_bounds__(kChunkThreads) group_place_kernel(const PermuteArgs a, int CT,
+                                                                  const int *chunk_cnt) {
+    __shared__ int s_base[kMaxE];   // first row of this chunk's pairs of each expert
+    __shared__ int s_off[kMaxE], s_toff[kMaxE], s_soff[kMaxE];
+    __shared__ unsigned s_mask[kMaxE][8];  // tokens of the chunk per expert (CT <= 256)
+    __shared__ int s_tmp[4][kChunkThreads / 32];
+    const int tid = threadIdx.x, c = blockIdx.x, nchunk = gridDim.x;
+    griddep_wait();
+    griddep_launch_dependents();
+    // per-expert offsets over the padded rows, tiles and sub-tiles (E <= 256)
+    const int cnt = tid < a.E ? a.counts[tid] : 0;
+    const int ntile = (cnt + a.BN - 1) / a.BN;
+    const int nsub = a.tiles_sub ? (cnt + a.sub_bn - 1) / a.sub_bn : 0;
+    const int vals[4] = {ntile * a.BN, ntile, nsub, cnt};
+    int pre[4], tot[4];
+    chunk_block_scan<4>(vals, pre, tot, s_tmp);
+    const int off = pre[0], toff = pre[1], soff = pre[2];
+    const int tot_rows = tot[0], tot_tiles = tot[1], tot_sub = tot[2], tot_pairs = tot[3];
+    if (tid < a.E) {
+        s_off[tid] = off;
+        s_toff[tid] = toff;
+        s_soff[tid] = soff;
+    }
+    for (int i = tid; i < a.E * 8; i += kChunkThreads) s_mask[i / 8][i % 8] = 0u;
+    const int ncp = (nchunk + 3) & ~3;
+    if (tid < a.E) {
+        // this expert's pairs in earlier chunks: its contiguous counts, four
+        // chunks per load
+        const int4 *row = reinterpret_cast<const int4 *>(chunk_cnt + (long long)tid * ncp);
+        int before = 0;
+#pragma unroll 8
+        for (int q4 = 0; q4 < (c + 3) / 4; ++q4) {
+            const int4 v = row[q4];
+            const int q = 4 * q4;
+            before += (q < c ? v.x : 0) + (q + 1 < c ? v.y : 0) + (q + 2 < c ? v.z : 0) +
+                      (q + 3 < c ? v.w : 0);
+        }
+        s_base[tid] = off + before;
+    }
+    __syncthreads();
+    if (c == 0 && tid == 0) {
+        a.meta[0] = tot_tiles;
+        a.meta[1] = tot_rows;
+        a.meta[2] = tot_pairs;
+        if (a.tiles_sub) a.meta[3] = tot_sub;
+    }
+    __syncthreads();
+    const int t0 = c * CT, t1 = min(a.T, t0 + CT);
+    for (long long i = (long long)t0 * a.K + tid; i < (long long)t1 * a.K; i += kChunkThreads) {
+        const int e = a.idx[i];
+        if (e >= 0) {
+            const int lt = int(i / a.K) - t0;
+            atomicOr(&s_mask[e][lt >> 5], 1u << (lt & 31));
+        }
+    }
+    __syncthreads();
+    for (long long i = (long long)t0 * a.K + tid; i < (long long)t1 * a.K; i += kChunkThreads) {
+        const int e = a.idx[i];
+        if (e >= 0) {
+            const int lt = int(i / a.K) - t0, wd = lt >> 5;
+            int rank = __popc(s_mask[e][wd] & ((1u << (lt & 31)) - 1u));
+            for (int q = 0; q < wd; ++q) rank += __popc(s_mask[e][q]);
+            const int pos = s_base[e] + rank;
+            a.pair[pos] = int(i);
+            a.pair_pos[i] = pos;
+        }
+    }
+    // Experts e = c, c + nchunk, ...: padding rows, tiles, sub-tiles, and the
+    // check that the chunks' counts add up to the expert's count.
+    for (int e = c; e < a.E; e += nchunk) {
+        const int count_e = a.counts[e];
+        if (tid < 32) {  // the chunks' counts of e add up to its count
+            int listed = 0;
+            for (int q = tid; q < nchunk; q += 32) listed += chunk_cnt[(long long)e * ncp + q];
+#pragma unroll
+            for (int off2 = 16; off2 > 0; off2 >>= 1)
+                listed += __shfl_xor_sync(0xffffffffu, listed, off2);
+            if (tid == 0 && listed != count_e) atomicExch(a.err, DEV_ERR_INTERNAL);
+        }
+        const int padded = (count_e + a.BN - 1) / a.BN * a.BN;
+        for (int r = count_e + tid; r < padded; r += kChunkThreads) a.pair[s_off[e] + r] = -1;
+        for (int j = tid; j * a.BN < count_e; j += kChunkThreads) {
+            a.tiles[s_toff[e] + j] =
+                make_int4(e, s_off[e] + j * a.BN, min(a.BN, count_e - j * a.BN), 0);
+            a.tile_done[s_toff[e] + j] = 0;
+        }
+        if (a.tiles_sub)
+            for (int j = tid; j * a.sub_bn < count_e; j += kChunkThreads)
+                a.tiles_sub[s_soff[e] + j] = make_int4(e, s_off[e] + j * a.sub_bn,
+                                                       min(a.sub_bn, count_e - j * a.sub_bn), 0);
+    }
+}
+
 // ------------------------------------------------------------------ gather --
 // One warp per permuted row, 16-byte vectors; padding rows are skipped (they
 // only feed padding columns of the GEMMs, which are never stored).
@@ -202,12 +369,14 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *x, const int *
 }
 
 // ----------------------------------------------------------------- combine --
-// One block per token; each thread owns 8 consecutive features.  The kept
+// A group of threads per token; each thread owns 8-feature chunks.  The kept
 // candidates' fp32 expert outputs are added in slot order k = 0..K-1 in fp32,
 // then rounded once to the output type.
-__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
-    const float4 a = *reinterpret_cast<const float4 *>(p);
-    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+
+// 8 floats through the read-only path (the data is not written in the kernel).
+__device__ __forceinline__ void load8_ro(const float *p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4 *>(p + 4));
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
@@ -223,15 +392,23 @@ __device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
     *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <typename Tout>
+// G threads per token (a power of two, 32..256), 256 / G tokens per block
+// and pass: the group's first warp lists the token's kept slots in slot order
+// (ballot, no serial loop), then every thread of the group owns 8-feature
+// chunks v = tig, tig + G, ...  Large batches take small groups, so that
+// every token of the batch is in flight at once; small batches take whole
+// blocks, so that a token's rows are read by many threads.
+template <typename Tout, int G>
 __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int *idx,
                                                       const float *w, const int *pair_pos, int T,
                                                       int K, int d, const float *Ys, int n_shared,
                                                       Tout *out, int *hdr) {
-    __shared__ int s_row[kMaxK], s_slot[kMaxK];
-    __shared__ float s_w[kMaxK], s_slotw[kMaxK];
-    __shared__ int s_n;
+    constexpr int TPB = 256 / G;
+    __shared__ int s_row[TPB][kMaxK];
+    __shared__ float s_w[TPB][kMaxK];
+    __shared__ int s_n[TPB];
     const int nvec = d / 8;
+    const int grp = threadIdx.x / G, tig = threadIdx.x % G, lane = threadIdx.x & 31;
     griddep_wait();
     griddep_launch_dependents();
     if (hdr && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -240,55 +417,67 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
         if (hdr[kHdrErrShared] == kSharedTimeoutTag) atomicExch(hdr + kHdrErr, DEV_ERR_TIMEOUT);
         hdr[kHdrErrShared] = 0;
     }
-    for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < K) {  // slot metadata, one thread per slot
-            const long long o = (long long)t * K + threadIdx.x;
-            s_slot[threadIdx.x] = idx[o] >= 0 ? pair_pos[o] : -1;
-            s_slotw[threadIdx.x] = w[o];
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {  // kept candidates of token t, in slot order
-            int n = 0;
-            for (int k = 0; k < K; ++k)
-                if (s_slot[k] >= 0) {
-                    s_row[n] = s_slot[k];
-                    s_w[n] = s_slotw[k];
-                    ++n;
-                }
-            s_n = n;
-        }
-        __syncthreads();
-        const int n = s_n;
-        for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            int j = 0;
-            for (; j + 4 <= n; j += 4) {  // four rows in flight, added in slot order
-                float y[4][8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) load8(Y + (long long)s_row[j + q] * d + v * 8, y[q]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float wk = s_w[j + q];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[q][i], acc[i]);
+    for (int t0 = blockIdx.x * TPB; t0 < T; t0 += gridDim.x * TPB) {
+        const int t = t0 + grp;
+        // G == 32: each warp owns its tokens and its slot lists; nothing is
+        // shared between warps, so they never wait for one another
+        if (G == 32) __syncwarp();
+        else __syncthreads();  // the slot lists are rewritten below
+        if (tig < 32) {  // kept candidates of token t, in slot order
+            int row = -1;
+            float wk = 0.0f;
+            if (t < T && lane < K) {
+                const long long o = (long long)t * K + lane;
+                if (idx[o] >= 0) {
+                    row = pair_pos[o];
+                    wk = w[o];
                 }
             }
-            for (; j < n; ++j) {
-                float y[8];
-                load8(Y + (long long)s_row[j] * d + v * 8, y);
-                const float wk = s_w[j];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
+            const unsigned kept = __ballot_sync(0xffffffffu, row >= 0);
+            if (row >= 0) {
+                const int p = __popc(kept & ((1u << lane) - 1u));
+                s_row[grp][p] = row;
+                s_w[grp][p] = wk;
             }
-            for (int sx = 0; sx < n_shared; ++sx) {  // shared experts, weight 1, in order
-                float y[8];
-                load8(Ys + ((long long)sx * T + t) * d + v * 8, y);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] += y[i];
-            }
-            store8(out + (long long)t * d + v * 8, acc);
+            if (lane == 0) s_n[grp] = __popc(kept);
         }
-        __syncthreads();
+        if (G == 32) __syncwarp();
+        else __syncthreads();
+        if (t < T) {
+            const int n = s_n[grp];
+            const int *rows = s_row[grp];
+            const float *ws = s_w[grp];
+#pragma unroll 2
+            for (int v = tig; v < nvec; v += G) {
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                int j = 0;
+                for (; j + 4 <= n; j += 4) {  // four rows in flight, added in slot order
+                    float y[4][8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) load8_ro(Y + (long long)rows[j + q] * d + v * 8, y[q]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float wk = ws[j + q];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[q][i], acc[i]);
+                    }
+                }
+                for (; j < n; ++j) {
+                    float y[8];
+                    load8_ro(Y + (long long)rows[j] * d + v * 8, y);
+                    const float wk = ws[j];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
+                }
+                for (int sx = 0; sx < n_shared; ++sx) {  // shared experts, weight 1, in order
+                    float y[8];
+                    load8_ro(Ys + ((long long)sx * T + t) * d + v * 8, y);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] += y[i];
+                }
+                store8(out + (long long)t * d + v * 8, acc);
+            }
+        }
     }
 }
 
@@ -465,6 +654,20 @@ cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream) {
     return launch_pdl(permute_kernel, dim3(a.E * a.R), dim3(kPermThreads), 0, stream, a);
 }
 
+bool group_chunked_fits(int T) { return group_chunk_tokens(T) > 0; }
+
+cudaError_t launch_group_chunked(const PermuteArgs &a, int *chunk_cnt, cudaStream_t stream) {
+    if (a.T <= 0) return cudaSuccess;
+    const int CT = group_chunk_tokens(a.T);
+    if (CT == 0) return cudaErrorInvalidValue;
+    const int nchunk = (a.T + CT - 1) / CT;
+    cudaError_t e = launch_pdl(group_count_kernel, dim3(nchunk), dim3(kChunkThreads), 0, stream,
+                               a.idx, a.T, a.K, a.E, CT, chunk_cnt);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(group_place_kernel, dim3(nchunk), dim3(kChunkThreads), 0, stream, a, CT,
+                      static_cast<const int *>(chunk_cnt));
+}
+
 cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K,
                           long long row_bytes, int p_cap, void *xp, int n_sm,
                           cudaStream_t stream) {
@@ -476,19 +679,42 @@ cudaError_t launch_gather(const void *x, const int *pair, const int *meta, int K
                       static_cast<uint4 *>(xp));
 }
 
+template <typename Tout>
+cudaError_t launch_combine_t(const float *Y, const int *idx, const float *w, const int *pair_pos,
+                             int T, int K, int d, const float *Ys, int n_shared, Tout *out,
+                             int *hdr, int n_sm, cudaStream_t stream) {
+    // Threads per token: the largest G that keeps every token of the batch
+    // in flight at once (8 blocks of 256 threads per SM), and no more than
+    // the token's 8-feature chunks need.
+    const long long slots = 8LL * n_sm * 256;
+    int G = 256;
+    while (G > 32 && (long long)T * G > slots) G >>= 1;
+    while (G > 32 && d / 8 <= G / 2) G >>= 1;
+    const int tpb = 256 / G;
+    long long blocks = ((long long)T + tpb - 1) / tpb;
+    if (blocks > 8LL * n_sm) blocks = 8LL * n_sm;
+    const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+    switch (G) {
+        case 256: return launch_pdl(combine_kernel<Tout, 256>, grid, block, 0, stream, Y, idx, w,
+                                    pair_pos, T, K, d, Ys, n_shared, out, hdr);
+        case 128: return launch_pdl(combine_kernel<Tout, 128>, grid, block, 0, stream, Y, idx, w,
+                                    pair_pos, T, K, d, Ys, n_shared, out, hdr);
+        case 64: return launch_pdl(combine_kernel<Tout, 64>, grid, block, 0, stream, Y, idx, w,
+                                   pair_pos, T, K, d, Ys, n_shared, out, hdr);
+        default: return launch_pdl(combine_kernel<Tout, 32>, grid, block, 0, stream, Y, idx, w,
+                                   pair_pos, T, K, d, Ys, n_shared, out, hdr);
+    }
+}
+
 cudaError_t launch_combine(int dtype, const float *Y, const int *idx, const float *w,
                            const int *pair_pos, int T, int K, int d, const float *Ys,
                            int n_shared, void *out, int *hdr, int n_sm, cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
-    int threads = d / 8;
-    threads = threads >= 256 ? 256 : ((threads + 31) / 32) * 32;
-    int blocks = T < 8 * n_sm ? T : 8 * n_sm;
     if (dtype == BEAM_BF16)
-        return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), 0, stream,
-                          Y, idx, w, pair_pos, T, K, d, Ys, n_shared,
-                          static_cast<__nv_bfloat16 *>(out), hdr);
-    return launch_pdl(combine_kernel<float>, dim3(blocks), dim3(threads), 0, stream, Y, idx, w,
-                      pair_pos, T, K, d, Ys, n_shared, static_cast<float *>(out), hdr);
+        return launch_combine_t(Y, idx, w, pair_pos, T, K, d, Ys, n_shared,
+                                static_cast<__nv_bfloat16 *>(out), hdr, n_sm, stream);
+    return launch_combine_t(Y, idx, w, pair_pos, T, K, d, Ys, n_shared, static_cast<float *>(out),
+                            hdr, n_sm, stream);
 }
 
 cudaError_t launch_shared_swiglu(const float *A, const float *B, int splits, long long n,

@@ -109,8 +109,9 @@ def test_argument_errors_return_before_any_launch():
 
 def test_kernel_count_per_path():
     assert abi.kernel_count(abi.desc(128, 2048, 128, 768, 8, "bf16", 1)) == 5  # fused, no gather
-    assert abi.kernel_count(abi.desc(8192, 2048, 128, 768, 8, "bf16", 1)) == 7
-    assert abi.kernel_count(abi.desc(64, 128, 8, 256, 2, "f32", 0)) == 7
+    # prefill and fp32: the grouping in two launches (per-chunk counts, placement)
+    assert abi.kernel_count(abi.desc(8192, 2048, 128, 768, 8, "bf16", 1)) == 8
+    assert abi.kernel_count(abi.desc(64, 128, 8, 256, 2, "f32", 0)) == 8
     assert abi.kernel_count(abi.desc(0, 2048, 128, 768, 8, "bf16", 1)) == 0
     assert abi.kernel_count(abi.desc(4, 2000, 128, 768, 8, "bf16", 1)) == 0
 
