@@ -494,10 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 MODE == MODE_GEMM1_IL || (MODE == MODE_EXPERTS && w.phase == 0);
             const bool down = MODE == MODE_GEMM2 || MODE == MODE_GEMM2T || MODE == MODE_GEMM1T ||
                               (MODE == MODE_EXPERTS && w.phase == 1);
-            // Split unit (MODE_EXPERTS, few tiles): store this split's fp32
-            // partial, free the accumulator and count the arrival.  The split
-            // that arrives last sums the group's partials in split order and
-            // finishes the unit from that sum; the others are done.
             const int ncol = unit_cols<MODE, BN>(w, p);  // same in the 4 epilogue warps
 #pragma unroll 1
             for (int c0 = 0; c0 < ncol; c0 += 16) {
