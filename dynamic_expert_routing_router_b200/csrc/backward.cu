@@ -670,15 +670,17 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
     }
 }
 
-// dW_gate[e] += sum_t dr[t][e] x_t (tokens ascending); dW_mask[e] += sum over
-// the candidate rows of e (token order) dz x.  Block (expert, 1024 columns):
-// 256 threads x 4 columns.  Each round of 256 tokens first lists the nonzero
-// dr[t][e] in token order (with renorm only the tokens that have e as a
-// candidate), so the sums run without branches and load eight rows at a time
-// (a popular expert has a term for nearly every token); zero terms add
-// nothing, so the order of the others is unchanged.
+// dW_gate[e] += sum_t dr[t][e] x_t; dW_mask[e] += sum over the candidate
+// rows of e (token order) dz x.  Block (expert, 128 columns): each warp holds
+// all 128 columns (4 per lane) for its own contiguous share of the terms, and
+// warp 0 adds the eight partial sums in warp order before the one
+// read-modify-write; a popular expert's terms are thus summed by eight warps
+// at once.  Each round of 256 tokens first lists the nonzero dr[t][e] in
+// token order (with renorm only the tokens that have e as a candidate), so
+// the sums run without branches and load eight rows at a time.  The order is
+// fixed: the same inputs give the same bits.
 constexpr int kDrChunk = 256;
-constexpr int kDrCols = 1024;
+constexpr int kDrCols = 128;
 // g[0..3] += sum over q < n (in order) c[q] * X[r[q]][j .. j+3]: the rows are
 // loaded eight at a time before their terms are added.
 template <typename TIn>
@@ -710,13 +712,14 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
     __shared__ int s_first, s_warp[8];
     __shared__ float s_c[kDrChunk];
     __shared__ int s_r[kDrChunk];
+    __shared__ __align__(16) float s_pg[8][kDrCols], s_pm[8][kDrCols];
     griddep_wait();
     griddep_launch_dependents();
-    const int e = blockIdx.x;
-    const int j = blockIdx.y * kDrCols + threadIdx.x * 4;
+    const int e = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int j = blockIdx.y * kDrCols + lane * 4;
     const bool active = j < a.d;
     const int d = a.d, E = a.E;
-    if (active) {
+    if (active && warp == 0) {
         prefetch_l2(dWg + (long long)e * d + j);
         if (dWm) prefetch_l2(dWm + (long long)e * d + j);
     }
@@ -731,7 +734,8 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
             s_r[pos] = t;
         }
         __syncthreads();
-        if (active) sum_rows(x, d, j, s_r, s_c, nz, gg);
+        const int q0 = warp * nz / 8, q1 = (warp + 1) * nz / 8;
+        if (active) sum_rows(x, d, j, s_r + q0, s_c + q0, q1 - q0, gg);
         __syncthreads();
     }
     const int n = a.counts_all[e];
@@ -745,19 +749,33 @@ __global__ void __launch_bounds__(256) bw_drouter_kernel(const BwArgs a, const T
                 s_c[q] = a.dz[a.pair[r]];
             }
             __syncthreads();
-            if (active) sum_rows(xp, d, j, s_r, s_c, cnt, gm);
+            const int q0 = warp * cnt / 8, q1 = (warp + 1) * cnt / 8;
+            if (active) sum_rows(xp, d, j, s_r + q0, s_c + q0, q1 - q0, gm);
             __syncthreads();
         }
     }
     if (active) {
+        *reinterpret_cast<float4 *>(&s_pg[warp][lane * 4]) = make_float4(gg[0], gg[1], gg[2], gg[3]);
+        *reinterpret_cast<float4 *>(&s_pm[warp][lane * 4]) = make_float4(gm[0], gm[1], gm[2], gm[3]);
+    }
+    __syncthreads();
+    if (warp == 0 && active) {
+        float4 sg = make_float4(0.f, 0.f, 0.f, 0.f), sm = sg;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {  // partial sums in warp order
+            const float4 pg = *reinterpret_cast<const float4 *>(&s_pg[w][lane * 4]);
+            const float4 pm = *reinterpret_cast<const float4 *>(&s_pm[w][lane * 4]);
+            sg.x += pg.x; sg.y += pg.y; sg.z += pg.z; sg.w += pg.w;
+            sm.x += pm.x; sm.y += pm.y; sm.z += pm.z; sm.w += pm.w;
+        }
         float4 *pg = reinterpret_cast<float4 *>(dWg + (long long)e * d + j);
         float4 u = *pg;
-        u.x += gg[0]; u.y += gg[1]; u.z += gg[2]; u.w += gg[3];
+        u.x += sg.x; u.y += sg.y; u.z += sg.z; u.w += sg.w;
         *pg = u;
         if (dWm) {
             float4 *pm = reinterpret_cast<float4 *>(dWm + (long long)e * d + j);
             float4 v = *pm;
-            v.x += gm[0]; v.y += gm[1]; v.z += gm[2]; v.w += gm[3];
+            v.x += sm.x; v.y += sm.y; v.z += sm.z; v.w += sm.w;
             *pm = v;
         }
     }
