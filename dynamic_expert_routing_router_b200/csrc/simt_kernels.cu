@@ -427,10 +427,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *Y, const int 
             int row = -1;
             float wk = 0.0f;
             if (t < T && lane < K) {
+                // three independent loads; a masked slot's pair_pos and w
+                // are read but not used
                 const long long o = (long long)t * K + lane;
-                if (idx[o] >= 0) {
-                    row = pair_pos[o];
-                    wk = w[o];
+                const int e = idx[o], pp = pair_pos[o];
+                const float ww = w[o];
+                if (e >= 0) {
+                    row = pp;
+                    wk = ww;
                 }
             }
             const unsigned kept = __ballot_sync(0xffffffffu, row >= 0);

@@ -38,14 +38,15 @@
 // expiry the CTA records DEV_ERR_TIMEOUT, drains its own copies and MMAs,
 // frees TMEM and returns.
 //
-// MODE_EXPERTS hands units out dynamically: the producer takes the next index
-// from a global counter (all gate/up units first, then the smaller down
-// units, so the tail is made of small units) and passes it to the MMA and
-// epilogue warps through a 4-slot ring in shared memory.  It cannot deadlock:
-// indices are handed out in increasing order, so every gate/up unit a down
-// unit waits for was already taken by a running CTA whose producer issued
-// all of that unit's loads before taking another index, and gate/up units
-// wait on nothing outside their CTA.  The other modes deal units round-robin.
+// MODE_EXPERTS hands units out dynamically: CTA b starts with unit b, then
+// its producer takes the next index from a global counter (all gate/up units
+// first, then the smaller down units, so the tail is made of small units) and
+// passes it to the MMA and epilogue warps through a 4-slot ring in shared
+// memory.  It cannot deadlock: gate/up units wait on nothing outside their
+// CTA; a down unit waits only for lower-numbered gate/up units, each of which
+// is a CTA's first unit (that CTA owns an SM of its own: the grid is at most
+// one CTA per SM) or was taken from the counter by a running CTA whose
+// producer issued all of that unit's loads before taking another index.  The other modes deal units round-robin.
 #include <cuda_bf16.h>
 
 #include "beam_internal.h"
@@ -301,7 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    u = atomicAdd(p.work_ctr, 1);
+                    // The first unit of CTA b is unit b (no global round trip
+                    // before the first loads); later ones come from the
+                    // counter, after the gridDim.x first units.
+                    u = lu == 0 ? int(blockIdx.x) : int(gridDim.x) + atomicAdd(p.work_ctr, 1);
                     if (u >= n_units) u = -1;
                     unit_ring[slot] = u;
                     mbar_arrive(&unit_full[slot]);
