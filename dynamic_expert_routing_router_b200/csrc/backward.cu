@@ -529,7 +529,12 @@ __device__ int stage_expert_chunk(const BwArgs &a, int first, int r0, int cnt, i
 }
 
 // dW1_e[i] += sum over kept rows (in order) da[r][i] x_r, dW3 likewise with db.
-// Block (expert, 4 rows of I); each thread owns 8 consecutive columns of d.
+// Block (expert, kDw13Groups groups of 4 rows of I); each thread owns 8
+// consecutive columns of d.  The expert's kept rows are listed once (when
+// they fit one chunk) and serve every group; each group's gradient rows are
+// prefetched into L2 while the previous group is summed, so the block's
+// read-modify-writes follow one another without a fresh staging chain.
+constexpr int kDw13Groups = 3;
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn *xp, float *dW1,
                                                       float *dW3) {
@@ -540,73 +545,90 @@ __global__ void __launch_bounds__(256) bw_dw13_kernel(const BwArgs a, const TIn 
     griddep_launch_dependents();
     const int e = blockIdx.x;
     if (a.counts_kept[e] == 0) return;  // no kept pair: no gradient, rows untouched
-    const int i0 = blockIdx.y * 4;
+    const int d = a.d, I = a.I;
+    const int ig0 = blockIdx.y * kDw13Groups * 4;  // first row of I of the block
+    // gradient rows of group g, this thread's columns, into L2
+    auto prefetch_group = [&](int i0, int j) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (i0 + i < I) {
+                const long long o = ((long long)e * I + i0 + i) * d + j;
+                prefetch_l2(dW1 + o);
+                prefetch_l2(dW3 + o);
+            }
+    };
+    if (threadIdx.x * 8 < d) prefetch_group(ig0, threadIdx.x * 8);
     const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
     const int n = a.counts_all[e];
-    const int d = a.d, I = a.I;
+    const bool one_chunk = n <= kWgChunk;
+    int nk = one_chunk ? stage_expert_chunk(a, first, 0, n, s_wc, s_kr) : 0;
     for (int jb = 0; jb < d; jb += 8 * blockDim.x) {
         const int j = jb + threadIdx.x * 8;
         const bool active = j < d;
-        if (active)
+        for (int g = 0; g < kDw13Groups; ++g) {
+            const int i0 = ig0 + 4 * g;
+            if (i0 >= I) break;
+            // this group's rows were prefetched one group ahead (or at the
+            // start); a new column pass prefetches its first group here
+            if (active && g == 0 && jb > 0) prefetch_group(i0, j);
+            if (active && g + 1 < kDw13Groups && i0 + 4 < I) prefetch_group(i0 + 4, j);
+            float g1[4][8], g3[4][8];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (i0 + i < I) {
-                    const long long o = ((long long)e * I + i0 + i) * d + j;
-                    prefetch_l2(dW1 + o);
-                    prefetch_l2(dW3 + o);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) g1[i][c] = g3[i][c] = 0.0f;
+            for (int r0 = 0; r0 < n; r0 += kWgChunk) {
+                if (!one_chunk)
+                    nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_wc, s_kr);
+                for (int q = threadIdx.x; q < 4 * nk; q += blockDim.x) {
+                    const int kq = q >> 2, i = q & 3;
+                    const bool ok = i0 + i < I;
+                    s_da[kq][i] = ok ? a.da[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
+                    s_db[kq][i] = ok ? a.db[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
                 }
-        float g1[4][8], g3[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) g1[i][c] = g3[i][c] = 0.0f;
-        for (int r0 = 0; r0 < n; r0 += kWgChunk) {
-            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_wc, s_kr);
-            for (int q = threadIdx.x; q < 4 * nk; q += blockDim.x) {
-                const int kq = q >> 2, i = q & 3;
-                const bool ok = i0 + i < I;
-                s_da[kq][i] = ok ? a.da[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
-                s_db[kq][i] = ok ? a.db[(long long)s_kr[kq] * I + i0 + i] : 0.0f;
-            }
-            __syncthreads();
-            if (active) {
+                __syncthreads();
+                if (active) {
 #pragma unroll 4
-                for (int kq = 0; kq < nk; ++kq) {
-                    float xv[8];
-                    load8(xp + (long long)s_kr[kq] * d + j, xv);
+                    for (int kq = 0; kq < nk; ++kq) {
+                        float xv[8];
+                        load8(xp + (long long)s_kr[kq] * d + j, xv);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float va = s_da[kq][i], vb = s_db[kq][i];
+                        for (int i = 0; i < 4; ++i) {
+                            const float va = s_da[kq][i], vb = s_db[kq][i];
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            g1[i][c] = fmaf(va, xv[c], g1[i][c]);
-                            g3[i][c] = fmaf(vb, xv[c], g3[i][c]);
+                            for (int c = 0; c < 8; ++c) {
+                                g1[i][c] = fmaf(va, xv[c], g1[i][c]);
+                                g3[i][c] = fmaf(vb, xv[c], g3[i][c]);
+                            }
                         }
                     }
                 }
+                __syncthreads();
             }
-            __syncthreads();
-        }
-        if (active) {
+            if (active) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if (i0 + i >= I) continue;
-                const long long o = ((long long)e * I + i0 + i) * d + j;
-                float4 *p1 = reinterpret_cast<float4 *>(dW1 + o);
-                float4 *p3 = reinterpret_cast<float4 *>(dW3 + o);
-                float4 u0 = p1[0], u1 = p1[1], v0 = p3[0], v1 = p3[1];
-                u0.x += g1[i][0]; u0.y += g1[i][1]; u0.z += g1[i][2]; u0.w += g1[i][3];
-                u1.x += g1[i][4]; u1.y += g1[i][5]; u1.z += g1[i][6]; u1.w += g1[i][7];
-                v0.x += g3[i][0]; v0.y += g3[i][1]; v0.z += g3[i][2]; v0.w += g3[i][3];
-                v1.x += g3[i][4]; v1.y += g3[i][5]; v1.z += g3[i][6]; v1.w += g3[i][7];
-                p1[0] = u0; p1[1] = u1; p3[0] = v0; p3[1] = v1;
+                for (int i = 0; i < 4; ++i) {
+                    if (i0 + i >= I) continue;
+                    const long long o = ((long long)e * I + i0 + i) * d + j;
+                    float4 *p1 = reinterpret_cast<float4 *>(dW1 + o);
+                    float4 *p3 = reinterpret_cast<float4 *>(dW3 + o);
+                    float4 u0 = p1[0], u1 = p1[1], v0 = p3[0], v1 = p3[1];
+                    u0.x += g1[i][0]; u0.y += g1[i][1]; u0.z += g1[i][2]; u0.w += g1[i][3];
+                    u1.x += g1[i][4]; u1.y += g1[i][5]; u1.z += g1[i][6]; u1.w += g1[i][7];
+                    v0.x += g3[i][0]; v0.y += g3[i][1]; v0.z += g3[i][2]; v0.w += g3[i][3];
+                    v1.x += g3[i][4]; v1.y += g3[i][5]; v1.z += g3[i][6]; v1.w += g3[i][7];
+                    p1[0] = u0; p1[1] = u1; p3[0] = v0; p3[1] = v1;
+                }
             }
         }
     }
 }
 
 // dW2_e[j] += sum over kept rows (in order) w_r dy_r[j] h_r (h fp32 from the
-// finalize step).  Block (expert, 8 rows of d); each thread owns 4 columns of I.
+// finalize step).  Block (expert, kDw2Groups groups of 8 rows of d); each
+// thread owns 4 columns of I.  As in bw_dw13_kernel, the kept rows are listed
+// once and each group's gradient rows are prefetched one group ahead.
+constexpr int kDw2Groups = 3;
 template <typename TIn>
 __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *dyp, float *dW2) {
     __shared__ int s_first;
@@ -616,55 +638,71 @@ __global__ void __launch_bounds__(256) bw_dw2_kernel(const BwArgs a, const TIn *
     griddep_launch_dependents();
     const int e = blockIdx.x;
     if (a.counts_kept[e] == 0) return;
-    const int j0 = blockIdx.y * 8;
-    const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
-    const int n = a.counts_all[e];
     const int d = a.d, I = a.I;
-    for (int ib = 0; ib < I; ib += 4 * blockDim.x) {
-        const int i = ib + threadIdx.x * 4;
-        const bool active = i < I;
-        if (active && (threadIdx.x & 1) == 0)  // one request per 32-byte sector
+    const int jg0 = blockIdx.y * kDw2Groups * 8;  // first row of d of the block
+    auto prefetch_group = [&](int j0, int i) {  // one request per 32-byte sector
+        if ((threadIdx.x & 1) == 0)
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj)
                 if (j0 + jj < d) prefetch_l2(dW2 + ((long long)e * d + j0 + jj) * I + i);
-        float g[8][4];
+    };
+    if (threadIdx.x * 4 < I) prefetch_group(jg0, threadIdx.x * 4);
+    const int first = expert_first_row(a.tiles, a.meta[0], e, &s_first);
+    const int n = a.counts_all[e];
+    const bool one_chunk = n <= kWgChunk;
+    int nk = one_chunk ? stage_expert_chunk(a, first, 0, n, s_wc, s_kr) : 0;
+    for (int ib = 0; ib < I; ib += 4 * blockDim.x) {
+        const int i = ib + threadIdx.x * 4;
+        const bool active = i < I;
+        for (int gq = 0; gq < kDw2Groups; ++gq) {
+            const int j0 = jg0 + 8 * gq;
+            if (j0 >= d) break;
+            // this group's rows were prefetched one group ahead (or at the
+            // start); a new column pass prefetches its first group here
+            if (active && gq == 0 && ib > 0) prefetch_group(j0, i);
+            if (active && gq + 1 < kDw2Groups && j0 + 8 < d) prefetch_group(j0 + 8, i);
+            float g[8][4];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
+            for (int jj = 0; jj < 8; ++jj)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) g[jj][c] = 0.0f;
-        for (int r0 = 0; r0 < n; r0 += kWgChunk) {
-            const int nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_wc, s_kr);
-            for (int q = threadIdx.x; q < 8 * nk; q += blockDim.x) {
-                const int kq = q >> 3, jj = q & 7;
-                const int r = s_kr[kq];
-                const float wk = a.w[a.pair[r]];
-                s_dy[kq][jj] = (j0 + jj < d) ? wk * load_f(dyp, (long long)r * d + j0 + jj) : 0.0f;
-            }
-            __syncthreads();
-            if (active) {
+                for (int c = 0; c < 4; ++c) g[jj][c] = 0.0f;
+            for (int r0 = 0; r0 < n; r0 += kWgChunk) {
+                if (!one_chunk)
+                    nk = stage_expert_chunk(a, first, r0, min(kWgChunk, n - r0), s_wc, s_kr);
+                for (int q = threadIdx.x; q < 8 * nk; q += blockDim.x) {
+                    const int kq = q >> 3, jj = q & 7;
+                    const int r = s_kr[kq];
+                    const float wk = a.w[a.pair[r]];
+                    s_dy[kq][jj] =
+                        (j0 + jj < d) ? wk * load_f(dyp, (long long)r * d + j0 + jj) : 0.0f;
+                }
+                __syncthreads();
+                if (active) {
 #pragma unroll 4
-                for (int kq = 0; kq < nk; ++kq) {
-                    const float4 hv = *reinterpret_cast<const float4 *>(a.h + (long long)s_kr[kq] * I + i);
+                    for (int kq = 0; kq < nk; ++kq) {
+                        const float4 hv =
+                            *reinterpret_cast<const float4 *>(a.h + (long long)s_kr[kq] * I + i);
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        const float dv = s_dy[kq][jj];
-                        g[jj][0] = fmaf(dv, hv.x, g[jj][0]);
-                        g[jj][1] = fmaf(dv, hv.y, g[jj][1]);
-                        g[jj][2] = fmaf(dv, hv.z, g[jj][2]);
-                        g[jj][3] = fmaf(dv, hv.w, g[jj][3]);
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const float dv = s_dy[kq][jj];
+                            g[jj][0] = fmaf(dv, hv.x, g[jj][0]);
+                            g[jj][1] = fmaf(dv, hv.y, g[jj][1]);
+                            g[jj][2] = fmaf(dv, hv.z, g[jj][2]);
+                            g[jj][3] = fmaf(dv, hv.w, g[jj][3]);
+                        }
                     }
                 }
+                __syncthreads();
             }
-            __syncthreads();
-        }
-        if (active) {
+            if (active) {
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                if (j0 + jj >= d) continue;
-                float4 *p = reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
-                float4 v = *p;
-                v.x += g[jj][0]; v.y += g[jj][1]; v.z += g[jj][2]; v.w += g[jj][3];
-                *p = v;
+                for (int jj = 0; jj < 8; ++jj) {
+                    if (j0 + jj >= d) continue;
+                    float4 *p = reinterpret_cast<float4 *>(dW2 + ((long long)e * d + j0 + jj) * I + i);
+                    float4 v = *p;
+                    v.x += g[jj][0]; v.y += g[jj][1]; v.z += g[jj][2]; v.w += g[jj][3];
+                    *p = v;
+                }
             }
         }
     }
@@ -886,10 +924,11 @@ cudaError_t backward_stages(const BwArgs &a, const T *x, const T *xp, const T *d
     }
     if ((e = launch_pdl(bw_dx_kernel<T>, dim3(tb), dim3(256), 0, st, a, Wg, Wm, a.dx_tc ? 1 : a.S)))
         return e;
-    if ((e = launch_pdl(bw_dw13_kernel<T>, dim3(a.E, (a.I + 3) / 4), dim3(256), 0, st, a, xp, dW1,
-                        dW3)))
+    if ((e = launch_pdl(bw_dw13_kernel<T>, dim3(a.E, (a.I + 4 * kDw13Groups - 1) / (4 * kDw13Groups)),
+                        dim3(256), 0, st, a, xp, dW1, dW3)))
         return e;
-    if ((e = launch_pdl(bw_dw2_kernel<T>, dim3(a.E, (a.d + 7) / 8), dim3(256), 0, st, a, dyp, dW2)))
+    if ((e = launch_pdl(bw_dw2_kernel<T>, dim3(a.E, (a.d + 8 * kDw2Groups - 1) / (8 * kDw2Groups)),
+                        dim3(256), 0, st, a, dyp, dW2)))
         return e;
     return launch_pdl(bw_drouter_kernel<T>, dim3(a.E, (a.d + kDrCols - 1) / kDrCols), dim3(256), 0,
                       st, a, x, xp, dWg, dWm);
