@@ -377,22 +377,42 @@ __global__ void __launch_bounds__(256) dh_finalize_kernel(const BwArgs a, int S)
     const int nk = stage_kept_rows(a, tile.y, tile.z, s_flag, s_fw, s_row, s_w, &s_n);
     const int I = a.I;
     const long long split = (long long)a.p_cap * I;
-    // Every (kept row, column) of the tile in one loop: the loads of all rows
-    // are independent.
-    for (int qi = threadIdx.x; qi < nk * I; qi += blockDim.x) {
-        const int q = qi / I, i = qi - q * I;
-        {
-            const long long o = (long long)s_row[q] * I + i;
-            float c = 0.0f;
-            for (int sp = 0; sp < S; ++sp) c += a.part[sp * split + o];
-            const float dh = s_w[q] * c;
-            const float av = a.A[o], bv = a.B[o], sa = sigm(av);
-            a.da[o] = dh * bv * sa * (1.0f + av * (1.0f - sa));
-            a.db[o] = dh * av * sa;
-            a.h[o] = av * sa * bv;
+    // Every (kept row, column) of the tile in one loop, kFinBatch items per
+    // thread and pass: all their loads are issued before any result is
+    // stored (the stores would otherwise hold back the next item's loads).
+    constexpr int kFinBatch = 4;
+    const int n_items = nk * I;
+    for (int qb = threadIdx.x; qb < n_items; qb += kFinBatch * blockDim.x) {
+        long long o[kFinBatch];
+        float c[kFinBatch], av[kFinBatch], bv[kFinBatch], wq[kFinBatch];
+#pragma unroll
+        for (int u = 0; u < kFinBatch; ++u) {
+            const int qi = qb + u * blockDim.x;
+            o[u] = -1;
+            if (qi < n_items) {
+                const int q = qi / I, i = qi - q * I;
+                o[u] = (long long)s_row[q] * I + i;
+                wq[u] = s_w[q];
+                float cs = 0.0f;
+                for (int sp = 0; sp < S; ++sp) cs += a.part[sp * split + o[u]];
+                c[u] = cs;
+                av[u] = a.A[o[u]];
+                bv[u] = a.B[o[u]];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kFinBatch; ++u) {
+            if (o[u] < 0) continue;
+            const float dh = wq[u] * c[u];
+            const float sa = sigm(av[u]);
+            const float da = dh * bv[u] * sa * (1.0f + av[u] * (1.0f - sa));
+            const float db = dh * av[u] * sa;
+            a.da[o[u]] = da;
+            a.db[o[u]] = db;
+            a.h[o[u]] = av[u] * sa * bv[u];
             if (a.da_bf) {  // operands of the tensor-core dx product
-                static_cast<__nv_bfloat16 *>(a.da_bf)[o] = __float2bfloat16_rn(a.da[o]);
-                static_cast<__nv_bfloat16 *>(a.db_bf)[o] = __float2bfloat16_rn(a.db[o]);
+                static_cast<__nv_bfloat16 *>(a.da_bf)[o[u]] = __float2bfloat16_rn(da);
+                static_cast<__nv_bfloat16 *>(a.db_bf)[o[u]] = __float2bfloat16_rn(db);
             }
         }
     }
