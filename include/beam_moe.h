@@ -186,9 +186,20 @@ beam_status beam_moe_forward(const beam_moe_desc *desc, const void *x, const voi
 /* beam_moe_forward with shared experts (desc->n_shared > 0): out = routed sum
  * (Eq. 8) + sum over the shared experts of E_s(x), the shared experts run for
  * every token.  W1s (gate), W3s (up) [n_shared, I_shared, d], W2s (down)
- * [n_shared, d, I_shared], bf16.  Two more launches than beam_moe_forward
- * (a gate/up and a down GEMM over all tokens), inside the down-GEMM stage slot.
- * With n_shared == 0 it is beam_moe_forward (the shared pointers may be NULL). */
+ * [n_shared, d, I_shared], bf16.  Two or three more launches than
+ * beam_moe_forward (a gate/up GEMM, when its reduction is split a SwiGLU
+ * kernel, and a down GEMM over all tokens; see beam_moe_forward_kernel_count).
+ * They read no routing, so they run on a second stream that the library owns
+ * (one per device, created by the first such call made outside a stream
+ * capture): the call records an event on `stream` at its start, the second
+ * stream waits for it, and `stream` waits for the second stream's event
+ * before the combine.  Work issued on `stream` after the call therefore
+ * follows all of it, as with any other call; a captured call records the
+ * fork and the join as graph edges.  A first call made inside a capture runs
+ * the shared experts on `stream` itself.  Calls are serialised on the host
+ * from the fork to the end of their enqueue (a lock), so concurrent callers
+ * never interleave their events.  With n_shared == 0 it is beam_moe_forward
+ * (the shared pointers may be NULL). */
 beam_status beam_moe_forward_shared(const beam_moe_desc *desc, const void *x,
                                     const void *W_gate, const void *W_mask, const void *W1,
                                     const void *W3, const void *W2, const void *W1s,
