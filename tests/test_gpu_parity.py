@@ -330,6 +330,10 @@ EDGE = [
     ("T1_all_kept", 1, 2048, 128, 768, 8, 1, 1.0),
     ("bn64_T600", 600, 1024, 128, 256, 8, 1, 0.35),
     ("bn32_T400", 400, 2048, 128, 768, 8, 1, 0.6),
+    # the chunked grouping's larger chunks: 128 tokens (T > 16384) and 256
+    # tokens (T > 32768), with a ragged last chunk
+    ("chunked_T20000_ct128", 20000, 128, 8, 128, 2, 0, 0.5),
+    ("chunked_T40003_ct256", 40003, 128, 16, 128, 2, 1, 0.35),
 ]
 
 
