@@ -539,3 +539,48 @@ def test_shared_experts_second_stream_graph_replay_and_dirty_workspace():
         torch.cuda.synchronize()
         abi.check(dsc, ws)
         assert torch.equal(gout, ref)
+
+
+_FIRST_CALL_CAPTURED = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from dynamic_expert_routing_router_b200 import abi, inputs
+sh, S, T = inputs.DSV2_LITE, inputs.DSV2_LITE_SHARED, 24
+x = inputs.make_tokens(sh, T, seed=41, device="cuda")
+Wg = inputs.make_gate(sh, seed=3, device="cuda")
+Wm = inputs.make_mask(sh, 0.35, seed=3, device="cuda")
+W1, W3, W2 = inputs.make_experts(sh, seed=3, device="cuda")
+W1s, W3s, W2s = inputs.make_shared_experts(sh, S, seed=3, device="cuda")
+dsc = abi.desc(T, sh.d, sh.E, sh.I, sh.K, "bf16", sh.renorm, n_shared=S, I_shared=sh.I)
+ws = abi.alloc_workspace(dsc, "cuda")
+gout = torch.zeros((T, sh.d), dtype=torch.bfloat16, device="cuda")
+torch.cuda.synchronize()
+s = torch.cuda.Stream()
+s.wait_stream(torch.cuda.current_stream())
+g = torch.cuda.CUDAGraph()
+with torch.cuda.stream(s):
+    with torch.cuda.graph(g, stream=s):  # the process's first shared-expert call
+        abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, gout, ws, stream=s)
+g.replay()
+torch.cuda.synchronize()
+abi.check(dsc, ws)
+ref = torch.empty_like(gout)
+abi.forward_shared(dsc, x, Wg, Wm, W1, W3, W2, W1s, W3s, W2s, ref, ws)  # eager: second stream
+abi.check(dsc, ws)
+assert torch.equal(gout, ref)
+print("ok")
+"""
+
+
+def test_shared_experts_first_call_inside_a_capture():
+    """A process whose first shared-expert call is captured: the library
+    creates no stream inside the capture and runs the shared experts on the
+    caller's stream; the replay equals a later eager call (second stream)
+    bit for bit."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FIRST_CALL_CAPTURED, root], capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
